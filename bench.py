@@ -1,0 +1,392 @@
+"""Benchmark of the ASM hot path on B200.
+
+Headline: the decode step of Attention State Memory at the LLaMA-3.1-8B
+single-layer shape (32 query heads, 8 KV heads, head dim 128, K=1024
+centroids per head, local KV cache of 2048 tokens, batch 1, bf16).  One
+benchmark step decodes one token through 32 such layers, each with its own
+memory and KV cache (537 MB in all, more than the 126 MB L2, so every step
+streams its bytes from HBM); the 32 launches are replayed from a CUDA graph.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl asm|reference]
+
+Prints ONE JSON line (rank 0).  `value` is decode query-heads/s over all
+ranks (each rank runs its own independent replica: weak scaling), timed with
+CUDA events between barriers; `roofline` is the decode kernel's algorithmic
+HBM bytes per launch over its average launch time against the measured HBM
+copy peak; `e2e` repeats the measurement through the public API with the
+per-step queries copied from pinned host memory and the outputs copied back;
+`cpu_baseline` times the fp64 oracle on the host cores (a bounded sample);
+`build` times the offline memory build at its full shape (32/8 heads,
+N=65536, L=16384 in 4 chunks, K=8192, 10 Lloyd rounds).
+``--impl reference`` times the fp64 CPU oracle on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_prefix_attention_b200 import inputs  # noqa: E402
+
+METRIC = "decode attention query-heads/sec and HBM GB/s vs 8 TB/s; build queries/sec"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", 0)), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def decode_bytes(B, Hq, Hkv, K, T, d, eb=2):
+    """Algorithmic HBM bytes of one decode step of one layer."""
+    centroids = Hq * K * d * eb
+    local_kv = B * Hkv * T * 2 * d * eb
+    gathered = B * Hq * (d * eb + 4)
+    q_out = 2 * B * Hq * d * eb
+    return centroids + local_kv + gathered + q_out
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        self.gpu = gpu_index
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- distributed --
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------- workloads --
+
+class DecodeStack:
+    """`layers` independent C1-shaped layers resident in HBM, one graph per step."""
+
+    def __init__(self, cfg, layers, seed_base):
+        from long_prefix_attention_b200 import ops
+        self.ops = ops
+        self.cfg = cfg
+        self.layers = []
+        for l in range(layers):
+            ins = inputs.decode_inputs(cfg, seed=seed_base + l)
+            dev = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in ins.items()}
+            B, Hq, d = dev["q"].shape
+            _, Hkv, T, _ = dev["k_cache"].shape
+            K = dev["centroids"].shape[1]
+            dev["out"] = torch.empty_like(dev["q"])
+            dev["ws"] = ops.alloc_workspace(
+                ops.asm_decode_workspace_size(B, Hq, Hkv, K, T, d, dev["q"].dtype), "cuda")
+            self.layers.append(dev)
+        self.B, self.Hq, self.d = self.layers[0]["q"].shape
+        self.Hkv, self.T = self.layers[0]["k_cache"].shape[1:3]
+        self.K = self.layers[0]["centroids"].shape[1]
+        self.graph = None
+
+    def launch_all(self):
+        for L in self.layers:
+            self.ops.asm_decode_step(L["q"], L["centroids"], L["a_bar"], L["logz_bar"], L["k_cache"],
+                                     L["v_cache"], L["local_len"], L["scale"], L["out"], L["ws"])
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.launch_all()  # warm the per-kernel attributes outside capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.launch_all()
+        torch.cuda.synchronize()
+
+    def step(self):
+        self.graph.replay()
+
+    def bytes_per_launch(self):
+        return decode_bytes(self.B, self.Hq, self.Hkv, self.K, self.T, self.d)
+
+
+def time_steps(fn, steps, warmup, world):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        fn()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3
+
+
+def cpu_decode_baseline(cfg, budget_s=12.0):
+    """fp64 oracle decode of C1-shaped layers on the host cores (bounded sample)."""
+    from oracle import asm_oracle as O
+    ins = inputs.decode_inputs(cfg, seed=inputs.BASE_SEED + 1)
+    args = (ins["q"], ins["centroids"], ins["a_bar"], ins["logz_bar"], ins["k_cache"], ins["v_cache"],
+            ins["local_len"], ins["scale"])
+    # marshal once (the oracle's own fp64 copies), then time whole-layer calls
+    f = [O._f64(a) if torch.is_tensor(a) else a for a in args]
+    f[6] = O._i32(ins["local_len"])
+    O.decode(*f)
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        O.decode(*f)
+        n += 1
+    dt = time.perf_counter() - t0
+    B, Hq = ins["q"].shape[:2]
+    return {"value": n * B * Hq / dt, "unit": "query-heads/s", "cores": O.max_threads(), "kind": "oracle",
+            "sample": f"{n} single-layer decode steps of the K=1024/T=2048/B=1 layer shape "
+                      f"({dt:.1f} s of fp64 CPU work)"}
+
+
+def run_build(cfg):
+    """Full offline build at the 32/8-head, N=65536, L=16384, K=8192 shape."""
+    from long_prefix_attention_b200 import ops
+    bi = inputs.build_inputs(cfg)
+    x, k, v, u = bi["q"].cuda(), bi["k"].cuda(), bi["v"].cuda(), bi["u"].cuda()
+    H, N, d = x.shape
+    K, iters, L = cfg["K"], cfg["iters"], cfg["L"]
+    chunks = cfg["chunks"]
+    a = torch.empty_like(x)
+    logz = torch.empty(H, N, dtype=torch.float32, device="cuda")
+    init = torch.empty(H, K, dtype=torch.int32, device="cuda")
+    ws_s = ops.alloc_workspace(ops.asm_kmeanspp_workspace_size(H, N, d, K), "cuda", zero=False)
+    cen = torch.empty(H, K, d, dtype=torch.float32, device="cuda")
+    cdt = torch.empty(H, K, d, dtype=x.dtype, device="cuda")
+    assign = torch.empty(H, N, dtype=torch.int32, device="cuda")
+    counts = torch.empty(H, K, dtype=torch.int32, device="cuda")
+    perm = torch.empty(H, N, dtype=torch.int32, device="cuda")
+    seg = torch.empty(H, K + 1, dtype=torch.int32, device="cuda")
+    ws = ops.alloc_workspace(ops.asm_kmeans_workspace_size(H, N, d, K), "cuda", zero=False)
+    a_bar = torch.empty(H, K, d, dtype=x.dtype, device="cuda")
+    lz_bar = torch.empty(H, K, dtype=torch.float32, device="cuda")
+    cl = L // chunks
+    kc = [k[:, i * cl:(i + 1) * cl].contiguous() for i in range(chunks)]
+    vc = [v[:, i * cl:(i + 1) * cl].contiguous() for i in range(chunks)]
+
+    def stage_times():
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record()
+        for i in range(chunks):
+            ops.asm_build_states(x, kc[i], vc[i], bi["scale"], a, logz, accumulate=i > 0)
+        ev[1].record()
+        ops.asm_kmeanspp_seed(x, u, init, ws_s)
+        ev[2].record()
+        ops.asm_kmeans(x, init, iters, cen, cdt, assign, counts, perm, seg, ws)
+        ev[3].record()
+        ops.asm_aggregate(a, logz, perm, seg, a_bar, lz_bar)
+        ev[4].record()
+        torch.cuda.synchronize()
+        return [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
+
+    stage_times()  # warm-up
+    t = stage_times()
+    total = sum(t)
+    hbm, tf, tfs, src = peaks()
+    states_flops = 4.0 * N * L * d * H
+    assign_flops = 2.0 * N * K * d * H * iters
+    return {
+        "workload": cfg["name"], "queries": H * N,
+        "value": H * N / (total / 1e3), "unit": "queries/s",
+        "ms": {"states_4chunks": t[0], "kmeanspp_seed": t[1], "lloyd_10": t[2], "aggregate": t[3],
+               "total": total},
+        "states_tflops": states_flops / (t[0] / 1e3) / 1e12,
+        "states_frac_of_bf16_peak": states_flops / (t[0] / 1e3) / 1e12 / tf,
+        "lloyd_assign_tflops_incl_update": assign_flops / (t[2] / 1e3) / 1e12,
+        "peak_source": src,
+    }
+
+
+# -------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="asm", choices=["asm", "reference"])
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--no-build", action="store_true", help="skip the offline-build measurement")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    args = ap.parse_args()
+    cfg = inputs.CONFIGS[1]
+    world, rank, local = dist_setup(args.gpus)
+    hbm, tf, tfs, peak_src = peaks()
+    config = {"workload": cfg["name"] + f" x {args.layers} layers", "layers": args.layers,
+              "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "d": cfg["d"], "K": cfg["K"], "local_len": cfg["T"],
+              "batch": cfg["B"], "l2": f"inputs larger than L2: {args.layers} distinct layer buffers",
+              "parallelism": f"replicas x{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = cpu_decode_baseline(cfg, budget_s=max(3.0, min(20.0, 0.05 * args.steps)))
+        line = {"metric": METRIC, "value": cb["value"], "unit": "query-heads/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "impl": "reference",
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config,
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "query-heads/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    stack = DecodeStack(cfg, args.layers, seed_base=inputs.BASE_SEED + 1000 + 100 * rank)
+    stack.capture()
+    with ClockSampler(local) as clk:
+        secs = time_steps(stack.step, args.steps, max(3, args.warmup), world)
+    secs = max_over_ranks(secs, world)
+    launches = args.steps * args.layers
+    qh = stack.B * stack.Hq * args.layers * args.steps * world
+    value = qh / secs
+    ms_per_step = secs * 1e3 / args.steps
+    per_launch_s = secs / launches
+    bpl = stack.bytes_per_launch()
+    achieved = bpl / per_launch_s / 1e9
+
+    # end to end: per-step queries H2D from pinned memory, outputs D2H
+    qh_host = torch.stack([L["q"].cpu() for L in stack.layers]).pin_memory()
+    out_host = torch.empty_like(qh_host).pin_memory()
+
+    def e2e_step():
+        for i, L in enumerate(stack.layers):
+            L["q"].copy_(qh_host[i], non_blocking=True)
+        stack.graph.replay()
+        for i, L in enumerate(stack.layers):
+            out_host[i].copy_(L["out"], non_blocking=True)
+
+    e2e_secs = max_over_ranks(time_steps(e2e_step, max(10, args.steps // 4), 3, world), world)
+    e2e_steps = max(10, args.steps // 4)
+    h2d = qh_host[0].numel() * qh_host.element_size() * args.layers
+    d2h = h2d
+
+    build = None
+    if not args.no_build and rank == 0:
+        try:
+            build = run_build(inputs.CONFIGS[3])
+        except Exception as e:  # report, do not hide
+            build = {"error": repr(e)}
+    cpu = None
+    if not args.no_cpu and rank == 0 and world == 1:
+        cpu = cpu_decode_baseline(cfg)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "query-heads/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config,
+            "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": None,
+                         "kernel": "decode_kernel<bf16,128,4>",
+                         "bytes_per_launch": bpl, "us_per_launch": per_launch_s * 1e6,
+                         "peak_source": f"{peak_src} HBM copy"},
+            "e2e": {"value": stack.B * stack.Hq * args.layers * e2e_steps * world / e2e_secs,
+                    "unit": "query-heads/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+            "build": build,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        stack.graph = None
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

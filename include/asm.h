@@ -1,0 +1,253 @@
+/*
+ * asm.h -- C ABI of the Attention State Memory (ASM) hot path on NVIDIA B200
+ * (sm_100a).
+ *
+ * Method: "Context Memorization for Efficient Long Context Generation"
+ * (technical summary of arXiv 2605.18226), section "Metodologia: Memoria de
+ * Estado de Atencion (ASM)".  A long conditioning prefix is replaced by a
+ * lookup memory of K query centroids per head, each carrying a precomputed
+ * attention state (a, Z) of the prefix; every decode step retrieves the
+ * nearest centroid and merges its state with attention over the locally
+ * generated tokens by the online-softmax identity.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every array argument is a DEVICE pointer unless marked "host".  The caller
+ *   allocates and owns every buffer; the library never allocates, frees or
+ *   keeps state between calls.
+ * - Layouts are row-major and contiguous with the head dimension d innermost.
+ *   Hq query heads share Hkv key/value heads; query head h reads KV head
+ *   h / (Hq / Hkv) (grouped-query attention).
+ * - Storage dtype `dt` (fp32 or bf16) applies to q, k, v, a, centroids_dt,
+ *   a_bar and out.  logZ-type arrays and the centroid master copy are fp32.
+ *   Arithmetic is fp32 (k-means++ distances: fp64).
+ * - Z is stored as its natural logarithm logZ = ln sum_j exp(scale <q, k_j>),
+ *   and `a` is the normalised attention output.  The empty state is
+ *   (a = 0, logZ = -inf).
+ * - Calls are asynchronous on `stream`.  All arguments are validated on the
+ *   host before anything is enqueued; an invalid call returns an error code
+ *   and touches no buffer.  Kernel launch failures return ASM_ERR_CUDA;
+ *   faults inside a kernel surface at the caller's next synchronisation.
+ * - Pointers must be 16-byte aligned; d must be 64 or 128; Hq % Hkv == 0 and
+ *   Hq / Hkv must be 1, 2, 4 or 8.
+ * - Calls that take a workspace `ws` of `ws_bytes` bytes document its size
+ *   function.  Workspaces of asm_decode_step and asm_flash_decode hold
+ *   self-resetting counters: zero them once with asm_workspace_init before
+ *   the first call, then reuse them for any number of calls on one stream.
+ *   Two calls that overlap on the GPU must not share a workspace.
+ */
+#ifndef ASM_B200_H
+#define ASM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ASM_OK = 0,
+    ASM_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or enum   */
+    ASM_ERR_UNSUPPORTED = 2, /* valid but unsupported shape (d, group size) */
+    ASM_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required  */
+    ASM_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    ASM_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up          */
+} asm_status;
+
+typedef enum { ASM_F32 = 0, ASM_BF16 = 1 } asm_dtype;
+
+/* Retrieval metric ("Recuperacion" bullet).  The page names cosine
+ * similarity; squared L2 is the default here, matching k-means.
+ *   ASM_L2:     argmax_c <q, c> - |c|^2 / 2   (== argmin |q - c|^2)
+ *   ASM_COSINE: argmax_c <q, c> / |c|         (0 for a zero centre)
+ * Ties go to the smallest centre index. */
+typedef enum { ASM_L2 = 0, ASM_COSINE = 1 } asm_metric;
+
+/* Normalisation term of an aggregated cluster ("Agregacion" bullet).
+ *   ASM_ZBAR_MEAN: Z_bar = mean of the members' Z (default)
+ *   ASM_ZBAR_SUM:  Z_bar = sum of the members' Z (plain state merge) */
+typedef enum { ASM_ZBAR_MEAN = 0, ASM_ZBAR_SUM = 1 } asm_zbar_mode;
+
+/* ------------------------------------------------------------------------ */
+/* Offline memory build                                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * asm_build_states -- attention state of every calibration query over one
+ * block of the prefix ("Recoleccion" bullet: for each query its state over
+ * the prefix; "Eficiencia" bullet: a long prefix is encoded chunk by chunk and
+ * the chunk states are merged with the online-softmax identity).
+ *   q      [Hq, N, d]  dt   calibration queries
+ *   k, v   [Hkv, L, d] dt   the prefix block (non-causal: all L keys are seen)
+ *   scale               softmax scale (typically 1/sqrt(d))
+ *   accumulate          0: overwrite (a, logz) with this block's state;
+ *                       1: merge this block's state into the stored (a, logz)
+ *                          (a is re-rounded to dt after each merge)
+ *   a      [Hq, N, d]  dt   output / in-out when accumulate
+ *   logz   [Hq, N]     fp32 output / in-out when accumulate
+ * L == 0 with accumulate == 0 writes the empty state.  No workspace.
+ */
+asm_status asm_build_states(const void *q, const void *k, const void *v,
+                            int Hq, int Hkv, int N, int L, int d, float scale,
+                            asm_dtype dt, int accumulate, void *a, float *logz,
+                            cudaStream_t stream);
+
+/*
+ * asm_kmeanspp_seed -- k-means++ initial centres of every head's points
+ * (the clustering of the "Agrupamiento" bullet; seeding by D^2 sampling,
+ * Arthur & Vassilvitskii 2007).  Round 0 takes point floor(u[h,0] * N); round
+ * r takes the smallest i whose running sum of D2 (index order) exceeds
+ * u[h,r] * sum(D2), where D2_i is the squared distance (fp64) of point i to
+ * its nearest chosen centre; if sum(D2) == 0 the smallest unchosen index.
+ *   x        [H, N, d] dt   points
+ *   u        [H, K]    fp64 uniform draws in [0, 1), one per round
+ *   init_idx [H, K]    int32 output
+ *   ws       asm_kmeanspp_workspace_size(H, N, d, K) bytes
+ * Requires 1 <= K <= N.
+ */
+size_t asm_kmeanspp_workspace_size(int H, int N, int d, int K);
+asm_status asm_kmeanspp_seed(const void *x, int H, int N, int d, int K,
+                             const double *u, asm_dtype dt, int32_t *init_idx,
+                             void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * asm_kmeans_assign -- nearest centre of every point ("Agrupamiento"
+ * bullet), with the metric rule above, against the storage-dtype centres.
+ *   x [H, N, d] dt, centroids_dt [H, K, d] dt -> assign [H, N] int32.
+ *   ws asm_kmeans_workspace_size(H, N, d, K) bytes (holds centre norms).
+ */
+asm_status asm_kmeans_assign(const void *x, const void *centroids_dt, int H,
+                             int N, int d, int K, asm_metric metric,
+                             asm_dtype dt, int32_t *assign, void *ws,
+                             size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * asm_kmeans_update -- every centre moves to the mean of its members
+ * ("Agregacion" bullet: a cluster's query vector is the mean of its
+ * members' queries); an empty cluster keeps its centre.  Also produces the
+ * members of each cluster in index order: perm[h, seg_off[h,c] ..
+ * seg_off[h,c+1]) lists the points of cluster c ascending.
+ *   x [H,N,d] dt, assign [H,N]
+ *   centroids    [H, K, d] fp32 in/out (master copy)
+ *   centroids_dt [H, K, d] dt   out (storage rounding of the master)
+ *   counts [H, K], perm [H, N], seg_off [H, K+1] int32 out
+ *   ws asm_kmeans_workspace_size(H, N, d, K) bytes
+ */
+asm_status asm_kmeans_update(const void *x, const int32_t *assign, int H,
+                             int N, int d, int K, asm_dtype dt,
+                             float *centroids, void *centroids_dt,
+                             int32_t *counts, int32_t *perm, int32_t *seg_off,
+                             void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * asm_kmeans -- Lloyd's algorithm from the points x[h, init_idx[h, :]]:
+ * `iters` rounds of asm_kmeans_assign then asm_kmeans_update.  On return the
+ * assignment is the last round's and the centres are the means of exactly
+ * those members.  Arguments as in the two calls above; iters >= 1.
+ */
+size_t asm_kmeans_workspace_size(int H, int N, int d, int K);
+asm_status asm_kmeans(const void *x, int H, int N, int d, int K, int iters,
+                      asm_metric metric, asm_dtype dt, const int32_t *init_idx,
+                      float *centroids, void *centroids_dt, int32_t *assign,
+                      int32_t *counts, int32_t *perm, int32_t *seg_off,
+                      void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * asm_aggregate -- attention-aware aggregation of each cluster's member
+ * states ("Agregacion" bullet: members are fused by the online-softmax update
+ * rule into one lossless average):
+ *   m = max_i logz_i,  w_i = exp(logz_i - m)
+ *   a_bar = sum_i w_i a_i / sum_i w_i           (Z-weighted mean of a)
+ *   logz_bar = m + ln sum_i w_i [- ln |members| in ASM_ZBAR_MEAN mode]
+ * Members come from perm / seg_off of asm_kmeans_update.  An empty cluster
+ * gets (0, -inf).
+ *   a [H, N, d] dt, logz [H, N] fp32 -> a_bar [H, K, d] dt, logz_bar [H, K]
+ * No workspace.
+ */
+asm_status asm_aggregate(const void *a, const float *logz, const int32_t *perm,
+                         const int32_t *seg_off, int H, int N, int d, int K,
+                         asm_zbar_mode zmode, asm_dtype dt, void *a_bar,
+                         float *logz_bar, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Online decode                                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * asm_decode_step -- one decode step for a batch ("Fase de Inferencia
+ * Online": Recuperacion then Fusion).  For every row b and query head h
+ * (KV head g = h / (Hq / Hkv)):
+ *   idx      = nearest centre of q[b,h] in centroids[h] (metric rule above)
+ *   local    = state of q[b,h] over k_cache[b,g,0:T_b), v_cache[b,g,0:T_b)
+ *              with T_b = local_len[b] (the row's non-prefix tokens)
+ *   out, lse = merge((a_bar[h,idx], logz_bar[h,idx]), local)
+ * so the prefix is never read: per-step cost depends on K and T_b only.
+ *   q         [B, Hq, d]       dt
+ *   centroids [Hq, K, d]       dt
+ *   a_bar     [Hq, K, d]       dt
+ *   logz_bar  [Hq, K]          fp32
+ *   k_cache, v_cache [B, Hkv, Tmax, d] dt
+ *   local_len [B]              int32, device, 0 <= T_b <= Tmax
+ *   out       [B, Hq, d]       dt   output
+ *   lse_out   [B, Hq]          fp32 output (natural log of the merged Z), or NULL
+ *   idx_out   [B, Hq]          int32 output, or NULL
+ *   ws        asm_decode_workspace_size(...) bytes, zeroed once by
+ *             asm_workspace_init.
+ * One kernel launch.  T_b == 0 returns the retrieved state itself.
+ */
+size_t asm_decode_workspace_size(int B, int Hq, int Hkv, int K, int Tmax,
+                                 int d, asm_dtype dt);
+asm_status asm_decode_step(const void *q, const void *centroids,
+                           const void *a_bar, const float *logz_bar,
+                           const void *k_cache, const void *v_cache,
+                           const int32_t *local_len, int B, int Hq, int Hkv,
+                           int K, int Tmax, int d, float scale,
+                           asm_metric metric, asm_dtype dt, void *out,
+                           float *lse_out, int32_t *idx_out, void *ws,
+                           size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * asm_flash_decode -- the quantity the memory stands in for: decode attention
+ * over an explicit prefix shared by the whole batch followed by each row's
+ * local tokens ("Fusion" bullet: the exact output as if the prefix were
+ * present).  Used as the full-attention comparison.
+ *   k_prefix, v_prefix [Hkv, Lp, d] dt (read once per call for all rows)
+ *   other arguments as asm_decode_step; lse_out may be NULL.
+ *   ws asm_flash_decode_workspace_size(...) bytes, zeroed once by
+ *   asm_workspace_init.
+ */
+size_t asm_flash_decode_workspace_size(int B, int Hq, int Hkv, int Lp,
+                                       int Tmax, int d, asm_dtype dt);
+asm_status asm_flash_decode(const void *q, const void *k_prefix,
+                            const void *v_prefix, int Lp, const void *k_cache,
+                            const void *v_cache, const int32_t *local_len,
+                            int B, int Hq, int Hkv, int Tmax, int d,
+                            float scale, asm_dtype dt, void *out,
+                            float *lse_out, void *ws, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Utilities                                                                */
+/* ------------------------------------------------------------------------ */
+
+/* Zero a decode / flash-decode workspace (its counters and error word). */
+asm_status asm_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Error word of a decode / flash-decode workspace, copied to the host
+ * pointer `code` (0 = no device-side error; otherwise ASM_ERR_TIMEOUT).
+ * Synchronises `stream`. */
+asm_status asm_workspace_error(const void *ws, size_t ws_bytes, int *code,
+                               cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char *asm_status_string(asm_status s);
+
+/* Library version, "major.minor.patch". */
+const char *asm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ASM_B200_H */

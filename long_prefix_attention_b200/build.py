@@ -1,0 +1,100 @@
+"""Build the sm_100a shared library ``libasm_b200.so`` in-tree with nvcc.
+
+Usage:  python -m long_prefix_attention_b200.build [--force] [-v]
+
+Every ``csrc/*.cu`` file is compiled for ``arch=compute_100a,code=sm_100a``
+(objects under ``_build/`` at the repository root), then linked into
+``long_prefix_attention_b200/libasm_b200.so`` against the CUDA runtime.  Only
+files whose source or headers changed are recompiled.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import glob
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+BUILD = os.path.join(ROOT, "_build")
+LIB = os.path.join(PKG, "libasm_b200.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
+         "-I", INCLUDE, "-I", CSRC]
+
+
+def _cutlass_include() -> str | None:
+    """CUTLASS/CuTe headers vendored with the Python environment (header-only use)."""
+    import site
+    cands = []
+    for sp in site.getsitepackages() + [site.getusersitepackages()]:
+        cands.append(os.path.join(sp, "flashinfer", "data", "cutlass", "include"))
+    for c in cands:
+        if os.path.exists(os.path.join(c, "cute", "arch", "mma_sm100_desc.hpp")):
+            return c
+    return None
+
+
+def _headers() -> list[str]:
+    return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
+        glob.glob(os.path.join(INCLUDE, "*.h"))
+
+
+def _stale(obj: str, src: str, hdr_mtime: float) -> bool:
+    if not os.path.exists(obj):
+        return True
+    m = os.path.getmtime(obj)
+    return m < os.path.getmtime(src) or m < hdr_mtime
+
+
+def build(force: bool = False, verbose: bool = False, jobs: int | None = None) -> str:
+    os.makedirs(BUILD, exist_ok=True)
+    srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    hdr_mtime = max([os.path.getmtime(h) for h in _headers()] + [0.0])
+    flags = list(FLAGS)
+    cut = _cutlass_include()
+    if cut:
+        flags += ["-isystem", cut, "-DASM_HAVE_CUTLASS=1"]
+    objs, todo = [], []
+    for s in srcs:
+        o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")
+        objs.append(o)
+        if force or _stale(o, s, hdr_mtime):
+            todo.append((s, o))
+
+    def _compile(so):
+        s, o = so
+        cmd = [NVCC] + ARCH + flags + ["-c", s, "-o", o]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        return s, r
+
+    if todo:
+        with cf.ThreadPoolExecutor(max_workers=jobs or min(8, len(todo))) as ex:
+            for s, r in ex.map(_compile, todo):
+                if verbose or r.returncode != 0:
+                    sys.stderr.write(r.stdout + r.stderr)
+                if r.returncode != 0:
+                    raise RuntimeError(f"nvcc failed on {os.path.basename(s)}")
+    if force or todo or not os.path.exists(LIB):
+        cmd = [NVCC] + ARCH + ["-shared", "-o", LIB] + objs + ["-lcudart", "-lcuda"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            sys.stderr.write(r.stdout + r.stderr)
+            raise RuntimeError("link of libasm_b200.so failed")
+    return LIB
+
+
+if __name__ == "__main__":
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("-v", "--verbose", action="store_true")
+    a = ap.parse_args()
+    print(build(force=a.force, verbose=a.verbose))

@@ -1,0 +1,517 @@
+// kmeans.cu -- clustering of the calibration queries into K centroids.
+//
+// "Context Memorization for Efficient Long Context Generation", Metodologia,
+// "Agrupamiento" (the query vectors are clustered, e.g. by k-means, into K
+// centroids) and "Agregacion" (a centroid's query vector is the mean of its
+// cluster's queries).  Seeding is k-means++ (D^2 sampling) with the uniform
+// draws supplied by the caller.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace asmk {
+
+namespace {
+inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+}
+
+// ============================================================ k-means++ ===
+//
+// One launch per round.  Every block refreshes D2 for its slice of points
+// against the centre chosen in the previous round (fp64, exact for bf16
+// inputs) and publishes its slice sum; the last block of each head to arrive
+// (arrival counter, no waiting) scans the slice sums, finds the slice that
+// holds the threshold u * sum(D2) and the first index inside it whose running
+// sum exceeds the threshold, and records the pick for the next round.
+
+constexpr int kSeedThreads = 256;
+constexpr int kSeedPts = 1024;  // points per block (4 per thread)
+
+struct SeedWs {
+    size_t off_d2, off_bsum, off_cnt, off_taken, total;
+};
+SeedWs seed_ws(int H, int N) {
+    const int nblk = (N + kSeedPts - 1) / kSeedPts;
+    SeedWs w;
+    w.off_d2 = 0;
+    w.off_bsum = al256(w.off_d2 + sizeof(double) * (size_t)H * N);
+    w.off_cnt = al256(w.off_bsum + sizeof(double) * (size_t)H * nblk);
+    w.off_taken = al256(w.off_cnt + sizeof(int) * (size_t)H);
+    w.total = al256(w.off_taken + (size_t)H * N);
+    return w;
+}
+
+__device__ __forceinline__ double block_sum_d(double v, double *red) {
+    for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    double t = 0.0;
+    if (threadIdx.x == 0)
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    return t;  // valid in thread 0
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSeedThreads)
+kmeanspp_round(const T *__restrict__ x, int N, int K, int r, const double *__restrict__ u,
+               int32_t *idx, double *d2, double *bsum, int *cnt, unsigned char *taken) {
+    const int h = blockIdx.y, nblk = gridDim.x;
+    const T *xh = x + (size_t)h * N * D;
+    double *d2h = d2 + (size_t)h * N;
+    unsigned char *tk = taken + (size_t)h * N;
+    __shared__ double cs[D];
+    __shared__ double red[kSeedThreads / 32];
+    __shared__ int last;
+    const int p0 = blockIdx.x * kSeedPts;
+
+    if (r == 0) {
+        // round 0: clear the slice state; the last block records floor(u*N)
+        for (int i = p0 + threadIdx.x; i < min(N, p0 + kSeedPts); i += blockDim.x) {
+            d2h[i] = __longlong_as_double(0x7ff0000000000000LL);  // +inf
+            tk[i] = 0;
+        }
+    } else {
+        const int c = idx[(size_t)h * K + r - 1];
+        for (int i = threadIdx.x; i < D; i += blockDim.x) cs[i] = (double)Elem<T>::to_f(xh[(size_t)c * D + i]);
+        __syncthreads();
+        double local = 0.0;
+        for (int i = p0 + threadIdx.x; i < min(N, p0 + kSeedPts); i += blockDim.x) {
+            const T *xi = xh + (size_t)i * D;
+            double s = 0.0;
+#pragma unroll 8
+            for (int e = 0; e < D; ++e) {
+                const double t = (double)Elem<T>::to_f(xi[e]) - cs[e];
+                s = fma(t, t, s);
+            }
+            const double nd = fmin(d2h[i], s);
+            d2h[i] = nd;
+            local += nd;
+        }
+        const double tot = block_sum_d(local, red);
+        if (threadIdx.x == 0) bsum[(size_t)h * nblk + blockIdx.x] = tot;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int old = atomicAdd(&cnt[h], 1);
+        last = (old == nblk - 1);
+        __threadfence();
+    }
+    __syncthreads();
+    if (!last) return;
+
+    // ---------------- last block of head h: choose this round's centre
+    if (threadIdx.x == 0) {
+        cnt[h] = 0;
+        int pk = -1;
+        const double ur = u[(size_t)h * K + r];
+        if (r == 0) {
+            pk = (int)floor(ur * (double)N);
+            pk = min(max(pk, 0), N - 1);
+        } else {
+            double total = 0.0;
+            for (int b = 0; b < nblk; ++b) total += __ldcg(bsum + (size_t)h * nblk + b);
+            if (total > 0.0) {
+                const double thr = ur * total;
+                double run = 0.0;
+                for (int b = 0; b < nblk && pk < 0; ++b) {
+                    const double bs = __ldcg(bsum + (size_t)h * nblk + b);
+                    if (run + bs > thr) {
+                        // the threshold falls in this slice: walk its points
+                        double r2 = run;
+                        for (int i = b * kSeedPts; i < min(N, (b + 1) * kSeedPts); ++i) {
+                            r2 += __ldcg(d2h + i);
+                            if (r2 > thr) { pk = i; break; }
+                        }
+                        run = r2;  // (a rounding miss continues in the next slice)
+                    } else {
+                        run += bs;
+                    }
+                }
+                if (pk < 0) {
+                    // threshold at the very top of the CDF: the last point with D2 > 0
+                    for (int i = N - 1; i >= 0; --i)
+                        if (__ldcg(d2h + i) > 0.0) { pk = i; break; }
+                    if (pk < 0) pk = 0;
+                }
+            } else {
+                for (int i = 0; i < N; ++i)
+                    if (!__ldcg(tk + i)) { pk = i; break; }
+                if (pk < 0) pk = 0;
+            }
+        }
+        idx[(size_t)h * K + r] = pk;
+        tk[pk] = 1;
+    }
+}
+
+}  // namespace asmk
+
+// ============================================================ init / norms ==
+namespace asmk {
+
+template <typename T, int D>
+__global__ void kmeans_init(const T *__restrict__ x, int N, int K, const int32_t *__restrict__ init_idx,
+                            float *centroids, T *centroids_dt) {
+    const int h = blockIdx.y;
+    const int c = blockIdx.x * (blockDim.x / D) + threadIdx.x / D;
+    const int e = threadIdx.x % D;
+    if (c >= K) return;
+    const int src = init_idx[(size_t)h * K + c];
+    const T v = x[((size_t)h * N + src) * D + e];
+    centroids[((size_t)h * K + c) * D + e] = Elem<T>::to_f(v);
+    centroids_dt[((size_t)h * K + c) * D + e] = v;
+}
+
+// |c|^2 of every storage-dtype centre (fp32), one warp per centre.
+template <typename T, int D>
+__global__ void centroid_norms(const T *__restrict__ c, int HK, float *norms) {
+    constexpr int EPL = D / 32;
+    const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (w >= HK) return;
+    float f[EPL];
+    load_vec<T, EPL>(c + (size_t)w * D + lane * EPL, f);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) s = fmaf(f[e], f[e], s);
+    s = warp_sum(s);
+    if (lane == 0) norms[w] = s;
+}
+
+// ================================================================ assign ===
+//
+// Portable CUDA-core assignment: a 64-point x 64-centre register-tiled
+// fp32 contraction per step, with the arg-max of <x,c> - |c|^2/2 (or
+// <x,c>/|c|) carried across all centre tiles; ties go to the smaller index.
+
+constexpr int kAsP = 64, kAsC = 64, kAsDK = 32;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+assign_simple(const T *__restrict__ x, const T *__restrict__ c, const float *__restrict__ norms,
+              int N, int K, int metric, int32_t *assign) {
+    __shared__ float xs[kAsDK][kAsP + 4];
+    __shared__ float cs[kAsDK][kAsC + 4];
+    __shared__ float bs_s[16][kAsP];
+    __shared__ int bi_s[16][kAsP];
+    const int h = blockIdx.y;
+    const int p0 = blockIdx.x * kAsP;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;  // ty: points, tx: centres
+    const T *xh = x + (size_t)h * N * D;
+    const T *ch = c + (size_t)h * K * D;
+    float best[4];
+    int bidx[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { best[i] = kNegInf; bidx[i] = 0x7fffffff; }
+
+    for (int c0 = 0; c0 < K; c0 += kAsC) {
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+        for (int k0 = 0; k0 < D; k0 += kAsDK) {
+            __syncthreads();
+            for (int i = threadIdx.x; i < kAsP * kAsDK; i += 256) {
+                const int row = i / kAsDK, col = i % kAsDK;
+                const int p = p0 + row, cc = c0 + row;
+                xs[col][row] = p < N ? Elem<T>::to_f(xh[(size_t)p * D + k0 + col]) : 0.f;
+                cs[col][row] = cc < K ? Elem<T>::to_f(ch[(size_t)cc * D + k0 + col]) : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 8
+            for (int kk = 0; kk < kAsDK; ++kk) {
+                float xv[4], cv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) xv[i] = xs[kk][ty * 4 + i];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) cv[j] = cs[kk][tx + 16 * j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xv[i], cv[j], acc[i][j]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int cc = c0 + tx + 16 * j;
+            if (cc >= K) continue;
+            const float nr = norms[(size_t)h * K + cc];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float s;
+                if (metric == 0) s = acc[i][j] - 0.5f * nr;
+                else s = nr > 0.f ? acc[i][j] / sqrtf(nr) : 0.f;
+                if (better(s, cc, best[i], bidx[i])) { best[i] = s; bidx[i] = cc; }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        bs_s[tx][ty * 4 + i] = best[i];
+        bi_s[tx][ty * 4 + i] = bidx[i];
+    }
+    __syncthreads();
+    if (threadIdx.x < kAsP) {
+        const int p = p0 + threadIdx.x;
+        float bs = kNegInf;
+        int bi = 0x7fffffff;
+        for (int t = 0; t < 16; ++t)
+            if (better(bs_s[t][threadIdx.x], bi_s[t][threadIdx.x], bs, bi)) {
+                bs = bs_s[t][threadIdx.x];
+                bi = bi_s[t][threadIdx.x];
+            }
+        if (p < N) assign[(size_t)h * N + p] = (bi == 0x7fffffff) ? 0 : bi;
+    }
+}
+
+// ================================================================ update ===
+//
+// Counting sort of the points by cluster (histogram, exclusive scan, scatter,
+// then each cluster's member list put in ascending index order), followed
+// by the fp32 mean of each cluster's members in that order.
+
+__global__ void hist_kernel(const int32_t *__restrict__ assign, int H, int N, int K, int32_t *counts) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (size_t)H * N) return;
+    const int h = (int)(i / N);
+    atomicAdd(&counts[(size_t)h * K + assign[i]], 1);
+}
+
+// Exclusive scan of counts[h, 0:K) into seg_off[h, 0:K] (one block per head)
+// and a copy of the offsets into the scatter cursors.
+__global__ void scan_kernel(const int32_t *__restrict__ counts, int K, int32_t *seg_off, int32_t *cursor) {
+    const int h = blockIdx.x;
+    __shared__ int warp_tot[32];
+    __shared__ int carry;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int base = 0; base < K; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const int v = i < K ? counts[(size_t)h * K + i] : 0;
+        int x = v;
+        for (int m = 1; m < 32; m <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, x, m);
+            if (lane >= m) x += y;
+        }
+        if (lane == 31) warp_tot[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int t = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+            for (int m = 1; m < 32; m <<= 1) {
+                int y = __shfl_up_sync(0xffffffffu, t, m);
+                if (lane >= m) t += y;
+            }
+            warp_tot[lane] = t;  // inclusive prefix of warp totals
+        }
+        __syncthreads();
+        const int excl = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + x - v;
+        if (i < K) {
+            seg_off[(size_t)h * (K + 1) + i] = excl;
+            cursor[(size_t)h * K + i] = excl;
+        }
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = excl + v;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) seg_off[(size_t)h * (K + 1) + K] = carry;
+}
+
+__global__ void scatter_kernel(const int32_t *__restrict__ assign, int H, int N, int K, int32_t *cursor,
+                               int32_t *perm) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (size_t)H * N) return;
+    const int h = (int)(i / N), p = (int)(i % N);
+    const int pos = atomicAdd(&cursor[(size_t)h * K + assign[i]], 1);
+    perm[(size_t)h * N + pos] = p;
+}
+
+// Put every cluster's member list in ascending order (insertion sort; the
+// lists are short, about N / K entries).
+__global__ void segsort_kernel(const int32_t *__restrict__ seg_off, int H, int N, int K, int32_t *perm) {
+    const size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= (size_t)H * K) return;
+    const int h = (int)(t / K), c = (int)(t % K);
+    int32_t *p = perm + (size_t)h * N;
+    const int lo = seg_off[(size_t)h * (K + 1) + c], hi = seg_off[(size_t)h * (K + 1) + c + 1];
+    for (int i = lo + 1; i < hi; ++i) {
+        const int v = p[i];
+        int j = i - 1;
+        while (j >= lo && p[j] > v) { p[j + 1] = p[j]; --j; }
+        p[j + 1] = v;
+    }
+}
+
+// One warp per cluster: fp32 mean of its members (member order), or the
+// previous centre if empty; writes the fp32 master and its storage copy.
+template <typename T, int D>
+__global__ void means_kernel(const T *__restrict__ x, const int32_t *__restrict__ perm,
+                             const int32_t *__restrict__ seg_off, int H, int N, int K,
+                             float *centroids, T *centroids_dt) {
+    constexpr int EPL = D / 32;
+    const size_t w = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= (size_t)H * K) return;
+    const int h = (int)(w / K), c = (int)(w % K);
+    const int lo = seg_off[(size_t)h * (K + 1) + c], hi = seg_off[(size_t)h * (K + 1) + c + 1];
+    float acc[EPL];
+    float *cm = centroids + w * D + lane * EPL;
+    if (hi > lo) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+        for (int i = lo; i < hi; ++i) {
+            const int p = perm[(size_t)h * N + i];
+            float f[EPL];
+            load_vec<T, EPL>(x + ((size_t)h * N + p) * D + lane * EPL, f);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] += f[e];
+        }
+        const float inv = 1.f / (float)(hi - lo);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] *= inv;
+    } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = cm[e];
+    }
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) cm[e] = acc[e];
+    store_vec<T, EPL>(centroids_dt + w * D + lane * EPL, acc);
+}
+
+struct KmWs {
+    size_t off_norm, off_cursor, total;
+};
+KmWs km_ws(int H, int N, int K) {
+    (void)N;
+    KmWs w;
+    w.off_norm = 0;
+    w.off_cursor = al256(w.off_norm + sizeof(float) * (size_t)H * K);
+    w.total = al256(w.off_cursor + sizeof(int) * (size_t)H * K);
+    return w;
+}
+
+}  // namespace asmk
+
+// ============================================================== host side ==
+using namespace asmk;
+
+size_t asm_kmeanspp_ws_bytes(int H, int N, int d, int K) {
+    (void)d; (void)K;
+    return seed_ws(H, N).total;
+}
+
+cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const double *u,
+                                asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st) {
+    SeedWs w = seed_ws(H, N);
+    char *b = static_cast<char *>(ws);
+    double *d2 = reinterpret_cast<double *>(b + w.off_d2);
+    double *bsum = reinterpret_cast<double *>(b + w.off_bsum);
+    int *cnt = reinterpret_cast<int *>(b + w.off_cnt);
+    unsigned char *taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
+    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int) * (size_t)H, st);
+    if (e != cudaSuccess) return e;
+    dim3 grid((N + kSeedPts - 1) / kSeedPts, H);
+    for (int r = 0; r < K; ++r) {
+        if (dt == ASM_BF16) {
+            using T = __nv_bfloat16;
+            if (d == 128) kmeanspp_round<T, 128><<<grid, kSeedThreads, 0, st>>>((const T *)x, N, K, r, u, init_idx, d2, bsum, cnt, taken);
+            else kmeanspp_round<T, 64><<<grid, kSeedThreads, 0, st>>>((const T *)x, N, K, r, u, init_idx, d2, bsum, cnt, taken);
+        } else {
+            if (d == 128) kmeanspp_round<float, 128><<<grid, kSeedThreads, 0, st>>>((const float *)x, N, K, r, u, init_idx, d2, bsum, cnt, taken);
+            else kmeanspp_round<float, 64><<<grid, kSeedThreads, 0, st>>>((const float *)x, N, K, r, u, init_idx, d2, bsum, cnt, taken);
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+size_t asm_kmeans_ws_bytes(int H, int N, int d, int K) {
+    (void)d;
+    return km_ws(H, N, K).total;
+}
+
+cudaError_t asm_kmeans_init_launch(const void *x, int H, int N, int d, int K, asm_dtype dt,
+                                   const int32_t *init_idx, float *centroids, void *centroids_dt,
+                                   cudaStream_t st) {
+    const int per_block = 256 / d;
+    dim3 grid((K + per_block - 1) / per_block, H);
+    if (dt == ASM_BF16) {
+        using T = __nv_bfloat16;
+        if (d == 128) kmeans_init<T, 128><<<grid, 256, 0, st>>>((const T *)x, N, K, init_idx, centroids, (T *)centroids_dt);
+        else kmeans_init<T, 64><<<grid, 256, 0, st>>>((const T *)x, N, K, init_idx, centroids, (T *)centroids_dt);
+    } else {
+        if (d == 128) kmeans_init<float, 128><<<grid, 256, 0, st>>>((const float *)x, N, K, init_idx, centroids, (float *)centroids_dt);
+        else kmeans_init<float, 64><<<grid, 256, 0, st>>>((const float *)x, N, K, init_idx, centroids, (float *)centroids_dt);
+    }
+    return cudaGetLastError();
+}
+
+#ifdef ASM_HAVE_TC_ASSIGN
+cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, int H, int N,
+                                 int K, int metric, int32_t *assign, int num_sms, cudaStream_t st);
+#endif
+
+cudaError_t asm_kmeans_assign_launch(const void *x, const void *centroids_dt, int H, int N, int d,
+                                     int K, int metric, asm_dtype dt, int32_t *assign, void *ws,
+                                     int num_sms, cudaStream_t st) {
+    (void)num_sms;
+    KmWs w = km_ws(H, N, K);
+    float *norms = reinterpret_cast<float *>(static_cast<char *>(ws) + w.off_norm);
+    const int HK = H * K;
+    const int nb = (HK * 32 + 255) / 256;
+    if (dt == ASM_BF16) {
+        using T = __nv_bfloat16;
+        if (d == 128) centroid_norms<T, 128><<<nb, 256, 0, st>>>((const T *)centroids_dt, HK, norms);
+        else centroid_norms<T, 64><<<nb, 256, 0, st>>>((const T *)centroids_dt, HK, norms);
+    } else {
+        if (d == 128) centroid_norms<float, 128><<<nb, 256, 0, st>>>((const float *)centroids_dt, HK, norms);
+        else centroid_norms<float, 64><<<nb, 256, 0, st>>>((const float *)centroids_dt, HK, norms);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+#ifdef ASM_HAVE_TC_ASSIGN
+    if (dt == ASM_BF16 && d == 128)
+        return asm_assign_tc_launch(x, centroids_dt, norms, H, N, K, metric, assign, num_sms, st);
+#endif
+    dim3 grid((N + kAsP - 1) / kAsP, H);
+    if (dt == ASM_BF16) {
+        using T = __nv_bfloat16;
+        if (d == 128) assign_simple<T, 128><<<grid, 256, 0, st>>>((const T *)x, (const T *)centroids_dt, norms, N, K, metric, assign);
+        else assign_simple<T, 64><<<grid, 256, 0, st>>>((const T *)x, (const T *)centroids_dt, norms, N, K, metric, assign);
+    } else {
+        if (d == 128) assign_simple<float, 128><<<grid, 256, 0, st>>>((const float *)x, (const float *)centroids_dt, norms, N, K, metric, assign);
+        else assign_simple<float, 64><<<grid, 256, 0, st>>>((const float *)x, (const float *)centroids_dt, norms, N, K, metric, assign);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t asm_kmeans_update_launch(const void *x, const int32_t *assign, int H, int N, int d,
+                                     int K, asm_dtype dt, float *centroids, void *centroids_dt,
+                                     int32_t *counts, int32_t *perm, int32_t *seg_off, void *ws,
+                                     cudaStream_t st) {
+    KmWs w = km_ws(H, N, K);
+    int32_t *cursor = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + w.off_cursor);
+    cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)H * K, st);
+    if (e != cudaSuccess) return e;
+    const size_t HN = (size_t)H * N, HK = (size_t)H * K;
+    hist_kernel<<<(unsigned)((HN + 255) / 256), 256, 0, st>>>(assign, H, N, K, counts);
+    scan_kernel<<<H, 1024, 0, st>>>(counts, K, seg_off, cursor);
+    scatter_kernel<<<(unsigned)((HN + 255) / 256), 256, 0, st>>>(assign, H, N, K, cursor, perm);
+    segsort_kernel<<<(unsigned)((HK + 255) / 256), 256, 0, st>>>(seg_off, H, N, K, perm);
+    const unsigned nb = (unsigned)((HK * 32 + 255) / 256);
+    if (dt == ASM_BF16) {
+        using T = __nv_bfloat16;
+        if (d == 128) means_kernel<T, 128><<<nb, 256, 0, st>>>((const T *)x, perm, seg_off, H, N, K, centroids, (T *)centroids_dt);
+        else means_kernel<T, 64><<<nb, 256, 0, st>>>((const T *)x, perm, seg_off, H, N, K, centroids, (T *)centroids_dt);
+    } else {
+        if (d == 128) means_kernel<float, 128><<<nb, 256, 0, st>>>((const float *)x, perm, seg_off, H, N, K, centroids, (float *)centroids_dt);
+        else means_kernel<float, 64><<<nb, 256, 0, st>>>((const float *)x, perm, seg_off, H, N, K, centroids, (float *)centroids_dt);
+    }
+    return cudaGetLastError();
+}

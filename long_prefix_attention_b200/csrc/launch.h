@@ -1,0 +1,47 @@
+// launch.h -- internal launch entry points between the C ABI (api.cu) and the
+// kernel files.  Arguments are validated by the caller.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "asm.h"
+
+// decode.cu: mode 0 = memory lookup + local attention, 1 = explicit prefix + local.
+size_t asm_decode_ws_bytes(int mode, int B, int Hq, int Hkv, int K, int Lp, int Tmax, int d,
+                           asm_dtype dt);
+cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, const void *a_bar,
+                              const float *logz_bar, const void *k_prefix, const void *v_prefix,
+                              int Lp, const void *k_cache, const void *v_cache,
+                              const int32_t *local_len, int B, int Hq, int Hkv, int K, int Tmax,
+                              int d, float scale, int metric, asm_dtype dt, void *out,
+                              float *lse_out, int32_t *idx_out, void *ws, int num_sms,
+                              cudaStream_t st);
+
+// build_states.cu
+cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v, int Hq, int Hkv,
+                                    int N, int L, int d, float scale, asm_dtype dt,
+                                    int accumulate, void *a, float *logz, int num_sms,
+                                    cudaStream_t st);
+
+// kmeans.cu
+size_t asm_kmeanspp_ws_bytes(int H, int N, int d, int K);
+cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const double *u,
+                                asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st);
+size_t asm_kmeans_ws_bytes(int H, int N, int d, int K);
+cudaError_t asm_kmeans_init_launch(const void *x, int H, int N, int d, int K, asm_dtype dt,
+                                   const int32_t *init_idx, float *centroids, void *centroids_dt,
+                                   cudaStream_t st);
+cudaError_t asm_kmeans_assign_launch(const void *x, const void *centroids_dt, int H, int N, int d,
+                                     int K, int metric, asm_dtype dt, int32_t *assign, void *ws,
+                                     int num_sms, cudaStream_t st);
+cudaError_t asm_kmeans_update_launch(const void *x, const int32_t *assign, int H, int N, int d,
+                                     int K, asm_dtype dt, float *centroids, void *centroids_dt,
+                                     int32_t *counts, int32_t *perm, int32_t *seg_off, void *ws,
+                                     cudaStream_t st);
+
+// aggregate.cu
+cudaError_t asm_aggregate_launch(const void *a, const float *logz, const int32_t *perm,
+                                 const int32_t *seg_off, int H, int N, int d, int K, int zmode,
+                                 asm_dtype dt, void *a_bar, float *logz_bar, cudaStream_t st);

@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/asm.h declares, and rejects invalid arguments with
+the documented status before any CUDA call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_prefix_attention_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "asm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(asm_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ["asm_build_states", "asm_kmeanspp_seed", "asm_kmeans", "asm_kmeans_assign",
+              "asm_kmeans_update", "asm_aggregate", "asm_decode_step", "asm_flash_decode",
+              "asm_decode_workspace_size", "asm_workspace_init", "asm_status_string"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"binding lacks {n}"
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.asm_status_string(s)
+    assert lib.asm_version().decode().count(".") == 2
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+ODD = ctypes.c_void_p(0x10008)       # 8-byte aligned only
+NULL = None
+
+
+def decode(lib, **kw):
+    a = dict(q=FAKE, c=FAKE, ab=FAKE, lz=FAKE, kc=FAKE, vc=FAKE, ll=FAKE, B=1, Hq=32, Hkv=8,
+             K=1024, Tmax=2048, d=128, scale=0.088, metric=0, dt=1, out=FAKE, lse=NULL, idx=NULL,
+             ws=FAKE, wsb=1 << 30)
+    a.update(kw)
+    return lib.asm_decode_step(a["q"], a["c"], a["ab"], a["lz"], a["kc"], a["vc"], a["ll"], a["B"],
+                               a["Hq"], a["Hkv"], a["K"], a["Tmax"], a["d"], a["scale"],
+                               a["metric"], a["dt"], a["out"], a["lse"], a["idx"], a["ws"],
+                               a["wsb"], None)
+
+
+def test_decode_validation(lib):
+    assert decode(lib, d=96) == UNSUPPORTED
+    assert decode(lib, Hq=32, Hkv=5) == INVALID
+    assert decode(lib, Hq=48, Hkv=3) == UNSUPPORTED    # group of 16
+    assert decode(lib, q=NULL) == INVALID
+    assert decode(lib, c=ODD) == INVALID
+    assert decode(lib, K=0) == INVALID
+    assert decode(lib, B=0) == INVALID
+    assert decode(lib, metric=7) == INVALID
+    assert decode(lib, dt=3) == INVALID
+    assert decode(lib, wsb=16) == WORKSPACE
+    assert decode(lib, ws=NULL) == WORKSPACE
+    assert decode(lib, scale=float("nan")) == INVALID
+
+
+def test_workspace_sizes_grow_with_the_problem(lib):
+    s1 = lib.asm_decode_workspace_size(1, 32, 8, 1024, 2048, 128, 1)
+    s2 = lib.asm_decode_workspace_size(16, 32, 8, 8192, 4096, 128, 1)
+    assert 0 < s1 < s2 and s1 % 256 == 0
+    assert lib.asm_decode_workspace_size(0, 32, 8, 1024, 2048, 128, 1) == 0
+    assert lib.asm_flash_decode_workspace_size(1, 32, 8, 32768, 2048, 128, 1) > 0
+    assert lib.asm_kmeans_workspace_size(32, 65536, 128, 8192) > 0
+    assert lib.asm_kmeanspp_workspace_size(32, 65536, 128, 8192) > 0
+
+
+def test_build_and_kmeans_validation(lib):
+    P = FAKE
+    # build states: bad group / d
+    assert lib.asm_build_states(P, P, P, 32, 6, 16, 16, 128, 0.1, 1, 0, P, P, None) == INVALID
+    assert lib.asm_build_states(P, P, P, 32, 8, 16, 16, 80, 0.1, 1, 0, P, P, None) == UNSUPPORTED
+    assert lib.asm_build_states(P, P, P, 32, 8, 0, 16, 128, 0.1, 1, 0, P, P, None) == 0  # N=0: no-op
+    # k-means++: K > N, small workspace
+    assert lib.asm_kmeanspp_seed(P, 2, 10, 64, 11, P, 0, P, P, 1 << 30, None) == INVALID
+    assert lib.asm_kmeanspp_seed(P, 2, 10, 64, 4, P, 0, P, P, 8, None) == WORKSPACE
+    # k-means: iters < 1, bad metric
+    assert lib.asm_kmeans(P, 2, 10, 64, 4, 0, 0, 0, P, P, P, P, P, P, P, P, 1 << 30, None) == INVALID
+    assert lib.asm_kmeans(P, 2, 10, 64, 4, 3, 5, 0, P, P, P, P, P, P, P, P, 1 << 30, None) == INVALID
+    # aggregate: bad z mode
+    assert lib.asm_aggregate(P, P, P, P, 2, 10, 64, 4, 9, 0, P, P, None) == INVALID
+    # flash decode: nothing to attend
+    assert lib.asm_flash_decode(P, P, P, 0, P, P, P, 1, 32, 8, 0, 128, 0.1, 1, P, NULL, P,
+                                1 << 30, None) == INVALID
