@@ -149,9 +149,10 @@ def max_over_ranks(x, world):
 class DecodeStack:
     """`layers` independent C1-shaped layers resident in HBM, one graph per step."""
 
-    def __init__(self, cfg, layers, seed_base):
+    def __init__(self, cfg, layers, seed_base, flags=0):
         from long_prefix_attention_b200 import ops
         self.ops = ops
+        self.flags = flags
         self.cfg = cfg
         self.layers = []
         for l in range(layers):
@@ -172,7 +173,8 @@ class DecodeStack:
     def launch_all(self):
         for L in self.layers:
             self.ops.asm_decode_step(L["q"], L["centroids"], L["a_bar"], L["logz_bar"], L["k_cache"],
-                                     L["v_cache"], L["local_len"], L["scale"], L["out"], L["ws"])
+                                     L["v_cache"], L["local_len"], L["scale"], L["out"], L["ws"],
+                                     flags=self.flags)
 
     def capture(self):
         s = torch.cuda.Stream()
@@ -301,6 +303,9 @@ def main():
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--no-build", action="store_true", help="skip the offline-build measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--no-prefetch", action="store_true",
+                    help="do not let a layer's kernel stream its (static) centroids before the "
+                         "preceding kernel finishes")
     args = ap.parse_args()
     cfg = inputs.CONFIGS[1]
     world, rank, local = dist_setup(args.gpus)
@@ -324,7 +329,9 @@ def main():
         print(json.dumps(line))
         return
 
-    stack = DecodeStack(cfg, args.layers, seed_base=inputs.BASE_SEED + 1000 + 100 * rank)
+    flags = 0 if args.no_prefetch else 1  # ASM_DECODE_PREFETCH_CENTROIDS
+    config["prefetch_centroids"] = bool(flags)
+    stack = DecodeStack(cfg, args.layers, seed_base=inputs.BASE_SEED + 1000 + 100 * rank, flags=flags)
     stack.capture()
     with ClockSampler(local) as clk:
         secs = time_steps(stack.step, args.steps, max(3, args.warmup), world)

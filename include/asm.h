@@ -193,10 +193,18 @@ asm_status asm_aggregate(const void *a, const float *logz, const int32_t *perm,
  *   out       [B, Hq, d]       dt   output
  *   lse_out   [B, Hq]          fp32 output (natural log of the merged Z), or NULL
  *   idx_out   [B, Hq]          int32 output, or NULL
+ *   flags     0, or ASM_DECODE_PREFETCH_CENTROIDS
  *   ws        asm_decode_workspace_size(...) bytes, zeroed once by
  *             asm_workspace_init.
- * One kernel launch.  T_b == 0 returns the retrieved state itself.
+ * One kernel launch, with programmatic dependent launch enabled: the kernel
+ * may start while the preceding kernel in `stream` finishes, and reads no
+ * argument before that kernel has completed -- except, with
+ * ASM_DECODE_PREFETCH_CENTROIDS, the `centroids` array, which it may start
+ * streaming early.  Pass that flag only when the preceding kernel in the
+ * stream does not write `centroids` (the memory is normally built once and
+ * then only read).  T_b == 0 returns the retrieved state itself.
  */
+#define ASM_DECODE_PREFETCH_CENTROIDS 1u
 size_t asm_decode_workspace_size(int B, int Hq, int Hkv, int K, int Tmax,
                                  int d, asm_dtype dt);
 asm_status asm_decode_step(const void *q, const void *centroids,
@@ -205,8 +213,8 @@ asm_status asm_decode_step(const void *q, const void *centroids,
                            const int32_t *local_len, int B, int Hq, int Hkv,
                            int K, int Tmax, int d, float scale,
                            asm_metric metric, asm_dtype dt, void *out,
-                           float *lse_out, int32_t *idx_out, void *ws,
-                           size_t ws_bytes, cudaStream_t stream);
+                           float *lse_out, int32_t *idx_out, unsigned flags,
+                           void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
  * asm_flash_decode -- the quantity the memory stands in for: decode attention

@@ -154,9 +154,11 @@ asm_status asm_decode_step(const void *q, const void *centroids, const void *a_b
                            const float *logz_bar, const void *k_cache, const void *v_cache,
                            const int32_t *local_len, int B, int Hq, int Hkv, int K, int Tmax, int d,
                            float scale, asm_metric metric, asm_dtype dt, void *out, float *lse_out,
-                           int32_t *idx_out, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                           int32_t *idx_out, unsigned flags, void *ws, size_t ws_bytes,
+                           cudaStream_t stream) {
     if (!dt_ok(dt) || B < 1 || B > 4096 || K < 1 || Tmax < 0 || !(scale == scale)) return ASM_ERR_INVALID_ARG;
     if (metric != ASM_L2 && metric != ASM_COSINE) return ASM_ERR_INVALID_ARG;
+    if ((flags & ~ASM_DECODE_PREFETCH_CENTROIDS) != 0) return ASM_ERR_INVALID_ARG;
     if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ASM_ERR_INVALID_ARG;
     if (!d_ok(d) || !group_ok(Hq, Hkv)) return ASM_ERR_UNSUPPORTED;
     if (!aligned(q, 16) || !aligned(centroids, 16) || !aligned(a_bar, 16) || !aligned(logz_bar, 4) ||
@@ -168,7 +170,7 @@ asm_status asm_decode_step(const void *q, const void *centroids, const void *a_b
         return ASM_ERR_WORKSPACE;
     return cuda_status(asm_decode_launch(0, q, centroids, a_bar, logz_bar, nullptr, nullptr, 0, k_cache,
                                          v_cache, local_len, B, Hq, Hkv, K, Tmax, d, scale, (int)metric,
-                                         dt, out, lse_out, idx_out, ws, num_sms(), stream));
+                                         dt, out, lse_out, idx_out, flags, ws, num_sms(), stream));
 }
 
 size_t asm_flash_decode_workspace_size(int B, int Hq, int Hkv, int Lp, int Tmax, int d, asm_dtype dt) {
@@ -192,7 +194,7 @@ asm_status asm_flash_decode(const void *q, const void *k_prefix, const void *v_p
         return ASM_ERR_WORKSPACE;
     return cuda_status(asm_decode_launch(1, q, nullptr, nullptr, nullptr, k_prefix, v_prefix, Lp, k_cache,
                                          v_cache, local_len, B, Hq, Hkv, 1, Tmax, d, scale, 0, dt, out,
-                                         lse_out, nullptr, ws, num_sms(), stream));
+                                         lse_out, nullptr, 0u, ws, num_sms(), stream));
 }
 
 asm_status asm_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream) {

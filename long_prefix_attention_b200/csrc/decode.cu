@@ -7,22 +7,34 @@
 // online-softmax merge (Fusion).
 //
 // One launch does the whole step.  The bytes that must stream from HBM are
-// cut into 16 KB work units laid out group by group (g = KV head):
+// cut into 16 KB work units laid out KV group by KV group (g = KV head):
 //     [centroid rows of the G query heads of g] [local K/V of (b=0,g)] ...
 // (flash-decode mode instead has, per (b,g), [prefix K/V units][local units]).
-// CTA i owns the contiguous unit range [i*upc, (i+1)*upc).  A producer warp
-// streams the units through a ring of shared-memory stages with 1-D bulk
-// copies (cp.async.bulk + mbarrier transaction counts); four consumer warps
-// process each unit.  Consecutive units of one key (a head for centroid
-// scans, a (b,g) pair for attention) are reduced in registers and written as
-// ONE partial per CTA run, into the slot of the run's first unit.  Each CTA
-// then adds the run length to the (b,g) arrival counter; the CTA that
-// completes a counter merges all partials of that (b,g) -- argmax of the
-// centroid scores, log-sum-exp of the attention partials, the gather of
+// CTA i owns the contiguous unit range [i*upc, (i+1)*upc), one CTA per SM.
+// A producer warp streams the units through a ring of shared-memory stages
+// (bf16: 3-D TMA tensor loads with 128-byte swizzling; fp32: 1-D bulk
+// copies), completing on mbarrier transaction counts; four consumer warps
+// process each unit -- bf16 on tensor cores with warp-level m16n8k16 MMAs
+// (q.c and |c|^2 from the same ldmatrix fragments, then q.k and p.v), fp32 on
+// CUDA cores.  Consecutive units of one key (a head for centroid scans, a
+// (b,g) pair for attention) are reduced in registers and written as ONE
+// partial per CTA run, into the slot of the run's first unit.  Each CTA then
+// adds the run length to the (b,g) arrival counter; the CTA that completes a
+// counter merges the partials of that (b,g) -- arg-max of the centroid
+// scores, log-sum-exp of the attention partials, the gather of
 // (a_bar, logZ_bar)[idx] and the final state merge -- writes the outputs and
 // resets the counter for the next call.  No CTA ever waits for another.
+//
+// Launched with programmatic dependent launch: every thread waits for the
+// preceding grid before reading inputs; with ASM_DECODE_PREFETCH_CENTROIDS
+// the producer may stream the first centroid units before that wait.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "launch.h"
@@ -32,20 +44,32 @@ namespace asmk {
 constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
 constexpr int kUnitBytes = 16384;
+constexpr int kDecodeStages = 8;
 
 template <typename T, int D, int G>
 struct DCfg {
-    static constexpr int EPL = D / 32;                         // dims per lane
+    static constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;
+    static constexpr int EPL = D / 32;                         // dims per lane (CUDA-core path)
     static constexpr int ROWB = D * (int)sizeof(T);            // bytes per row
     static constexpr int CS = kUnitBytes / ROWB;               // centroid rows / unit
     static constexpr int TS = kUnitBytes / (2 * ROWB);         // tokens / unit
+    // CUDA-core path
     static constexpr int TSW = (32 / G) < TS ? (32 / G) : TS;  // tokens / warp step
     static constexpr int NV = G * TSW;                         // values reduced / step
     static constexpr int R = 32 / NV;                          // lanes per value
     static constexpr int NTG = TS / TSW;                       // token groups / unit
     static constexpr int CSW = CS / kDecodeConsumerWarps;      // centroid rows / warp
+    // tensor-core path (bf16)
+    static constexpr int HALVES = D / 64;                      // 128-byte column halves
+    static constexpr int TW = TS / kDecodeConsumerWarps;       // tokens / warp / unit (8 or 16)
+    static constexpr int NTS = TW / 8;                         // S n-tiles / warp
+    static constexpr int RB = CS / kDecodeConsumerWarps / 16;  // 16-row scan blocks / warp
+    static constexpr int KSTEPS = D / 16;
+    static constexpr int NTO = D / 8;                          // O n-tiles
     static_assert(NV <= 32 && (NV & (NV - 1)) == 0, "NV");
     static_assert(CSW >= 1 && CSW <= 32 && (CSW & (CSW - 1)) == 0, "CSW");
+    static_assert(!TC || (TW == 8 || TW == 16), "TW");
+    static_assert(!TC || G <= 8, "G");
 };
 
 struct DecodeArgs {
@@ -62,21 +86,29 @@ struct DecodeArgs {
     float *lse_out;
     int *idx_out;
     int B, Hq, Hkv, K, Tmax, Lp;
+    float scale;   // softmax scale
     float qscale;  // scale * log2(e): attention logits are kept in base 2
     int metric;
     int mode;      // 0: memory lookup + local; 1: explicit prefix + local
+    int flags;
     int nS;        // centroid units per head (mode 0)
     int nP;        // prefix units per (b,g) (mode 1)
     int nA;        // local units per (b,g)
     int UG;        // units per KV group
     int U;         // total units
     int upc;       // units per CTA
-    int stages;
+    int ccap;      // (b, g) pairs one CTA may have to merge
     float2 *ws_srch;  // [B][Hq][nS]   (score, idx bits)
     float2 *ws_ml;    // [B][Hq][nP+nA] (m, l), base-2 logits
     float *ws_o;      // [B][Hq][nP+nA][D] unnormalised outputs
     int *ws_cnt;      // [B][Hkv] arrival counters (self-resetting)
     int *ws_err;
+};
+
+// TMA descriptors (bf16 path): centroids [Hq][K][D], caches [B*Hkv][Tmax][D],
+// prefix [Hkv][Lp][D]; boxes of 64 columns (128 bytes) x unit rows.
+struct DecodeMaps {
+    CUtensorMap c, k, v, kp, vp;
 };
 
 // Decoded work unit.
@@ -87,8 +119,7 @@ struct Unit {
     int slot;   // slot within the key's partial array
     int first;  // first row (scan) / first token (attention) within its source
     int valid;  // valid rows / tokens in this unit (may be <= 0)
-    const char *src_k;  // first byte to copy (scan: centroid rows; attn: K rows)
-    const char *src_v;  // attention: V rows
+    int prefix; // attention unit over the explicit prefix (mode 1)
     int key;    // run key
 };
 
@@ -98,7 +129,7 @@ __device__ __forceinline__ Unit decode_unit(const DecodeArgs &a, int u, const in
     Unit x;
     x.g = u / a.UG;
     int r = u - x.g * a.UG;
-    x.src_v = nullptr;
+    x.prefix = 0;
     if (a.mode == 0 && r < G * a.nS) {
         x.kind = 0;
         x.h = x.g * G + r / a.nS;
@@ -106,41 +137,86 @@ __device__ __forceinline__ Unit decode_unit(const DecodeArgs &a, int u, const in
         x.b = 0;
         x.first = x.slot * C::CS;
         x.valid = min(C::CS, a.K - x.first);
-        x.src_k = (const char *)a.centroids + ((size_t)x.h * a.K + x.first) * C::ROWB;
         x.key = x.h;  // centroid keys: 0 .. Hq-1
         return x;
     }
     x.kind = 1;
     x.h = 0;
-    int per_b = a.nP + a.nA;
-    int r2 = (a.mode == 0) ? r - G * a.nS : r;
+    const int per_b = a.nP + a.nA;
+    const int r2 = (a.mode == 0) ? r - G * a.nS : r;
     x.b = r2 / per_b;
     x.slot = r2 % per_b;
     x.key = a.Hq + x.b * a.Hkv + x.g;  // attention keys follow the centroid keys
     if (x.slot < a.nP) {
+        x.prefix = 1;
         x.first = x.slot * C::TS;
         x.valid = min(C::TS, a.Lp - x.first);
-        size_t off = ((size_t)x.g * a.Lp + x.first) * C::ROWB;
-        x.src_k = (const char *)a.k_prefix + off;
-        x.src_v = (const char *)a.v_prefix + off;
     } else {
         x.first = (x.slot - a.nP) * C::TS;
-        x.valid = min(C::TS, lens[x.b] - x.first);
-        size_t off = (((size_t)x.b * a.Hkv + x.g) * a.Tmax + x.first) * C::ROWB;
-        x.src_k = (const char *)a.k_cache + off;
-        x.src_v = (const char *)a.v_cache + off;
+        x.valid = lens ? min(C::TS, min(max(__ldg(lens + x.b), 0), a.Tmax) - x.first) : C::TS;
     }
     return x;
 }
 
 __device__ __forceinline__ void set_error(int *err) { atomicExch(err, (int)ASM_ERR_TIMEOUT); }
 
+// Runs recorded per CTA before their arrivals are published together.
+constexpr int kMaxRuns = 32;
+
+// Publish one run immediately (used only when a CTA has more than kMaxRuns
+// runs): fence, count, and queue the (b, g) pairs it completes.
+__device__ void publish_run(const DecodeArgs &a, int kind, int g, int b, int len, int G,
+                            int *combine_list) {
+    __threadfence();
+    const int target = (a.mode == 0 ? G * a.nS : a.nP) + a.nA;
+    for (int bb = 0; bb < a.B; ++bb) {
+        if (kind == 1 && bb != b) continue;
+        const int old = atomicAdd(&a.ws_cnt[bb * a.Hkv + g], len);
+        if (old + len == target) {
+            const int slot = combine_list[0]++;
+            if (slot < a.ccap) {
+                combine_list[1 + 2 * slot] = bb;
+                combine_list[2 + 2 * slot] = g;
+            } else {
+                set_error(a.ws_err);
+            }
+        }
+    }
+}
+
 // Consumer-only barrier (named barrier 1, the four consumer warps).
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kDecodeConsumerWarps * 32) : "memory");
 }
 
-// Merge all partials of (b, g) and write the outputs (consumer warps).
+// Slots of a key holding partials: slot 0 and every slot whose unit starts a
+// CTA range.  operator()(j) is the j-th such slot (j < count).
+struct SlotSeq {
+    int first, step, count;
+    __device__ SlotSeq(int base, int nslots, int upc) {
+        step = upc;
+        const int f = (upc - base % upc) % upc;
+        if (nslots <= 0) {
+            first = 0;
+            count = 0;
+        } else if (f == 0) {
+            first = 0;
+            count = (nslots + upc - 1) / upc;
+        } else {
+            first = f;
+            count = 1 + (f < nslots ? (nslots - f + upc - 1) / upc : 0);
+        }
+    }
+    __device__ int operator()(int j) const {
+        return first == 0 ? j * step : (j == 0 ? 0 : first + (j - 1) * step);
+    }
+};
+
+// Merge all partials of (b, g) and write the outputs (consumer warps).  All
+// partial reads of a head are issued together (one round trip), then the
+// retrieved state is gathered (a second one).
+constexpr int kCombineBatch = 16;
+
 template <typename T, int D, int G>
 __device__ void combine(const DecodeArgs &a, int b, int g, int warp, int lane) {
     using C = DCfg<T, D, G>;
@@ -148,30 +224,45 @@ __device__ void combine(const DecodeArgs &a, int b, int g, int warp, int lane) {
     for (int hh = warp; hh < G; hh += kDecodeConsumerWarps) {
         const int h = g * G + hh;
         const size_t bh = (size_t)b * a.Hq + h;
-        // ---- retrieval: arg-max over the scan partials of head h
+        const SlotSeq as(g * a.UG + (a.mode == 0 ? G * a.nS : 0) + b * nslots, nslots, a.upc);
+        // ---- round 1: scan partials, (m, l) and the first output rows
+        float bs = kNegInf;
+        int bi = 0x7fffffff;
+        if (a.mode == 0) {
+            const SlotSeq ss(g * a.UG + hh * a.nS, a.nS, a.upc);
+            for (int j = lane; j < ss.count; j += 32) {
+                const float2 v = __ldcg(a.ws_srch + bh * a.nS + ss(j));
+                const int vi = __float_as_int(v.y);
+                if (better(v.x, vi, bs, bi)) { bs = v.x; bi = vi; }
+            }
+        }
+        float2 ml = make_float2(kNegInf, 0.f);
+        if (lane < as.count) ml = __ldcg(a.ws_ml + bh * nslots + as(lane));
+        float ov[kCombineBatch][C::EPL];
+#pragma unroll
+        for (int k = 0; k < kCombineBatch; ++k) {
+            const bool use = k < as.count;
+            const float *os = a.ws_o + (bh * nslots + as(use ? k : 0)) * D + lane * C::EPL;
+#pragma unroll
+            for (int e = 0; e < C::EPL; ++e) ov[k][e] = use ? __ldcg(os + e) : 0.f;
+        }
         int idx = 0;
         if (a.mode == 0) {
-            float bs = kNegInf;
-            int bi = 0x7fffffff;
-            const int ubase = g * a.UG + hh * a.nS;
-            for (int s = lane; s < a.nS; s += 32) {
-                if (s == 0 || (ubase + s) % a.upc == 0) {
-                    float2 v = __ldcg(a.ws_srch + bh * a.nS + s);
-                    int vi = __float_as_int(v.y);
-                    if (better(v.x, vi, bs, bi)) { bs = v.x; bi = vi; }
-                }
-            }
             warp_argmax(bs, bi);
             idx = (bi == 0x7fffffff) ? 0 : bi;
         }
-        // ---- local (and prefix) attention: log-sum-exp of the partials
-        const int abase = g * a.UG + (a.mode == 0 ? G * a.nS : 0) + b * nslots;
-        float M = kNegInf;
-        for (int s = lane; s < nslots; s += 32) {
-            if (s == 0 || (abase + s) % a.upc == 0) {
-                float2 ml = __ldcg(a.ws_ml + bh * nslots + s);
-                if (ml.y > 0.f) M = fmaxf(M, ml.x);
-            }
+        // ---- round 2: the retrieved state
+        float ab[C::EPL];
+        float zb = kNegInf;
+        if (a.mode == 0) {
+            zb = __ldg(a.logz_bar + (size_t)h * a.K + idx);
+            load_vec<T, C::EPL>((const T *)a.a_bar + ((size_t)h * a.K + idx) * D + lane * C::EPL, ab);
+        }
+        // log-sum-exp of the attention partials (slots beyond 32 in later rounds)
+        float M = (ml.y > 0.f) ? ml.x : kNegInf;
+        for (int j = lane + 32; j < as.count; j += 32) {
+            const float2 m2 = __ldcg(a.ws_ml + bh * nslots + as(j));
+            if (m2.y > 0.f) M = fmaxf(M, m2.x);
         }
         M = warp_max(M);
         float L = 0.f;
@@ -179,24 +270,29 @@ __device__ void combine(const DecodeArgs &a, int b, int g, int warp, int lane) {
 #pragma unroll
         for (int e = 0; e < C::EPL; ++e) o[e] = 0.f;
         if (M != kNegInf) {
-            for (int s = 0; s < nslots; ++s) {
-                if (!(s == 0 || (abase + s) % a.upc == 0)) continue;
-                float2 ml = __ldcg(a.ws_ml + bh * nslots + s);
-                if (!(ml.y > 0.f)) continue;
-                float w = exp2f(ml.x - M);
-                L += ml.y * w;
-                const float *os = a.ws_o + (bh * nslots + s) * D + lane * C::EPL;
+            const float w = (ml.y > 0.f) ? exp2f(ml.x - M) : 0.f;
+            L = warp_sum(ml.y * w);
 #pragma unroll
-                for (int e = 0; e < C::EPL; ++e) o[e] += w * __ldcg(os + e);
+            for (int k = 0; k < kCombineBatch; ++k) {
+                const float wk = __shfl_sync(0xffffffffu, w, k);
+#pragma unroll
+                for (int e = 0; e < C::EPL; ++e) o[e] = fmaf(wk, ov[k][e], o[e]);
+            }
+            for (int j = kCombineBatch; j < as.count; ++j) {  // rare: more than 16 partials
+                const float2 m2 = __ldcg(a.ws_ml + bh * nslots + as(j));
+                if (!(m2.y > 0.f)) continue;
+                const float wj = exp2f(m2.x - M);
+                if (j >= 32) L += m2.y * wj;
+                const float *os = a.ws_o + (bh * nslots + as(j)) * D + lane * C::EPL;
+#pragma unroll
+                for (int e = 0; e < C::EPL; ++e) o[e] = fmaf(wj, __ldcg(os + e), o[e]);
             }
         }
-        float zl = (L > 0.f) ? (M + log2f(L)) * kLn2 : kNegInf;  // natural log
+        const float zl = (L > 0.f) ? (M + log2f(L)) * kLn2 : kNegInf;  // natural log
         float res[C::EPL];
         float lse;
+        const float invL = (L > 0.f) ? 1.f / L : 0.f;
         if (a.mode == 0) {
-            const float zb = a.logz_bar[(size_t)h * a.K + idx];
-            float ab[C::EPL];
-            load_vec<T, C::EPL>((const T *)a.a_bar + ((size_t)h * a.K + idx) * D + lane * C::EPL, ab);
             if (zb == kNegInf && zl == kNegInf) {
                 lse = kNegInf;
 #pragma unroll
@@ -206,13 +302,11 @@ __device__ void combine(const DecodeArgs &a, int b, int g, int warp, int lane) {
                 const float eb = expf(zb - m), el = expf(zl - m);
                 lse = m + logf(eb + el);
                 const float wb = eb / (eb + el), wl = el / (eb + el);
-                const float invL = (L > 0.f) ? 1.f / L : 0.f;
 #pragma unroll
                 for (int e = 0; e < C::EPL; ++e) res[e] = wb * ab[e] + wl * (o[e] * invL);
             }
         } else {
             lse = zl;
-            const float invL = (L > 0.f) ? 1.f / L : 0.f;
 #pragma unroll
             for (int e = 0; e < C::EPL; ++e) res[e] = o[e] * invL;
         }
@@ -224,12 +318,17 @@ __device__ void combine(const DecodeArgs &a, int b, int g, int warp, int lane) {
     }
 }
 
+// ---------------------------------------------------------------- kernel --
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads, 3)
-decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
     using C = DCfg<T, D, G>;
-    extern __shared__ __align__(128) unsigned char smem[];
-    const int S = a.stages;
+    constexpr int S = kDecodeStages;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte alignment for the 128-byte-swizzled TMA tiles
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     unsigned char *stage_buf = smem;                                   // S * kUnitBytes
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * kUnitBytes);
     uint64_t *empty = full + S;
@@ -237,44 +336,102 @@ decode_kernel(const DecodeArgs a) {
     float *flush_m = flush_o + kDecodeConsumerWarps * G * D;           // [W][G]
     float *flush_l = flush_m + kDecodeConsumerWarps * G;               // [W][G]
     float2 *best = reinterpret_cast<float2 *>(flush_l + kDecodeConsumerWarps * G);  // [W][B]
-    int *lens = reinterpret_cast<int *>(best + kDecodeConsumerWarps * a.B);         // [B]
-    int *combine_list = lens + a.B;                                    // [B+1]
+    int *combine_list = reinterpret_cast<int *>(best + kDecodeConsumerWarps * a.B);  // [1 + 2*ccap]
+    int4 *runs = reinterpret_cast<int4 *>(combine_list + ((2 * a.ccap + 4) & ~3));  // (kind, g, b, len)
+    int *n_runs = reinterpret_cast<int *>(runs + kMaxRuns);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int u_begin = blockIdx.x * a.upc;
     const int u_end = min(a.U, u_begin + a.upc);
     const int n_units = u_end - u_begin;
 
-    for (int i = tid; i < a.B; i += blockDim.x) lens[i] = min(max(a.local_len[i], 0), a.Tmax);
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kDecodeConsumerWarps);
         }
         fence_mbar_init();
+        *n_runs = 0;
+        combine_list[0] = 0;
     }
     __syncthreads();
+
+    // Units issued before the dependency wait: leading centroid units only,
+    // and only when the caller allows it (the memory is not written by the
+    // preceding kernel).
+    int pre = 0;
+    if constexpr (C::TC) {
+        if (warp == kDecodeConsumerWarps && lane == 0 && (a.flags & 1)) {
+            for (; pre < min(n_units, S); ++pre) {
+                const Unit x = decode_unit<T, D, G>(a, u_begin + pre, nullptr);
+                if (x.kind != 0) break;
+                unsigned char *dst = stage_buf + (size_t)pre * kUnitBytes;
+                mbar_arrive_expect_tx(&full[pre], C::CS * C::ROWB);
+#pragma unroll
+                for (int hf = 0; hf < C::HALVES; ++hf)
+                    tma_load_3d(dst + hf * C::CS * 128, &maps.c, 64 * hf, x.first, x.h, &full[pre]);
+            }
+        }
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+    const int *lens = a.local_len;
 
     if (warp == kDecodeConsumerWarps) {
         // ------------------------------------------------ producer warp
         if (lane == 0) {
-            for (int i = 0; i < n_units; ++i) {
+            // start fetching the row lengths the local units of this range need
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(lens));
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(lens + (a.B - 1)));
+            for (int i = pre; i < n_units; ++i) {
                 const int s = i % S;
                 if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) set_error(a.ws_err);
-                Unit x = decode_unit<T, D, G>(a, u_begin + i, lens);
+                const Unit x = decode_unit<T, D, G>(a, u_begin + i, lens);
                 unsigned char *dst = stage_buf + (size_t)s * kUnitBytes;
-                if (x.valid > 0) {
-                    const uint32_t rb = (uint32_t)x.valid * C::ROWB;
+                if (x.valid <= 0) {
+                    mbar_arrive(&full[s]);
+                    continue;
+                }
+                if constexpr (C::TC) {
                     if (x.kind == 0) {
-                        mbar_arrive_expect_tx(&full[s], rb);
-                        bulk_g2s(dst, x.src_k, rb, &full[s]);
+                        mbar_arrive_expect_tx(&full[s], C::CS * C::ROWB);
+#pragma unroll
+                        for (int hf = 0; hf < C::HALVES; ++hf)
+                            tma_load_3d(dst + hf * C::CS * 128, &maps.c, 64 * hf, x.first, x.h, &full[s]);
                     } else {
-                        mbar_arrive_expect_tx(&full[s], 2 * rb);
-                        bulk_g2s(dst, x.src_k, rb, &full[s]);
-                        bulk_g2s(dst + C::TS * C::ROWB, x.src_v, rb, &full[s]);
+                        mbar_arrive_expect_tx(&full[s], 2 * C::TS * C::ROWB);
+                        const CUtensorMap *mk = x.prefix ? &maps.kp : &maps.k;
+                        const CUtensorMap *mv = x.prefix ? &maps.vp : &maps.v;
+                        const int c2 = x.prefix ? x.g : x.b * a.Hkv + x.g;
+#pragma unroll
+                        for (int hf = 0; hf < C::HALVES; ++hf) {
+                            tma_load_3d(dst + hf * C::TS * 128, mk, 64 * hf, x.first, c2, &full[s]);
+                            tma_load_3d(dst + kUnitBytes / 2 + hf * C::TS * 128, mv, 64 * hf, x.first, c2,
+                                        &full[s]);
+                        }
                     }
                 } else {
-                    mbar_arrive(&full[s]);
+                    const uint32_t rb = (uint32_t)x.valid * C::ROWB;
+                    if (x.kind == 0) {
+                        const char *src = (const char *)a.centroids + ((size_t)x.h * a.K + x.first) * C::ROWB;
+                        mbar_arrive_expect_tx(&full[s], rb);
+                        bulk_g2s(dst, src, rb, &full[s]);
+                    } else {
+                        size_t off;
+                        const char *kb, *vb;
+                        if (x.prefix) {
+                            off = ((size_t)x.g * a.Lp + x.first) * C::ROWB;
+                            kb = (const char *)a.k_prefix;
+                            vb = (const char *)a.v_prefix;
+                        } else {
+                            off = (((size_t)x.b * a.Hkv + x.g) * a.Tmax + x.first) * C::ROWB;
+                            kb = (const char *)a.k_cache;
+                            vb = (const char *)a.v_cache;
+                        }
+                        mbar_arrive_expect_tx(&full[s], 2 * rb);
+                        bulk_g2s(dst, kb + off, rb, &full[s]);
+                        bulk_g2s(dst + kUnitBytes / 2, vb + off, rb, &full[s]);
+                    }
                 }
             }
             // Drain: every issued copy has landed before the CTA may exit.
@@ -285,39 +442,56 @@ decode_kernel(const DecodeArgs a) {
     }
 
     // ---------------------------------------------------- consumer warps
+    const int gid = lane >> 2, quad = lane & 3;
     int cur_key = -1;
     Unit run{};
     int run_len = 0;
-    // attention running state (one (m, l, o) per head of the group, per warp)
+    // CUDA-core attention state: (m, l, o) per head of the group, lanes = dims
     float m_run[G], l_run[G], o_run[G][C::EPL];
     float qreg[G][C::EPL];
+    // tensor-core attention state: row gid (= head of the group), O fragments
+    float tm_run = kNegInf, tl_run = 0.f;
+    float to[C::NTO][4];
+    uint32_t qa0[C::KSTEPS], qa2[C::KSTEPS];
 
     auto flush = [&](const Unit &rx, int len) {
         // Publish this CTA's partial of the run's key, then count arrivals.
         if (rx.kind == 0) {
             consumer_sync();
-            // merge the per-warp bests for every row b
             for (int b = tid; b < a.B; b += kDecodeConsumerWarps * 32) {
                 float bs = kNegInf;
                 int bi = 0x7fffffff;
                 for (int w = 0; w < kDecodeConsumerWarps; ++w) {
-                    float2 v = best[w * a.B + b];
-                    int vi = __float_as_int(v.y);
+                    const float2 v = best[w * a.B + b];
+                    const int vi = __float_as_int(v.y);
                     if (better(v.x, vi, bs, bi)) { bs = v.x; bi = vi; }
                 }
-                a.ws_srch[((size_t)b * a.Hq + rx.h) * a.nS + rx.slot] =
-                    make_float2(bs, __int_as_float(bi));
+                a.ws_srch[((size_t)b * a.Hq + rx.h) * a.nS + rx.slot] = make_float2(bs, __int_as_float(bi));
             }
         } else {
+            if constexpr (C::TC) {
+                if (gid < G) {
+                    if (quad == 0) {
+                        flush_m[warp * G + gid] = tm_run;
+                        flush_l[warp * G + gid] = tl_run;
+                    }
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                if (lane == 0) {
-                    flush_m[warp * G + h] = m_run[h];
-                    flush_l[warp * G + h] = l_run[h];
+                    for (int c = 0; c < C::NTO; ++c) {
+                        flush_o[(warp * G + gid) * D + 8 * c + 2 * quad] = to[c][0];
+                        flush_o[(warp * G + gid) * D + 8 * c + 2 * quad + 1] = to[c][1];
+                    }
                 }
+            } else {
 #pragma unroll
-                for (int e = 0; e < C::EPL; ++e)
-                    flush_o[(warp * G + h) * D + lane * C::EPL + e] = o_run[h][e];
+                for (int h = 0; h < G; ++h) {
+                    if (lane == 0) {
+                        flush_m[warp * G + h] = m_run[h];
+                        flush_l[warp * G + h] = l_run[h];
+                    }
+#pragma unroll
+                    for (int e = 0; e < C::EPL; ++e)
+                        flush_o[(warp * G + h) * D + lane * C::EPL + e] = o_run[h][e];
+                }
             }
             consumer_sync();
             const int nslots = a.nP + a.nA;
@@ -330,7 +504,7 @@ decode_kernel(const DecodeArgs a) {
                 if (M != kNegInf) {
                     for (int w = 0; w < kDecodeConsumerWarps; ++w) {
                         if (!(flush_l[w * G + h] > 0.f)) continue;
-                        float sc = exp2f(flush_m[w * G + h] - M);
+                        const float sc = exp2f(flush_m[w * G + h] - M);
                         L += flush_l[w * G + h] * sc;
                         o += flush_o[(w * G + h) * D + dd] * sc;
                     }
@@ -340,33 +514,20 @@ decode_kernel(const DecodeArgs a) {
                 if (dd == 0) a.ws_ml[bh * nslots + rx.slot] = make_float2(M, L);
             }
         }
-        // make the partial visible, then count this run's units
-        __threadfence();
+        // record the run; its arrival is published once, at the end of the CTA
+        consumer_sync();
+        if (*n_runs >= kMaxRuns) __threadfence();  // overflow: published right away below
         consumer_sync();
         if (tid == 0) {
-            int n = 0;
-            const int target = (a.mode == 0 ? G * a.nS : a.nP) + a.nA;
-            if (rx.kind == 0) {
-                for (int b = 0; b < a.B; ++b) {
-                    int old = atomicAdd(&a.ws_cnt[b * a.Hkv + rx.g], len);
-                    if (old + len == target) combine_list[1 + n++] = b;
-                }
+            const int r = *n_runs;
+            if (r < kMaxRuns) {
+                runs[r] = make_int4(rx.kind, rx.g, rx.b, len);
+                *n_runs = r + 1;
             } else {
-                int old = atomicAdd(&a.ws_cnt[rx.b * a.Hkv + rx.g], len);
-                if (old + len == target) combine_list[1 + n++] = rx.b;
+                publish_run(a, rx.kind, rx.g, rx.b, len, G, combine_list);  // overflow: at once
             }
-            combine_list[0] = n;
-            __threadfence();
         }
         consumer_sync();
-        const int n = combine_list[0];
-        for (int j = 0; j < n; ++j) {
-            const int b = combine_list[1 + j];
-            combine<T, D, G>(a, b, rx.g, warp, lane);
-        }
-        consumer_sync();
-        if (tid == 0)
-            for (int j = 0; j < n; ++j) atomicExch(&a.ws_cnt[combine_list[1 + j] * a.Hkv + rx.g], 0);
     };
 
     for (int i = 0; i < n_units; ++i) {
@@ -377,22 +538,35 @@ decode_kernel(const DecodeArgs a) {
             cur_key = x.key;
             run = x;
             run_len = 0;
-            // start a new run
             if (x.kind == 0) {
                 for (int b = lane; b < a.B; b += 32)
                     best[warp * a.B + b] = make_float2(kNegInf, __int_as_float(0x7fffffff));
             } else {
+                if constexpr (C::TC) {
+                    tm_run = kNegInf;
+                    tl_run = 0.f;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    m_run[h] = kNegInf;
-                    l_run[h] = 0.f;
-                    float qv[C::EPL];
-                    load_vec<T, C::EPL>((const T *)a.q + ((size_t)x.b * a.Hq + x.g * G + h) * D +
-                                            lane * C::EPL, qv);
+                    for (int c = 0; c < C::NTO; ++c) to[c][0] = to[c][1] = to[c][2] = to[c][3] = 0.f;
+                    // A fragments of the group's queries: row gid = head gid of the group
+                    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
+                        (const T *)a.q + ((size_t)x.b * a.Hq + x.g * G + min(gid, G - 1)) * D);
 #pragma unroll
-                    for (int e = 0; e < C::EPL; ++e) {
-                        o_run[h][e] = 0.f;
-                        qreg[h][e] = qv[e] * a.qscale;
+                    for (int j = 0; j < C::KSTEPS; ++j) {
+                        qa0[j] = gid < G ? __ldg(qrow + 8 * j + quad) : 0u;
+                        qa2[j] = gid < G ? __ldg(qrow + 8 * j + 4 + quad) : 0u;
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        m_run[h] = kNegInf;
+                        l_run[h] = 0.f;
+                        float qv[C::EPL];
+                        load_vec<T, C::EPL>((const T *)a.q + ((size_t)x.b * a.Hq + x.g * G + h) * D + lane * C::EPL, qv);
+#pragma unroll
+                        for (int e = 0; e < C::EPL; ++e) {
+                            o_run[h][e] = 0.f;
+                            qreg[h][e] = qv[e] * a.qscale;
+                        }
                     }
                 }
             }
@@ -402,121 +576,285 @@ decode_kernel(const DecodeArgs a) {
         if (!mbar_wait(&full[s], (i / S) & 1)) set_error(a.ws_err);
         const unsigned char *buf = stage_buf + (size_t)s * kUnitBytes;
 
-        if (x.kind == 0) {
-            // ---------------- centroid scan: CSW rows per warp, all rows b
-            const int r0 = warp * C::CSW;
-            float nrm[C::CSW];
-            float cf[C::CSW][C::EPL];
+        if constexpr (C::TC) {
+            const uint32_t sbuf = smem_addr(buf);
+            if (x.kind == 0) {
+                // -------- centroid scan on tensor cores: 16-row blocks, all rows b
 #pragma unroll
-            for (int r = 0; r < C::CSW; ++r) {
-                if (r0 + r < x.valid) {
-                    load_vec<T, C::EPL>(reinterpret_cast<const T *>(buf + (size_t)(r0 + r) * C::ROWB) +
-                                            lane * C::EPL, cf[r]);
-                } else {
+                for (int rb = 0; rb < C::RB; ++rb) {
+                    const int r0 = (warp * C::RB + rb) * 16;
+                    if (r0 >= x.valid) break;
+                    uint32_t bf[C::KSTEPS][2][2];  // [k-step][n-tile][lo/hi]
 #pragma unroll
-                    for (int e = 0; e < C::EPL; ++e) cf[r][e] = 0.f;
+                    for (int j = 0; j < C::KSTEPS; ++j) {
+                        const int i4 = lane >> 3;
+                        const int row = r0 + 8 * (i4 >> 1) + (lane & 7);
+                        const int col = 16 * j + 8 * (i4 & 1);
+                        const uint32_t addr = sbuf + (col >> 6) * (C::CS * 128) + swz128(row, (col & 63) >> 3);
+                        ldsm_x4(addr, bf[j][0][0], bf[j][0][1], bf[j][1][0], bf[j][1][1]);
+                    }
+                    // |c|^2 as the diagonal of C C^T (same fragments as A and B)
+                    float dn[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                    for (int j = 0; j < C::KSTEPS; ++j)
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+                            mma_bf16_16816(dn[nt], bf[j][0][0], bf[j][1][0], bf[j][0][1], bf[j][1][1],
+                                           bf[j][nt][0], bf[j][nt][1]);
+                    const float diag0 = dn[0][gid & 1], diag1 = dn[1][2 + (gid & 1)];
+                    float nrm[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int rr = 2 * quad + e;
+                            nrm[nt][e] = __shfl_sync(0xffffffffu, nt == 0 ? diag0 : diag1, 4 * rr + (rr >> 1));
+                        }
+                    for (int mt = 0; mt * 16 < a.B; ++mt) {
+                        const int b0 = mt * 16 + gid, b1 = b0 + 8;
+                        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(
+                            (const T *)a.q + ((size_t)min(b0, a.B - 1) * a.Hq + x.h) * D);
+                        const uint32_t *q1 = reinterpret_cast<const uint32_t *>(
+                            (const T *)a.q + ((size_t)min(b1, a.B - 1) * a.Hq + x.h) * D);
+                        float dd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                        for (int j = 0; j < C::KSTEPS; ++j) {
+                            const uint32_t a0 = b0 < a.B ? __ldg(q0 + 8 * j + quad) : 0u;
+                            const uint32_t a1 = b1 < a.B ? __ldg(q1 + 8 * j + quad) : 0u;
+                            const uint32_t a2 = b0 < a.B ? __ldg(q0 + 8 * j + 4 + quad) : 0u;
+                            const uint32_t a3 = b1 < a.B ? __ldg(q1 + 8 * j + 4 + quad) : 0u;
+#pragma unroll
+                            for (int nt = 0; nt < 2; ++nt)
+                                mma_bf16_16816(dd[nt], a0, a1, a2, a3, bf[j][nt][0], bf[j][nt][1]);
+                        }
+#pragma unroll
+                        for (int hr = 0; hr < 2; ++hr) {  // rows b0 (hr 0) and b1
+                            float bs = kNegInf;
+                            int bi = 0x7fffffff;
+#pragma unroll
+                            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int rloc = r0 + 8 * nt + 2 * quad + e;
+                                    const float dot = dd[nt][2 * hr + e];
+                                    const float nr = nrm[nt][e];
+                                    float sc = (a.metric == 0) ? dot - 0.5f * nr
+                                                               : (nr > 0.f ? dot / sqrtf(nr) : 0.f);
+                                    int ci = x.first + rloc;
+                                    if (rloc >= x.valid) { sc = kNegInf; ci = 0x7fffffff; }
+                                    if (better(sc, ci, bs, bi)) { bs = sc; bi = ci; }
+                                }
+#pragma unroll
+                            for (int m = 1; m <= 2; m <<= 1) {
+                                const float os = __shfl_xor_sync(0xffffffffu, bs, m);
+                                const int oi = __shfl_xor_sync(0xffffffffu, bi, m);
+                                if (better(os, oi, bs, bi)) { bs = os; bi = oi; }
+                            }
+                            const int bb = hr ? b1 : b0;
+                            if (quad == 0 && bb < a.B) {
+                                const float2 cur = best[warp * a.B + bb];
+                                if (better(bs, bi, cur.x, __float_as_int(cur.y)))
+                                    best[warp * a.B + bb] = make_float2(bs, __int_as_float(bi));
+                            }
+                        }
+                    }
                 }
-                float t = 0.f;
+            } else {
+                // -------- attention on tensor cores: TW tokens per warp
+                const int t0 = warp * C::TW;
+                if (t0 < x.valid) {
+                    float sf[C::NTS][4];
 #pragma unroll
-                for (int e = 0; e < C::EPL; ++e) t = fmaf(cf[r][e], cf[r][e], t);
-                nrm[r] = t;
-            }
-            const float nr = transpose_reduce<C::CSW>(nrm, lane);
-            const int my_row = lane / (32 / C::CSW);
-            const int my_c = x.first + r0 + my_row;
-            const bool my_valid = (r0 + my_row) < x.valid;
-            for (int b = 0; b < a.B; ++b) {
-                float qv[C::EPL];
-                load_vec<T, C::EPL>((const T *)a.q + ((size_t)b * a.Hq + x.h) * D + lane * C::EPL, qv);
-                float dp[C::CSW];
+                    for (int nt = 0; nt < C::NTS; ++nt) sf[nt][0] = sf[nt][1] = sf[nt][2] = sf[nt][3] = 0.f;
 #pragma unroll
-                for (int r = 0; r < C::CSW; ++r) {
-                    float t = 0.f;
+                    for (int j = 0; j < C::KSTEPS; j += 2) {
 #pragma unroll
-                    for (int e = 0; e < C::EPL; ++e) t = fmaf(qv[e], cf[r][e], t);
-                    dp[r] = t;
-                }
-                const float dot = transpose_reduce<C::CSW>(dp, lane);
-                float sc;
-                if (a.metric == 0) sc = dot - 0.5f * nr;
-                else sc = nr > 0.f ? dot / sqrtf(nr) : 0.f;
-                int ci = my_c;
-                if (!my_valid) { sc = kNegInf; ci = 0x7fffffff; }
-                warp_argmax(sc, ci);
-                if (lane == 0) {
-                    float2 cur = best[warp * a.B + b];
-                    if (better(sc, ci, cur.x, __float_as_int(cur.y)))
-                        best[warp * a.B + b] = make_float2(sc, __int_as_float(ci));
+                        for (int nt = 0; nt < C::NTS; ++nt) {
+                            const int i4 = lane >> 3;
+                            const int row = t0 + 8 * nt + (lane & 7);
+                            const int col = 16 * (j + (i4 >> 1)) + 8 * (i4 & 1);
+                            const uint32_t addr = sbuf + (col >> 6) * (C::TS * 128) + swz128(row, (col & 63) >> 3);
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4(addr, b0, b1, b2, b3);
+                            mma_bf16_16816(sf[nt], qa0[j], 0u, qa2[j], 0u, b0, b1);
+                            mma_bf16_16816(sf[nt], qa0[j + 1], 0u, qa2[j + 1], 0u, b2, b3);
+                        }
+                    }
+                    // online softmax for row gid (head), base-2 logits
+                    float p[C::NTS][2];
+                    float mx = kNegInf;
+#pragma unroll
+                    for (int nt = 0; nt < C::NTS; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int tok = t0 + 8 * nt + 2 * quad + e;
+                            p[nt][e] = tok < x.valid ? sf[nt][e] * a.qscale : kNegInf;
+                            mx = fmaxf(mx, p[nt][e]);
+                        }
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    const float mnew = fmaxf(tm_run, mx);
+                    const float alpha = (mnew == kNegInf) ? 1.f : exp2f(tm_run - mnew);
+                    float rs = 0.f;
+#pragma unroll
+                    for (int nt = 0; nt < C::NTS; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            p[nt][e] = (p[nt][e] == kNegInf) ? 0.f : exp2f(p[nt][e] - mnew);
+                            rs += p[nt][e];
+                        }
+                    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+                    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+                    tl_run = tl_run * alpha + rs;
+                    tm_run = mnew;
+#pragma unroll
+                    for (int c = 0; c < C::NTO; ++c) {
+                        to[c][0] *= alpha;
+                        to[c][1] *= alpha;
+                    }
+                    const uint32_t pa0 = pack_bf16(p[0][0], p[0][1]);
+                    const uint32_t pa2 = C::NTS == 2 ? pack_bf16(p[C::NTS - 1][0], p[C::NTS - 1][1]) : 0u;
+                    const uint32_t vbase = sbuf + kUnitBytes / 2;
+                    if constexpr (C::NTS == 1) {
+#pragma unroll
+                        for (int c = 0; c < C::NTO; c += 4) {
+                            const int i4 = lane >> 3;
+                            const int row = t0 + (lane & 7);
+                            const int col = 8 * (c + i4);
+                            const uint32_t addr = vbase + (col >> 6) * (C::TS * 128) + swz128(row, (col & 63) >> 3);
+                            uint32_t v0, v1, v2, v3;
+                            ldsm_x4_t(addr, v0, v1, v2, v3);
+                            mma_bf16_16816(to[c], pa0, 0u, 0u, 0u, v0, 0u);
+                            mma_bf16_16816(to[c + 1], pa0, 0u, 0u, 0u, v1, 0u);
+                            mma_bf16_16816(to[c + 2], pa0, 0u, 0u, 0u, v2, 0u);
+                            mma_bf16_16816(to[c + 3], pa0, 0u, 0u, 0u, v3, 0u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < C::NTO; c += 2) {
+                            const int i4 = lane >> 3;
+                            const int row = t0 + 8 * (i4 & 1) + (lane & 7);
+                            const int col = 8 * (c + (i4 >> 1));
+                            const uint32_t addr = vbase + (col >> 6) * (C::TS * 128) + swz128(row, (col & 63) >> 3);
+                            uint32_t v0, v1, v2, v3;
+                            ldsm_x4_t(addr, v0, v1, v2, v3);
+                            mma_bf16_16816(to[c], pa0, 0u, pa2, 0u, v0, v1);
+                            mma_bf16_16816(to[c + 1], pa0, 0u, pa2, 0u, v2, v3);
+                        }
+                    }
                 }
             }
         } else {
-            // ---------------- attention over TS tokens: warp takes token groups
-            const unsigned char *kb = buf;
-            const unsigned char *vb = buf + C::TS * C::ROWB;
-            for (int tg = warp; tg < C::NTG; tg += kDecodeConsumerWarps) {
-                const int t0 = tg * C::TSW;
-                if (t0 >= x.valid) break;
-                float part[C::NV];
+            if (x.kind == 0) {
+                // ---------------- centroid scan (CUDA cores): CSW rows per warp
+                const int r0 = warp * C::CSW;
+                float nrm[C::CSW];
+                float cf[C::CSW][C::EPL];
 #pragma unroll
-                for (int t = 0; t < C::TSW; ++t) {
-                    float kf[C::EPL];
-                    if (t0 + t < x.valid) {
-                        load_vec<T, C::EPL>(reinterpret_cast<const T *>(kb + (size_t)(t0 + t) * C::ROWB) +
-                                                lane * C::EPL, kf);
+                for (int r = 0; r < C::CSW; ++r) {
+                    if (r0 + r < x.valid) {
+                        load_vec<T, C::EPL>(reinterpret_cast<const T *>(buf + (size_t)(r0 + r) * C::ROWB) + lane * C::EPL, cf[r]);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) kf[e] = 0.f;
+                        for (int e = 0; e < C::EPL; ++e) cf[r][e] = 0.f;
                     }
+                    float t = 0.f;
+#pragma unroll
+                    for (int e = 0; e < C::EPL; ++e) t = fmaf(cf[r][e], cf[r][e], t);
+                    nrm[r] = t;
+                }
+                const float nr = transpose_reduce<C::CSW>(nrm, lane);
+                const int my_row = lane / (32 / C::CSW);
+                const int my_c = x.first + r0 + my_row;
+                const bool my_valid = (r0 + my_row) < x.valid;
+                for (int b = 0; b < a.B; ++b) {
+                    float qv[C::EPL];
+                    load_vec<T, C::EPL>((const T *)a.q + ((size_t)b * a.Hq + x.h) * D + lane * C::EPL, qv);
+                    float dp[C::CSW];
+#pragma unroll
+                    for (int r = 0; r < C::CSW; ++r) {
+                        float t = 0.f;
+#pragma unroll
+                        for (int e = 0; e < C::EPL; ++e) t = fmaf(qv[e], cf[r][e], t);
+                        dp[r] = t;
+                    }
+                    const float dot = transpose_reduce<C::CSW>(dp, lane);
+                    float sc = (a.metric == 0) ? dot - 0.5f * nr : (nr > 0.f ? dot / sqrtf(nr) : 0.f);
+                    int ci = my_c;
+                    if (!my_valid) { sc = kNegInf; ci = 0x7fffffff; }
+                    warp_argmax(sc, ci);
+                    if (lane == 0) {
+                        const float2 cur = best[warp * a.B + b];
+                        if (better(sc, ci, cur.x, __float_as_int(cur.y)))
+                            best[warp * a.B + b] = make_float2(sc, __int_as_float(ci));
+                    }
+                }
+            } else {
+                // ---------------- attention (CUDA cores): warps take token groups
+                const unsigned char *kb = buf;
+                const unsigned char *vb = buf + kUnitBytes / 2;
+                for (int tg = warp; tg < C::NTG; tg += kDecodeConsumerWarps) {
+                    const int t0 = tg * C::TSW;
+                    if (t0 >= x.valid) break;
+                    float part[C::NV];
+#pragma unroll
+                    for (int t = 0; t < C::TSW; ++t) {
+                        float kf[C::EPL];
+                        if (t0 + t < x.valid) {
+                            load_vec<T, C::EPL>(reinterpret_cast<const T *>(kb + (size_t)(t0 + t) * C::ROWB) + lane * C::EPL, kf);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < C::EPL; ++e) kf[e] = 0.f;
+                        }
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            float acc = 0.f;
+#pragma unroll
+                            for (int e = 0; e < C::EPL; ++e) acc = fmaf(qreg[h][e], kf[e], acc);
+                            part[h * C::TSW + t] = acc;
+                        }
+                    }
+                    float sv = transpose_reduce<C::NV>(part, lane);
+                    const int vidx = lane / C::R;
+                    const int my_t = vidx % C::TSW;
+                    if (t0 + my_t >= x.valid) sv = kNegInf;
+                    float mx = sv;
+#pragma unroll
+                    for (int m = 16 / G; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+                    float mnew[G], alpha[G];
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        float acc = 0.f;
-#pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) acc = fmaf(qreg[h][e], kf[e], acc);
-                        part[h * C::TSW + t] = acc;
+                        const float mh = __shfl_sync(0xffffffffu, mx, h * (32 / G));
+                        mnew[h] = fmaxf(m_run[h], mh);
+                        alpha[h] = (mnew[h] == kNegInf) ? 1.f : exp2f(m_run[h] - mnew[h]);
                     }
-                }
-                float sv = transpose_reduce<C::NV>(part, lane);
-                const int vidx = lane / C::R;
-                const int my_t = vidx % C::TSW;
-                if (t0 + my_t >= x.valid) sv = kNegInf;
-                // per-head max over this step's tokens (lanes of a head are contiguous)
-                float mx = sv;
+                    const int my_h = vidx / C::TSW;
+                    float mh_l = mnew[0];
 #pragma unroll
-                for (int m = 16 / G; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-                float mnew[G], alpha[G];
+                    for (int h = 1; h < G; ++h) if (my_h == h) mh_l = mnew[h];
+                    const float p = (sv == kNegInf) ? 0.f : exp2f(sv - mh_l);
+                    float ps = p;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float mh = __shfl_sync(0xffffffffu, mx, h * (32 / G));
-                    mnew[h] = fmaxf(m_run[h], mh);
-                    alpha[h] = (mnew[h] == kNegInf) ? 1.f : exp2f(m_run[h] - mnew[h]);
-                }
-                const int my_h = vidx / C::TSW;
-                float mh_l = mnew[0];
-#pragma unroll
-                for (int h = 1; h < G; ++h) if (my_h == h) mh_l = mnew[h];
-                const float p = (sv == kNegInf) ? 0.f : exp2f(sv - mh_l);
-                float ps = p;
-#pragma unroll
-                for (int m = 16 / G; m >= C::R; m >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float sh = __shfl_sync(0xffffffffu, ps, h * (32 / G));
-                    l_run[h] = l_run[h] * alpha[h] + sh;
-                    m_run[h] = mnew[h];
-#pragma unroll
-                    for (int e = 0; e < C::EPL; ++e) o_run[h][e] *= alpha[h];
-                }
-#pragma unroll
-                for (int t = 0; t < C::TSW; ++t) {
-                    if (t0 + t >= x.valid) break;
-                    float vf[C::EPL];
-                    load_vec<T, C::EPL>(reinterpret_cast<const T *>(vb + (size_t)(t0 + t) * C::ROWB) +
-                                            lane * C::EPL, vf);
+                    for (int m = 16 / G; m >= C::R; m >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        const float ph = __shfl_sync(0xffffffffu, p, (h * C::TSW + t) * C::R);
+                        const float sh = __shfl_sync(0xffffffffu, ps, h * (32 / G));
+                        l_run[h] = l_run[h] * alpha[h] + sh;
+                        m_run[h] = mnew[h];
 #pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) o_run[h][e] = fmaf(ph, vf[e], o_run[h][e]);
+                        for (int e = 0; e < C::EPL; ++e) o_run[h][e] *= alpha[h];
+                    }
+#pragma unroll
+                    for (int t = 0; t < C::TSW; ++t) {
+                        if (t0 + t >= x.valid) break;
+                        float vf[C::EPL];
+                        load_vec<T, C::EPL>(reinterpret_cast<const T *>(vb + (size_t)(t0 + t) * C::ROWB) + lane * C::EPL, vf);
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float ph = __shfl_sync(0xffffffffu, p, (h * C::TSW + t) * C::R);
+#pragma unroll
+                            for (int e = 0; e < C::EPL; ++e) o_run[h][e] = fmaf(ph, vf[e], o_run[h][e]);
+                        }
                     }
                 }
             }
@@ -525,37 +863,122 @@ decode_kernel(const DecodeArgs a) {
         if (lane == 0) mbar_arrive(&empty[s]);
     }
     if (cur_key >= 0) flush(run, run_len);
+
+    // Publish: make this CTA's partials visible, then add every run's length
+    // to its arrival counters in parallel; a counter that reaches its target
+    // marks (b, g) for merging by this CTA.
+    __threadfence();
+    consumer_sync();
+    const int nr = *n_runs;
+    for (int t = tid; t < nr * a.B; t += kDecodeConsumerWarps * 32) {
+        const int4 rr = runs[t / a.B];
+        const int b = t % a.B;
+        if (rr.x == 1 && b != rr.z) continue;  // attention runs count for their own row only
+        const int target = (a.mode == 0 ? G * a.nS : a.nP) + a.nA;
+        const int old = atomicAdd(&a.ws_cnt[b * a.Hkv + rr.y], rr.w);
+        if (old + rr.w == target) {
+            const int slot = atomicAdd(&combine_list[0], 1);
+            if (slot < a.ccap) {
+                combine_list[1 + 2 * slot] = b;
+                combine_list[2 + 2 * slot] = rr.y;
+            } else {
+                set_error(a.ws_err);  // cannot happen: ccap bounds the pairs of one CTA
+            }
+        }
+    }
+    __threadfence();
+    consumer_sync();
+    const int nc = min(combine_list[0], a.ccap);
+    for (int j = 0; j < nc; ++j) combine<T, D, G>(a, combine_list[1 + 2 * j], combine_list[2 + 2 * j], warp, lane);
+    consumer_sync();
+    for (int j = tid; j < nc; j += kDecodeConsumerWarps * 32)
+        atomicExch(&a.ws_cnt[combine_list[1 + 2 * j] * a.Hkv + combine_list[2 + 2 * j]], 0);
 }
 
 // ------------------------------------------------------------- host side --
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 3-D bf16 map [d2][d1][d0] with a box of 64 columns x `rows` rows x 1.
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows) {
+    auto fn = encode_fn();
+    if (!fn || base == nullptr || d1 == 0 || d2 == 0) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {64, rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T, int D, int G>
-static void decode_geometry(DecodeArgs &a, int num_sms, int ctas_per_sm) {
+static void decode_geometry(DecodeArgs &a, int workers) {
     using C = DCfg<T, D, G>;
     a.nS = (a.mode == 0) ? (a.K + C::CS - 1) / C::CS : 0;
     a.nP = (a.mode == 1) ? (a.Lp + C::TS - 1) / C::TS : 0;
     a.nA = (a.Tmax + C::TS - 1) / C::TS;
     a.UG = (a.mode == 0 ? G * a.nS : 0) + a.B * (a.nP + a.nA);
     a.U = a.Hkv * a.UG;
-    const int workers = num_sms * ctas_per_sm;
     a.upc = (a.U + workers - 1) / workers;
     if (a.upc < 1) a.upc = 1;
+    // KV groups one CTA range can touch, times the rows of each
+    const int groups = min(a.Hkv, (a.upc + a.UG - 1) / a.UG + 1);
+    a.ccap = a.B * groups;
 }
 
 template <typename T, int D, int G>
 static cudaError_t decode_launch_t(DecodeArgs a, int num_sms, cudaStream_t st) {
-    const int ctas_per_sm = 3;
-    a.stages = 4;
-    decode_geometry<T, D, G>(a, num_sms, ctas_per_sm);
+    using C = DCfg<T, D, G>;
+    decode_geometry<T, D, G>(a, num_sms);
+    DecodeMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if constexpr (C::TC) {
+        if (a.mode == 0 && !make_map_3d(&maps.c, a.centroids, D, a.K, a.Hq, C::CS)) return cudaErrorInvalidValue;
+        if (a.Tmax > 0) {
+            if (!make_map_3d(&maps.k, a.k_cache, D, a.Tmax, (uint64_t)a.B * a.Hkv, C::TS) ||
+                !make_map_3d(&maps.v, a.v_cache, D, a.Tmax, (uint64_t)a.B * a.Hkv, C::TS))
+                return cudaErrorInvalidValue;
+        }
+        if (a.mode == 1 && a.Lp > 0) {
+            if (!make_map_3d(&maps.kp, a.k_prefix, D, a.Lp, a.Hkv, C::TS) ||
+                !make_map_3d(&maps.vp, a.v_prefix, D, a.Lp, a.Hkv, C::TS))
+                return cudaErrorInvalidValue;
+        }
+    }
     const int grid = (a.U + a.upc - 1) / a.upc;
-    const size_t smem = (size_t)a.stages * kUnitBytes + 2 * a.stages * sizeof(uint64_t) +
+    const size_t smem = 1024 + (size_t)kDecodeStages * kUnitBytes + 2 * kDecodeStages * sizeof(uint64_t) +
                         sizeof(float) * kDecodeConsumerWarps * G * (D + 2) +
-                        sizeof(float2) * kDecodeConsumerWarps * a.B + sizeof(int) * (2 * a.B + 1);
+                        sizeof(float2) * kDecodeConsumerWarps * a.B + sizeof(int) * ((2 * a.ccap + 4) & ~3) +
+                        sizeof(int4) * (kMaxRuns + 1);
     auto kern = decode_kernel<T, D, G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, kDecodeThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    static size_t attr_smem = 0;  // largest dynamic smem opted in so far (per instantiation)
+    if (smem > attr_smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_smem = smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, maps);
 }
 
 template <typename T, int D>
@@ -578,8 +1001,7 @@ struct DecodeWs {
 };
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-DecodeWs decode_ws_layout(int mode, int B, int Hq, int Hkv, int K, int Lp, int Tmax, int d,
-                          asm_dtype dt) {
+DecodeWs decode_ws_layout(int mode, int B, int Hq, int Hkv, int K, int Lp, int Tmax, int d, asm_dtype dt) {
     const int rowb = d * (dt == ASM_BF16 ? 2 : 4);
     const int CS = asmk::kUnitBytes / rowb, TS = asmk::kUnitBytes / (2 * rowb);
     const size_t nS = mode == 0 ? (size_t)(K + CS - 1) / CS : 0;
@@ -595,18 +1017,16 @@ DecodeWs decode_ws_layout(int mode, int B, int Hq, int Hkv, int K, int Lp, int T
 }
 }  // namespace
 
-size_t asm_decode_ws_bytes(int mode, int B, int Hq, int Hkv, int K, int Lp, int Tmax, int d,
-                           asm_dtype dt) {
+size_t asm_decode_ws_bytes(int mode, int B, int Hq, int Hkv, int K, int Lp, int Tmax, int d, asm_dtype dt) {
     return decode_ws_layout(mode, B, Hq, Hkv, K, Lp, Tmax, d, dt).total;
 }
 
 cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, const void *a_bar,
-                              const float *logz_bar, const void *k_prefix, const void *v_prefix,
-                              int Lp, const void *k_cache, const void *v_cache,
-                              const int32_t *local_len, int B, int Hq, int Hkv, int K, int Tmax,
-                              int d, float scale, int metric, asm_dtype dt, void *out,
-                              float *lse_out, int32_t *idx_out, void *ws, int num_sms,
-                              cudaStream_t st) {
+                              const float *logz_bar, const void *k_prefix, const void *v_prefix, int Lp,
+                              const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
+                              int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, asm_dtype dt,
+                              void *out, float *lse_out, int32_t *idx_out, unsigned flags, void *ws,
+                              int num_sms, cudaStream_t st) {
     using namespace asmk;
     DecodeWs w = decode_ws_layout(mode, B, Hq, Hkv, K, Lp, Tmax, d, dt);
     DecodeArgs a{};
@@ -614,7 +1034,7 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
     a.k_prefix = k_prefix; a.v_prefix = v_prefix; a.k_cache = k_cache; a.v_cache = v_cache;
     a.local_len = local_len; a.out = out; a.lse_out = lse_out; a.idx_out = idx_out;
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.K = K; a.Tmax = Tmax; a.Lp = Lp;
-    a.qscale = scale * kLog2e; a.metric = metric; a.mode = mode;
+    a.scale = scale; a.qscale = scale * kLog2e; a.metric = metric; a.mode = mode; a.flags = (int)flags;
     char *base = static_cast<char *>(ws);
     a.ws_err = reinterpret_cast<int *>(base);
     a.ws_cnt = reinterpret_cast<int *>(base + w.off_cnt);

@@ -16,8 +16,8 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
                               int Lp, const void *k_cache, const void *v_cache,
                               const int32_t *local_len, int B, int Hq, int Hkv, int K, int Tmax,
                               int d, float scale, int metric, asm_dtype dt, void *out,
-                              float *lse_out, int32_t *idx_out, void *ws, int num_sms,
-                              cudaStream_t st);
+                              float *lse_out, int32_t *idx_out, unsigned flags, void *ws,
+                              int num_sms, cudaStream_t st);
 
 // build_states.cu
 cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v, int Hq, int Hkv,

@@ -18,6 +18,7 @@ from . import _lib
 ASM_F32, ASM_BF16 = 0, 1
 ASM_L2, ASM_COSINE = 0, 1
 ASM_ZBAR_MEAN, ASM_ZBAR_SUM = 0, 1
+ASM_DECODE_PREFETCH_CENTROIDS = 1
 
 _DT = {torch.float32: ASM_F32, torch.bfloat16: ASM_BF16}
 
@@ -155,7 +156,8 @@ def asm_workspace_error(ws, stream=None) -> int:
 
 
 def asm_decode_step(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, scale: float,
-                    out, ws, lse_out=None, idx_out=None, metric: int = ASM_L2, stream=None):
+                    out, ws, lse_out=None, idx_out=None, metric: int = ASM_L2, flags: int = 0,
+                    stream=None):
     """One decode step: lookup + merge with local attention, into out[B,Hq,d]."""
     _contig(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, out, lse_out, idx_out)
     B, Hq, d = q.shape
@@ -164,7 +166,7 @@ def asm_decode_step(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, 
     _check("asm_decode_step", _lib.load().asm_decode_step(
         _p(q), _p(centroids), _p(a_bar), _p(logz_bar), _p(k_cache), _p(v_cache), _p(local_len),
         B, Hq, Hkv, K, Tmax, d, float(scale), int(metric), _dt(q), _p(out), _p(lse_out),
-        _p(idx_out), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+        _p(idx_out), int(flags), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def asm_flash_decode(q, k_prefix, v_prefix, k_cache, v_cache, local_len, scale: float, out, ws,

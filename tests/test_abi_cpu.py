@@ -53,12 +53,12 @@ NULL = None
 def decode(lib, **kw):
     a = dict(q=FAKE, c=FAKE, ab=FAKE, lz=FAKE, kc=FAKE, vc=FAKE, ll=FAKE, B=1, Hq=32, Hkv=8,
              K=1024, Tmax=2048, d=128, scale=0.088, metric=0, dt=1, out=FAKE, lse=NULL, idx=NULL,
-             ws=FAKE, wsb=1 << 30)
+             flags=0, ws=FAKE, wsb=1 << 30)
     a.update(kw)
     return lib.asm_decode_step(a["q"], a["c"], a["ab"], a["lz"], a["kc"], a["vc"], a["ll"], a["B"],
                                a["Hq"], a["Hkv"], a["K"], a["Tmax"], a["d"], a["scale"],
-                               a["metric"], a["dt"], a["out"], a["lse"], a["idx"], a["ws"],
-                               a["wsb"], None)
+                               a["metric"], a["dt"], a["out"], a["lse"], a["idx"], a["flags"],
+                               a["ws"], a["wsb"], None)
 
 
 def test_decode_validation(lib):
@@ -74,6 +74,7 @@ def test_decode_validation(lib):
     assert decode(lib, wsb=16) == WORKSPACE
     assert decode(lib, ws=NULL) == WORKSPACE
     assert decode(lib, scale=float("nan")) == INVALID
+    assert decode(lib, flags=6) == INVALID
 
 
 def test_workspace_sizes_grow_with_the_problem(lib):

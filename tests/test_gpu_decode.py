@@ -20,7 +20,7 @@ from gpu_common import TOL, check_indices, dev, f64, host, max_abs
 pytestmark = pytest.mark.gpu
 
 
-def run_decode(ins, metric=ops.ASM_L2, with_lse=True, with_idx=True, calls=1):
+def run_decode(ins, metric=ops.ASM_L2, with_lse=True, with_idx=True, calls=1, flags=0):
     q, C, Ab, lz = (dev(ins[k]) for k in ("q", "centroids", "a_bar", "logz_bar"))
     kc, vc, ll = dev(ins["k_cache"]), dev(ins["v_cache"]), dev(ins["local_len"])
     B, Hq, d = q.shape
@@ -33,14 +33,14 @@ def run_decode(ins, metric=ops.ASM_L2, with_lse=True, with_idx=True, calls=1):
     for _ in range(calls):
         out.fill_(float("nan"))
         ops.asm_decode_step(q, C, Ab, lz, kc, vc, ll, ins["scale"], out, ws, lse_out=lse,
-                            idx_out=idx, metric=metric)
+                            idx_out=idx, metric=metric, flags=flags)
     torch.cuda.synchronize()
     assert ops.asm_workspace_error(ws) == 0
     return out, lse, idx
 
 
-def check_decode(ins, metric=ops.ASM_L2, calls=1):
-    out, lse, idx = run_decode(ins, metric, calls=calls)
+def check_decode(ins, metric=ops.ASM_L2, calls=1, flags=0):
+    out, lse, idx = run_decode(ins, metric, calls=calls, flags=flags)
     o_out, o_lse, o_idx, o_gap = O.decode(ins["q"], ins["centroids"], ins["a_bar"], ins["logz_bar"],
                                           ins["k_cache"], ins["v_cache"], ins["local_len"],
                                           ins["scale"], metric)
@@ -73,6 +73,14 @@ def test_decode_tiny_fp32_config():
 
 def test_decode_llama_layer_k1024_t2048_b1():
     check_decode(inputs.decode_inputs(inputs.CONFIGS[1]), calls=3)
+
+
+def test_decode_llama_layer_prefetching_centroids():
+    """ASM_DECODE_PREFETCH_CENTROIDS streams centroid units before the
+    dependency wait; the results are those of the plain call."""
+    check_decode(inputs.decode_inputs(inputs.CONFIGS[1]), calls=2, flags=ops.ASM_DECODE_PREFETCH_CENTROIDS)
+    check_decode(small_case("bf16", B=3, K=700, T=90, local_len=[90, 0, 45]),
+                 flags=ops.ASM_DECODE_PREFETCH_CENTROIDS)
 
 
 def test_decode_llama_layer_k8192_t4096_b16():
