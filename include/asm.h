@@ -217,6 +217,37 @@ asm_status asm_decode_step(const void *q, const void *centroids,
                            void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * asm_decode_step_noalloc -- asm_decode_step without a caller workspace.
+ * The paper has no counterpart: this is a convenience of the library.
+ * It exists for callers that cannot allocate device memory at the point where
+ * they decode -- for example a plug-in inside a host framework that owns all
+ * device allocations and hands none to extensions, or a latency-critical loop
+ * where cudaMalloc is ruled out because it may synchronise the device.
+ * Instead of `ws`, the call uses a scratch array of 8 MiB compiled into the
+ * library (a file-scope __device__ array: every GPU that loads the library
+ * holds it until the process exits).  Problems whose
+ * asm_decode_workspace_size(...) exceeds 8 MiB are rejected with
+ * ASM_ERR_WORKSPACE.  The call allocates and frees nothing.
+ * Arguments, outputs and errors are those of asm_decode_step.
+ * - The first call on a device looks up the array's device address for that
+ *   device (with the device current); make that first call before any stream
+ *   capture.
+ * - Every call on a device shares the one array and it keeps the previous
+ *   call's contents; the call clears the part that must start at zero.  Calls
+ *   that overlap on the GPU (other streams, other host threads) race on it and
+ *   must be serialised by the caller.
+ */
+asm_status asm_decode_step_noalloc(const void *q, const void *centroids,
+                                   const void *a_bar, const float *logz_bar,
+                                   const void *k_cache, const void *v_cache,
+                                   const int32_t *local_len, int B, int Hq,
+                                   int Hkv, int K, int Tmax, int d,
+                                   float scale, asm_metric metric,
+                                   asm_dtype dt, void *out, float *lse_out,
+                                   int32_t *idx_out, unsigned flags,
+                                   cudaStream_t stream);
+
+/*
  * asm_flash_decode -- the quantity the memory stands in for: decode attention
  * over an explicit prefix shared by the whole batch followed by each row's
  * local tokens ("Fusion" bullet: the exact output as if the prefix were

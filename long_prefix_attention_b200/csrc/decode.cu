@@ -1049,3 +1049,9 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
     if (d == 128) return decode_launch_g<float, 128>(a, G, num_sms, st);
     return decode_launch_g<float, 64>(a, G, num_sms, st);
 }
+
+// Bytes at the start of a decode workspace that must be zero before a call:
+// the error word and the (b, g) arrival counters.
+size_t asm_decode_ws_header_bytes(int B, int Hkv) {
+    return align256(256 + sizeof(int) * (size_t)B * Hkv);
+}

@@ -19,6 +19,8 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
                               float *lse_out, int32_t *idx_out, unsigned flags, void *ws,
                               int num_sms, cudaStream_t st);
 
+size_t asm_decode_ws_header_bytes(int B, int Hkv);
+
 // build_states.cu
 cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v, int Hq, int Hkv,
                                     int N, int L, int d, float scale, asm_dtype dt,

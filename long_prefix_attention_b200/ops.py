@@ -169,6 +169,20 @@ def asm_decode_step(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, 
         _p(idx_out), int(flags), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def asm_decode_step_noalloc(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len,
+                            scale: float, out, lse_out=None, idx_out=None, metric: int = ASM_L2,
+                            flags: int = 0, stream=None):
+    """asm_decode_step using the library's built-in scratch (no workspace argument)."""
+    _contig(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, out, lse_out, idx_out)
+    B, Hq, d = q.shape
+    K = centroids.shape[1]
+    _, Hkv, Tmax, _ = k_cache.shape
+    _check("asm_decode_step_noalloc", _lib.load().asm_decode_step_noalloc(
+        _p(q), _p(centroids), _p(a_bar), _p(logz_bar), _p(k_cache), _p(v_cache), _p(local_len),
+        B, Hq, Hkv, K, Tmax, d, float(scale), int(metric), _dt(q), _p(out), _p(lse_out),
+        _p(idx_out), int(flags), _stream(stream)))
+
+
 def asm_flash_decode(q, k_prefix, v_prefix, k_cache, v_cache, local_len, scale: float, out, ws,
                      lse_out=None, stream=None):
     """Full attention over a shared explicit prefix plus each row's local tokens."""
