@@ -181,6 +181,20 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
 }
 
+// Hardware base-2 exponential and logarithm (approximate, flush-to-zero;
+// relative error about 2^-22): single instructions, used where code size and
+// latency matter more than the last bits (softmax weights, merge weights).
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2f(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float ld_cg(const float *p) { return __ldcg(p); }
 __device__ __forceinline__ int ld_cg(const int *p) { return __ldcg(p); }
 

@@ -98,6 +98,7 @@ struct DecodeArgs {
     int U;         // total units
     int upc;       // units per CTA
     int ccap;      // (b, g) pairs one CTA may have to merge
+    float inv_UG, inv_nS, inv_perb;  // reciprocals for the unit-index divisions
     float2 *ws_srch;  // [B][Hq][nS]   (score, idx bits)
     float2 *ws_ml;    // [B][Hq][nP+nA] (m, l), base-2 logits
     float *ws_o;      // [B][Hq][nP+nA][D] unnormalised outputs
@@ -110,6 +111,15 @@ struct DecodeArgs {
 struct DecodeMaps {
     CUtensorMap c, k, v, kp, vp;
 };
+
+// n / d for 0 <= n < 2^31 and d >= 1, from a float reciprocal and an exact fix-up.
+__device__ __forceinline__ int fdiv(int n, int d, float inv) {
+    int q = __float2int_rz((float)n * inv);
+    int r = n - q * d;
+    while (r < 0) { --q; r += d; }
+    while (r >= d) { ++q; r -= d; }
+    return q;
+}
 
 // Decoded work unit.
 struct Unit {
@@ -124,16 +134,17 @@ struct Unit {
 };
 
 template <typename T, int D, int G>
-__device__ __forceinline__ Unit decode_unit(const DecodeArgs &a, int u, const int *lens) {
+__device__ __noinline__ Unit decode_unit(const DecodeArgs &a, int u, const int *lens) {
     using C = DCfg<T, D, G>;
     Unit x;
-    x.g = u / a.UG;
+    x.g = fdiv(u, a.UG, a.inv_UG);
     int r = u - x.g * a.UG;
     x.prefix = 0;
     if (a.mode == 0 && r < G * a.nS) {
         x.kind = 0;
-        x.h = x.g * G + r / a.nS;
-        x.slot = r % a.nS;
+        const int hh = fdiv(r, a.nS, a.inv_nS);
+        x.h = x.g * G + hh;
+        x.slot = r - hh * a.nS;
         x.b = 0;
         x.first = x.slot * C::CS;
         x.valid = min(C::CS, a.K - x.first);
@@ -144,8 +155,8 @@ __device__ __forceinline__ Unit decode_unit(const DecodeArgs &a, int u, const in
     x.h = 0;
     const int per_b = a.nP + a.nA;
     const int r2 = (a.mode == 0) ? r - G * a.nS : r;
-    x.b = r2 / per_b;
-    x.slot = r2 % per_b;
+    x.b = fdiv(r2, per_b, a.inv_perb);
+    x.slot = r2 - x.b * per_b;
     x.key = a.Hq + x.b * a.Hkv + x.g;  // attention keys follow the centroid keys
     if (x.slot < a.nP) {
         x.prefix = 1;
@@ -212,57 +223,47 @@ struct SlotSeq {
     }
 };
 
-// Merge all partials of (b, g) and write the outputs (consumer warps).  All
-// partial reads of a head are issued together (one round trip), then the
-// retrieved state is gathered (a second one).
-constexpr int kCombineBatch = 16;
+// Merge all partials of (b, g) and write the outputs (consumer warps).  The
+// partial rows of a head are read in batches of 8 issued together, then the
+// retrieved state is gathered; all weights are computed in base 2.
+constexpr int kCombineBatch = 8;
 
-template <typename T, int D, int G>
-__device__ void combine(const DecodeArgs &a, int b, int g, int warp, int lane) {
+template <typename T, int D, int G, int NW = kDecodeConsumerWarps>
+__device__ __noinline__ void combine(const DecodeArgs &a, int b, int g, int warp, int lane) {
     using C = DCfg<T, D, G>;
     const int nslots = a.nP + a.nA;
-    for (int hh = warp; hh < G; hh += kDecodeConsumerWarps) {
+#pragma unroll 1
+    for (int hh = warp; hh < G; hh += NW) {
         const int h = g * G + hh;
         const size_t bh = (size_t)b * a.Hq + h;
         const SlotSeq as(g * a.UG + (a.mode == 0 ? G * a.nS : 0) + b * nslots, nslots, a.upc);
-        // ---- round 1: scan partials, (m, l) and the first output rows
-        float bs = kNegInf;
-        int bi = 0x7fffffff;
+        // retrieval: arg-max over the scan partials of head h
+        int idx = 0;
         if (a.mode == 0) {
             const SlotSeq ss(g * a.UG + hh * a.nS, a.nS, a.upc);
+            float bs = kNegInf;
+            int bi = 0x7fffffff;
+#pragma unroll 1
             for (int j = lane; j < ss.count; j += 32) {
                 const float2 v = __ldcg(a.ws_srch + bh * a.nS + ss(j));
                 const int vi = __float_as_int(v.y);
                 if (better(v.x, vi, bs, bi)) { bs = v.x; bi = vi; }
             }
-        }
-        float2 ml = make_float2(kNegInf, 0.f);
-        if (lane < as.count) ml = __ldcg(a.ws_ml + bh * nslots + as(lane));
-        float ov[kCombineBatch][C::EPL];
-#pragma unroll
-        for (int k = 0; k < kCombineBatch; ++k) {
-            const bool use = k < as.count;
-            const float *os = a.ws_o + (bh * nslots + as(use ? k : 0)) * D + lane * C::EPL;
-#pragma unroll
-            for (int e = 0; e < C::EPL; ++e) ov[k][e] = use ? __ldcg(os + e) : 0.f;
-        }
-        int idx = 0;
-        if (a.mode == 0) {
             warp_argmax(bs, bi);
             idx = (bi == 0x7fffffff) ? 0 : bi;
         }
-        // ---- round 2: the retrieved state
         float ab[C::EPL];
-        float zb = kNegInf;
+        float zb2 = kNegInf;  // retrieved log Z in base 2
         if (a.mode == 0) {
-            zb = __ldg(a.logz_bar + (size_t)h * a.K + idx);
+            zb2 = __ldg(a.logz_bar + (size_t)h * a.K + idx) * kLog2e;
             load_vec<T, C::EPL>((const T *)a.a_bar + ((size_t)h * a.K + idx) * D + lane * C::EPL, ab);
         }
-        // log-sum-exp of the attention partials (slots beyond 32 in later rounds)
-        float M = (ml.y > 0.f) ? ml.x : kNegInf;
-        for (int j = lane + 32; j < as.count; j += 32) {
-            const float2 m2 = __ldcg(a.ws_ml + bh * nslots + as(j));
-            if (m2.y > 0.f) M = fmaxf(M, m2.x);
+        // log-sum-exp of the attention partials (base 2)
+        float M = kNegInf;
+#pragma unroll 1
+        for (int j = lane; j < as.count; j += 32) {
+            const float2 ml = __ldcg(a.ws_ml + bh * nslots + as(j));
+            if (ml.y > 0.f) M = fmaxf(M, ml.x);
         }
         M = warp_max(M);
         float L = 0.f;
@@ -270,49 +271,57 @@ __device__ void combine(const DecodeArgs &a, int b, int g, int warp, int lane) {
 #pragma unroll
         for (int e = 0; e < C::EPL; ++e) o[e] = 0.f;
         if (M != kNegInf) {
-            const float w = (ml.y > 0.f) ? exp2f(ml.x - M) : 0.f;
-            L = warp_sum(ml.y * w);
+#pragma unroll 1
+            for (int j0 = 0; j0 < as.count; j0 += kCombineBatch) {
+                // lanes 0..7 hold the batch's weights, every lane its dims of each row
+                float w = 0.f;
+                if (lane < kCombineBatch && j0 + lane < as.count) {
+                    const float2 ml = __ldcg(a.ws_ml + bh * nslots + as(j0 + lane));
+                    if (ml.y > 0.f) {
+                        w = ex2f(ml.x - M);
+                        L += ml.y * w;
+                    }
+                }
+                float v[kCombineBatch][C::EPL];
 #pragma unroll
-            for (int k = 0; k < kCombineBatch; ++k) {
-                const float wk = __shfl_sync(0xffffffffu, w, k);
+                for (int k = 0; k < kCombineBatch; ++k) {
+                    const bool use = j0 + k < as.count;
+                    const float *os = a.ws_o + (bh * nslots + as(use ? j0 + k : 0)) * D + lane * C::EPL;
 #pragma unroll
-                for (int e = 0; e < C::EPL; ++e) o[e] = fmaf(wk, ov[k][e], o[e]);
+                    for (int e = 0; e < C::EPL; ++e) v[k][e] = use ? __ldcg(os + e) : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < kCombineBatch; ++k) {
+                    const float wk = __shfl_sync(0xffffffffu, w, k);
+#pragma unroll
+                    for (int e = 0; e < C::EPL; ++e) o[e] = fmaf(wk, v[k][e], o[e]);
+                }
             }
-            for (int j = kCombineBatch; j < as.count; ++j) {  // rare: more than 16 partials
-                const float2 m2 = __ldcg(a.ws_ml + bh * nslots + as(j));
-                if (!(m2.y > 0.f)) continue;
-                const float wj = exp2f(m2.x - M);
-                if (j >= 32) L += m2.y * wj;
-                const float *os = a.ws_o + (bh * nslots + as(j)) * D + lane * C::EPL;
-#pragma unroll
-                for (int e = 0; e < C::EPL; ++e) o[e] = fmaf(wj, __ldcg(os + e), o[e]);
-            }
+            L = warp_sum(L);
         }
-        const float zl = (L > 0.f) ? (M + log2f(L)) * kLn2 : kNegInf;  // natural log
-        float res[C::EPL];
-        float lse;
+        const float zl2 = (L > 0.f) ? M + lg2f(L) : kNegInf;
         const float invL = (L > 0.f) ? 1.f / L : 0.f;
-        if (a.mode == 0) {
-            if (zb == kNegInf && zl == kNegInf) {
-                lse = kNegInf;
+        float res[C::EPL];
+        float lse2;
+        if (a.mode == 0 && !(zb2 == kNegInf && zl2 == kNegInf)) {
+            const float m = fmaxf(zb2, zl2);
+            const float eb = ex2f(zb2 - m), el = ex2f(zl2 - m);
+            lse2 = m + lg2f(eb + el);
+            const float inv = 1.f / (eb + el);
 #pragma unroll
-                for (int e = 0; e < C::EPL; ++e) res[e] = 0.f;
-            } else {
-                const float m = fmaxf(zb, zl);
-                const float eb = expf(zb - m), el = expf(zl - m);
-                lse = m + logf(eb + el);
-                const float wb = eb / (eb + el), wl = el / (eb + el);
+            for (int e = 0; e < C::EPL; ++e) res[e] = (eb * ab[e] + el * (o[e] * invL)) * inv;
+        } else if (a.mode == 0) {
+            lse2 = kNegInf;
 #pragma unroll
-                for (int e = 0; e < C::EPL; ++e) res[e] = wb * ab[e] + wl * (o[e] * invL);
-            }
+            for (int e = 0; e < C::EPL; ++e) res[e] = 0.f;
         } else {
-            lse = zl;
+            lse2 = zl2;
 #pragma unroll
             for (int e = 0; e < C::EPL; ++e) res[e] = o[e] * invL;
         }
         store_vec<T, C::EPL>((T *)a.out + bh * D + lane * C::EPL, res);
         if (lane == 0) {
-            if (a.lse_out) a.lse_out[bh] = lse;
+            if (a.lse_out) a.lse_out[bh] = lse2 * kLn2;
             if (a.idx_out && a.mode == 0) a.idx_out[bh] = idx;
         }
     }
@@ -935,6 +944,9 @@ static void decode_geometry(DecodeArgs &a, int workers) {
     // KV groups one CTA range can touch, times the rows of each
     const int groups = min(a.Hkv, (a.upc + a.UG - 1) / a.UG + 1);
     a.ccap = a.B * groups;
+    a.inv_UG = 1.f / (float)a.UG;
+    a.inv_nS = a.nS > 0 ? 1.f / (float)a.nS : 0.f;
+    a.inv_perb = (a.nP + a.nA) > 0 ? 1.f / (float)(a.nP + a.nA) : 0.f;
 }
 
 template <typename T, int D, int G>
@@ -957,6 +969,15 @@ static cudaError_t decode_launch_t(DecodeArgs a, int num_sms, cudaStream_t st) {
         }
     }
     const int grid = (a.U + a.upc - 1) / a.upc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    {
     const size_t smem = 1024 + (size_t)kDecodeStages * kUnitBytes + 2 * kDecodeStages * sizeof(uint64_t) +
                         sizeof(float) * kDecodeConsumerWarps * G * (D + 2) +
                         sizeof(float2) * kDecodeConsumerWarps * a.B + sizeof(int) * ((2 * a.ccap + 4) & ~3) +
@@ -968,17 +989,10 @@ static cudaError_t decode_launch_t(DecodeArgs a, int num_sms, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr_smem = smem;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kDecodeThreads);
     cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, a, maps);
+    }
 }
 
 template <typename T, int D>
@@ -1018,6 +1032,7 @@ DecodeWs decode_ws_layout(int mode, int B, int Hq, int Hkv, int K, int Lp, int T
 }  // namespace
 
 size_t asm_decode_ws_bytes(int mode, int B, int Hq, int Hkv, int K, int Lp, int Tmax, int d, asm_dtype dt) {
+    if (dt == ASM_BF16) return asm_decode_tc_ws_bytes(mode, B, Hq, K, Lp, Tmax, d);
     return decode_ws_layout(mode, B, Hq, Hkv, K, Lp, Tmax, d, dt).total;
 }
 
@@ -1042,10 +1057,10 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
     a.ws_ml = reinterpret_cast<float2 *>(base + w.off_ml);
     a.ws_o = reinterpret_cast<float *>(base + w.off_o);
     const int G = Hq / Hkv;
-    if (dt == ASM_BF16) {
-        if (d == 128) return decode_launch_g<__nv_bfloat16, 128>(a, G, num_sms, st);
-        return decode_launch_g<__nv_bfloat16, 64>(a, G, num_sms, st);
-    }
+    if (dt == ASM_BF16)
+        return asm_decode_tc_launch(mode, q, centroids, a_bar, logz_bar, k_prefix, v_prefix, Lp, k_cache, v_cache,
+                                    local_len, B, Hq, Hkv, K, Tmax, d, scale, metric, out, lse_out, idx_out, flags,
+                                    ws, st);
     if (d == 128) return decode_launch_g<float, 128>(a, G, num_sms, st);
     return decode_launch_g<float, 64>(a, G, num_sms, st);
 }

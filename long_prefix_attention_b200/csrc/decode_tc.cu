@@ -1,0 +1,603 @@
+// decode_tc.cu -- bf16 decode step on tensor cores: split units, then merge.
+//
+// "Context Memorization for Efficient Long Context Generation", Metodologia,
+// "Fase de Inferencia Online": every query head retrieves its nearest memory
+// centroid (Recuperacion) and merges that centroid's stored prefix state with
+// its attention over the non-prefix tokens by the online-softmax merge
+// (Fusion).
+//
+// Kernel 1 (asm_decode_units) streams the bytes of the step in 32 KB units,
+// one unit per CTA: 128 (d=128) or 256 (d=64) centroid rows of one head, or
+// 64 / 128 tokens of K and V for one (row b, KV head g).  The unit arrives
+// by TMA (128-byte swizzled boxes) while the warps fetch their query
+// fragments; four warps then contract it on tensor cores with the streamed
+// operand on the 16-row M side ("swapped" tiles, nothing wasted at batch 1):
+//   centroids  D[c, b] = C[c, :] q[b, :]   and |c|^2 = diag(C C^T) from the same fragments
+//   attention  S^T[t, h] = K[t, :] q[h, :],   O^T[d, h] = V^T[d, t] P^T[t, h]
+// and write one partial per unit: the best (score, index) per row b, or the
+// unnormalised (m, l, o) per head.  Centroid units come first in the grid;
+// with ASM_DECODE_PREFETCH_CENTROIDS they start their loads before the
+// programmatic-dependent-launch wait.
+//
+// Kernel 2 (asm_decode_merge), one CTA per (b, h), reads every partial of the
+// pair in one round (arg-max of the scores, log-sum-exp of the attention
+// partials), gathers (a_bar, logZ_bar)[idx] in a second round and writes the
+// merged state.  Both kernels use programmatic dependent launch, so the merge
+// of one call and the centroid loads of the next overlap the tail of the
+// previous kernel.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace asmk {
+namespace tc {
+
+constexpr int kUnit = 32768;     // bytes per unit
+constexpr int kWarps = 4;        // compute warps per unit CTA
+constexpr int kThreads = kWarps * 32;
+
+template <int D>
+struct Geo {
+    static constexpr int ROWB = 2 * D;             // bytes per bf16 row
+    static constexpr int CS = kUnit / ROWB;        // centroid rows per unit
+    static constexpr int TS = kUnit / (2 * ROWB);  // tokens per unit
+    static constexpr int HALVES = D / 64;          // 128-byte column halves
+    static constexpr int KS = D / 16;              // k-steps over the head dim
+    static constexpr int RMT = CS / kWarps / 16;   // 16-row centroid tiles per warp
+    static constexpr int TMT = TS / kWarps / 16;   // 16-token tiles per warp
+};
+
+struct Args {
+    const __nv_bfloat16 *q;       // [B][Hq][D]
+    const __nv_bfloat16 *a_bar;   // [Hq][K][D]
+    const float *logz_bar;        // [Hq][K]
+    const int *local_len;         // [B]
+    __nv_bfloat16 *out;           // [B][Hq][D]
+    float *lse_out;               // [B][Hq] or null
+    int *idx_out;                 // [B][Hq] or null
+    int B, Hq, Hkv, K, Tmax, Lp;
+    float qscale;                 // softmax scale * log2(e)
+    int metric, mode, flags;
+    int nS;                       // centroid units per head (mode 0)
+    int nP, nA;                   // prefix / local units per (b, g)
+    int n_scan;                   // Hq * nS
+    float2 *ws_srch;              // [B][Hq][nS]
+    float2 *ws_ml;                // [B][Hq][nP+nA]
+    float *ws_o;                  // [B][Hq][nP+nA][D]
+    int *ws_err;
+};
+
+struct Maps {
+    CUtensorMap c, k, v, kp, vp;
+};
+
+__device__ __forceinline__ void set_error(int *err) { atomicExch(err, (int)ASM_ERR_TIMEOUT); }
+
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// ------------------------------------------------------------ unit kernel --
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads)
+asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
+    using Gm = Geo<D>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *tile = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(tile + kUnit);
+    float *wo = reinterpret_cast<float *>(bar + 2);       // [W][G][D]
+    float *wm = wo + kWarps * G * D;                      // [W][G]
+    float *wl = wm + kWarps * G;                          // [W][G]
+    float2 *wb = reinterpret_cast<float2 *>(wl + kWarps * G);  // [W][B]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, quad = lane & 3, i4 = lane >> 3;
+    const uint32_t sbuf = smem_addr(tile);
+
+    // ---- which unit
+    const int u = blockIdx.x;
+    const bool scan = u < a.n_scan;
+    int h = 0, b = 0, g = 0, slot, first, valid;
+    bool prefix = false;
+    if (scan) {
+        h = u / a.nS;
+        slot = u - h * a.nS;
+        first = slot * Gm::CS;
+        valid = min(Gm::CS, a.K - first);
+        g = h / G;
+    } else {
+        const int v = u - a.n_scan, ns = a.nP + a.nA;
+        const int bg = v / ns;
+        slot = v - bg * ns;
+        b = bg / a.Hkv;
+        g = bg - b * a.Hkv;
+        prefix = slot < a.nP;
+        first = (prefix ? slot : slot - a.nP) * Gm::TS;
+        valid = prefix ? min(Gm::TS, a.Lp - first) : Gm::TS;  // refined by the row length below
+    }
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int vrows) {
+        if (scan) {
+            mbar_arrive_expect_tx(bar, Gm::CS * Gm::ROWB);
+#pragma unroll
+            for (int hf = 0; hf < Gm::HALVES; ++hf)
+                tma_load_3d(tile + hf * Gm::CS * 128, &maps.c, 64 * hf, first, h, bar);
+        } else if (vrows > 0) {
+            mbar_arrive_expect_tx(bar, 2 * Gm::TS * Gm::ROWB);
+            const CUtensorMap *mk = prefix ? &maps.kp : &maps.k;
+            const CUtensorMap *mv = prefix ? &maps.vp : &maps.v;
+            const int c2 = prefix ? g : b * a.Hkv + g;
+#pragma unroll
+            for (int hf = 0; hf < Gm::HALVES; ++hf) {
+                tma_load_3d(tile + hf * Gm::TS * 128, mk, 64 * hf, first, c2, bar);
+                tma_load_3d(tile + kUnit / 2 + hf * Gm::TS * 128, mv, 64 * hf, first, c2, bar);
+            }
+        } else {
+            mbar_arrive(bar);
+        }
+    };
+    // static centroids may stream before the dependency wait (caller's choice)
+    const bool early = scan && (a.flags & 1);
+    if (early && tid == 0) issue(valid);
+    pdl_wait();
+    pdl_launch_dependents();
+    if (!scan && !prefix) valid = min(Gm::TS, min(max(__ldg(a.local_len + b), 0), a.Tmax) - first);
+    if (!early && tid == 0) issue(valid);
+
+    if (scan) {
+        // ------------------------------------------- centroid unit
+        constexpr int KS = Gm::KS, RMT = Gm::RMT;
+        float nrl[RMT], nrh[RMT];
+        const int src = 4 * gid + (gid >> 1);  // lane holding the diagonal entry of row gid
+#pragma unroll 1
+        for (int nt = 0; nt * 8 < a.B; ++nt) {
+            const int bq = 8 * nt + gid;
+            const uint32_t *qr = reinterpret_cast<const uint32_t *>(
+                a.q + ((size_t)min(bq, a.B - 1) * a.Hq + h) * D);
+            uint32_t qb0[KS], qb1[KS];
+#pragma unroll
+            for (int j = 0; j < KS; ++j) {
+                qb0[j] = bq < a.B ? __ldg(qr + 8 * j + quad) : 0u;
+                qb1[j] = bq < a.B ? __ldg(qr + 8 * j + 4 + quad) : 0u;
+            }
+            if (nt == 0 && !mbar_wait(bar, 0)) set_error(a.ws_err);
+            float bs[2] = {kNegInf, kNegInf};
+            int bi[2] = {0x7fffffff, 0x7fffffff};
+#pragma unroll
+            for (int mt = 0; mt < RMT; ++mt) {
+                const int r0 = (warp * RMT + mt) * 16;
+                const int row = r0 + 8 * (i4 & 1) + (lane & 7);
+                float dd[4] = {0.f, 0.f, 0.f, 0.f};
+                float dn0[4] = {0.f, 0.f, 0.f, 0.f}, dn1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < KS; ++j) {
+                    const int col = 16 * j + 8 * (i4 >> 1);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(sbuf + (col >> 6) * (Gm::CS * 128) + swz128(row, (col & 63) >> 3), a0, a1, a2, a3);
+                    mma_bf16_16816(dd, a0, a1, a2, a3, qb0[j], qb1[j]);
+                    if (nt == 0) {
+                        // the same fragments as B operands give C C^T (rows 0-7 / 8-15)
+                        mma_bf16_16816(dn0, a0, a1, a2, a3, a0, a2);
+                        mma_bf16_16816(dn1, a0, a1, a2, a3, a1, a3);
+                    }
+                }
+                if (nt == 0) {
+                    nrl[mt] = __shfl_sync(0xffffffffu, dn0[gid & 1], src);
+                    nrh[mt] = __shfl_sync(0xffffffffu, dn1[2 + (gid & 1)], src);
+                }
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int rloc = r0 + gid + 8 * hr;
+                    const float nr = hr ? nrh[mt] : nrl[mt];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float dot = dd[2 * hr + e];
+                        float sc = (a.metric == 0) ? dot - 0.5f * nr : (nr > 0.f ? dot / sqrtf(nr) : 0.f);
+                        int ci = first + rloc;
+                        if (rloc >= valid) { sc = kNegInf; ci = 0x7fffffff; }
+                        if (better(sc, ci, bs[e], bi[e])) { bs[e] = sc; bi[e] = ci; }
+                    }
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+#pragma unroll
+                for (int m = 4; m <= 16; m <<= 1) {
+                    const float os = __shfl_xor_sync(0xffffffffu, bs[e], m);
+                    const int oi = __shfl_xor_sync(0xffffffffu, bi[e], m);
+                    if (better(os, oi, bs[e], bi[e])) { bs[e] = os; bi[e] = oi; }
+                }
+                const int bb = 8 * nt + 2 * quad + e;
+                if (gid == 0 && bb < a.B) wb[warp * a.B + bb] = make_float2(bs[e], __int_as_float(bi[e]));
+            }
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int bb = tid; bb < a.B; bb += kThreads) {
+            float bs = kNegInf;
+            int bi = 0x7fffffff;
+            for (int w = 0; w < kWarps; ++w) {
+                const float2 v = wb[w * a.B + bb];
+                if (better(v.x, __float_as_int(v.y), bs, bi)) { bs = v.x; bi = __float_as_int(v.y); }
+            }
+            a.ws_srch[((size_t)bb * a.Hq + h) * a.nS + slot] = make_float2(bs, __int_as_float(bi));
+        }
+        return;
+    }
+
+    // ------------------------------------------------ attention unit
+    constexpr int KS = Gm::KS, TMT = Gm::TMT, NMD = D / 16;
+    const int nslots = a.nP + a.nA;
+    float *so = wo + warp * G * D;
+    if (valid <= 0) {
+        // nothing to attend in this unit: an empty partial
+        for (int i = tid; i < G * D; i += kThreads) {
+            const int hh = i / D, dd = i - hh * D;
+            const size_t bh = (size_t)b * a.Hq + g * G + hh;
+            a.ws_o[(bh * nslots + slot) * D + dd] = 0.f;
+            if (dd == 0) a.ws_ml[bh * nslots + slot] = make_float2(kNegInf, 0.f);
+        }
+        return;
+    }
+    // B fragments of Q^T: n = head gid of the group (heads >= G are zero)
+    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(a.q + ((size_t)b * a.Hq + g * G + min(gid, G - 1)) * D);
+    uint32_t qb0[KS], qb1[KS];
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+        qb0[j] = gid < G ? __ldg(qrow + 8 * j + quad) : 0u;
+        qb1[j] = gid < G ? __ldg(qrow + 8 * j + 4 + quad) : 0u;
+    }
+    if (!mbar_wait(bar, 0)) set_error(a.ws_err);
+    const int t0 = warp * TMT * 16;  // first token of this warp
+    float sf[TMT][4];
+#pragma unroll
+    for (int mt = 0; mt < TMT; ++mt) {
+        sf[mt][0] = sf[mt][1] = sf[mt][2] = sf[mt][3] = 0.f;
+        const int row = t0 + 16 * mt + 8 * (i4 & 1) + (lane & 7);
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+            const int col = 16 * j + 8 * (i4 >> 1);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(sbuf + (col >> 6) * (Gm::TS * 128) + swz128(row, (col & 63) >> 3), a0, a1, a2, a3);
+            mma_bf16_16816(sf[mt], a0, a1, a2, a3, qb0[j], qb1[j]);
+        }
+    }
+    // base-2 softmax statistics per head (2quad + e) over this warp's tokens
+    float mx[2] = {kNegInf, kNegInf};
+#pragma unroll
+    for (int mt = 0; mt < TMT; ++mt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int tok = t0 + 16 * mt + gid + 8 * (k >> 1);
+            const float v = tok < valid ? sf[mt][k] * a.qscale : kNegInf;
+            sf[mt][k] = v;
+            mx[k & 1] = fmaxf(mx[k & 1], v);
+        }
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int m = 4; m <= 16; m <<= 1) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], m));
+    float ls[2] = {0.f, 0.f};
+#pragma unroll
+    for (int mt = 0; mt < TMT; ++mt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float v = sf[mt][k];
+            const float p = (v == kNegInf) ? 0.f : ex2f(v - mx[k & 1]);
+            sf[mt][k] = p;
+            ls[k & 1] += p;
+        }
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int m = 4; m <= 16; m <<= 1) ls[e] += __shfl_xor_sync(0xffffffffu, ls[e], m);
+    // P^T as B fragments (movmatrix turns (token, head) pairs into (head, token))
+    uint32_t pb0[TMT], pb1[TMT];
+#pragma unroll
+    for (int kk = 0; kk < TMT; ++kk) {
+        pb0[kk] = movm_t(pack_bf16(sf[kk][0], sf[kk][1]));
+        pb1[kk] = movm_t(pack_bf16(sf[kk][2], sf[kk][3]));
+    }
+    const uint32_t vbase = sbuf + kUnit / 2;
+#pragma unroll
+    for (int md = 0; md < NMD; ++md) {
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
+        const int col = 16 * md + 8 * (i4 & 1);
+#pragma unroll
+        for (int kk = 0; kk < TMT; ++kk) {
+            const int row = t0 + 16 * kk + 8 * (i4 >> 1) + (lane & 7);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vbase + (col >> 6) * (Gm::TS * 128) + swz128(row, (col & 63) >> 3), a0, a1, a2, a3);
+            mma_bf16_16816(o, a0, a1, a2, a3, pb0[kk], pb1[kk]);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int hh = 2 * quad + e;
+            if (hh < G) {
+                so[hh * D + 16 * md + gid] = o[e];
+                so[hh * D + 16 * md + gid + 8] = o[2 + e];
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int hh = 2 * quad + e;
+        if (gid == 0 && hh < G) {
+            wm[warp * G + hh] = mx[e];
+            wl[warp * G + hh] = ls[e];
+        }
+    }
+    __syncthreads();
+    // fold the four warps' states into the unit's partial
+#pragma unroll 1
+    for (int i = tid; i < G * D; i += kThreads) {
+        const int hh = i / D, dd = i - hh * D;
+        float M = kNegInf;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            if (wl[w * G + hh] > 0.f) M = fmaxf(M, wm[w * G + hh]);
+        float L = 0.f, o = 0.f;
+        if (M != kNegInf) {
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                if (!(wl[w * G + hh] > 0.f)) continue;
+                const float sc = ex2f(wm[w * G + hh] - M);
+                L += wl[w * G + hh] * sc;
+                o += wo[(w * G + hh) * D + dd] * sc;
+            }
+        }
+        const size_t bh = (size_t)b * a.Hq + g * G + hh;
+        a.ws_o[(bh * nslots + slot) * D + dd] = o;
+        if (dd == 0) a.ws_ml[bh * nslots + slot] = make_float2(M, L);
+    }
+}
+
+// ----------------------------------------------------------- merge kernel --
+//
+// One CTA of D threads per (b, h); thread t owns output dim t.
+
+constexpr int kMergeSlots = 32;  // partial rows a thread keeps in flight
+
+template <int D>
+__global__ void __launch_bounds__(D)
+asm_decode_merge(const Args a) {
+    const int bh = blockIdx.x;
+    const int b = bh / a.Hq, h = bh - b * a.Hq;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = D / 32;
+    __shared__ float red_m[NW];
+    __shared__ int sidx;
+    __shared__ float2 sb[NW];
+    __shared__ float2 sml[kMergeSlots];
+    const int nslots = a.nP + a.nA;
+    pdl_wait();
+    pdl_launch_dependents();
+    // ---- round 1: every partial of (b, h)
+    float2 best = make_float2(kNegInf, __int_as_float(0x7fffffff));
+    if (a.mode == 0) {
+        for (int s = tid; s < a.nS; s += D) {
+            const float2 v = __ldcg(a.ws_srch + (size_t)bh * a.nS + s);
+            if (better(v.x, __float_as_int(v.y), best.x, __float_as_int(best.y))) best = v;
+        }
+    }
+    const float2 *mlp = a.ws_ml + (size_t)bh * nslots;
+    const float *op = a.ws_o + (size_t)bh * nslots * D + tid;
+    float ov[kMergeSlots];
+#pragma unroll
+    for (int s = 0; s < kMergeSlots; ++s) ov[s] = s < nslots ? __ldcg(op + (size_t)s * D) : 0.f;
+    float mloc = kNegInf;
+    for (int s = tid; s < nslots; s += D) {
+        const float2 ml = __ldcg(mlp + s);
+        if (s < kMergeSlots) sml[s] = ml;
+        if (ml.y > 0.f) mloc = fmaxf(mloc, ml.x);
+    }
+    // block reductions: arg-max of the scores, max of the attention partials
+    {
+        float bs = best.x;
+        int bi = __float_as_int(best.y);
+        warp_argmax(bs, bi);
+        mloc = warp_max(mloc);
+        if (lane == 0) {
+            sb[warp] = make_float2(bs, __int_as_float(bi));
+            red_m[warp] = mloc;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float s0 = kNegInf;
+            int i0 = 0x7fffffff;
+            float m0 = kNegInf;
+            for (int w = 0; w < NW; ++w) {
+                if (better(sb[w].x, __float_as_int(sb[w].y), s0, i0)) { s0 = sb[w].x; i0 = __float_as_int(sb[w].y); }
+                m0 = fmaxf(m0, red_m[w]);
+            }
+            sidx = (i0 == 0x7fffffff) ? 0 : i0;
+            red_m[0] = m0;
+        }
+        __syncthreads();
+    }
+    const int idx = sidx;
+    const float M = red_m[0];
+    // ---- round 2: the retrieved state (issued before the weighted sums)
+    float zb2 = kNegInf, ab = 0.f;
+    if (a.mode == 0) {
+        zb2 = __ldg(a.logz_bar + (size_t)h * a.K + idx) * kLog2e;
+        ab = __bfloat162float(a.a_bar[((size_t)h * a.K + idx) * D + tid]);
+    }
+    float L = 0.f, o = 0.f;
+    if (M != kNegInf) {
+#pragma unroll
+        for (int s = 0; s < kMergeSlots; ++s) {
+            if (s >= nslots) break;
+            const float2 ml = sml[s];
+            if (ml.y > 0.f) {
+                const float w = ex2f(ml.x - M);
+                L += ml.y * w;
+                o = fmaf(w, ov[s], o);
+            }
+        }
+        for (int s = kMergeSlots; s < nslots; ++s) {  // more than 32 partials
+            const float2 ml = __ldcg(mlp + s);
+            if (ml.y > 0.f) {
+                const float w = ex2f(ml.x - M);
+                L += ml.y * w;
+                o = fmaf(w, __ldcg(op + (size_t)s * D), o);
+            }
+        }
+    }
+    const float zl2 = (L > 0.f) ? M + lg2f(L) : kNegInf;
+    const float loc = (L > 0.f) ? o / L : 0.f;
+    float res, lse2;
+    if (a.mode == 0 && !(zb2 == kNegInf && zl2 == kNegInf)) {
+        const float m = fmaxf(zb2, zl2);
+        const float eb = ex2f(zb2 - m), el = ex2f(zl2 - m);
+        lse2 = m + lg2f(eb + el);
+        res = (eb * ab + el * loc) / (eb + el);
+    } else if (a.mode == 0) {
+        lse2 = kNegInf;
+        res = 0.f;
+    } else {
+        lse2 = zl2;
+        res = loc;
+    }
+    a.out[(size_t)bh * D + tid] = __float2bfloat16_rn(res);
+    if (tid == 0) {
+        if (a.lse_out) a.lse_out[bh] = lse2 * kLn2;
+        if (a.idx_out && a.mode == 0) a.idx_out[bh] = idx;
+    }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------- host side --
+
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows);
+
+namespace {
+struct TcWs {
+    size_t off_srch, off_ml, off_o, total;
+};
+inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+TcWs tc_ws_layout(int mode, int B, int Hq, int K, int Lp, int Tmax, int d) {
+    const int CS = tc::kUnit / (2 * d), TS = tc::kUnit / (4 * d);
+    const size_t nS = mode == 0 ? (size_t)(K + CS - 1) / CS : 0;
+    const size_t nP = mode == 1 ? (size_t)(Lp + TS - 1) / TS : 0;
+    const size_t nA = (size_t)(Tmax + TS - 1) / TS;
+    TcWs w;
+    w.off_srch = 256;  // word 0: device-side error code
+    w.off_ml = al256(w.off_srch + sizeof(float2) * (size_t)B * Hq * nS);
+    w.off_o = al256(w.off_ml + sizeof(float2) * (size_t)B * Hq * (nP + nA));
+    w.total = al256(w.off_o + sizeof(float) * (size_t)B * Hq * (nP + nA) * d);
+    return w;
+}
+
+template <int D, int G>
+cudaError_t tc_launch(tc::Args a, const void *centroids, const void *k_prefix, const void *v_prefix,
+                      const void *k_cache, const void *v_cache, cudaStream_t st) {
+    using Gm = tc::Geo<D>;
+    tc::Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (a.mode == 0 && !make_map_3d(&maps.c, centroids, D, a.K, a.Hq, Gm::CS)) return cudaErrorInvalidValue;
+    if (a.Tmax > 0 && (!make_map_3d(&maps.k, k_cache, D, a.Tmax, (uint64_t)a.B * a.Hkv, Gm::TS) ||
+                       !make_map_3d(&maps.v, v_cache, D, a.Tmax, (uint64_t)a.B * a.Hkv, Gm::TS)))
+        return cudaErrorInvalidValue;
+    if (a.mode == 1 && a.Lp > 0 && (!make_map_3d(&maps.kp, k_prefix, D, a.Lp, a.Hkv, Gm::TS) ||
+                                    !make_map_3d(&maps.vp, v_prefix, D, a.Lp, a.Hkv, Gm::TS)))
+        return cudaErrorInvalidValue;
+    const int units = a.n_scan + a.B * a.Hkv * (a.nP + a.nA);
+    const size_t smem = 1024 + tc::kUnit + 16 + sizeof(float) * tc::kWarps * G * (D + 2) +
+                        sizeof(float2) * tc::kWarps * a.B;
+    auto k1 = tc::asm_decode_units<D, G>;
+    static size_t k1_smem = 0;
+    if (smem > k1_smem) {
+        cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k1_smem = smem;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c1 = {};
+    c1.gridDim = dim3(units);
+    c1.blockDim = dim3(tc::kThreads);
+    c1.dynamicSmemBytes = smem;
+    c1.stream = st;
+    c1.attrs = attr;
+    c1.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&c1, k1, a, maps);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t c2 = {};
+    c2.gridDim = dim3(a.B * a.Hq);
+    c2.blockDim = dim3(D);
+    c2.stream = st;
+    c2.attrs = attr;
+    c2.numAttrs = 1;
+    return cudaLaunchKernelEx(&c2, tc::asm_decode_merge<D>, a);
+}
+
+template <int D>
+cudaError_t tc_launch_g(int G, const tc::Args &a, const void *c, const void *kp, const void *vp, const void *kc,
+                        const void *vc, cudaStream_t st) {
+    switch (G) {
+        case 1: return tc_launch<D, 1>(a, c, kp, vp, kc, vc, st);
+        case 2: return tc_launch<D, 2>(a, c, kp, vp, kc, vc, st);
+        case 4: return tc_launch<D, 4>(a, c, kp, vp, kc, vc, st);
+        case 8: return tc_launch<D, 8>(a, c, kp, vp, kc, vc, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+}  // namespace
+
+}  // namespace asmk
+
+size_t asm_decode_tc_ws_bytes(int mode, int B, int Hq, int K, int Lp, int Tmax, int d) {
+    return asmk::tc_ws_layout(mode, B, Hq, K, Lp, Tmax, d).total;
+}
+
+cudaError_t asm_decode_tc_launch(int mode, const void *q, const void *centroids, const void *a_bar,
+                                 const float *logz_bar, const void *k_prefix, const void *v_prefix, int Lp,
+                                 const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
+                                 int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, void *out,
+                                 float *lse_out, int32_t *idx_out, unsigned flags, void *ws, cudaStream_t st) {
+    using namespace asmk;
+    const TcWs w = tc_ws_layout(mode, B, Hq, K, Lp, Tmax, d);
+    tc::Args a{};
+    a.q = (const __nv_bfloat16 *)q;
+    a.a_bar = (const __nv_bfloat16 *)a_bar;
+    a.logz_bar = logz_bar;
+    a.local_len = local_len;
+    a.out = (__nv_bfloat16 *)out;
+    a.lse_out = lse_out;
+    a.idx_out = idx_out;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.K = K; a.Tmax = Tmax; a.Lp = Lp;
+    a.qscale = scale * kLog2e;
+    a.metric = metric;
+    a.mode = mode;
+    a.flags = (int)flags;
+    const int CS = tc::kUnit / (2 * d), TS = tc::kUnit / (4 * d);
+    a.nS = mode == 0 ? (K + CS - 1) / CS : 0;
+    a.nP = mode == 1 ? (Lp + TS - 1) / TS : 0;
+    a.nA = (Tmax + TS - 1) / TS;
+    a.n_scan = Hq * a.nS;
+    char *base = static_cast<char *>(ws);
+    a.ws_err = reinterpret_cast<int *>(base);
+    a.ws_srch = reinterpret_cast<float2 *>(base + w.off_srch);
+    a.ws_ml = reinterpret_cast<float2 *>(base + w.off_ml);
+    a.ws_o = reinterpret_cast<float *>(base + w.off_o);
+    const int G = Hq / Hkv;
+    if (d == 128) return tc_launch_g<128>(G, a, centroids, k_prefix, v_prefix, k_cache, v_cache, st);
+    return tc_launch_g<64>(G, a, centroids, k_prefix, v_prefix, k_cache, v_cache, st);
+}

@@ -21,6 +21,14 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
 
 size_t asm_decode_ws_header_bytes(int B, int Hkv);
 
+// decode_tc.cu: the bf16 path (split units on tensor cores, then a merge kernel)
+size_t asm_decode_tc_ws_bytes(int mode, int B, int Hq, int K, int Lp, int Tmax, int d);
+cudaError_t asm_decode_tc_launch(int mode, const void *q, const void *centroids, const void *a_bar,
+                                 const float *logz_bar, const void *k_prefix, const void *v_prefix, int Lp,
+                                 const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
+                                 int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, void *out,
+                                 float *lse_out, int32_t *idx_out, unsigned flags, void *ws, cudaStream_t st);
+
 // build_states.cu
 cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v, int Hq, int Hkv,
                                     int N, int L, int d, float scale, asm_dtype dt,
