@@ -235,6 +235,13 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
                 if (better(v.x, __float_as_int(v.y), bs, bi)) { bs = v.x; bi = __float_as_int(v.y); }
             }
             a.ws_srch[((size_t)bb * a.Hq + h) * a.nS + slot] = make_float2(bs, __int_as_float(bi));
+            if (bi != 0x7fffffff) {
+                // warm L2 with this unit's candidate state for the merge's gather
+                const __nv_bfloat16 *row = a.a_bar + ((size_t)h * a.K + bi) * D;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(row));
+                if (D * 2 > 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + 64));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.logz_bar + (size_t)h * a.K + bi));
+            }
         }
         return;
     }
