@@ -34,6 +34,8 @@
  *   function.  Workspaces of asm_decode_step and asm_flash_decode hold
  *   self-resetting counters: zero them once with asm_workspace_init before
  *   the first call, then reuse them for any number of calls on one stream.
+ *   The k-means workspace (asm_kmeans_workspace_size) starts with the same
+ *   error word; zero it once too if that word is to be read.
  *   Two calls that overlap on the GPU must not share a workspace.
  */
 #ifndef ASM_B200_H
@@ -116,7 +118,10 @@ asm_status asm_kmeanspp_seed(const void *x, int H, int N, int d, int K,
  * asm_kmeans_assign -- nearest centre of every point ("Agrupamiento"
  * bullet), with the metric rule above, against the storage-dtype centres.
  *   x [H, N, d] dt, centroids_dt [H, K, d] dt -> assign [H, N] int32.
- *   ws asm_kmeans_workspace_size(H, N, d, K) bytes (holds centre norms).
+ *   ws asm_kmeans_workspace_size(H, N, d, K) bytes (error word, centre norms).
+ * bf16 with d = 128 runs on the tcgen05 tensor cores (bf16 products, fp32
+ * accumulation); other cases on CUDA cores in fp32.  A tensor-core pipeline
+ * wait that times out sets the workspace error word to ASM_ERR_TIMEOUT.
  */
 asm_status asm_kmeans_assign(const void *x, const void *centroids_dt, int H,
                              int N, int d, int K, asm_metric metric,
@@ -271,10 +276,10 @@ asm_status asm_flash_decode(const void *q, const void *k_prefix,
 /* Utilities                                                                */
 /* ------------------------------------------------------------------------ */
 
-/* Zero a decode / flash-decode workspace (its counters and error word). */
+/* Zero a decode / flash-decode / k-means workspace (counters, error word). */
 asm_status asm_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Error word of a decode / flash-decode workspace, copied to the host
+/* Error word of a decode / flash-decode / k-means workspace, copied to the host
  * pointer `code` (0 = no device-side error; otherwise ASM_ERR_TIMEOUT).
  * Synchronises `stream`. */
 asm_status asm_workspace_error(const void *ws, size_t ws_bytes, int *code,

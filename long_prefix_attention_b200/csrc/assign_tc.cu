@@ -1,0 +1,290 @@
+// assign_tc.cu -- k-means assignment on the 5th-generation tensor cores.
+//
+// "Context Memorization for Efficient Long Context Generation", Metodologia,
+// "Agrupamiento": each calibration query joins its nearest centroid.  The L2
+// arg-min over centroids is the arg-max of <x, c> - |c|^2 / 2 (cosine: the
+// arg-max of <x, c> / |c|), so the work is a dense X C^T contraction (bf16
+// in, fp32 accumulate) followed by a row-wise arg-max with a per-column term.
+//
+// One CTA owns 256 points of one head (two M=128 halves that share every
+// centroid tile, which halves the L2 -> shared traffic per flop) and sweeps
+// all K centroids in tiles of 128.  Warp roles:
+//   warp 0     producer: TMA of the 256x128 point tile once, then the 128x128
+//              centroid tiles (128-byte swizzle, 4 stages); its lanes copy the
+//              tile's |c|^2 (or |c|) into a 4-deep shared ring;
+//   warp 1     allocates 512 TMEM columns and one lane issues tcgen05.mma
+//              (M=128, N=128, K=16 x 8, both halves) into two ping-pong
+//              accumulator pairs, committing to mbarriers;
+//   warps 2-9  epilogue: warp w reads TMEM lane quarter w%4 of one half,
+//              folds the per-column term and keeps a running arg-max (ties
+//              go to the smaller index) while the next tile is multiplied.
+// Every wait is bounded; a timeout sets the workspace error word to 5.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace asmk {
+namespace atc {
+
+constexpr int kMH = 128;         // rows per MMA (one half)
+constexpr int kM = 2 * kMH;      // points per CTA
+constexpr int kN = 128;          // centroids per tile (MMA N)
+constexpr int kD = 128;          // head dim (MMA K = 8 x 16)
+constexpr int kStages = 4;
+constexpr int kBias = 4;         // depth of the per-column term ring
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr uint32_t kTmemCols = 512;   // 2 buffers x 2 halves x 128 fp32 columns
+
+constexpr int kSub = 128 * 128;       // one 128-row x 64-column swizzled box (16 KB)
+constexpr int kABytes = 4 * kSub;     // [half][k-half]
+constexpr int kBBytes = 2 * kSub;     // [k-half]
+
+struct Smem {
+    unsigned char a[kABytes];
+    unsigned char b[kStages][kBBytes];
+    float bias[kBias][kN];
+    uint64_t a_full, b_full[kStages], b_empty[kStages], acc_full[2], acc_empty[2];
+    uint64_t bias_full[kBias], bias_empty[kBias];
+    uint32_t tmem_base;
+};
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes in 8-row groups 1024 bytes apart; Blackwell descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// D[tmem] (+)= A * B^T, bf16 operands from shared memory, fp32 accumulator
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive on `bar` once every tcgen05 operation this thread issued so far is done.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (no wait)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+struct Maps {
+    CUtensorMap x, c;
+};
+
+// Fold 32 accumulator columns (global centre indices col0 ..) into the
+// running arg-max; only the first `nv` of them are real centres.
+template <int METRIC>
+__device__ __forceinline__ void fold32(const uint32_t (&r)[32], const float *bias, int col0, int nv,
+                                       float &best, int &bidx) {
+    float v[32];
+    float cm = kNegInf;
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+        const float4 bn = *reinterpret_cast<const float4 *>(bias + k);
+        const float bb[4] = {bn.x, bn.y, bn.z, bn.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float acc = __uint_as_float(r[k + u]);
+            float s;
+            if (METRIC == 0) s = fmaf(-0.5f, bb[u], acc);   // exact product: acc - |c|^2 / 2
+            else s = bb[u] > 0.f ? acc / bb[u] : 0.f;     // the term holds |c|
+            v[k + u] = (k + u < nv) ? s : kNegInf;
+            cm = fmaxf(cm, v[k + u]);
+        }
+    }
+    if (cm > best) {
+        int first = 31;
+#pragma unroll
+        for (int k = 31; k >= 0; --k)
+            if (v[k] == cm) first = k;
+        best = cm;
+        bidx = col0 + first;
+    }
+}
+
+template <int METRIC>
+__global__ void __launch_bounds__(kThreads, 1)
+assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ norms, int N, int K,
+                 int32_t *__restrict__ assign, int *err) {
+    extern __shared__ unsigned char smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y;
+    const int p0 = blockIdx.x * kM;
+    const int ntiles = (K + kN - 1) / kN;
+
+    if (tid == 0) {
+        mbar_init(&sm.a_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.b_full[s], 1);
+            mbar_init(&sm.b_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], kEpiWarps);
+        }
+        for (int s = 0; s < kBias; ++s) {
+            mbar_init(&sm.bias_full[s], 32);
+            mbar_init(&sm.bias_empty[s], kEpiWarps);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_addr(&sm.tmem_base)), "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&sm.a_full, kABytes);
+            for (int m = 0; m < 2; ++m)
+                for (int kh = 0; kh < 2; ++kh)
+                    tma_load_3d(sm.a + (m * 2 + kh) * kSub, &maps.x, kh * 64, p0 + m * kMH, h, &sm.a_full);
+        }
+        const float *nh = norms + (size_t)h * K;
+        for (int t = 0; t < ntiles; ++t) {
+            const int s = t % kStages, r = t % kBias;
+            if (lane == 0) {
+                if (t >= kStages) ok &= mbar_wait(&sm.b_empty[s], ((t / kStages) - 1) & 1);
+                mbar_arrive_expect_tx(&sm.b_full[s], kBBytes);
+                tma_load_3d(sm.b[s], &maps.c, 0, t * kN, h, &sm.b_full[s]);
+                tma_load_3d(sm.b[s] + kSub, &maps.c, 64, t * kN, h, &sm.b_full[s]);
+            }
+            if (t >= kBias) ok &= mbar_wait(&sm.bias_empty[r], ((t / kBias) - 1) & 1);
+#pragma unroll
+            for (int u = 0; u < kN / 32; ++u) {
+                const int col = t * kN + u * 32 + lane;
+                float nr = col < K ? __ldg(nh + col) : 0.f;
+                if (METRIC == 1) nr = sqrtf(nr);
+                sm.bias[r][u * 32 + lane] = nr;
+            }
+            mbar_arrive(&sm.bias_full[r]);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B,
+            // both K-major, N = 128, M = 128
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kN >> 3) << 17) |
+                                   ((uint32_t)(kMH >> 4) << 24);
+            ok &= mbar_wait(&sm.a_full, 0);
+            const uint32_t a_base = smem_addr(sm.a);
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % kStages, b = t & 1;
+                ok &= mbar_wait(&sm.b_full[s], (t / kStages) & 1);
+                if (t >= 2) ok &= mbar_wait(&sm.acc_empty[b], ((t >> 1) - 1) & 1);
+                tc_fence_after();
+                const uint32_t b_base = smem_addr(sm.b[s]);
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+#pragma unroll
+                    for (int j = 0; j < kD / 16; ++j) {
+                        // k-step j: box j/4, +32 bytes per 16 elements inside the 128-byte row
+                        const uint32_t koff = (uint32_t)((j >> 2) * kSub + (j & 3) * 32);
+                        const uint64_t ad = sdesc_sw128(a_base + (uint32_t)(m * 2 * kSub) + koff);
+                        const uint64_t bd = sdesc_sw128(b_base + koff);
+                        umma_bf16(tmem + (uint32_t)((b * 2 + m) * kN), ad, bd, idesc, j > 0 ? 1u : 0u);
+                    }
+                }
+                umma_commit(&sm.b_empty[s]);   // the centroid stage is free once these MMAs finish
+                umma_commit(&sm.acc_full[b]);  // and the accumulator pair is ready for the epilogue
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int e = warp - 2;
+        const int m = e >> 2;                // M-half
+        const int q = warp & 3;              // TMEM lane quarter this warp may access
+        const int row = m * kMH + q * 32 + lane;
+        float best = kNegInf;
+        int bidx = 0;
+        for (int t = 0; t < ntiles; ++t) {
+            const int b = t & 1, r = t % kBias;
+            ok &= mbar_wait(&sm.acc_full[b], (t >> 1) & 1);
+            ok &= mbar_wait(&sm.bias_full[r], (t / kBias) & 1);
+            tc_fence_after();
+            const int nv = min(kN, K - t * kN);
+            const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((b * 2 + m) * kN);
+#pragma unroll 1
+            for (int c0 = 0; c0 < kN; c0 += 64) {
+                if (c0 >= nv) break;
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tb + (uint32_t)c0, r0);
+                tmem_ld32(tb + (uint32_t)c0 + 32, r1);
+                tmem_wait_ld();
+                fold32<METRIC>(r0, sm.bias[r] + c0, t * kN + c0, nv - c0, best, bidx);
+                fold32<METRIC>(r1, sm.bias[r] + c0 + 32, t * kN + c0 + 32, nv - c0 - 32, best, bidx);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.acc_empty[b]);
+                mbar_arrive(&sm.bias_empty[r]);
+            }
+        }
+        if (p0 + row < N) assign[(size_t)h * N + p0 + row] = bidx;
+    }
+    if (!ok) atomicExch(err, (int)ASM_ERR_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+}  // namespace atc
+
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows);
+
+}  // namespace asmk
+
+// bf16, d = 128.  `norms` [H, K] holds |c|^2 of the stored (bf16) centres.
+cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, int H, int N, int K, int metric,
+                                 int32_t *assign, int *err, cudaStream_t st) {
+    using namespace asmk;
+    atc::Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!make_map_3d(&maps.x, x, atc::kD, N, H, atc::kMH) || !make_map_3d(&maps.c, c, atc::kD, K, H, atc::kN))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(atc::Smem) + 1024;
+    auto kern = metric == 0 ? atc::assign_tc_kernel<0> : atc::assign_tc_kernel<1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((N + atc::kM - 1) / atc::kM, H);
+    kern<<<grid, atc::kThreads, smem, st>>>(maps, norms, N, K, assign, err);
+    return cudaGetLastError();
+}

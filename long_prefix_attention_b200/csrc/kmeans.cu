@@ -27,7 +27,8 @@ inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 // sum exceeds the threshold, and records the pick for the next round.
 
 constexpr int kSeedThreads = 256;
-constexpr int kSeedPts = 1024;  // points per block (4 per thread)
+constexpr int kSeedWarps = kSeedThreads / 32;
+constexpr int kSeedPts = 1024;  // points per block: 8 warps x 4 steps of 32 points
 
 struct SeedWs {
     size_t off_d2, off_bsum, off_cnt, off_taken, total;
@@ -43,60 +44,113 @@ SeedWs seed_ws(int H, int N) {
     return w;
 }
 
-__device__ __forceinline__ double block_sum_d(double v, double *red) {
-    for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Inclusive prefix sum over the block (fp64); every thread gets its value.
+__device__ __forceinline__ double block_scan_d(double v, double *sh) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, v, m);
+        if (lane >= m) v += y;
+    }
     __syncthreads();
-    if (lane == 0) red[warp] = v;
+    if (lane == 31) sh[warp] = v;
     __syncthreads();
-    double t = 0.0;
-    if (threadIdx.x == 0)
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
-    return t;  // valid in thread 0
+    double off = 0.0;
+    for (int w = 0; w < warp; ++w) off += sh[w];
+    return v + off;
+}
+
+// Sum of D2 over exactly the dims a lane owns, for one point (fp64, exact for
+// bf16 inputs): lane owns dims [EPL*lane, EPL*lane + EPL).
+template <typename T, int D>
+__device__ __forceinline__ double lane_sqdist(const T *xi, const double (&c)[D / 32], int lane) {
+    constexpr int EPL = D / 32;
+    float f[EPL];
+    load_vec<T, EPL>(xi + lane * EPL, f);
+    double s = 0.0;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        const double t = (double)f[e] - c[e];
+        s = fma(t, t, s);
+    }
+    return s;
 }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kSeedThreads)
 kmeanspp_round(const T *__restrict__ x, int N, int K, int r, const double *__restrict__ u,
                int32_t *idx, double *d2, double *bsum, int *cnt, unsigned char *taken) {
+    constexpr int EPL = D / 32;
     const int h = blockIdx.y, nblk = gridDim.x;
     const T *xh = x + (size_t)h * N * D;
     double *d2h = d2 + (size_t)h * N;
     unsigned char *tk = taken + (size_t)h * N;
-    __shared__ double cs[D];
-    __shared__ double red[kSeedThreads / 32];
-    __shared__ int last;
+    __shared__ double sh[kSeedWarps];
+    __shared__ int last, pick_blk;
+    __shared__ double sh_base;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p0 = blockIdx.x * kSeedPts;
+    const int p1 = min(N, p0 + kSeedPts);
 
+    double local = 0.0;
     if (r == 0) {
-        // round 0: clear the slice state; the last block records floor(u*N)
-        for (int i = p0 + threadIdx.x; i < min(N, p0 + kSeedPts); i += blockDim.x) {
+        // round 0: clear the state; the last block records floor(u * N)
+        for (int i = p0 + tid; i < p1; i += kSeedThreads) {
             d2h[i] = __longlong_as_double(0x7ff0000000000000LL);  // +inf
             tk[i] = 0;
         }
     } else {
+        // D2_i = min(D2_i, |x_i - c|^2): a warp takes 32 points at a time, lanes
+        // own dims, then a transpose-reduction leaves point `lane` in lane `lane`
         const int c = idx[(size_t)h * K + r - 1];
-        for (int i = threadIdx.x; i < D; i += blockDim.x) cs[i] = (double)Elem<T>::to_f(xh[(size_t)c * D + i]);
-        __syncthreads();
-        double local = 0.0;
-        for (int i = p0 + threadIdx.x; i < min(N, p0 + kSeedPts); i += blockDim.x) {
-            const T *xi = xh + (size_t)i * D;
-            double s = 0.0;
-#pragma unroll 8
-            for (int e = 0; e < D; ++e) {
-                const double t = (double)Elem<T>::to_f(xi[e]) - cs[e];
-                s = fma(t, t, s);
-            }
-            const double nd = fmin(d2h[i], s);
-            d2h[i] = nd;
-            local += nd;
+        double cv[EPL];
+        {
+            float f[EPL];
+            load_vec<T, EPL>(xh + (size_t)c * D + lane * EPL, f);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) cv[e] = (double)f[e];
         }
-        const double tot = block_sum_d(local, red);
-        if (threadIdx.x == 0) bsum[(size_t)h * nblk + blockIdx.x] = tot;
+        for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
+            double part[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const int i = base + k;
+                part[k] = i < p1 ? lane_sqdist<T, D>(xh + (size_t)i * D, cv, lane) : 0.0;
+            }
+            // transpose-reduce in fp64: after 5 halvings lane l holds point l
+            int mask = 16;
+#pragma unroll
+            for (int n = 32; n > 1; n >>= 1) {
+                const int half = n >> 1;
+                const bool up = (lane & mask) != 0;
+#pragma unroll
+                for (int k = 0; k < half; ++k) {
+                    const double send = up ? part[k] : part[k + half];
+                    const double keep = up ? part[k + half] : part[k];
+                    part[k] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+                }
+                mask >>= 1;
+            }
+            const int i = base + lane;
+            if (i < p1) {
+                const double nd = fmin(d2h[i], part[0]);
+                d2h[i] = nd;
+                local += nd;
+            }
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) local += __shfl_xor_sync(0xffffffffu, local, m);
+        if (lane == 0) sh[warp] = local;
+        __syncthreads();
+        if (tid == 0) {
+            double t = 0.0;
+            for (int w = 0; w < kSeedWarps; ++w) t += sh[w];
+            bsum[(size_t)h * nblk + blockIdx.x] = t;
+        }
     }
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         const int old = atomicAdd(&cnt[h], 1);
         last = (old == nblk - 1);
         __threadfence();
@@ -105,47 +159,113 @@ kmeanspp_round(const T *__restrict__ x, int N, int K, int r, const double *__res
     if (!last) return;
 
     // ---------------- last block of head h: choose this round's centre
-    if (threadIdx.x == 0) {
-        cnt[h] = 0;
-        int pk = -1;
-        const double ur = u[(size_t)h * K + r];
-        if (r == 0) {
-            pk = (int)floor(ur * (double)N);
+    const double ur = u[(size_t)h * K + r];
+    if (r == 0) {
+        if (tid == 0) {
+            int pk = (int)floor(ur * (double)N);
             pk = min(max(pk, 0), N - 1);
-        } else {
-            double total = 0.0;
-            for (int b = 0; b < nblk; ++b) total += __ldcg(bsum + (size_t)h * nblk + b);
-            if (total > 0.0) {
-                const double thr = ur * total;
-                double run = 0.0;
-                for (int b = 0; b < nblk && pk < 0; ++b) {
-                    const double bs = __ldcg(bsum + (size_t)h * nblk + b);
-                    if (run + bs > thr) {
-                        // the threshold falls in this slice: walk its points
-                        double r2 = run;
-                        for (int i = b * kSeedPts; i < min(N, (b + 1) * kSeedPts); ++i) {
-                            r2 += __ldcg(d2h + i);
-                            if (r2 > thr) { pk = i; break; }
-                        }
-                        run = r2;  // (a rounding miss continues in the next slice)
-                    } else {
-                        run += bs;
-                    }
+            idx[(size_t)h * K] = pk;
+            tk[pk] = 1;
+            cnt[h] = 0;
+        }
+        return;
+    }
+    // slice sums -> the slice holding the threshold u * sum(D2)
+    double total = 0.0;
+    {
+        double v = 0.0;
+        for (int bb = tid; bb < nblk; bb += kSeedThreads) v += __ldcg(bsum + (size_t)h * nblk + bb);
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+        __syncthreads();
+        if (lane == 0) sh[warp] = v;
+        __syncthreads();
+        for (int w = 0; w < kSeedWarps; ++w) total += sh[w];
+    }
+    if (total > 0.0) {
+        const double thr = ur * total;
+        if (tid == 0) pick_blk = 0x7fffffff;
+        // inclusive running sums of the slice sums, chunk by chunk; the first
+        // slice whose running sum exceeds thr holds the pick
+        double carry = 0.0;
+        for (int c0 = 0; c0 < nblk; c0 += kSeedThreads) {
+            const int bb = c0 + tid;
+            const double v = bb < nblk ? __ldcg(bsum + (size_t)h * nblk + bb) : 0.0;
+            const double inc = block_scan_d(v, sh) + carry;
+            __syncthreads();
+            if (bb < nblk && inc > thr) atomicMin(&pick_blk, bb);
+            if (tid == kSeedThreads - 1) sh[0] = inc;  // carry into the next chunk
+            __syncthreads();
+            carry = sh[0];
+            if (bb == pick_blk) sh_base = inc - v;  // exclusive running sum of the slice
+            __syncthreads();
+        }
+        int blk = pick_blk;
+        double base_run = blk != 0x7fffffff ? sh_base : 0.0;
+        if (blk == 0x7fffffff) {  // rounding put the threshold past the last sum
+            blk = nblk - 1;
+            base_run = -1.0;      // marks "take the last point with D2 > 0"
+        }
+        __syncthreads();
+        // inside the slice: the first point whose running sum exceeds thr
+        const int q0 = blk * kSeedPts, q1 = min(N, q0 + kSeedPts);
+        constexpr int PT = kSeedPts / kSeedThreads;  // points per thread (4)
+        double dv[PT];
+        double tsum = 0.0;
+#pragma unroll
+        for (int k = 0; k < PT; ++k) {
+            const int i = q0 + tid * PT + k;
+            dv[k] = i < q1 ? __ldcg(d2h + i) : 0.0;
+            tsum += dv[k];
+        }
+        const double inc = block_scan_d(tsum, sh);
+        __syncthreads();
+        if (tid == 0) pick_blk = 0x7fffffff;
+        __syncthreads();
+        if (base_run >= 0.0) {
+            double run = base_run + inc - tsum;
+#pragma unroll
+            for (int k = 0; k < PT; ++k) {
+                run += dv[k];
+                if (run > thr) {
+                    atomicMin(&pick_blk, q0 + tid * PT + k);
+                    break;
                 }
-                if (pk < 0) {
-                    // threshold at the very top of the CDF: the last point with D2 > 0
-                    for (int i = N - 1; i >= 0; --i)
-                        if (__ldcg(d2h + i) > 0.0) { pk = i; break; }
-                    if (pk < 0) pk = 0;
-                }
-            } else {
-                for (int i = 0; i < N; ++i)
-                    if (!__ldcg(tk + i)) { pk = i; break; }
-                if (pk < 0) pk = 0;
             }
         }
+        __syncthreads();
+        if (pick_blk == 0x7fffffff) {
+            // no point crossed thr by rounding: the last point with D2 > 0
+            if (tid == 0) pick_blk = -1;
+            __syncthreads();
+            for (int i = N - 1 - tid; i >= 0; i -= kSeedThreads) {
+                if (__ldcg(d2h + i) > 0.0) {
+                    atomicMax(&pick_blk, i);
+                    break;
+                }
+            }
+            __syncthreads();
+            if (tid == 0 && pick_blk < 0) pick_blk = 0;
+            __syncthreads();
+        }
+    } else {
+        // every remaining point coincides with a centre: the smallest unchosen index
+        if (tid == 0) pick_blk = 0x7fffffff;
+        __syncthreads();
+        for (int i = tid; i < N; i += kSeedThreads)
+            if (!__ldcg(tk + i)) {
+                atomicMin(&pick_blk, i);
+                break;
+            }
+        __syncthreads();
+        if (tid == 0 && pick_blk == 0x7fffffff) pick_blk = 0;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        const int pk = pick_blk;
         idx[(size_t)h * K + r] = pk;
         tk[pk] = 1;
+        cnt[h] = 0;
     }
 }
 
@@ -383,13 +503,16 @@ __global__ void means_kernel(const T *__restrict__ x, const int32_t *__restrict_
     store_vec<T, EPL>(centroids_dt + w * D + lane * EPL, acc);
 }
 
+// Lloyd workspace: a 256-byte header whose first int is the error word
+// (5 = a tensor-core wait timed out), the |c|^2 of every centre, and the
+// scatter cursors.
 struct KmWs {
     size_t off_norm, off_cursor, total;
 };
 KmWs km_ws(int H, int N, int K) {
     (void)N;
     KmWs w;
-    w.off_norm = 0;
+    w.off_norm = 256;
     w.off_cursor = al256(w.off_norm + sizeof(float) * (size_t)H * K);
     w.total = al256(w.off_cursor + sizeof(int) * (size_t)H * K);
     return w;
@@ -452,10 +575,6 @@ cudaError_t asm_kmeans_init_launch(const void *x, int H, int N, int d, int K, as
     return cudaGetLastError();
 }
 
-#ifdef ASM_HAVE_TC_ASSIGN
-cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, int H, int N,
-                                 int K, int metric, int32_t *assign, int num_sms, cudaStream_t st);
-#endif
 
 cudaError_t asm_kmeans_assign_launch(const void *x, const void *centroids_dt, int H, int N, int d,
                                      int K, int metric, asm_dtype dt, int32_t *assign, void *ws,
@@ -475,10 +594,8 @@ cudaError_t asm_kmeans_assign_launch(const void *x, const void *centroids_dt, in
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-#ifdef ASM_HAVE_TC_ASSIGN
     if (dt == ASM_BF16 && d == 128)
-        return asm_assign_tc_launch(x, centroids_dt, norms, H, N, K, metric, assign, num_sms, st);
-#endif
+        return asm_assign_tc_launch(x, centroids_dt, norms, H, N, K, metric, assign, static_cast<int *>(ws), st);
     dim3 grid((N + kAsP - 1) / kAsP, H);
     if (dt == ASM_BF16) {
         using T = __nv_bfloat16;

@@ -35,6 +35,10 @@ cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v,
                                     int accumulate, void *a, float *logz, int num_sms,
                                     cudaStream_t st);
 
+// build_states_tc.cu: bf16, d = 128, L > 0 on tcgen05
+cudaError_t asm_build_states_tc_launch(const void *q, const void *k, const void *v, int Hq, int Hkv, int N, int L,
+                                       float scale, int accumulate, void *a, float *logz, cudaStream_t st);
+
 // kmeans.cu
 size_t asm_kmeanspp_ws_bytes(int H, int N, int d, int K);
 cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const double *u,
@@ -50,6 +54,10 @@ cudaError_t asm_kmeans_update_launch(const void *x, const int32_t *assign, int H
                                      int K, asm_dtype dt, float *centroids, void *centroids_dt,
                                      int32_t *counts, int32_t *perm, int32_t *seg_off, void *ws,
                                      cudaStream_t st);
+
+// assign_tc.cu: bf16, d = 128 assignment on tcgen05; `err` is the workspace error word
+cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, int H, int N, int K,
+                                 int metric, int32_t *assign, int *err, cudaStream_t st);
 
 // aggregate.cu
 cudaError_t asm_aggregate_launch(const void *a, const float *logz, const int32_t *perm,

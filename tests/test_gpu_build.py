@@ -57,6 +57,20 @@ def test_states_shapes(dt, d, Hq, Hkv, N, L):
         assert max_abs(f64(logz), olz) <= tol
 
 
+def test_states_running_max_rises():
+    """Key norms grow along the prefix, so later key tiles raise the row
+    maximum by many units: exercises the rescale of the stored numerator."""
+    cfg = dict(inputs.CONFIGS[3], Hq=2, Hkv=1, n_mix=8)
+    bi = inputs.build_inputs(cfg, seed=11, N=300, L=1000, K=4)
+    ramp = torch.linspace(0.1, 6.0, 1000, dtype=torch.float64)[None, :, None]
+    k = (bi["k"].to(torch.float64) * ramp).to(torch.bfloat16)
+    for chunks in (1, 2):
+        a, logz = gpu_states(dev(bi["q"]), dev(k), dev(bi["v"]), bi["scale"], chunks)
+        oa, olz = O.build_states(bi["q"], k, bi["v"], bi["scale"])
+        assert max_abs(f64(a), oa) <= 2e-2
+        assert max_abs(f64(logz), olz) <= 2e-2
+
+
 def test_states_llama_build_config_sampled_rows():
     """Full build shape (32/8 heads, N=65536, L=16384 as 4 chunks of 4096),
     checked on sampled (head, query) rows against the single-pass oracle."""
@@ -176,6 +190,46 @@ def test_kmeans_teacher_forced_llama_shape_subset():
     cfg = inputs.CONFIGS[3]
     bi = inputs.build_inputs(cfg, N=16384, K=2048, H=4)
     teacher_forced(bi, iters=2, heads=[0, 3])
+
+
+@pytest.mark.parametrize("metric", [ops.ASM_L2, ops.ASM_COSINE])
+@pytest.mark.parametrize("N,K", [(1000, 300), (513, 5), (256, 128), (2304, 1153)])
+def test_assign_tensor_core_ragged(metric, N, K):
+    """bf16, d = 128 (the tcgen05 path): ragged point tail (N % 256), ragged
+    centre tail (K % 128), a single partial centre tile, several tiles; the
+    workspace error word stays 0."""
+    cfg = inputs.CONFIGS[3]
+    bi = inputs.build_inputs(cfg, N=N, K=K, H=3, L=64)
+    x = dev(bi["q"])
+    H, _, d = x.shape
+    # centres: K distinct calibration points plus noise, in storage precision
+    rng = np.random.default_rng(N * 7 + K)
+    pick = np.stack([rng.choice(N, K, replace=False) for _ in range(H)])
+    cen = bi["q"].to(torch.float64)[torch.arange(H)[:, None], torch.from_numpy(pick)]
+    cen = cen + 0.05 * torch.from_numpy(rng.standard_normal(cen.shape))
+    cdt = dev(cen.to(torch.bfloat16))
+    assign = torch.full((H, N), -1, dtype=torch.int32, device="cuda")
+    ws = ops.alloc_workspace(ops.asm_kmeans_workspace_size(H, N, d, K), "cuda", zero=True)
+    ops.asm_kmeans_assign(x, cdt, assign, ws, metric)
+    torch.cuda.synchronize()
+    assert ops.asm_workspace_error(ws) == 0
+    g = host(assign).numpy()
+    xs, cs = f64(bi["q"]), f64(cdt)
+    for h in range(H):
+        o, gap = O.assign(xs[h], cs[h], metric)
+        check_indices(g[h], o, gap)
+
+
+def test_kmeans_every_point_a_centre_tensor_core():
+    bi = inputs.build_inputs(inputs.CONFIGS[3], N=300, K=300, H=2, L=64)
+    x = dev(bi["q"])
+    H, N, d = x.shape
+    c, cdt, assign, counts, perm, seg, ws = kmeans_buffers(H, N, d, N, x.dtype)
+    init = torch.arange(N, dtype=torch.int32).repeat(H, 1).contiguous()
+    ops.asm_kmeans(x, dev(init), 2, c, cdt, assign, counts, perm, seg, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(host(assign), init)
+    assert (host(counts) == 1).all()
 
 
 def test_kmeans_free_running_tiny_fp32_config():
