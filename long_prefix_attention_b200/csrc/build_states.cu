@@ -8,7 +8,7 @@
 //
 // This file holds the portable CUDA-core kernel, used for fp32 storage and
 // for head dim 64; bf16 with head dim 128 is dispatched to the tcgen05
-// kernel in build_states_tc.cu when it is available.
+// kernel in build_states_tc.cu.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -131,11 +131,6 @@ build_states_simple(const T *__restrict__ q, const T *__restrict__ k, const T *_
 
 }  // namespace asmk
 
-#ifdef ASM_HAVE_TC_STATES
-cudaError_t asm_build_states_tc_launch(const void *q, const void *k, const void *v, int Hq,
-                                       int Hkv, int N, int L, float scale, int accumulate, void *a,
-                                       float *logz, int num_sms, cudaStream_t st);
-#endif
 
 cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v, int Hq, int Hkv,
                                     int N, int L, int d, float scale, asm_dtype dt,
@@ -143,11 +138,8 @@ cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v,
                                     cudaStream_t st) {
     using namespace asmk;
     (void)num_sms;
-#ifdef ASM_HAVE_TC_STATES
     if (dt == ASM_BF16 && d == 128 && L > 0)
-        return asm_build_states_tc_launch(q, k, v, Hq, Hkv, N, L, scale, accumulate, a, logz,
-                                          num_sms, st);
-#endif
+        return asm_build_states_tc_launch(q, k, v, Hq, Hkv, N, L, scale, accumulate, a, logz, st);
     dim3 grid((N + kBsQ - 1) / kBsQ, Hq);
     const float qs = scale * kLog2e;
     if (dt == ASM_BF16) {
