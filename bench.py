@@ -5,20 +5,24 @@ single-layer shape (32 query heads, 8 KV heads, head dim 128, K=1024
 centroids per head, local KV cache of 2048 tokens, batch 1, bf16).  One
 benchmark step decodes one token through 32 such layers, each with its own
 memory and KV cache (537 MB in all, more than the 126 MB L2, so every step
-streams its bytes from HBM); the 32 launches are replayed from a CUDA graph.
+streams its bytes from HBM); the 32 layer steps (two kernels each) are
+replayed from a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl asm|reference]
+    python bench.py --only states|assign|seed [--steps K] [--warmup W]
 
 Prints ONE JSON line (rank 0).  `value` is decode query-heads/s over all
 ranks (each rank runs its own independent replica: weak scaling), timed with
-CUDA events between barriers; `roofline` is the decode kernel's algorithmic
-HBM bytes per launch over its average launch time against the measured HBM
-copy peak; `e2e` repeats the measurement through the public API with the
+CUDA events between barriers; `roofline` is the decode step's algorithmic
+HBM bytes per layer over its average time per layer against the measured
+HBM copy peak; `e2e` repeats the measurement through the public API with the
 per-step queries copied from pinned host memory and the outputs copied back;
 `cpu_baseline` times the fp64 oracle on the host cores (a bounded sample);
 `build` times the offline memory build at its full shape (32/8 heads,
 N=65536, L=16384 in 4 chunks, K=8192, 10 Lloyd rounds).
 ``--impl reference`` times the fp64 CPU oracle on the same workload.
+``--only`` times one build stage alone at the build shape (for profiling a
+single kernel) and prints its own JSON line.
 """
 from __future__ import annotations
 
@@ -292,6 +296,55 @@ def run_build(cfg):
     }
 
 
+def run_stage(name, steps, warmup):
+    """One build stage at the full build shape, `steps` timed launches (for
+    profiling single kernels): states = one 4096-key block of the prefix
+    (fresh states, no merge); assign = one Lloyd assignment against K
+    calibration points; seed = the whole k-means++ seeding."""
+    from long_prefix_attention_b200 import ops
+    cfg = inputs.CONFIGS[3]
+    bi = inputs.build_inputs(cfg)
+    x = bi["q"].cuda()
+    H, N, d = x.shape
+    K, L = cfg["K"], cfg["L"] // cfg["chunks"]
+    hbm, tf, tfs, src = peaks()
+    if name == "states":
+        k, v = bi["k"][:, :L].contiguous().cuda(), bi["v"][:, :L].contiguous().cuda()
+        a = torch.empty_like(x)
+        logz = torch.empty(H, N, dtype=torch.float32, device="cuda")
+        fn = lambda: ops.asm_build_states(x, k, v, bi["scale"], a, logz, accumulate=False)
+        flops = 4.0 * N * L * d * H
+    elif name == "assign":
+        g = torch.Generator().manual_seed(5)
+        pick = torch.stack([torch.randperm(N, generator=g)[:K] for _ in range(H)])
+        cdt = x[torch.arange(H, device="cuda")[:, None], pick.cuda()].contiguous()
+        assign = torch.empty(H, N, dtype=torch.int32, device="cuda")
+        ws = ops.alloc_workspace(ops.asm_kmeans_workspace_size(H, N, d, K), "cuda")
+        fn = lambda: ops.asm_kmeans_assign(x, cdt, assign, ws)
+        flops = 2.0 * N * K * d * H
+    else:
+        u = bi["u"].cuda()
+        init = torch.empty(H, K, dtype=torch.int32, device="cuda")
+        ws = ops.alloc_workspace(ops.asm_kmeanspp_workspace_size(H, N, d, K), "cuda", zero=False)
+        fn = lambda: ops.asm_kmeanspp_seed(x, u, init, ws)
+        flops = None
+    for _ in range(max(1, warmup)):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    out = {"stage": name, "workload": cfg["name"], "ms_per_launch": ms, "steps": steps}
+    if flops is not None:
+        out.update({"tflops": flops / (ms / 1e3) / 1e12, "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf,
+                    "peak_tflops": tf, "peak_source": src})
+    print(json.dumps(out))
+
+
 # -------------------------------------------------------------------- main --
 
 def main():
@@ -306,7 +359,12 @@ def main():
     ap.add_argument("--no-prefetch", action="store_true",
                     help="do not let a layer's kernel stream its (static) centroids before the "
                          "preceding kernel finishes")
+    ap.add_argument("--only", choices=["states", "assign", "seed"],
+                    help="time one build stage alone (single-kernel profiling) and exit")
     args = ap.parse_args()
+    if args.only:
+        run_stage(args.only, args.steps, args.warmup)
+        return
     cfg = inputs.CONFIGS[1]
     world, rank, local = dist_setup(args.gpus)
     hbm, tf, tfs, peak_src = peaks()
@@ -336,11 +394,11 @@ def main():
     with ClockSampler(local) as clk:
         secs = time_steps(stack.step, args.steps, max(3, args.warmup), world)
     secs = max_over_ranks(secs, world)
-    launches = args.steps * args.layers
+    launches = args.steps * args.layers * 2  # asm_decode_units + asm_decode_merge per layer
     qh = stack.B * stack.Hq * args.layers * args.steps * world
     value = qh / secs
     ms_per_step = secs * 1e3 / args.steps
-    per_launch_s = secs / launches
+    per_launch_s = secs / (args.steps * args.layers)  # one decode step (both kernels) of one layer
     bpl = stack.bytes_per_launch()
     achieved = bpl / per_launch_s / 1e9
 
@@ -379,7 +437,7 @@ def main():
             "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": None,
-                         "kernel": "decode_kernel<bf16,128,4>",
+                         "kernel": "asm_decode_step = asm_decode_units<128,4> + asm_decode_merge<128>",
                          "bytes_per_launch": bpl, "us_per_launch": per_launch_s * 1e6,
                          "peak_source": f"{peak_src} HBM copy"},
             "e2e": {"value": stack.B * stack.Hq * args.layers * e2e_steps * world / e2e_secs,

@@ -60,27 +60,39 @@ __device__ __forceinline__ double block_scan_d(double v, double *sh) {
     return v + off;
 }
 
-// Sum of D2 over exactly the dims a lane owns, for one point (fp64, exact for
-// bf16 inputs): lane owns dims [EPL*lane, EPL*lane + EPL).
+// D2 update geometry: a point is LPP lanes x 16 bytes; one 16-byte load per
+// lane covers PPL = 32 / LPP points, so a warp reads its 32 points with LPP
+// independent loads, all issued before any arithmetic (memory parallelism:
+// every round streams the whole of x from HBM).
 template <typename T, int D>
-__device__ __forceinline__ double lane_sqdist(const T *xi, const double (&c)[D / 32], int lane) {
-    constexpr int EPL = D / 32;
-    float f[EPL];
-    load_vec<T, EPL>(xi + lane * EPL, f);
-    double s = 0.0;
+struct SeedGeo {
+    static constexpr int E16 = 16 / (int)sizeof(T);   // elements per 16-byte load
+    static constexpr int LPP = D / E16;                // lanes per point
+    static constexpr int PPL = 32 / LPP;               // points per load
+};
+
+// Widen the E16 elements of a 16-byte chunk to fp64.
+template <typename T>
+__device__ __forceinline__ void widen16(const uint4 &u, double *out) {
+    if constexpr (sizeof(T) == 4) {
+        out[0] = (double)__uint_as_float(u.x);
+        out[1] = (double)__uint_as_float(u.y);
+        out[2] = (double)__uint_as_float(u.z);
+        out[3] = (double)__uint_as_float(u.w);
+    } else {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-        const double t = (double)f[e] - c[e];
-        s = fma(t, t, s);
+        for (int e = 0; e < 4; ++e) {
+            out[2 * e] = (double)__uint_as_float(w[e] << 16);
+            out[2 * e + 1] = (double)__uint_as_float(w[e] & 0xFFFF0000u);
+        }
     }
-    return s;
 }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kSeedThreads)
 kmeanspp_round(const T *__restrict__ x, int N, int K, int r, const double *__restrict__ u,
                int32_t *idx, double *d2, double *bsum, int *cnt, unsigned char *taken) {
-    constexpr int EPL = D / 32;
     const int h = blockIdx.y, nblk = gridDim.x;
     const T *xh = x + (size_t)h * N * D;
     double *d2h = d2 + (size_t)h * N;
@@ -100,38 +112,49 @@ kmeanspp_round(const T *__restrict__ x, int N, int K, int r, const double *__res
             tk[i] = 0;
         }
     } else {
-        // D2_i = min(D2_i, |x_i - c|^2): a warp takes 32 points at a time, lanes
-        // own dims, then a transpose-reduction leaves point `lane` in lane `lane`
+        // D2_i = min(D2_i, |x_i - c|^2) in fp64 (exact products for bf16 and
+        // fp32 inputs): lane l reads 16-byte chunk (l % LPP) of points
+        // base + i * PPL + l / LPP, then a transpose-reduction over the LPP
+        // lanes of a point leaves one point's distance in every lane.
+        using G = SeedGeo<T, D>;
         const int c = idx[(size_t)h * K + r - 1];
-        double cv[EPL];
-        {
-            float f[EPL];
-            load_vec<T, EPL>(xh + (size_t)c * D + lane * EPL, f);
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) cv[e] = (double)f[e];
-        }
+        const int sub = lane % G::LPP, grp = lane / G::LPP;
+        double cv[G::E16];
+        widen16<T>(*reinterpret_cast<const uint4 *>(xh + (size_t)c * D + sub * G::E16), cv);
         for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
-            double part[32];
+            uint4 buf[G::LPP];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const int i = base + k;
-                part[k] = i < p1 ? lane_sqdist<T, D>(xh + (size_t)i * D, cv, lane) : 0.0;
+            for (int i = 0; i < G::LPP; ++i) {
+                const int pt = base + i * G::PPL + grp;
+                buf[i] = pt < p1 ? __ldcs(reinterpret_cast<const uint4 *>(xh + (size_t)pt * D + sub * G::E16))
+                                 : make_uint4(0, 0, 0, 0);
             }
-            // transpose-reduce in fp64: after 5 halvings lane l holds point l
-            int mask = 16;
+            double part[G::LPP];
 #pragma unroll
-            for (int n = 32; n > 1; n >>= 1) {
+            for (int i = 0; i < G::LPP; ++i) {
+                double xv[G::E16];
+                widen16<T>(buf[i], xv);
+                double acc = 0.0;
+#pragma unroll
+                for (int e = 0; e < G::E16; ++e) {
+                    const double t = xv[e] - cv[e];
+                    acc = fma(t, t, acc);
+                }
+                part[i] = acc;
+            }
+            // transpose-reduce over the LPP lanes of each point group
+#pragma unroll
+            for (int n = G::LPP; n > 1; n >>= 1) {
                 const int half = n >> 1;
-                const bool up = (lane & mask) != 0;
+                const bool up = (lane & half) != 0;
 #pragma unroll
                 for (int k = 0; k < half; ++k) {
                     const double send = up ? part[k] : part[k + half];
                     const double keep = up ? part[k + half] : part[k];
-                    part[k] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+                    part[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
                 }
-                mask >>= 1;
             }
-            const int i = base + lane;
+            const int i = base + sub * G::PPL + grp;
             if (i < p1) {
                 const double nd = fmin(d2h[i], part[0]);
                 d2h[i] = nd;
