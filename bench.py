@@ -140,12 +140,24 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Largest value of `x` over the ranks (every rank gets it)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed_base(rank):
+    """Input seed of rank `rank`'s replica: each rank decodes its own layers."""
+    return inputs.BASE_SEED + 1000 + 100 * rank
+
+
+def job_throughput(units_per_rank, secs_per_rank, world, device="cuda"):
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time (ranks run the same workload; weak scaling)."""
+    return units_per_rank * world / max_over_ranks(secs_per_rank, world, device)
 
 
 # -------------------------------------------------------------- workloads --
@@ -389,14 +401,13 @@ def main():
 
     flags = 0 if args.no_prefetch else 1  # ASM_DECODE_PREFETCH_CENTROIDS
     config["prefetch_centroids"] = bool(flags)
-    stack = DecodeStack(cfg, args.layers, seed_base=inputs.BASE_SEED + 1000 + 100 * rank, flags=flags)
+    stack = DecodeStack(cfg, args.layers, seed_base=replica_seed_base(rank), flags=flags)
     stack.capture()
     with ClockSampler(local) as clk:
-        secs = time_steps(stack.step, args.steps, max(3, args.warmup), world)
-    secs = max_over_ranks(secs, world)
+        secs_rank = time_steps(stack.step, args.steps, max(3, args.warmup), world)
+    value = job_throughput(stack.B * stack.Hq * args.layers * args.steps, secs_rank, world)
+    secs = max_over_ranks(secs_rank, world)
     launches = args.steps * args.layers * 2  # asm_decode_units + asm_decode_merge per layer
-    qh = stack.B * stack.Hq * args.layers * args.steps * world
-    value = qh / secs
     ms_per_step = secs * 1e3 / args.steps
     per_launch_s = secs / (args.steps * args.layers)  # one decode step (both kernels) of one layer
     bpl = stack.bytes_per_launch()

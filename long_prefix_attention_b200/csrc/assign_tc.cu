@@ -96,27 +96,50 @@ struct Maps {
     CUtensorMap x, c;
 };
 
+// Three-input maximum and paired fp32 fused multiply-add (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+    return m;
+}
+__device__ __forceinline__ void fma2(float a0, float a1, float b, float c0, float c1, float &d0, float &d1) {
+    uint64_t d;
+    asm("{\n .reg .b64 a, b, c;\n mov.b64 a, {%1, %2};\n mov.b64 b, {%3, %3};\n mov.b64 c, {%4, %5};\n"
+        " fma.rn.f32x2 %0, a, b, c;\n}\n"
+        : "=l"(d) : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
 // Fold 32 accumulator columns (global centre indices col0 ..) into the
-// running arg-max; only the first `nv` of them are real centres.
-template <int METRIC>
+// running arg-max; only the first `nv` of them are real centres (FULL: all).
+template <int METRIC, bool FULL>
 __device__ __forceinline__ void fold32(const uint32_t (&r)[32], const float *bias, int col0, int nv,
                                        float &best, int &bidx) {
     float v[32];
-    float cm = kNegInf;
 #pragma unroll
     for (int k = 0; k < 32; k += 4) {
         const float4 bn = *reinterpret_cast<const float4 *>(bias + k);
-        const float bb[4] = {bn.x, bn.y, bn.z, bn.w};
+        if (METRIC == 0) {
+            // acc - |c|^2 / 2, two columns per instruction (the product is exact)
+            fma2(bn.x, bn.y, -0.5f, __uint_as_float(r[k]), __uint_as_float(r[k + 1]), v[k], v[k + 1]);
+            fma2(bn.z, bn.w, -0.5f, __uint_as_float(r[k + 2]), __uint_as_float(r[k + 3]), v[k + 2], v[k + 3]);
+        } else {
+            const float bb[4] = {bn.x, bn.y, bn.z, bn.w};   // the term holds |c|
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float acc = __uint_as_float(r[k + u]);
-            float s;
-            if (METRIC == 0) s = fmaf(-0.5f, bb[u], acc);   // exact product: acc - |c|^2 / 2
-            else s = bb[u] > 0.f ? acc / bb[u] : 0.f;     // the term holds |c|
-            v[k + u] = (k + u < nv) ? s : kNegInf;
-            cm = fmaxf(cm, v[k + u]);
+            for (int u = 0; u < 4; ++u) v[k + u] = bb[u] > 0.f ? __uint_as_float(r[k + u]) / bb[u] : 0.f;
         }
     }
+    if (!FULL) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            if (k >= nv) v[k] = kNegInf;
+    }
+    float m11[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) m11[i] = max3f(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    m11[10] = fmaxf(v[30], v[31]);
+    const float cm = max3f(max3f(m11[0], m11[1], m11[2]), max3f(m11[3], m11[4], m11[5]),
+                           max3f(max3f(m11[6], m11[7], m11[8]), m11[9], m11[10]));
     if (cm > best) {
         int first = 31;
 #pragma unroll
@@ -245,8 +268,13 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
                 tmem_ld32(tb + (uint32_t)c0, r0);
                 tmem_ld32(tb + (uint32_t)c0 + 32, r1);
                 tmem_wait_ld();
-                fold32<METRIC>(r0, sm.bias[r] + c0, t * kN + c0, nv - c0, best, bidx);
-                fold32<METRIC>(r1, sm.bias[r] + c0 + 32, t * kN + c0 + 32, nv - c0 - 32, best, bidx);
+                if (nv == kN) {
+                    fold32<METRIC, true>(r0, sm.bias[r] + c0, t * kN + c0, 32, best, bidx);
+                    fold32<METRIC, true>(r1, sm.bias[r] + c0 + 32, t * kN + c0 + 32, 32, best, bidx);
+                } else {
+                    fold32<METRIC, false>(r0, sm.bias[r] + c0, t * kN + c0, nv - c0, best, bidx);
+                    fold32<METRIC, false>(r1, sm.bias[r] + c0 + 32, t * kN + c0 + 32, nv - c0 - 32, best, bidx);
+                }
             }
             tc_fence_before();
             __syncwarp();

@@ -12,13 +12,15 @@
 // One CTA owns two 128-query tiles (X = 0, 1) of one query head and sweeps the
 // L keys of its KV head in tiles of 64.  Warp roles:
 //   warp 0     TMA producer: both Q tiles once, then K and V tiles (128-byte
-//              swizzle) through two 4-slot rings;
+//              swizzle) through two 3-slot rings;
 //   warp 1     allocates 512 TMEM columns; one lane issues the MMAs in the
 //              order S_0(j), S_1(j), PV_0(j-1), PV_1(j-1), so that the
 //              tensor core multiplies while the softmax warps work;
 //   warps 2-5  softmax of tile 0, warps 6-9 softmax of tile 1: one thread
 //              per query row (TMEM lane), which reads its 64 scores, forms
-//              P = exp2(t - m) in bf16 into shared memory, and rescales its
+//              P = exp2(t - m) in bf16 into one of two shared-memory buffers
+//              (so it never waits for the previous P V product unless it
+//              has to rescale), and rescales its
 //              O row in TMEM on the rare tiles where the running maximum
 //              rises by more than 8 (base-2 units; below that the stale
 //              maximum is kept, which is exact since numerator and
@@ -42,7 +44,7 @@ namespace stc {
 constexpr int kQT = 128;              // queries per tile (MMA M)
 constexpr int kKT = 64;               // keys per tile
 constexpr int kD = 128;
-constexpr int kRing = 4;
+constexpr int kRing = 3;
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescale = 8.f;       // lazy-rescale threshold (base-2 units)
@@ -55,9 +57,11 @@ struct Smem {
     unsigned char q[2][2][kQBox];     // [tile][d-half]
     unsigned char k[kRing][kKVBytes]; // [slot][d-half box]
     unsigned char v[kRing][kKVBytes];
-    unsigned char p[2][kQBox];        // P of each tile: 128 rows x 64 keys
+    unsigned char p[2][2][kQBox];     // P [tile][buffer]: 128 rows x 64 keys
     uint64_t q_full, k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
-    uint64_t s_full[2][2], s_free[2][2], p_full[2], pv_done[2];
+    // [tile][buffer]; a barrier per buffer, so no wait can be overtaken by
+    // the phase after the one it waits for
+    uint64_t s_full[2][2], s_free[2][2], p_full[2][2], pv_done[2][2];
     uint32_t tmem_base;
 };
 
@@ -115,6 +119,43 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// Three-input maximum and paired fp32 arithmetic (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+    return m;
+}
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+__device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
+    return v;
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo;
+}
+__device__ __forceinline__ float hi_f32(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return hi;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 struct Maps {
     CUtensorMap q, k, v;
 };
@@ -150,14 +191,13 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
             mbar_init(&sm.v_full[s], 1);
             mbar_init(&sm.v_empty[s], 1);
         }
-        for (int x = 0; x < 2; ++x) {
+        for (int x = 0; x < 2; ++x)
             for (int b = 0; b < 2; ++b) {
                 mbar_init(&sm.s_full[x][b], 1);
                 mbar_init(&sm.s_free[x][b], kQT);
+                mbar_init(&sm.p_full[x][b], kQT);
+                mbar_init(&sm.pv_done[x][b], 1);
             }
-            mbar_init(&sm.p_full[x], kQT);
-            mbar_init(&sm.pv_done[x], 1);
-        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -222,21 +262,21 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
                     umma_commit(&sm.k_empty[s]);
                 }
                 if (j >= 1) {
-                    const int jj = j - 1, s = jj % kRing;
+                    const int jj = j - 1, s = jj % kRing, pb = jj & 1;
                     ok &= mbar_wait(&sm.v_full[s], (jj / kRing) & 1);
                     const uint32_t vb = smem_addr(sm.v[s]);
                     for (int x = 0; x < 2; ++x) {
-                        ok &= mbar_wait(&sm.p_full[x], jj & 1);
+                        ok &= mbar_wait(&sm.p_full[x][pb], (jj >> 1) & 1);
                         tc_fence_after();
-                        const uint32_t pb = smem_addr(sm.p[x]);
+                        const uint32_t pa = smem_addr(sm.p[x][pb]);
 #pragma unroll
                         for (int kk = 0; kk < kKT / 16; ++kk) {
                             // 16 keys per step: +32 bytes along P's rows, +2 K-groups of V
-                            umma_bf16(tmem + (uint32_t)(x * 128), desc_k_sw128(pb + kk * 32),
+                            umma_bf16(tmem + (uint32_t)(x * 128), desc_k_sw128(pa + kk * 32),
                                       desc_mn_sw128(vb + kk * 2048, kKBox), idesc_o,
                                       (jj > 0 || kk > 0) ? 1u : 0u);
                         }
-                        umma_commit(&sm.pv_done[x]);
+                        umma_commit(&sm.pv_done[x][pb]);
                     }
                     umma_commit(&sm.v_empty[s]);
                 }
@@ -250,29 +290,36 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
         const int row = qd * 32 + lane;     // row within the tile
         const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
         const uint32_t t_o = tmem + lane_off + (uint32_t)(x * 128);
-        const uint32_t p_row = smem_addr(sm.p[x]) + (uint32_t)row * 128;
         float m_used = kNegInf, l = 0.f;
         for (int j = 0; j < J; ++j) {
             const int b = j & 1;
             ok &= mbar_wait(&sm.s_full[x][b], (j >> 1) & 1);
             tc_fence_after();
-            uint32_t r0[32], r1[32];
+            uint32_t r[64];
             const uint32_t t_s = tmem + lane_off + 256 + (uint32_t)(x * 128 + b * 64);
-            tmem_ld32(t_s, r0);
-            tmem_ld32(t_s + 32, r1);
+            tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.s_free[x][b]);
 
             const int valid = L - j * kKT;  // keys of this tile inside the block
-            float t[64];
-            float mt = kNegInf;
+            if (valid < kKT) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                t[c] = c < valid ? __uint_as_float(r0[c]) * sl2 : kNegInf;
-                t[c + 32] = c + 32 < valid ? __uint_as_float(r1[c]) * sl2 : kNegInf;
-                mt = fmaxf(mt, fmaxf(t[c], t[c + 32]));
+                for (int c = 0; c < 64; ++c)
+                    if (c >= valid) r[c] = 0xff800000u;  // -inf
             }
+            // row maximum of the raw scores (the scale is positive)
+            float m21[22];
+#pragma unroll
+            for (int i = 0; i < 21; ++i)
+                m21[i] = max3f(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
+            m21[21] = __uint_as_float(r[63]);
+            float m7[8];
+#pragma unroll
+            for (int i = 0; i < 7; ++i) m7[i] = max3f(m21[3 * i], m21[3 * i + 1], m21[3 * i + 2]);
+            m7[7] = m21[21];
+            const float mt = max3f(max3f(m7[0], m7[1], m7[2]), max3f(m7[3], m7[4], m7[5]), fmaxf(m7[6], m7[7])) * sl2;
             bool rescale = false;
             float alpha = 1.f;
             if (mt > m_used + kRescale) {
@@ -281,21 +328,26 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
                 m_used = mt;
                 l *= alpha;
             }
+            // p = 2^(s * scale * log2(e) - m), paired fp32 arithmetic
+            const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
+            const uint64_t negm2 = pack_f32x2(-m_used, -m_used);
             uint32_t pk[32];
-            float ls = 0.f;
+            uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                const float p0 = ex2f(t[2 * c] - m_used), p1 = ex2f(t[2 * c + 1] - m_used);
-                ls += p0 + p1;
+                const uint64_t t2 = fma_f32x2(pack_u32x2(r[2 * c], r[2 * c + 1]), sl2x2, negm2);
+                const float p0 = ex2f(lo_f32(t2)), p1 = ex2f(hi_f32(t2));
+                acc[c & 3] = add_f32x2(acc[c & 3], pack_f32x2(p0, p1));
                 pk[c] = pack_bf16(p0, p1);
             }
-            l += ls;
-            // P_x and O_x are free once PV(j-1) has finished
-            if (j >= 1) ok &= mbar_wait(&sm.pv_done[x], (j - 1) & 1);
-            tc_fence_after();
+            const uint64_t a01 = add_f32x2(add_f32x2(acc[0], acc[1]), add_f32x2(acc[2], acc[3]));
+            l += lo_f32(a01) + hi_f32(a01);
             // TMEM loads and stores are warp-collective: the warp rescales
-            // together, rows that keep their maximum by a factor of 1
+            // together, rows that keep their maximum by a factor of 1; O
+            // must hold PV(j-1) first
             if (__any_sync(0xffffffffu, rescale)) {
+                ok &= mbar_wait(&sm.pv_done[x][(j - 1) & 1], ((j - 1) >> 1) & 1);
+                tc_fence_after();
                 const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
                 for (int c0 = 0; c0 < kD; c0 += 32) {
@@ -308,6 +360,9 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
                 }
                 tmem_wait_st();
             }
+            // P buffer b is free once PV(j-2) has finished
+            if (j >= 2) ok &= mbar_wait(&sm.pv_done[x][b], ((j >> 1) - 1) & 1);
+            const uint32_t p_row = smem_addr(sm.p[x][b]) + (uint32_t)row * 128;
             // row of P: eight 16-byte chunks, 128-byte swizzle
 #pragma unroll
             for (int c = 0; c < 8; ++c)
@@ -315,10 +370,10 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
                              pk[4 * c + 3]);
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(&sm.p_full[x]);
+            mbar_arrive(&sm.p_full[x][b]);
         }
         // ------------------------------------------------------ epilogue
-        ok &= mbar_wait(&sm.pv_done[x], (J - 1) & 1);
+        ok &= mbar_wait(&sm.pv_done[x][(J - 1) & 1], ((J - 1) >> 1) & 1);
         tc_fence_after();
         const int n = n0 + x * kQT + row;
         const bool live = n < N;
