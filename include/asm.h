@@ -285,6 +285,11 @@ asm_status asm_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
 asm_status asm_workspace_error(const void *ws, size_t ws_bytes, int *code,
                                cudaStream_t stream);
 
+/* The CUDA runtime's message for the last CUDA error behind an ASM_ERR_CUDA
+ * returned on the calling thread ("no error" if there was none).  Static
+ * storage, never NULL. */
+const char *asm_last_cuda_error(void);
+
 /* Static description of a status code (never NULL). */
 const char *asm_status_string(asm_status s);
 

@@ -34,6 +34,7 @@ SIGNATURES = {
     "asm_workspace_init": (I, [P, SZ, P]),
     "asm_workspace_error": (I, [P, SZ, ctypes.POINTER(ctypes.c_int), P]),
     "asm_status_string": (ctypes.c_char_p, [I]),
+    "asm_last_cuda_error": (ctypes.c_char_p, []),
     "asm_version": (ctypes.c_char_p, []),
 }
 

@@ -31,11 +31,22 @@ int num_sms() {
     return cache[dev];
 }
 
-asm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ASM_OK : ASM_ERR_CUDA; }
+// The last CUDA error this thread's library calls observed (cudaSuccess if none).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+asm_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return ASM_OK;
+    t_last_cuda_error = e;
+    return ASM_ERR_CUDA;
+}
 
 }  // namespace
 
 extern "C" {
+
+const char *asm_last_cuda_error(void) {
+    return t_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda_error);
+}
 
 const char *asm_status_string(asm_status s) {
     switch (s) {

@@ -9,25 +9,28 @@
 // computed flash-attention style: S = Q K^T and O += P V on tcgen05.mma with
 // fp32 accumulators in tensor memory, the softmax in registers.
 //
-// One CTA owns two 128-query tiles (X = 0, 1) of one query head and sweeps the
-// L keys of its KV head in tiles of 64.  Warp roles:
-//   warp 0     TMA producer: both Q tiles once, then K and V tiles (128-byte
-//              swizzle) through two 3-slot rings;
+// One CTA owns two 128-query tiles (x = 0, 1) of one query head and sweeps the
+// L keys of its KV head in tiles of 128.  Warp roles:
+//   warp 0     TMA producer: both Q tiles once, then K_0, V_0, K_1, V_1, ...
+//              (128-byte swizzle) through a 4-slot ring;
 //   warp 1     allocates 512 TMEM columns; one lane issues the MMAs in the
-//              order S_0(j), S_1(j), PV_0(j-1), PV_1(j-1), so that the
-//              tensor core multiplies while the softmax warps work;
+//              order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): while one tile's
+//              softmax works, the tensor core multiplies the other tile;
 //   warps 2-5  softmax of tile 0, warps 6-9 softmax of tile 1: one thread
-//              per query row (TMEM lane), which reads its 64 scores, forms
-//              P = exp2(t - m) in bf16 into one of two shared-memory buffers
-//              (so it never waits for the previous P V product unless it
-//              has to rescale), and rescales its
-//              O row in TMEM on the rare tiles where the running maximum
-//              rises by more than 8 (base-2 units; below that the stale
-//              maximum is kept, which is exact since numerator and
-//              denominator share it).
-// TMEM columns: O_0 [0,128) O_1 [128,256) S_0 double buffer [256,384)
-// S_1 double buffer [384,512).  Every wait is bounded; a timeout writes NaN
-// into logZ of the CTA's rows.
+//              per query row (TMEM lane).  It loads its 128 scores, forms
+//              P = exp2(t - m) (three quarters on the MUFU unit, one quarter
+//              by a cubic on the FMA pipe) and stores P as bf16 over the
+//              first 64 columns of its own S region, from where the P V
+//              product reads it as the A operand; only V comes from shared
+//              memory.  Its O row is rescaled in TMEM on the rare tiles where
+//              the running maximum rises by more than 8 (base-2 units; below
+//              that the stale maximum is kept, which is exact since
+//              numerator and denominator share it).
+// The tensor pipe completes MMAs in issue order, so S_x(j+1) (issued after
+// PV_x(j)) overwrites P_x(j) only after it was read, and the completion of
+// S_x(j) also means PV_x(j-1) is done: O_x is stable when softmax x starts.
+// TMEM columns: O_0 [0,128) O_1 [128,256) S_0 / P_0 [256,384) S_1 / P_1 [384,512).
+// Every wait is bounded; a timeout writes NaN into logZ of the CTA's rows.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -42,26 +45,21 @@ namespace asmk {
 namespace stc {
 
 constexpr int kQT = 128;              // queries per tile (MMA M)
-constexpr int kKT = 64;               // keys per tile
+constexpr int kKT = 128;              // keys per tile (MMA N of S = Q K^T)
 constexpr int kD = 128;
-constexpr int kRing = 3;
+constexpr int kRing = 4;              // K/V slots
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescale = 8.f;       // lazy-rescale threshold (base-2 units)
 
-constexpr int kQBox = kQT * 128;      // 128 rows x 64 columns bf16 (16 KB)
-constexpr int kKBox = kKT * 128;      // 64 rows x 64 columns bf16 (8 KB)
-constexpr int kKVBytes = 2 * kKBox;   // one K or V tile
+constexpr int kBox = 128 * 128;       // 128 rows x 64 columns bf16 (16 KB)
+constexpr int kTile = 2 * kBox;       // a 128 x 128 bf16 tile as two 64-column boxes
 
 struct Smem {
-    unsigned char q[2][2][kQBox];     // [tile][d-half]
-    unsigned char k[kRing][kKVBytes]; // [slot][d-half box]
-    unsigned char v[kRing][kKVBytes];
-    unsigned char p[2][2][kQBox];     // P [tile][buffer]: 128 rows x 64 keys
-    uint64_t q_full, k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
-    // [tile][buffer]; a barrier per buffer, so no wait can be overtaken by
-    // the phase after the one it waits for
-    uint64_t s_full[2][2], s_free[2][2], p_full[2][2], pv_done[2][2];
+    unsigned char q[2][kTile];        // [query tile]: d-halves
+    unsigned char kv[kRing][kTile];   // K or V tile: d-halves, rows = keys
+    uint64_t q_full, kv_full[kRing], kv_empty[kRing];
+    uint64_t s_full[2], p_full[2], o_full[2];
     uint32_t tmem_base;
 };
 
@@ -84,13 +82,20 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint6
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
         ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+// D[tmem] (+)= A[tmem] * B^T: A (M x 16, bf16 pairs per column) from tensor memory
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
+        ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(smem_addr(bar)) : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -112,12 +117,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
           "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
 
 // Three-input maximum and paired fp32 arithmetic (sm_100).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -135,16 +144,8 @@ __device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
     asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
     return v;
 }
-__device__ __forceinline__ float lo_f32(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return lo;
-}
-__device__ __forceinline__ float hi_f32(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return hi;
-}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
 __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t d;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
@@ -154,6 +155,24 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
+}
+
+// 2^t for two arguments on the FMA pipe: t = n + f with n = round(t),
+// f in [-1/2, 1/2]; 2^f by a cubic fitted to 2^f over that interval
+// (relative error below 7.5e-5, under a quarter of a bf16 half-unit), and
+// 2^n added into the exponent field.  t is clamped at -125 (2^-125 counts as
+// 0 next to the row maximum's 2^0).
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t t2) {
+    const float t0 = fmaxf(lo_f32(t2), -125.f), t1 = fmaxf(hi_f32(t2), -125.f);
+    const uint64_t t = pack_f32x2(t0, t1);
+    const uint64_t y = add_f32x2(t, pack_f32x2(12582912.f, 12582912.f));   // 1.5 * 2^23: n in the low bits
+    const uint64_t n = add_f32x2(y, pack_f32x2(-12582912.f, -12582912.f));
+    const uint64_t f = fma_f32x2(n, pack_f32x2(-1.f, -1.f), t);
+    uint64_t p = fma_f32x2(pack_f32x2(0.0551716685f, 0.0551716685f), f, pack_f32x2(0.2426111251f, 0.2426111251f));
+    p = fma_f32x2(p, f, pack_f32x2(0.6932609678f, 0.6932609678f));
+    p = fma_f32x2(p, f, pack_f32x2(0.9999280572f, 0.9999280572f));
+    const uint32_t lo = (uint32_t)p + ((uint32_t)y << 23), hi = (uint32_t)(p >> 32) + ((uint32_t)(y >> 32) << 23);
+    return pack_u32x2(lo, hi);
 }
 
 struct Maps {
@@ -185,19 +204,15 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
 
     if (tid == 0) {
         mbar_init(&sm.q_full, 1);
-        for (int s = 0; s < kRing; ++s) {
-            mbar_init(&sm.k_full[s], 1);
-            mbar_init(&sm.k_empty[s], 1);
-            mbar_init(&sm.v_full[s], 1);
-            mbar_init(&sm.v_empty[s], 1);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(&sm.kv_full[i], 1);
+            mbar_init(&sm.kv_empty[i], 1);
         }
-        for (int x = 0; x < 2; ++x)
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(&sm.s_full[x][b], 1);
-                mbar_init(&sm.s_free[x][b], kQT);
-                mbar_init(&sm.p_full[x][b], kQT);
-                mbar_init(&sm.pv_done[x][b], 1);
-            }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&sm.s_full[x], 1);
+            mbar_init(&sm.p_full[x], kQT);
+            mbar_init(&sm.o_full[x], 1);
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -214,72 +229,73 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(&sm.q_full, 4 * kQBox);
+            mbar_arrive_expect_tx(&sm.q_full, 2 * kTile);
             for (int x = 0; x < 2; ++x)
                 for (int dh = 0; dh < 2; ++dh)
-                    tma_load_3d(sm.q[x][dh], &maps.q, dh * 64, n0 + x * kQT, h, &sm.q_full);
-            for (int j = 0; j < J; ++j) {
-                const int s = j % kRing;
-                const uint32_t par = ((j / kRing) - 1) & 1;
-                if (j >= kRing) ok &= mbar_wait(&sm.k_empty[s], par);
-                mbar_arrive_expect_tx(&sm.k_full[s], kKVBytes);
-                tma_load_3d(sm.k[s], &maps.k, 0, j * kKT, g, &sm.k_full[s]);
-                tma_load_3d(sm.k[s] + kKBox, &maps.k, 64, j * kKT, g, &sm.k_full[s]);
-                if (j >= kRing) ok &= mbar_wait(&sm.v_empty[s], par);
-                mbar_arrive_expect_tx(&sm.v_full[s], kKVBytes);
-                tma_load_3d(sm.v[s], &maps.v, 0, j * kKT, g, &sm.v_full[s]);
-                tma_load_3d(sm.v[s] + kKBox, &maps.v, 64, j * kKT, g, &sm.v_full[s]);
+                    tma_load_3d(sm.q[x] + dh * kBox, &maps.q, dh * 64, n0 + x * kQT, h, &sm.q_full);
+            // ring item n: K_{n/2} for even n, V_{n/2} for odd n
+            for (int n = 0; n < 2 * J; ++n) {
+                const int slot = n % kRing;
+                if (n >= kRing) ok &= mbar_wait(&sm.kv_empty[slot], ((n / kRing) - 1) & 1);
+                mbar_arrive_expect_tx(&sm.kv_full[slot], kTile);
+                const CUtensorMap *mp = (n & 1) ? &maps.v : &maps.k;
+                tma_load_3d(sm.kv[slot], mp, 0, (n >> 1) * kKT, g, &sm.kv_full[slot]);
+                tma_load_3d(sm.kv[slot] + kBox, mp, 64, (n >> 1) * kKT, g, &sm.kv_full[slot]);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer
         if (lane == 0) {
-            // S = Q K^T: M = 128, N = 64, both operands K-major
+            // S = Q K^T: M = 128, N = 128, both operands K-major (shared memory)
             const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kKT >> 3) << 17) |
                                      ((uint32_t)(kQT >> 4) << 24);
-            // O += P V: M = 128, N = 128; P K-major, V MN-major (d contiguous)
+            // O += P V: M = 128, N = 128; P K-major in TMEM, V MN-major (d contiguous)
             const uint32_t idesc_o = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                                      ((uint32_t)(kD >> 3) << 17) | ((uint32_t)(kQT >> 4) << 24);
+            auto issue_s = [&](int x, uint32_t kb) {
+                const uint32_t qb = smem_addr(sm.q[x]);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * kBox + (kk & 3) * 32);
+                    umma_bf16(tmem + 256 + (uint32_t)(x * 128), desc_k_sw128(qb + off), desc_k_sw128(kb + off),
+                              idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&sm.s_full[x]);
+            };
+            auto issue_pv = [&](int x, uint32_t vb, int j) {
+#pragma unroll
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    // 16 keys per step: 8 TMEM columns of P, 16 rows (2 K-groups) of V
+                    umma_bf16_ts(tmem + (uint32_t)(x * 128), tmem + 256 + (uint32_t)(x * 128 + kk * 8),
+                                 desc_mn_sw128(vb + (uint32_t)(kk * 2048), kBox), idesc_o,
+                                 (j > 0 || kk > 0) ? 1u : 0u);
+            };
             ok &= mbar_wait(&sm.q_full, 0);
-            for (int j = 0; j <= J; ++j) {
-                if (j < J) {
-                    const int s = j % kRing, b = j & 1;
-                    ok &= mbar_wait(&sm.k_full[s], (j / kRing) & 1);
-                    const uint32_t kb = smem_addr(sm.k[s]);
-                    for (int x = 0; x < 2; ++x) {
-                        if (j >= 2) ok &= mbar_wait(&sm.s_free[x][b], ((j >> 1) - 1) & 1);
-                        tc_fence_after();
-                        const uint32_t qb = smem_addr(sm.q[x][0]);
-                        const uint32_t td = tmem + 256 + (uint32_t)(x * 128 + b * 64);
-#pragma unroll
-                        for (int kk = 0; kk < kD / 16; ++kk) {
-                            const uint32_t off = (uint32_t)((kk & 3) * 32);
-                            umma_bf16(td, desc_k_sw128(qb + (kk >> 2) * kQBox + off),
-                                      desc_k_sw128(kb + (kk >> 2) * kKBox + off), idesc_s, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&sm.s_full[x][b]);
+            // scores of key tile 0
+            ok &= mbar_wait(&sm.kv_full[0], 0);
+            tc_fence_after();
+            issue_s(0, smem_addr(sm.kv[0]));
+            issue_s(1, smem_addr(sm.kv[0]));
+            umma_commit(&sm.kv_empty[0]);
+            for (int j = 0; j < J; ++j) {
+                const int nv = 2 * j + 1, nk = 2 * j + 2;          // ring items V_j and K_{j+1}
+                const int sv = nv % kRing, sk = nk % kRing;
+                const bool more = j + 1 < J;
+                ok &= mbar_wait(&sm.kv_full[sv], (nv / kRing) & 1);
+                const uint32_t vb = smem_addr(sm.kv[sv]), kb = smem_addr(sm.kv[sk]);
+                for (int x = 0; x < 2; ++x) {
+                    ok &= mbar_wait(&sm.p_full[x], j & 1);
+                    tc_fence_after();
+                    issue_pv(x, vb, j);
+                    if (more) {
+                        if (x == 0) ok &= mbar_wait(&sm.kv_full[sk], (nk / kRing) & 1);
+                        issue_s(x, kb);
+                    } else {
+                        umma_commit(&sm.o_full[x]);
                     }
-                    umma_commit(&sm.k_empty[s]);
                 }
-                if (j >= 1) {
-                    const int jj = j - 1, s = jj % kRing, pb = jj & 1;
-                    ok &= mbar_wait(&sm.v_full[s], (jj / kRing) & 1);
-                    const uint32_t vb = smem_addr(sm.v[s]);
-                    for (int x = 0; x < 2; ++x) {
-                        ok &= mbar_wait(&sm.p_full[x][pb], (jj >> 1) & 1);
-                        tc_fence_after();
-                        const uint32_t pa = smem_addr(sm.p[x][pb]);
-#pragma unroll
-                        for (int kk = 0; kk < kKT / 16; ++kk) {
-                            // 16 keys per step: +32 bytes along P's rows, +2 K-groups of V
-                            umma_bf16(tmem + (uint32_t)(x * 128), desc_k_sw128(pa + kk * 32),
-                                      desc_mn_sw128(vb + kk * 2048, kKBox), idesc_o,
-                                      (jj > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(&sm.pv_done[x][pb]);
-                    }
-                    umma_commit(&sm.v_empty[s]);
-                }
+                umma_commit(&sm.kv_empty[sv]);
+                if (more) umma_commit(&sm.kv_empty[sk]);
             }
         }
         __syncwarp();
@@ -290,36 +306,35 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
         const int row = qd * 32 + lane;     // row within the tile
         const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
         const uint32_t t_o = tmem + lane_off + (uint32_t)(x * 128);
+        const uint32_t t_s = tmem + lane_off + 256 + (uint32_t)(x * 128);
         float m_used = kNegInf, l = 0.f;
         for (int j = 0; j < J; ++j) {
-            const int b = j & 1;
-            ok &= mbar_wait(&sm.s_full[x][b], (j >> 1) & 1);
+            // S_x(j) done, and with it PV_x(j-1): O_x is stable, P_x's columns free
+            ok &= mbar_wait(&sm.s_full[x], j & 1);
             tc_fence_after();
-            uint32_t r[64];
-            const uint32_t t_s = tmem + lane_off + 256 + (uint32_t)(x * 128 + b * 64);
-            tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-            tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sm.s_free[x][b]);
-
             const int valid = L - j * kKT;  // keys of this tile inside the block
-            if (valid < kKT) {
+            // pass 1: row maximum of the raw scores (the scale is positive),
+            // 32 columns at a time
+            float mraw = kNegInf;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(t_s + (uint32_t)(32 * c), r);
+                tmem_wait_ld();
+                if (valid < kKT) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (c >= valid) r[c] = 0xff800000u;  // -inf
+                    for (int i = 0; i < 32; ++i)
+                        if (32 * c + i >= valid) r[i] = 0xff800000u;  // -inf
+                }
+                float m11[11];
+#pragma unroll
+                for (int i = 0; i < 10; ++i)
+                    m11[i] = max3f(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
+                m11[10] = fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31]));
+                mraw = max3f(mraw, max3f(max3f(m11[0], m11[1], m11[2]), max3f(m11[3], m11[4], m11[5]),
+                                         max3f(m11[6], m11[7], m11[8])), fmaxf(m11[9], m11[10]));
             }
-            // row maximum of the raw scores (the scale is positive)
-            float m21[22];
-#pragma unroll
-            for (int i = 0; i < 21; ++i)
-                m21[i] = max3f(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
-            m21[21] = __uint_as_float(r[63]);
-            float m7[8];
-#pragma unroll
-            for (int i = 0; i < 7; ++i) m7[i] = max3f(m21[3 * i], m21[3 * i + 1], m21[3 * i + 2]);
-            m7[7] = m21[21];
-            const float mt = max3f(max3f(m7[0], m7[1], m7[2]), max3f(m7[3], m7[4], m7[5]), fmaxf(m7[6], m7[7])) * sl2;
+            const float mt = mraw * sl2;
             bool rescale = false;
             float alpha = 1.f;
             if (mt > m_used + kRescale) {
@@ -328,26 +343,9 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
                 m_used = mt;
                 l *= alpha;
             }
-            // p = 2^(s * scale * log2(e) - m), paired fp32 arithmetic
-            const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
-            const uint64_t negm2 = pack_f32x2(-m_used, -m_used);
-            uint32_t pk[32];
-            uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const uint64_t t2 = fma_f32x2(pack_u32x2(r[2 * c], r[2 * c + 1]), sl2x2, negm2);
-                const float p0 = ex2f(lo_f32(t2)), p1 = ex2f(hi_f32(t2));
-                acc[c & 3] = add_f32x2(acc[c & 3], pack_f32x2(p0, p1));
-                pk[c] = pack_bf16(p0, p1);
-            }
-            const uint64_t a01 = add_f32x2(add_f32x2(acc[0], acc[1]), add_f32x2(acc[2], acc[3]));
-            l += lo_f32(a01) + hi_f32(a01);
             // TMEM loads and stores are warp-collective: the warp rescales
-            // together, rows that keep their maximum by a factor of 1; O
-            // must hold PV(j-1) first
+            // together, rows that keep their maximum by a factor of 1
             if (__any_sync(0xffffffffu, rescale)) {
-                ok &= mbar_wait(&sm.pv_done[x][(j - 1) & 1], ((j - 1) >> 1) & 1);
-                tc_fence_after();
                 const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
                 for (int c0 = 0; c0 < kD; c0 += 32) {
@@ -358,22 +356,45 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
                     tmem_st32(t_o + (uint32_t)c0, o);
                 }
-                tmem_wait_st();
             }
-            // P buffer b is free once PV(j-2) has finished
-            if (j >= 2) ok &= mbar_wait(&sm.pv_done[x][b], ((j >> 1) - 1) & 1);
-            const uint32_t p_row = smem_addr(sm.p[x][b]) + (uint32_t)row * 128;
-            // row of P: eight 16-byte chunks, 128-byte swizzle
+            // pass 2: p = 2^(s * scale * log2(e) - m), packed to bf16 pairs;
+            // chunk c's 16 columns of P land on S columns already read
+            const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
+            const uint64_t negm2 = pack_f32x2(-m_used, -m_used);
+            uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(t_s + (uint32_t)(32 * c), r);
+                tmem_wait_ld();
+                if (valid < kKT) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(p_row + (uint32_t)((c ^ (row & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                             pk[4 * c + 3]);
-            fence_async_smem();
+                    for (int i = 0; i < 32; ++i)
+                        if (32 * c + i >= valid) r[i] = 0xff800000u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint64_t t2 = fma_f32x2(pack_u32x2(r[2 * i], r[2 * i + 1]), sl2x2, negm2);
+                    uint64_t p2;
+                    if ((i & 3) == 3) {
+                        p2 = exp2_poly_x2(t2);
+                    } else {
+                        p2 = pack_f32x2(ex2f(lo_f32(t2)), ex2f(hi_f32(t2)));
+                    }
+                    acc[i & 3] = add_f32x2(acc[i & 3], p2);
+                    pk[i] = pack_bf16(lo_f32(p2), hi_f32(p2));
+                }
+                tmem_st16(t_s + (uint32_t)(16 * c), pk);
+            }
+            const uint64_t a01 = add_f32x2(add_f32x2(acc[0], acc[1]), add_f32x2(acc[2], acc[3]));
+            l += lo_f32(a01) + hi_f32(a01);
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sm.p_full[x][b]);
+            mbar_arrive(&sm.p_full[x]);
         }
         // ------------------------------------------------------ epilogue
-        ok &= mbar_wait(&sm.pv_done[x][(J - 1) & 1], ((J - 1) >> 1) & 1);
+        ok &= mbar_wait(&sm.o_full[x], 0);
         tc_fence_after();
         const int n = n0 + x * kQT + row;
         const bool live = n < N;

@@ -15,6 +15,7 @@ import torch
 
 from . import _lib
 
+ASM_OK, ASM_ERR_INVALID_ARG, ASM_ERR_UNSUPPORTED, ASM_ERR_WORKSPACE, ASM_ERR_CUDA, ASM_ERR_TIMEOUT = range(6)
 ASM_F32, ASM_BF16 = 0, 1
 ASM_L2, ASM_COSINE = 0, 1
 ASM_ZBAR_MEAN, ASM_ZBAR_SUM = 0, 1
@@ -25,7 +26,10 @@ _DT = {torch.float32: ASM_F32, torch.bfloat16: ASM_BF16}
 
 class AsmError(RuntimeError):
     def __init__(self, fn: str, status: int):
-        msg = _lib.load().asm_status_string(status).decode()
+        lib = _lib.load()
+        msg = lib.asm_status_string(status).decode()
+        if status == ASM_ERR_CUDA:
+            msg += ": " + lib.asm_last_cuda_error().decode()
         super().__init__(f"{fn}: status {status} ({msg})")
         self.status = status
 

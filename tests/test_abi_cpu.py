@@ -43,6 +43,8 @@ def test_status_strings(lib):
     for s in range(6):
         assert lib.asm_status_string(s)
     assert lib.asm_version().decode().count(".") == 2
+    # no CUDA call has failed on this thread
+    assert lib.asm_last_cuda_error().decode() == "no error"
 
 
 FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
