@@ -54,6 +54,9 @@ struct Geo {
 
 struct Args {
     const __nv_bfloat16 *q;       // [B][Hq][D]
+    const __nv_bfloat16 *centroids;             // [Hq][K][D]
+    const __nv_bfloat16 *k_cache, *v_cache;     // [B][Hkv][Tmax][D]
+    const __nv_bfloat16 *k_prefix, *v_prefix;   // [Hkv][Lp][D]
     const __nv_bfloat16 *a_bar;   // [Hq][K][D]
     const float *logz_bar;        // [Hq][K]
     const int *local_len;         // [B]
@@ -153,6 +156,33 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     // static centroids may stream before the dependency wait (caller's choice)
     const bool early = scan && (a.flags & 1);
     if (early && tid == 0) issue(valid);
+    if (!early) {
+        // Warm L2 with this unit's rows while the preceding kernel finishes.
+        // Always safe: L2 is the coherence point, so a row the preceding
+        // kernel still writes is read correctly after the wait below.  The
+        // row count of an attention unit comes from a relaxed read of the
+        // length, a hint only (a stale value costs bandwidth, not results).
+        int rows = valid;
+        const __nv_bfloat16 *kr = nullptr, *vr = nullptr;
+        if (scan) {
+            kr = a.centroids + ((size_t)h * a.K + first) * D;
+        } else if (prefix) {
+            kr = a.k_prefix + ((size_t)g * a.Lp + first) * D;
+            vr = a.v_prefix + ((size_t)g * a.Lp + first) * D;
+        } else {
+            int len;
+            asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(len) : "l"(a.local_len + b));
+            rows = min(Gm::TS, min(max(len, 0), a.Tmax) - first);
+            kr = a.k_cache + (((size_t)b * a.Hkv + g) * a.Tmax + first) * D;
+            vr = a.v_cache + (((size_t)b * a.Hkv + g) * a.Tmax + first) * D;
+        }
+        constexpr int LPR = Gm::ROWB / 128;  // 128-byte lines per row
+        for (int i = tid; i < rows * LPR; i += kThreads) {
+            const size_t off = (size_t)i * 64;  // elements: one line
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(kr + off));
+            if (vr) asm volatile("prefetch.global.L2 [%0];" ::"l"(vr + off));
+        }
+    }
     pdl_wait();
     pdl_launch_dependents();
     if (!scan && !prefix) valid = min(Gm::TS, min(max(__ldg(a.local_len + b), 0), a.Tmax) - first);
@@ -583,6 +613,11 @@ cudaError_t asm_decode_tc_launch(int mode, const void *q, const void *centroids,
     const TcWs w = tc_ws_layout(mode, B, Hq, K, Lp, Tmax, d);
     tc::Args a{};
     a.q = (const __nv_bfloat16 *)q;
+    a.centroids = (const __nv_bfloat16 *)centroids;
+    a.k_cache = (const __nv_bfloat16 *)k_cache;
+    a.v_cache = (const __nv_bfloat16 *)v_cache;
+    a.k_prefix = (const __nv_bfloat16 *)k_prefix;
+    a.v_prefix = (const __nv_bfloat16 *)v_prefix;
     a.a_bar = (const __nv_bfloat16 *)a_bar;
     a.logz_bar = logz_bar;
     a.local_len = local_len;
