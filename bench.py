@@ -10,6 +10,7 @@ replayed from a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl asm|reference]
     python bench.py --only states|assign|seed [--steps K] [--warmup W]
+    python bench.py --sweep [--steps K] [--warmup W]
 
 Prints ONE JSON line (rank 0).  `value` is decode query-heads/s over all
 ranks (each rank runs its own independent replica: weak scaling), timed with
@@ -357,6 +358,99 @@ def run_stage(name, steps, warmup):
     print(json.dumps(out))
 
 
+def run_sweep(steps, warmup):
+    """ASM decode over the 36-point grid of the 32-layer sweep (B x K x T at the
+    LLaMA layer shape), and full attention over an explicit 32K prefix plus
+    the local tokens at B = 1.  Each point cycles enough distinct layer
+    buffers (at least two, at least 3x L2 in all, at most the layer count and
+    60% of free HBM) that every step streams from HBM; inputs are generated on
+    the device.  Times are CUDA events around `steps` graph replays of all
+    layers, after `warmup` replays."""
+    from long_prefix_attention_b200 import ops
+    cfg = inputs.CONFIGS[4]
+    layers, Hq, Hkv, d, Lp = cfg["layers"], cfg["Hq"], cfg["Hkv"], cfg["d"], cfg["Lp"]
+    hbm, tf, tfs, src = peaks()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+
+    def time_graph(run_layer, nbuf):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for i in range(nbuf):
+                run_layer(i)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for l in range(layers):
+                run_layer(l % nbuf)
+        secs = time_steps(g.replay, steps, max(3, warmup), 1)
+        del g
+        return secs / (steps * layers)
+
+    def nbuf_for(bytes_per_layer, mem_per_layer):
+        free, _ = torch.cuda.mem_get_info()
+        n = max(2, math.ceil(3 * l2 / bytes_per_layer))
+        return max(1, min(layers, n, int(0.6 * free // mem_per_layer)))
+
+    points = []
+    for B in cfg["B"]:
+        for K in cfg["K"]:
+            for T in cfg["T"]:
+                byt = decode_bytes(B, Hq, Hkv, K, T, d)
+                mem = 2 * Hq * K * d * 2 + Hq * K * 4 + 2 * B * Hkv * T * d * 2
+                nbuf = nbuf_for(byt, mem)
+                bufs = []
+                for i in range(nbuf):
+                    L = inputs.decode_layer_device(cfg, inputs.BASE_SEED + 5000 + i, B, K, T)
+                    L["out"] = torch.empty_like(L["q"])
+                    L["ws"] = ops.alloc_workspace(ops.asm_decode_workspace_size(B, Hq, Hkv, K, T, d, L["q"].dtype),
+                                                  "cuda")
+                    bufs.append(L)
+
+                def asm_layer(i, bufs=bufs):
+                    L = bufs[i]
+                    ops.asm_decode_step(L["q"], L["centroids"], L["a_bar"], L["logz_bar"], L["k_cache"],
+                                        L["v_cache"], L["local_len"], L["scale"], L["out"], L["ws"], flags=1)
+
+                per = time_graph(asm_layer, nbuf)
+                pt = {"B": B, "K": K, "T": T, "asm_us_per_layer": per * 1e6, "asm_bytes_per_layer": byt,
+                      "asm_gbs": byt / per / 1e9, "asm_frac_of_hbm": byt / per / 1e9 / hbm, "buffers": nbuf}
+                del bufs
+                torch.cuda.empty_cache()
+                if B == 1 and K == cfg["K"][0]:
+                    # full attention: the explicit prefix plus the same local tokens
+                    fbyt = Hkv * Lp * 2 * d * 2 + B * Hkv * T * 2 * d * 2 + 2 * B * Hq * d * 2
+                    fmem = 2 * Hkv * Lp * d * 2 + 2 * B * Hkv * T * d * 2
+                    fnb = nbuf_for(fbyt, fmem)
+                    fb = []
+                    for i in range(fnb):
+                        L = inputs.decode_layer_device(cfg, inputs.BASE_SEED + 6000 + i, B, 1, T, Lp=Lp)
+                        L["out"] = torch.empty_like(L["q"])
+                        L["ws"] = ops.alloc_workspace(
+                            ops.asm_flash_decode_workspace_size(B, Hq, Hkv, Lp, T, d, L["q"].dtype), "cuda")
+                        fb.append(L)
+
+                    def fa_layer(i, fb=fb):
+                        L = fb[i]
+                        ops.asm_flash_decode(L["q"], L["k_prefix"], L["v_prefix"], L["k_cache"], L["v_cache"],
+                                             L["local_len"], L["scale"], L["out"], L["ws"])
+
+                    fper = time_graph(fa_layer, fnb)
+                    pt.update({"full_us_per_layer": fper * 1e6, "full_bytes_per_layer": fbyt,
+                               "full_gbs": fbyt / fper / 1e9, "speedup_vs_full": fper / per})
+                    del fb
+                    torch.cuda.empty_cache()
+                points.append(pt)
+                print(json.dumps(pt), file=sys.stderr, flush=True)
+    line = {"sweep": cfg["name"], "layers": layers, "prefix_len_full_attention": Lp, "steps": steps,
+            "warmup": max(3, warmup), "hbm_peak_gbs": hbm, "peak_source": src,
+            "note": "full attention timed at B=1, where its shared prefix is read once per layer; its "
+                    "prefix units are per batch row",
+            "points": points}
+    print(json.dumps(line))
+
+
 # -------------------------------------------------------------------- main --
 
 def main():
@@ -373,9 +467,14 @@ def main():
                          "preceding kernel finishes")
     ap.add_argument("--only", choices=["states", "assign", "seed"],
                     help="time one build stage alone (single-kernel profiling) and exit")
+    ap.add_argument("--sweep", action="store_true",
+                    help="decode over the 36-point B x K x T grid (and full attention at B=1) and exit")
     args = ap.parse_args()
     if args.only:
         run_stage(args.only, args.steps, args.warmup)
+        return
+    if args.sweep:
+        run_sweep(args.steps, args.warmup)
         return
     cfg = inputs.CONFIGS[1]
     world, rank, local = dist_setup(args.gpus)

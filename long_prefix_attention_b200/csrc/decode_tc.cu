@@ -405,41 +405,55 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
 
 // ----------------------------------------------------------- merge kernel --
 //
-// One CTA of D threads per (b, h); thread t owns output dim t.
+// One CTA per (b, h) of SG x D threads: thread (sg, t) owns output dim t of
+// the attention partials sg, sg + SG, ...; it keeps kMergeSlots of them in
+// flight per round.  SG grows with the partial count (1 for up to 32 partials,
+// up to 8 for 256 and more), so a long local window or prefix does not turn
+// the merge into a serial loop.
 
 constexpr int kMergeSlots = 32;  // partial rows a thread keeps in flight
+constexpr int kMergeMaxSG = 8;   // slot groups per CTA (up to 8 x D threads)
+constexpr int kMergeSml = 2048;  // (m, l) pairs staged in shared memory
 
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kMergeMaxSG * D)
 asm_decode_merge(const Args a) {
     const int bh = blockIdx.x;
     const int b = bh / a.Hq, h = bh - b * a.Hq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int NW = D / 32;
-    __shared__ float red_m[NW];
+    const int NT = blockDim.x, SG = NT / D, sg = tid / D, t = tid - sg * D;
+    constexpr int MW = kMergeMaxSG * D / 32;
+    __shared__ float red_m[MW];
+    __shared__ float2 sb[MW];
     __shared__ int sidx;
-    __shared__ float2 sb[NW];
-    __shared__ float2 sml[kMergeSlots];
+    __shared__ float sM;
+    __shared__ float2 sml[kMergeSml];
+    __shared__ float so[kMergeMaxSG][D];
+    __shared__ float sl[kMergeMaxSG];
     const int nslots = a.nP + a.nA;
     pdl_wait();
     pdl_launch_dependents();
-    // ---- round 1: every partial of (b, h)
+    // ---- round 1: the centroid scores, the attention maxima, and each
+    //      thread's first kMergeSlots partials
     float2 best = make_float2(kNegInf, __int_as_float(0x7fffffff));
     if (a.mode == 0) {
-        for (int s = tid; s < a.nS; s += D) {
+        for (int s = tid; s < a.nS; s += NT) {
             const float2 v = __ldcg(a.ws_srch + (size_t)bh * a.nS + s);
             if (better(v.x, __float_as_int(v.y), best.x, __float_as_int(best.y))) best = v;
         }
     }
     const float2 *mlp = a.ws_ml + (size_t)bh * nslots;
-    const float *op = a.ws_o + (size_t)bh * nslots * D + tid;
+    const float *op = a.ws_o + (size_t)bh * nslots * D + t;
     float ov[kMergeSlots];
 #pragma unroll
-    for (int s = 0; s < kMergeSlots; ++s) ov[s] = s < nslots ? __ldcg(op + (size_t)s * D) : 0.f;
+    for (int k = 0; k < kMergeSlots; ++k) {
+        const int s = sg + SG * k;
+        ov[k] = s < nslots ? __ldcg(op + (size_t)s * D) : 0.f;
+    }
     float mloc = kNegInf;
-    for (int s = tid; s < nslots; s += D) {
+    for (int s = tid; s < nslots; s += NT) {
         const float2 ml = __ldcg(mlp + s);
-        if (s < kMergeSlots) sml[s] = ml;
+        if (s < kMergeSml) sml[s] = ml;
         if (ml.y > 0.f) mloc = fmaxf(mloc, ml.x);
     }
     // block reductions: arg-max of the scores, max of the attention partials
@@ -457,42 +471,57 @@ asm_decode_merge(const Args a) {
             float s0 = kNegInf;
             int i0 = 0x7fffffff;
             float m0 = kNegInf;
-            for (int w = 0; w < NW; ++w) {
+            for (int w = 0; w < NT / 32; ++w) {
                 if (better(sb[w].x, __float_as_int(sb[w].y), s0, i0)) { s0 = sb[w].x; i0 = __float_as_int(sb[w].y); }
                 m0 = fmaxf(m0, red_m[w]);
             }
             sidx = (i0 == 0x7fffffff) ? 0 : i0;
-            red_m[0] = m0;
+            sM = m0;
         }
         __syncthreads();
     }
     const int idx = sidx;
-    const float M = red_m[0];
+    const float M = sM;
     // ---- round 2: the retrieved state (issued before the weighted sums)
     float zb2 = kNegInf, ab = 0.f;
-    if (a.mode == 0) {
+    if (a.mode == 0 && sg == 0) {
         zb2 = __ldg(a.logz_bar + (size_t)h * a.K + idx) * kLog2e;
-        ab = __bfloat162float(a.a_bar[((size_t)h * a.K + idx) * D + tid]);
+        ab = __bfloat162float(a.a_bar[((size_t)h * a.K + idx) * D + t]);
     }
     float L = 0.f, o = 0.f;
     if (M != kNegInf) {
+        for (int k0 = 0;; k0 += kMergeSlots) {
+            if (k0 > 0) {
+                if (sg + SG * k0 >= nslots) break;
 #pragma unroll
-        for (int s = 0; s < kMergeSlots; ++s) {
-            if (s >= nslots) break;
-            const float2 ml = sml[s];
-            if (ml.y > 0.f) {
-                const float w = ex2f(ml.x - M);
-                L += ml.y * w;
-                o = fmaf(w, ov[s], o);
+                for (int k = 0; k < kMergeSlots; ++k) {
+                    const int s = sg + SG * (k0 + k);
+                    ov[k] = s < nslots ? __ldcg(op + (size_t)s * D) : 0.f;
+                }
             }
+#pragma unroll
+            for (int k = 0; k < kMergeSlots; ++k) {
+                const int s = sg + SG * (k0 + k);
+                if (s >= nslots) break;
+                const float2 ml = s < kMergeSml ? sml[s] : __ldcg(mlp + s);
+                if (ml.y > 0.f) {
+                    const float w = ex2f(ml.x - M);
+                    L += ml.y * w;
+                    o = fmaf(w, ov[k], o);
+                }
+            }
+            if (sg + SG * (k0 + kMergeSlots) >= nslots) break;
         }
-        for (int s = kMergeSlots; s < nslots; ++s) {  // more than 32 partials
-            const float2 ml = __ldcg(mlp + s);
-            if (ml.y > 0.f) {
-                const float w = ex2f(ml.x - M);
-                L += ml.y * w;
-                o = fmaf(w, __ldcg(op + (size_t)s * D), o);
-            }
+    }
+    // slot groups meet in shared memory
+    if (SG > 1) {
+        so[sg][t] = o;
+        if (t == 0) sl[sg] = L;
+        __syncthreads();
+        if (sg != 0) return;
+        for (int gg = 1; gg < SG; ++gg) {
+            o += so[gg][t];
+            L += sl[gg];
         }
     }
     const float zl2 = (L > 0.f) ? M + lg2f(L) : kNegInf;
@@ -510,8 +539,8 @@ asm_decode_merge(const Args a) {
         lse2 = zl2;
         res = loc;
     }
-    a.out[(size_t)bh * D + tid] = __float2bfloat16_rn(res);
-    if (tid == 0) {
+    a.out[(size_t)bh * D + t] = __float2bfloat16_rn(res);
+    if (t == 0) {
         if (a.lse_out) a.lse_out[bh] = lse2 * kLn2;
         if (a.idx_out && a.mode == 0) a.idx_out[bh] = idx;
     }
@@ -577,8 +606,12 @@ cudaError_t tc_launch(tc::Args a, const void *centroids, const void *k_prefix, c
     cudaError_t e = cudaLaunchKernelEx(&c1, k1, a, maps);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t c2 = {};
+    // slot groups of the merge: one per 32 partials, at most kMergeMaxSG
+    const int nslots = a.nP + a.nA;
+    int sg = 1;
+    while (sg < tc::kMergeMaxSG && sg * tc::kMergeSlots < nslots) sg *= 2;
     c2.gridDim = dim3(a.B * a.Hq);
-    c2.blockDim = dim3(D);
+    c2.blockDim = dim3(sg * D);
     c2.stream = st;
     c2.attrs = attr;
     c2.numAttrs = 1;

@@ -106,6 +106,42 @@ def decode_inputs(cfg: dict, seed: int | None = None, B: int | None = None,
     return ins
 
 
+def decode_layer_device(cfg: dict, seed: int, B: int, K: int, T: int, device="cuda", Lp: int = 0) -> dict:
+    """One decode layer's inputs generated directly on the device (timing
+    workloads of gigabytes, where host generation would dominate): the same
+    distributions as :func:`decode_inputs` (N(0,1) centroids, states and
+    cache; logZ_bar ~ U(lo, hi); queries from a Gaussian mixture), drawn from
+    a seeded device generator, so the values differ from the host ones.
+    With Lp > 0 also an explicit prefix K/V [Hkv, Lp, d]."""
+    Hq, Hkv, d = cfg["Hq"], cfg["Hkv"], cfg["d"]
+    dt = torch.bfloat16 if cfg["dtype"] == "bf16" else torch.float32
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) & 0x7FFFFFFFFFFFFFFF)
+
+    def nrm(*shape):
+        return torch.randn(*shape, generator=g, device=device, dtype=torch.float32).to(dt)
+
+    means = torch.randn(Hq, cfg["n_mix"], d, generator=g, device=device)
+    comp = torch.randint(0, cfg["n_mix"], (Hq, B), generator=g, device=device)
+    q = means[torch.arange(Hq, device=device)[:, None], comp] + cfg["sigma"] * torch.randn(
+        Hq, B, d, generator=g, device=device)
+    lo, hi = cfg.get("logz_lo", 5.0), cfg.get("logz_hi", 10.0)
+    out = dict(
+        q=q.transpose(0, 1).contiguous().to(dt),
+        centroids=nrm(Hq, K, d),
+        a_bar=nrm(Hq, K, d),
+        logz_bar=lo + (hi - lo) * torch.rand(Hq, K, generator=g, device=device),
+        k_cache=nrm(B, Hkv, T, d),
+        v_cache=nrm(B, Hkv, T, d),
+        local_len=torch.full((B,), T, dtype=torch.int32, device=device),
+        scale=1.0 / math.sqrt(d),
+    )
+    if Lp > 0:
+        out["k_prefix"] = nrm(Hkv, Lp, d)
+        out["v_prefix"] = nrm(Hkv, Lp, d)
+    return out
+
+
 def build_inputs(cfg: dict, seed: int | None = None, N: int | None = None,
                  L: int | None = None, K: int | None = None, H: int | None = None) -> dict:
     """Calibration queries, prefix K/V and k-means++ draws of the memory build."""
