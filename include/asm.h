@@ -90,6 +90,10 @@ typedef enum { ASM_ZBAR_MEAN = 0, ASM_ZBAR_SUM = 1 } asm_zbar_mode;
  *   a      [Hq, N, d]  dt   output / in-out when accumulate
  *   logz   [Hq, N]     fp32 output / in-out when accumulate
  * L == 0 with accumulate == 0 writes the empty state.  No workspace.
+ * bf16 with d = 128 runs on the tcgen05 tensor cores (bf16 products, fp32
+ * accumulators and softmax statistics); a tensor-core pipeline wait that times
+ * out writes NaN into logz of the rows it covers.  Other cases run on CUDA
+ * cores in fp32.
  */
 asm_status asm_build_states(const void *q, const void *k, const void *v,
                             int Hq, int Hkv, int N, int L, int d, float scale,
@@ -261,6 +265,11 @@ asm_status asm_decode_step_noalloc(const void *q, const void *centroids,
  *   other arguments as asm_decode_step; lse_out may be NULL.
  *   ws asm_flash_decode_workspace_size(...) bytes, zeroed once by
  *   asm_workspace_init.
+ * bf16 with d = 128 and B >= 2: the prefix runs on the tcgen05 tensor cores
+ * in chunks, with the B * (Hq / Hkv) query rows of each KV head as the rows
+ * of one tile, then the local tokens and the merge: three kernel launches.
+ * Otherwise the prefix and local tokens are split into units that each
+ * serve one row (the rows of one prefix unit run together): two launches.
  */
 size_t asm_flash_decode_workspace_size(int B, int Hq, int Hkv, int Lp,
                                        int Tmax, int d, asm_dtype dt);

@@ -192,14 +192,35 @@ __device__ __forceinline__ void merge_weights(float za, float zb, float &wa, flo
     wb = eb / (ea + eb);
 }
 
+struct Params {
+    int Hq, Hkv, N, L;            // states: queries [Hq][N][d], keys [Hkv][L][d]
+    float sl2;                    // softmax scale * log2(e)
+    int accumulate;
+    __nv_bfloat16 *a;             // states: [Hq][N][d]
+    float *logz;                  // states: [Hq][N]
+    // decode partials: the (row b, head) pairs of KV group blockIdx.y against
+    // prefix chunk blockIdx.z (keys [z * chunk, z * chunk + chunk) of L)
+    int B, G, chunk, nslots;
+    float2 *ws_ml;                // [B][Hq][nslots] (m in base 2, l)
+    float *ws_o;                  // [B][Hq][nslots][d]
+};
+
+// MODE 0: prefix states of calibration queries (a, logZ), with the chunk merge.
+// MODE 1: decode partials of a shared prefix chunk for the batch's query rows:
+//         (m = log2 of the chunk's Z, l = 1, o = a), the form the decode merge reads.
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int L, float sl2, int accumulate,
-                 __nv_bfloat16 *__restrict__ a, float *__restrict__ logz) {
+states_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
     extern __shared__ unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.y, g = h / (Hq / Hkv);
+    const int Hq = p.Hq, N = p.N, accumulate = p.accumulate;
+    const float sl2 = p.sl2;
+    const int h = blockIdx.y;
+    const int g = MODE == 0 ? h / (Hq / p.Hkv) : blockIdx.y;
     const int n0 = blockIdx.x * (2 * kQT);
+    const int k0 = MODE == 0 ? 0 : blockIdx.z * p.chunk;                // first key of this CTA
+    const int L = MODE == 0 ? p.L : min(p.chunk, p.L - k0);             // keys of this CTA
     const int J = (L + kKT - 1) / kKT;
 
     if (tid == 0) {
@@ -231,16 +252,21 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
         if (lane == 0) {
             mbar_arrive_expect_tx(&sm.q_full, 2 * kTile);
             for (int x = 0; x < 2; ++x)
-                for (int dh = 0; dh < 2; ++dh)
-                    tma_load_3d(sm.q[x] + dh * kBox, &maps.q, dh * 64, n0 + x * kQT, h, &sm.q_full);
+                for (int dh = 0; dh < 2; ++dh) {
+                    if (MODE == 0)
+                        tma_load_3d(sm.q[x] + dh * kBox, &maps.q, dh * 64, n0 + x * kQT, h, &sm.q_full);
+                    else  // 128 (row, head) pairs of group g: rows (n0 + x * kQT) / G ..
+                        tma_load_4d(sm.q[x] + dh * kBox, &maps.q, dh * 64, 0, g, (n0 + x * kQT) / p.G,
+                                    &sm.q_full);
+                }
             // ring item n: K_{n/2} for even n, V_{n/2} for odd n
             for (int n = 0; n < 2 * J; ++n) {
                 const int slot = n % kRing;
                 if (n >= kRing) ok &= mbar_wait(&sm.kv_empty[slot], ((n / kRing) - 1) & 1);
                 mbar_arrive_expect_tx(&sm.kv_full[slot], kTile);
                 const CUtensorMap *mp = (n & 1) ? &maps.v : &maps.k;
-                tma_load_3d(sm.kv[slot], mp, 0, (n >> 1) * kKT, g, &sm.kv_full[slot]);
-                tma_load_3d(sm.kv[slot] + kBox, mp, 64, (n >> 1) * kKT, g, &sm.kv_full[slot]);
+                tma_load_3d(sm.kv[slot], mp, 0, k0 + (n >> 1) * kKT, g, &sm.kv_full[slot]);
+                tma_load_3d(sm.kv[slot] + kBox, mp, 64, k0 + (n >> 1) * kKT, g, &sm.kv_full[slot]);
             }
         }
     } else if (warp == 1) {
@@ -396,6 +422,32 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
         // ------------------------------------------------------ epilogue
         ok &= mbar_wait(&sm.o_full[x], 0);
         tc_fence_after();
+        if (MODE == 1) {
+            // row -> (batch row b, head g * G + hh); rows past the batch are padding
+            const int r = n0 + x * kQT + row;
+            const int b = r / p.G, hh = r - b * p.G;
+            const bool live = b < p.B;
+            const size_t bh = (size_t)b * Hq + (size_t)g * p.G + hh;
+            const size_t slot = (size_t)blockIdx.z;
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            float *orow = p.ws_o + ((live ? bh : 0) * p.nslots + slot) * kD;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kD; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(t_o + (uint32_t)c0, o);
+                tmem_wait_ld();
+                if (live) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4 *>(orow + c0 + i) =
+                            make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                                        __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                }
+            }
+            if (live)
+                p.ws_ml[bh * p.nslots + slot] = (l > 0.f && ok) ? make_float2(m_used + log2f(l), 1.f)
+                                                                : make_float2(ok ? kNegInf : __int_as_float(0x7fc00000), 0.f);
+        } else {
         const int n = n0 + x * kQT + row;
         const bool live = n < N;
         const size_t grow = (size_t)h * N + (size_t)(live ? n : 0);
@@ -404,10 +456,10 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
         float wa = 0.f, wb = 1.f;
         if (accumulate && live) {
             float zz;
-            merge_weights(logz[grow], z, wa, wb, zz);
+            merge_weights(p.logz[grow], z, wa, wb, zz);
             z = zz;
         }
-        __nv_bfloat16 *arow = a + grow * kD;
+        __nv_bfloat16 *arow = p.a + grow * kD;
 #pragma unroll 1
         for (int c0 = 0; c0 < kD; c0 += 32) {
             uint32_t o[32];
@@ -443,7 +495,8 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
                         make_uint4(packed[i], packed[i + 1], packed[i + 2], packed[i + 3]);
             }
         }
-        if (live) logz[grow] = ok ? z : __int_as_float(0x7fc00000);
+        if (live) p.logz[grow] = ok ? z : __int_as_float(0x7fc00000);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -456,6 +509,7 @@ states_tc_kernel(const __grid_constant__ Maps maps, int Hq, int Hkv, int N, int 
 }  // namespace stc
 
 bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows);
+bool make_map_qgroups(CUtensorMap *m, const void *q, int B, int Hkv, int G, int d);
 
 }  // namespace asmk
 
@@ -468,11 +522,45 @@ cudaError_t asm_build_states_tc_launch(const void *q, const void *k, const void 
         !make_map_3d(&maps.v, v, stc::kD, L, Hkv, stc::kKT))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(stc::Smem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(stc::states_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(stc::states_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
+    stc::Params p{};
+    p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.L = L;
+    p.sl2 = scale * kLog2e;
+    p.accumulate = accumulate;
+    p.a = static_cast<__nv_bfloat16 *>(a);
+    p.logz = logz;
     dim3 grid((N + 2 * stc::kQT - 1) / (2 * stc::kQT), Hq);
-    stc::states_tc_kernel<<<grid, stc::kThreads, smem, st>>>(maps, Hq, Hkv, N, L, scale * kLog2e, accumulate,
-                                                             static_cast<__nv_bfloat16 *>(a), logz);
+    stc::states_tc_kernel<0><<<grid, stc::kThreads, smem, st>>>(maps, p);
+    return cudaGetLastError();
+}
+
+// Decode partials of a shared explicit prefix for all B rows of a batch:
+// grid (row tiles, Hkv, chunks); partial slot z of pair (b, h) covers keys
+// [z * chunk, z * chunk + chunk).  q [B][Hq][128] bf16, prefix [Hkv][Lp][128].
+cudaError_t asm_prefix_partials_tc_launch(const void *q, const void *k_prefix, const void *v_prefix, int B, int Hq,
+                                          int Hkv, int Lp, int chunk, float scale, float2 *ws_ml, float *ws_o,
+                                          int nslots, cudaStream_t st) {
+    using namespace asmk;
+    const int G = Hq / Hkv;
+    stc::Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!make_map_qgroups(&maps.q, q, B, Hkv, G, stc::kD) ||
+        !make_map_3d(&maps.k, k_prefix, stc::kD, Lp, Hkv, stc::kKT) ||
+        !make_map_3d(&maps.v, v_prefix, stc::kD, Lp, Hkv, stc::kKT))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(stc::Smem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(stc::states_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    stc::Params p{};
+    p.Hq = Hq; p.Hkv = Hkv; p.N = B * G; p.L = Lp;
+    p.sl2 = scale * kLog2e;
+    p.B = B; p.G = G; p.chunk = chunk; p.nslots = nslots;
+    p.ws_ml = ws_ml;
+    p.ws_o = ws_o;
+    dim3 grid((B * G + 2 * stc::kQT - 1) / (2 * stc::kQT), Hkv, (Lp + chunk - 1) / chunk);
+    stc::states_tc_kernel<1><<<grid, stc::kThreads, smem, st>>>(maps, p);
     return cudaGetLastError();
 }

@@ -918,6 +918,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// 4-D bf16 map over decode queries q[B][Hq][d] seen as [B][Hkv][G][d]: a box
+// of 64 columns x G heads x 1 group x 128/G rows holds the 128 (row, head)
+// pairs of one KV group, row-major by (row, head).
+bool make_map_qgroups(CUtensorMap *m, const void *q, int B, int Hkv, int G, int d) {
+    auto fn = encode_fn();
+    if (!fn || q == nullptr || B < 1 || G < 1 || 128 % G != 0) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)Hkv, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2, (cuuint64_t)Hkv * G * d * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, 1, (cuuint32_t)(128 / G)};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D bf16 map [d2][d1][d0] with a box of 64 columns x `rows` rows x 1.
 bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows) {
     auto fn = encode_fn();

@@ -68,6 +68,7 @@ struct Args {
     int metric, mode, flags;
     int nS;                       // centroid units per head (mode 0)
     int nP, nA;                   // prefix / local units per (b, g)
+    int ext_prefix;               // the nP prefix partials come from the batched prefix kernel
     int n_scan;                   // Hq * nS
     float2 *ws_srch;              // [B][Hq][nS]
     float2 *ws_ml;                // [B][Hq][nP+nA]
@@ -118,12 +119,24 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
         valid = min(Gm::CS, a.K - first);
         g = h / G;
     } else {
-        const int v = u - a.n_scan, ns = a.nP + a.nA;
-        const int bg = v / ns;
-        slot = v - bg * ns;
-        b = bg / a.Hkv;
-        g = bg - b * a.Hkv;
-        prefix = slot < a.nP;
+        // prefix units (explicit shared prefix) first, ordered (g, slot, b)
+        // with b fastest: the B rows that read one prefix tile run together,
+        // so the tile comes from HBM once and from L2 for the other rows;
+        // then the local units, ordered (b, g, slot)
+        const int v = u - a.n_scan, npu = a.ext_prefix ? 0 : a.B * a.Hkv * a.nP;
+        if (v < npu) {
+            b = v % a.B;
+            const int r = v / a.B;
+            slot = r % a.nP;
+            g = r / a.nP;
+            prefix = true;
+        } else {
+            const int w = v - npu, bg = w / a.nA;
+            slot = a.nP + (w - bg * a.nA);
+            b = bg / a.Hkv;
+            g = bg - b * a.Hkv;
+            prefix = false;
+        }
         first = (prefix ? slot : slot - a.nP) * Gm::TS;
         valid = prefix ? min(Gm::TS, a.Lp - first) : Gm::TS;  // refined by the row length below
     }
@@ -583,7 +596,7 @@ cudaError_t tc_launch(tc::Args a, const void *centroids, const void *k_prefix, c
     if (a.mode == 1 && a.Lp > 0 && (!make_map_3d(&maps.kp, k_prefix, D, a.Lp, a.Hkv, Gm::TS) ||
                                     !make_map_3d(&maps.vp, v_prefix, D, a.Lp, a.Hkv, Gm::TS)))
         return cudaErrorInvalidValue;
-    const int units = a.n_scan + a.B * a.Hkv * (a.nP + a.nA);
+    const int units = a.n_scan + a.B * a.Hkv * ((a.ext_prefix ? 0 : a.nP) + a.nA);
     const size_t smem = 1024 + tc::kUnit + 16 + sizeof(float) * tc::kWarps * G * (D + 2) +
                         sizeof(float2) * tc::kWarps * a.B;
     auto k1 = tc::asm_decode_units<D, G>;
@@ -603,8 +616,10 @@ cudaError_t tc_launch(tc::Args a, const void *centroids, const void *k_prefix, c
     c1.stream = st;
     c1.attrs = attr;
     c1.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&c1, k1, a, maps);
-    if (e != cudaSuccess) return e;
+    if (units > 0) {
+        cudaError_t e = cudaLaunchKernelEx(&c1, k1, a, maps);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t c2 = {};
     // slot groups of the merge: one per 32 partials, at most kMergeMaxSG
     const int nslots = a.nP + a.nA;
@@ -673,6 +688,24 @@ cudaError_t asm_decode_tc_launch(int mode, const void *q, const void *centroids,
     a.ws_ml = reinterpret_cast<float2 *>(base + w.off_ml);
     a.ws_o = reinterpret_cast<float *>(base + w.off_o);
     const int G = Hq / Hkv;
+    if (mode == 1 && Lp > 0 && B >= 2 && d == 128) {
+        // A shared prefix read by several rows: tensor-core prefix chunks for
+        // all B * G query rows of each KV group at once (the prefix streams
+        // once per layer), about two waves of CTAs, written as the first
+        // partial slots; the units kernel then covers the local tokens only.
+        static int sms = 0;
+        if (sms == 0 && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, 0) != cudaSuccess) sms = 148;
+        const int row_tiles = (B * G + 255) / 256;
+        int nch = (2 * sms + Hkv * row_tiles - 1) / (Hkv * row_tiles);
+        int chunk = (Lp + nch - 1) / nch;
+        chunk = ((chunk + 127) / 128) * 128;
+        nch = (Lp + chunk - 1) / chunk;
+        a.nP = nch;
+        a.ext_prefix = 1;
+        cudaError_t e = asm_prefix_partials_tc_launch(q, k_prefix, v_prefix, B, Hq, Hkv, Lp, chunk, scale, a.ws_ml,
+                                                      a.ws_o, a.nP + a.nA, st);
+        if (e != cudaSuccess) return e;
+    }
     if (d == 128) return tc_launch_g<128>(G, a, centroids, k_prefix, v_prefix, k_cache, v_cache, st);
     return tc_launch_g<64>(G, a, centroids, k_prefix, v_prefix, k_cache, v_cache, st);
 }

@@ -39,6 +39,11 @@ cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v,
 cudaError_t asm_build_states_tc_launch(const void *q, const void *k, const void *v, int Hq, int Hkv, int N, int L,
                                        float scale, int accumulate, void *a, float *logz, cudaStream_t st);
 
+// build_states_tc.cu: decode partials of a shared prefix for all B rows (bf16, d = 128)
+cudaError_t asm_prefix_partials_tc_launch(const void *q, const void *k_prefix, const void *v_prefix, int B, int Hq,
+                                          int Hkv, int Lp, int chunk, float scale, float2 *ws_ml, float *ws_o,
+                                          int nslots, cudaStream_t st);
+
 // kmeans.cu
 size_t asm_kmeanspp_ws_bytes(int H, int N, int d, int K);
 cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const double *u,

@@ -171,6 +171,22 @@ def test_flash_decode_matches_full_attention(dt, Lp, T, B):
     assert max_abs(f64(lse), ref_lse) <= tol
 
 
+def test_flash_decode_batch_rows_share_the_prefix():
+    """Five rows with ragged local lengths over one explicit prefix whose
+    length is not a multiple of the tile: the rows that read a prefix tile
+    run together, each with its own local window."""
+    lens = [130, 0, 64, 129, 1]
+    ins = small_case("bf16", B=5, K=4, T=130, local_len=lens)
+    kp = inputs.normal(7, "kp", (2, 700, 128), "bf16")
+    vp = inputs.normal(7, "vp", (2, 700, 128), "bf16")
+    out, lse = run_flash(dev(ins["q"]), dev(kp), dev(vp), dev(ins["k_cache"]), dev(ins["v_cache"]),
+                         dev(ins["local_len"]), ins["scale"])
+    ref, ref_lse = O.full_attention(ins["q"], kp, vp, ins["k_cache"], ins["v_cache"], ins["local_len"],
+                                    ins["scale"])
+    assert max_abs(f64(out), ref) <= 2e-2
+    assert max_abs(f64(lse), ref_lse) <= 2e-2
+
+
 def test_identity_memory_recovers_full_attention():
     """K = N memory built on the GPU (states of the calibration queries
     themselves, singleton clusters): a decode query equal to calibration
