@@ -437,6 +437,98 @@ void oracle_aggregate(const double *A, const double *logZ,
 }
 
 /*
+ * Score of centre c for query x by the retrieval rule of oracle_assign,
+ * oriented so that smaller is better: |x - c|^2 (L2) or -<x, c>/|c| (cosine).
+ */
+static double retrieval_score(const double *x, const double *c, int d, int metric)
+{
+    if (metric == 0) return sqdist(x, c, d);
+    {
+        double nc = sqrt(dot(c, c, d));
+        return nc > 0.0 ? -dot(x, c, d) / nc : 0.0;
+    }
+}
+
+/*
+ * Two-level centroid search, the hierarchical lookup the pages name
+ * ("Complejidad": retrieval in O(log K) with a hierarchical index) without
+ * giving its construction; the plainest two-level reading is taken.  The K
+ * centres of a head are grouped into K1 clusters whose members are the rows
+ * seg_off[j] .. seg_off[j+1]-1 of the centre array (ordered by cluster), each
+ * cluster with a super-centre S[j].  The query scores every super-centre
+ * with the retrieval rule, keeps the P best clusters (ties to the smaller
+ * cluster index), and returns the best row among the members of those
+ * clusters by the same rule (ties to the smaller row).
+ * q[d], S[K1,d], seg_off[K1+1], C[K,d] -> idx, sel[P] (best cluster first),
+ * gap_sel: relative gap between the P-th and (P+1)-th cluster score (+inf
+ * when P >= K1), gap_idx: relative gap between the best and second-best
+ * member score (+inf with a single member).
+ */
+static void index_search_one(const double *q, const double *S, const int32_t *seg_off, const double *C,
+                             int K1, int d, int P, int metric, int32_t *idx, int32_t *sel, double *gap_sel,
+                             double *gap_idx)
+{
+    double *sc = (double *)malloc(sizeof(double) * (size_t)K1);
+    unsigned char *used = (unsigned char *)calloc((size_t)K1, 1);
+    int j, p, Psel = P < K1 ? P : K1;
+    double last = 0.0, next = INFINITY;
+    for (j = 0; j < K1; j++) sc[j] = retrieval_score(q, S + (size_t)j * d, d, metric);
+    for (p = 0; p < Psel; p++) {
+        int bj = -1;
+        for (j = 0; j < K1; j++)
+            if (!used[j] && (bj < 0 || sc[j] < sc[bj])) bj = j;
+        used[bj] = 1;
+        sel[p] = bj;
+        last = sc[bj];
+    }
+    for (p = Psel; p < P; p++) sel[p] = -1;
+    for (j = 0; j < K1; j++)
+        if (!used[j] && sc[j] < next) next = sc[j];
+    *gap_sel = (next - last) / (fabs(last) > 1e-30 ? fabs(last) : 1e-30);
+    {
+        int best = -1, r;
+        double b1 = INFINITY, b2 = INFINITY;
+        /* rows of the selected clusters, in row order (clusters are ordered) */
+        for (j = 0; j < K1; j++) {
+            if (!used[j]) continue;
+            for (r = seg_off[j]; r < seg_off[j + 1]; r++) {
+                double v = retrieval_score(q, C + (size_t)r * d, d, metric);
+                if (best < 0 || v < b1) {
+                    b2 = b1;
+                    b1 = v;
+                    best = r;
+                } else if (v < b2) {
+                    b2 = v;
+                }
+            }
+        }
+        *idx = best < 0 ? 0 : best;
+        *gap_idx = (b2 - b1) / (fabs(b1) > 1e-30 ? fabs(b1) : 1e-30);
+    }
+    free(sc);
+    free(used);
+}
+
+/*
+ * index_search_one for every batch row b and query head h:
+ * q[B,Hq,d], S[Hq,K1,d], seg_off[Hq,K1+1], C[Hq,K,d] -> idx[B,Hq],
+ * sel[B,Hq,P], gap_sel[B,Hq], gap_idx[B,Hq].
+ */
+void oracle_index_search(const double *q, const double *S, const int32_t *seg_off, const double *C, int B,
+                         int Hq, int K, int K1, int d, int P, int metric, int32_t *idx, int32_t *sel,
+                         double *gap_sel, double *gap_idx)
+{
+    long bh;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (bh = 0; bh < (long)B * Hq; bh++) {
+        int h = (int)(bh % Hq);
+        index_search_one(q + (size_t)bh * d, S + (size_t)h * K1 * d, seg_off + (size_t)h * (K1 + 1),
+                         C + (size_t)h * K * d, K1, d, P, metric, idx + bh, sel + (size_t)bh * P,
+                         gap_sel + bh, gap_idx + bh);
+    }
+}
+
+/*
  * One decode step ("Fase de Inferencia Online": Recuperacion, then Fusion).
  * For every batch row b and query head h (KV head g = h / (Hq / Hkv)):
  *   idx      = nearest centre of q[b,h] among C[h,0:K) (oracle_assign rule),

@@ -65,6 +65,7 @@ def _load():
                                       P, P, P, P, P]
         lib.oracle_full_attention.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, D,
                                               P, P]
+        lib.oracle_index_search.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -221,6 +222,24 @@ def decode(q, C, Abar, logZbar, Kc, Vc, local_len, scale: float, metric: int = L
                           K, Tmax, d, float(scale), int(metric), idx_p, _p(out), _p(lse),
                           _p(idx), _p(gap))
     return out, lse, idx, gap
+
+
+def index_search(q, S, seg_off, C, P: int, metric: int = L2):
+    """Two-level centroid search (C oracle ``oracle_index_search``).
+    q[B,Hq,d], S[Hq,K1,d], seg_off[Hq,K1+1] int32, C[Hq,K,d] (rows ordered by
+    cluster) -> idx[B,Hq], sel[B,Hq,P], gap_sel[B,Hq], gap_idx[B,Hq]."""
+    q, S, C = _f64(q), _f64(S), _f64(C)
+    so = _i32(seg_off)
+    B, Hq, d = q.shape
+    K1 = S.shape[1]
+    K = C.shape[1]
+    idx = np.zeros((B, Hq), dtype=np.int32)
+    sel = np.zeros((B, Hq, P), dtype=np.int32)
+    gs = np.zeros((B, Hq))
+    gi = np.zeros((B, Hq))
+    _load().oracle_index_search(_p(q), _p(S), _p(so), _p(C), B, Hq, K, K1, d, int(P), int(metric), _p(idx),
+                                _p(sel), _p(gs), _p(gi))
+    return idx, sel, gs, gi
 
 
 def full_attention(q, Kp, Vp, Kc, Vc, local_len, scale: float):

@@ -380,3 +380,64 @@ def test_decode_search_and_local_only_cases():
     forced = np.zeros((B, Hq), np.int32) + 3
     _, _, idx_f, _ = O.decode(q, C, np.zeros((Hq, K, d)), np.zeros((Hq, K)), Kc, Vc, ll, s, idx_in=forced)
     assert (idx_f == 3).all()
+
+
+# ------------------------------------------------- two-level (hierarchical) search
+
+def test_index_search_hand_case():
+    """Centres on a line: clusters {0, 4} (super-centre 2) and {6, 100}
+    (super-centre 53).  The query 5.2 is nearest to the super-centre 2, so
+    with one cluster kept the search returns 4 (row 1) although 6 (row 2) is
+    the nearest centre; keeping both clusters returns 6.  Distances by hand:
+    super 10.24 vs 2284.84; members 27.04, 1.44 | 0.64, 9063.04."""
+    C = np.array([[[0, 0], [4, 0], [6, 0], [100, 0]]], float)
+    S = np.array([[[2, 0], [53, 0]]], float)
+    so = np.array([[0, 2, 4]], np.int32)
+    q = np.array([[[5.2, 0]]], float)
+    idx, sel, gs, gi = O.index_search(q, S, so, C, 1)
+    assert idx[0, 0] == 1 and sel[0, 0, 0] == 0
+    assert gs[0, 0] == pytest.approx((2284.84 - 10.24) / 10.24)
+    assert gi[0, 0] == pytest.approx((27.04 - 1.44) / 1.44)
+    idx, sel, gs, gi = O.index_search(q, S, so, C, 2)
+    assert idx[0, 0] == 2 and list(sel[0, 0]) == [0, 1]
+    assert np.isinf(gs[0, 0])
+    assert gi[0, 0] == pytest.approx((1.44 - 0.64) / 0.64)
+
+
+def _clustered(rng, H, K, K1, d):
+    """Centres ordered by an arbitrary partition into K1 non-empty clusters."""
+    sizes = rng.multinomial(K - K1, np.ones(K1) / K1) + 1
+    so = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    C = rng.standard_normal((H, K, d))
+    S = rng.standard_normal((H, K1, d))
+    return C, S, np.tile(so, (H, 1))
+
+
+@pytest.mark.parametrize("metric", [O.L2, O.COSINE])
+def test_index_search_keeping_every_cluster_is_the_flat_search(metric):
+    rng = np.random.default_rng(3)
+    H, K, K1, d, B = 3, 97, 9, 16, 5
+    C, S, so = _clustered(rng, H, K, K1, d)
+    q = rng.standard_normal((B, H, d))
+    idx, sel, gs, gi = O.index_search(q, S, so, C, K1, metric)
+    for h in range(H):
+        flat, gap = O.assign(q[:, h], C[h], metric)
+        np.testing.assert_array_equal(idx[:, h], flat)
+        np.testing.assert_allclose(gi[:, h], gap)
+        assert all(sorted(s) == list(range(K1)) for s in sel[:, h])
+
+
+def test_index_search_singleton_clusters_is_the_flat_search():
+    """K1 = K, every centre its own cluster and super-centre, one cluster
+    kept: the first level alone is the flat search."""
+    rng = np.random.default_rng(4)
+    H, K, d, B = 2, 40, 8, 7
+    C = rng.standard_normal((H, K, d))
+    so = np.tile(np.arange(K + 1, dtype=np.int32), (H, 1))
+    q = rng.standard_normal((B, H, d))
+    idx, sel, gs, gi = O.index_search(q, C, so, C, 1)
+    for h in range(H):
+        flat, gap = O.assign(q[:, h], C[h])
+        np.testing.assert_array_equal(idx[:, h], flat)
+        np.testing.assert_array_equal(sel[:, h, 0], flat)
+        np.testing.assert_allclose(gs[:, h], gap)
