@@ -11,6 +11,7 @@ replayed from a CUDA graph.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl asm|reference]
     python bench.py --only states|assign|seed [--steps K] [--warmup W]
     python bench.py --sweep [--steps K] [--warmup W]
+    python bench.py --index [--steps K] [--warmup W]
 
 Prints ONE JSON line (rank 0).  `value` is decode query-heads/s over all
 ranks (each rank runs its own independent replica: weak scaling), timed with
@@ -455,6 +456,120 @@ def run_sweep(steps, warmup):
     print(json.dumps(line))
 
 
+def run_index(steps, warmup, Ps=(4, 8, 16)):
+    """Two-level (hierarchical) search against the flat search at the LLaMA
+    layer shape (B = 1, T = 2048) for K in {1024, 4096, 8192, 16384}: centres
+    drawn from a Gaussian mixture (clustered like k-means centres of real
+    queries), index built by the library's k-means on the centres with
+    K1 = round(sqrt(K)) clusters, memory ordered by cluster.  Times are per
+    layer step over 32 layers in one graph (distinct buffers cycled, each step
+    from HBM); recall@1 is the fraction of 64 x 32 queries from the same
+    mixture whose indexed retrieval equals the flat one."""
+    from long_prefix_attention_b200 import ops
+    cfg = dict(inputs.CONFIGS[1])
+    Hq, Hkv, d, T, layers = cfg["Hq"], cfg["Hkv"], cfg["d"], cfg["T"], 32
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    hbm, tf, tfs, src = peaks()
+
+    def mix(g, n, means):
+        comp = torch.randint(0, means.shape[1], (Hq, n), generator=g, device="cuda")
+        x = means[torch.arange(Hq, device="cuda")[:, None], comp]
+        return (x + 0.3 * torch.randn(Hq, n, d, generator=g, device="cuda")).to(torch.bfloat16)
+
+    def graph_time(run, nbuf):
+        run_all = lambda: [run(i % nbuf) for i in range(layers)]
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            run_all()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            run_all()
+        secs = time_steps(gr.replay, steps, max(3, warmup), 1)
+        del gr
+        return secs / (steps * layers)
+
+    rows = []
+    for K in (1024, 4096, 8192, 16384):
+        K1 = int(round(math.sqrt(K)))
+        per_layer = 2 * Hq * K * d * 2 + Hkv * T * 2 * d * 2
+        nbuf = min(layers, max(2, math.ceil(3 * l2 / per_layer)))
+        bufs = []
+        for i in range(nbuf):
+            g = torch.Generator(device="cuda")
+            g.manual_seed(inputs.BASE_SEED + 7000 + i)
+            means = torch.randn(Hq, 1024, d, generator=g, device="cuda")
+            L = inputs.decode_layer_device(cfg, inputs.BASE_SEED + 7100 + i, 1, K, T)
+            x = mix(g, K, means)
+            u = inputs.kmeanspp_uniforms(inputs.BASE_SEED + 7200 + i, Hq, K1).cuda()
+            init = torch.empty(Hq, K1, dtype=torch.int32, device="cuda")
+            wss = ops.alloc_workspace(ops.asm_kmeanspp_workspace_size(Hq, K, d, K1), "cuda", zero=False)
+            ops.asm_kmeanspp_seed(x, u, init, wss)
+            c = torch.empty(Hq, K1, d, dtype=torch.float32, device="cuda")
+            sdt = torch.empty(Hq, K1, d, dtype=torch.bfloat16, device="cuda")
+            asg = torch.empty(Hq, K, dtype=torch.int32, device="cuda")
+            cnt = torch.empty(Hq, K1, dtype=torch.int32, device="cuda")
+            perm = torch.empty(Hq, K, dtype=torch.int32, device="cuda")
+            seg = torch.empty(Hq, K1 + 1, dtype=torch.int32, device="cuda")
+            wsk = ops.alloc_workspace(ops.asm_kmeans_workspace_size(Hq, K, d, K1), "cuda")
+            ops.asm_kmeans(x, init, 4, c, sdt, asg, cnt, perm, seg, wsk)
+            co, ao, lo = torch.empty_like(x), torch.empty_like(L["a_bar"]), torch.empty_like(L["logz_bar"])
+            ops.asm_index_reorder(perm, x, L["a_bar"], L["logz_bar"], co, ao, lo)
+            L.update(centroids=co, a_bar=ao, logz_bar=lo, supers=sdt, seg=seg, max_seg=int(cnt.max().item()),
+                     q=mix(g, 1, means).transpose(0, 1).contiguous(), out=torch.empty(1, Hq, d, dtype=torch.bfloat16,
+                                                                                      device="cuda"))
+            L["ws"] = ops.alloc_workspace(ops.asm_decode_workspace_size(1, Hq, Hkv, K, T, d, torch.bfloat16), "cuda")
+            bufs.append(L)
+            if i == 0:
+                qr = mix(g, 64, means).transpose(0, 1).contiguous()
+        torch.cuda.synchronize()
+
+        def flat(i):
+            L = bufs[i]
+            ops.asm_decode_step(L["q"], L["centroids"], L["a_bar"], L["logz_bar"], L["k_cache"], L["v_cache"],
+                                L["local_len"], L["scale"], L["out"], L["ws"], flags=1)
+
+        t_flat = graph_time(flat, nbuf)
+        row = {"K": K, "K1": K1, "flat_us_per_layer": t_flat * 1e6, "buffers": nbuf, "indexed": []}
+        L0 = bufs[0]
+        kc64 = torch.zeros(64, Hkv, T, d, dtype=torch.bfloat16, device="cuda")
+        ll64 = torch.full((64,), 1, dtype=torch.int32, device="cuda")
+        ws64 = ops.alloc_workspace(ops.asm_decode_workspace_size(64, Hq, Hkv, K, T, d, torch.bfloat16), "cuda")
+        i_flat = torch.empty(64, Hq, dtype=torch.int32, device="cuda")
+        o64 = torch.empty_like(qr)
+        ops.asm_decode_step(qr, L0["centroids"], L0["a_bar"], L0["logz_bar"], kc64, kc64, ll64, L0["scale"], o64,
+                            ws64, idx_out=i_flat)
+        for P in Ps:
+            for L in bufs:
+                L["wsi"] = ops.alloc_workspace(ops.asm_decode_indexed_workspace_size(
+                    1, Hq, Hkv, K1, P, L["max_seg"], T, d, torch.bfloat16), "cuda")
+
+            def indexed(i, P=P):
+                L = bufs[i]
+                ops.asm_decode_step_indexed(L["q"], L["supers"], L["seg"], P, L["max_seg"], L["centroids"],
+                                            L["a_bar"], L["logz_bar"], L["k_cache"], L["v_cache"], L["local_len"],
+                                            L["scale"], L["out"], L["wsi"])
+
+            t_idx = graph_time(indexed, nbuf)
+            wsr = ops.alloc_workspace(ops.asm_decode_indexed_workspace_size(
+                64, Hq, Hkv, K1, P, L0["max_seg"], T, d, torch.bfloat16), "cuda")
+            i_idx = torch.empty_like(i_flat)
+            ops.asm_decode_step_indexed(qr, L0["supers"], L0["seg"], P, L0["max_seg"], L0["centroids"], L0["a_bar"],
+                                        L0["logz_bar"], kc64, kc64, ll64, L0["scale"], o64, wsr, idx_out=i_idx)
+            torch.cuda.synchronize()
+            recall = (i_idx == i_flat).float().mean().item()
+            row["indexed"].append({"P": P, "us_per_layer": t_idx * 1e6, "speedup": t_flat / t_idx,
+                                   "recall_at_1": recall})
+        rows.append(row)
+        print(json.dumps(row), file=sys.stderr, flush=True)
+        del bufs
+        torch.cuda.empty_cache()
+    print(json.dumps({"index": "two-level search vs flat, LLaMA layer shape, B=1, T=2048, 32 layers",
+                      "steps": steps, "warmup": max(3, warmup), "rows": rows}))
+
+
 # -------------------------------------------------------------------- main --
 
 def main():
@@ -471,6 +586,8 @@ def main():
                          "preceding kernel finishes")
     ap.add_argument("--only", choices=["states", "assign", "seed"],
                     help="time one build stage alone (single-kernel profiling) and exit")
+    ap.add_argument("--index", action="store_true",
+                    help="two-level (hierarchical) search against the flat search (time and recall) and exit")
     ap.add_argument("--sweep", action="store_true",
                     help="decode over the 36-point B x K x T grid (and full attention at B=1) and exit")
     args = ap.parse_args()
@@ -479,6 +596,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args.steps, args.warmup)
+        return
+    if args.index:
+        run_index(args.steps, args.warmup)
         return
     cfg = inputs.CONFIGS[1]
     world, rank, local = dist_setup(args.gpus)

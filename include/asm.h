@@ -282,6 +282,65 @@ asm_status asm_flash_decode(const void *q, const void *k_prefix,
                             cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Two-level (hierarchical) memory                                           */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The retrieval the pages describe is hierarchical, in O(log K)
+ * ("Complejidad"), without its construction; the plainest two-level reading
+ * is provided.  Index build: cluster each head's K centres into K1 clusters
+ * with asm_kmeanspp_seed + asm_kmeans run on the centres themselves (points =
+ * centroids_dt [Hq, K, d], clusters = K1); their centroids_dt are the
+ * super-centres, their perm / seg_off the members, their counts give
+ * max_seg.  Then asm_index_reorder lays the memory out by cluster.
+ *
+ * asm_index_reorder -- row i of head h of each output is row perm[h, i] of
+ * the corresponding input, so that cluster j occupies rows
+ * seg_off[h, j] .. seg_off[h, j+1]-1.
+ *   perm [H, K] int32; centroids, a_bar [H, K, d] dt; logz_bar [H, K] fp32
+ *   -> centroids_ord, a_bar_ord, logz_bar_ord of the same shapes (distinct
+ *   buffers).
+ */
+asm_status asm_index_reorder(const int32_t *perm, int H, int K, int d,
+                             asm_dtype dt, const void *centroids,
+                             const void *a_bar, const float *logz_bar,
+                             void *centroids_ord, void *a_bar_ord,
+                             float *logz_bar_ord, cudaStream_t stream);
+
+/*
+ * asm_decode_step_indexed -- asm_decode_step with the two-level search: each
+ * query head scores the K1 super-centres, keeps the P best clusters (ties to
+ * the smaller cluster index) and retrieves the best member of those clusters
+ * (ties to the smaller row), both by the retrieval metric; then the local
+ * attention and the merge as in asm_decode_step.  With P = K1 it is the flat
+ * search.
+ *   supers   [Hq, K1, d] dt   super-centres
+ *   seg_off  [Hq, K1 + 1]     int32, cluster j = rows seg_off[j] .. seg_off[j+1]-1
+ *   K1, P    1 <= P <= min(K1, 32), K1 <= min(K, 4096)
+ *   max_seg  at least the largest cluster (members beyond it are not read)
+ *   centroids, a_bar, logz_bar: the memory ordered by asm_index_reorder
+ *   idx_out  the retrieved row of the ordered memory (perm maps it back)
+ *   other arguments as asm_decode_step (no flags).  bf16 only.
+ *   ws asm_decode_indexed_workspace_size(...) bytes, zeroed once by
+ *   asm_workspace_init.
+ * Three kernel launches: the cluster choice, then the member and local units,
+ * then the merge.
+ */
+size_t asm_decode_indexed_workspace_size(int B, int Hq, int Hkv, int K1, int P,
+                                         int max_seg, int Tmax, int d,
+                                         asm_dtype dt);
+asm_status asm_decode_step_indexed(const void *q, const void *supers,
+                                   const int32_t *seg_off, int K1, int P,
+                                   int max_seg, const void *centroids,
+                                   const void *a_bar, const float *logz_bar,
+                                   const void *k_cache, const void *v_cache,
+                                   const int32_t *local_len, int B, int Hq,
+                                   int Hkv, int K, int Tmax, int d, float scale,
+                                   asm_metric metric, asm_dtype dt, void *out,
+                                   float *lse_out, int32_t *idx_out, void *ws,
+                                   size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Utilities                                                                */
 /* ------------------------------------------------------------------------ */
 

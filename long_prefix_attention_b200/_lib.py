@@ -31,6 +31,10 @@ SIGNATURES = {
     "asm_decode_step_noalloc": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, P, P, ctypes.c_uint, P]),
     "asm_flash_decode_workspace_size": (SZ, [I, I, I, I, I, I, I]),
     "asm_flash_decode": (I, [P, P, P, I, P, P, P, I, I, I, I, I, F, I, P, P, P, SZ, P]),
+    "asm_index_reorder": (I, [P, I, I, I, I, P, P, P, P, P, P, P]),
+    "asm_decode_indexed_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I]),
+    "asm_decode_step_indexed": (I, [P, P, P, I, I, I, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, P, P, P,
+                                    SZ, P]),
     "asm_workspace_init": (I, [P, SZ, P]),
     "asm_workspace_error": (I, [P, SZ, ctypes.POINTER(ctypes.c_int), P]),
     "asm_status_string": (ctypes.c_char_p, [I]),

@@ -184,6 +184,50 @@ asm_status asm_decode_step(const void *q, const void *centroids, const void *a_b
                                          dt, out, lse_out, idx_out, flags, ws, num_sms(), stream));
 }
 
+asm_status asm_index_reorder(const int32_t *perm, int H, int K, int d, asm_dtype dt, const void *centroids,
+                             const void *a_bar, const float *logz_bar, void *centroids_ord, void *a_bar_ord,
+                             float *logz_bar_ord, cudaStream_t stream) {
+    if (!dt_ok(dt) || H < 1 || K < 1) return ASM_ERR_INVALID_ARG;
+    if (!d_ok(d)) return ASM_ERR_UNSUPPORTED;
+    if (!aligned(perm, 4) || !aligned(centroids, 16) || !aligned(a_bar, 16) || !aligned(logz_bar, 4) ||
+        !aligned(centroids_ord, 16) || !aligned(a_bar_ord, 16) || !aligned(logz_bar_ord, 4))
+        return ASM_ERR_INVALID_ARG;
+    if (centroids_ord == centroids || a_bar_ord == a_bar || logz_bar_ord == logz_bar) return ASM_ERR_INVALID_ARG;
+    return cuda_status(asm_index_reorder_launch(perm, H, K, d, dt, centroids, a_bar, logz_bar, centroids_ord,
+                                                a_bar_ord, logz_bar_ord, stream));
+}
+
+size_t asm_decode_indexed_workspace_size(int B, int Hq, int Hkv, int K1, int P, int max_seg, int Tmax, int d,
+                                         asm_dtype dt) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || K1 < 1 || P < 1 || max_seg < 1 || Tmax < 0 || !d_ok(d) || dt != ASM_BF16)
+        return 0;
+    return asm_decode_indexed_tc_ws_bytes(B, Hq, P, max_seg, Tmax, d);
+}
+
+asm_status asm_decode_step_indexed(const void *q, const void *supers, const int32_t *seg_off, int K1, int P,
+                                   int max_seg, const void *centroids, const void *a_bar, const float *logz_bar,
+                                   const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
+                                   int Hq, int Hkv, int K, int Tmax, int d, float scale, asm_metric metric,
+                                   asm_dtype dt, void *out, float *lse_out, int32_t *idx_out, void *ws,
+                                   size_t ws_bytes, cudaStream_t stream) {
+    if (!dt_ok(dt) || B < 1 || B > 4096 || K < 1 || Tmax < 0 || !(scale == scale)) return ASM_ERR_INVALID_ARG;
+    if (metric != ASM_L2 && metric != ASM_COSINE) return ASM_ERR_INVALID_ARG;
+    if (K1 < 1 || K1 > K || K1 > 4096 || P < 1 || P > K1 || P > 32 || max_seg < 1 || max_seg > K)
+        return ASM_ERR_INVALID_ARG;
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ASM_ERR_INVALID_ARG;
+    if (dt != ASM_BF16 || !d_ok(d) || !group_ok(Hq, Hkv)) return ASM_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(supers, 16) || !aligned(seg_off, 4) || !aligned(centroids, 16) ||
+        !aligned(a_bar, 16) || !aligned(logz_bar, 4) || !aligned(local_len, 4) || !aligned(out, 16))
+        return ASM_ERR_INVALID_ARG;
+    if (Tmax > 0 && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return ASM_ERR_INVALID_ARG;
+    if ((lse_out && !aligned(lse_out, 4)) || (idx_out && !aligned(idx_out, 4))) return ASM_ERR_INVALID_ARG;
+    if (!aligned(ws, 16) || ws_bytes < asm_decode_indexed_tc_ws_bytes(B, Hq, P, max_seg, Tmax, d))
+        return ASM_ERR_WORKSPACE;
+    return cuda_status(asm_decode_indexed_tc_launch(q, supers, seg_off, K1, P, max_seg, centroids, a_bar, logz_bar,
+                                                    k_cache, v_cache, local_len, B, Hq, Hkv, K, Tmax, d, scale,
+                                                    (int)metric, out, lse_out, idx_out, ws, stream));
+}
+
 size_t asm_flash_decode_workspace_size(int B, int Hq, int Hkv, int Lp, int Tmax, int d, asm_dtype dt) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Lp < 0 || Tmax < 0 || !d_ok(d) || !dt_ok(dt)) return 0;
     return asm_decode_ws_bytes(1, B, Hq, Hkv, 0, Lp, Tmax, d, dt);

@@ -69,6 +69,12 @@ struct Args {
     int nS;                       // centroid units per head (mode 0)
     int nP, nA;                   // prefix / local units per (b, g)
     int ext_prefix;               // the nP prefix partials come from the batched prefix kernel
+    // mode 2 (two-level search): centroid units scan the members of the P
+    // clusters the select kernel kept for each (b, h), in nsub units each
+    int *sel;                     // [B][Hq][P] kept clusters (workspace)
+    const int *seg_off;           // [Hq][K1 + 1] member rows of each cluster
+    const __nv_bfloat16 *supers;  // [Hq][K1][D] super-centres
+    int K1, P, nsub;
     int n_scan;                   // Hq * nS
     float2 *ws_srch;              // [B][Hq][nS]
     float2 *ws_ml;                // [B][Hq][nP+nA]
@@ -112,7 +118,20 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     const bool scan = u < a.n_scan;
     int h = 0, b = 0, g = 0, slot, first, valid;
     bool prefix = false;
-    if (scan) {
+    int qrow0 = 0, nq = a.B;  // the query rows a centroid unit serves
+    if (scan && a.mode == 2) {
+        // one (b, h, kept cluster p, sub-range) per unit; its rows are known
+        // once the select kernel has finished
+        const int sub = u % a.nsub, r1 = u / a.nsub, p = r1 % a.P, r2 = r1 / a.P;
+        h = r2 % a.Hq;
+        b = r2 / a.Hq;
+        slot = p * a.nsub + sub;
+        qrow0 = b;
+        nq = 1;
+        g = h / G;
+        first = 0;
+        valid = 0;
+    } else if (scan) {
         h = u / a.nS;
         slot = u - h * a.nS;
         first = slot * Gm::CS;
@@ -147,11 +166,13 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     }
     __syncthreads();
     auto issue = [&](int vrows) {
-        if (scan) {
+        if (scan && vrows > 0) {
             mbar_arrive_expect_tx(bar, Gm::CS * Gm::ROWB);
 #pragma unroll
             for (int hf = 0; hf < Gm::HALVES; ++hf)
                 tma_load_3d(tile + hf * Gm::CS * 128, &maps.c, 64 * hf, first, h, bar);
+        } else if (scan) {
+            mbar_arrive(bar);  // a unit past its cluster's members: nothing to load
         } else if (vrows > 0) {
             mbar_arrive_expect_tx(bar, 2 * Gm::TS * Gm::ROWB);
             const CUtensorMap *mk = prefix ? &maps.kp : &maps.k;
@@ -167,9 +188,9 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
         }
     };
     // static centroids may stream before the dependency wait (caller's choice)
-    const bool early = scan && (a.flags & 1);
+    const bool early = scan && (a.flags & 1) && a.mode != 2;
     if (early && tid == 0) issue(valid);
-    if (!early) {
+    if (!early && !(scan && a.mode == 2)) {
         // Warm L2 with this unit's rows while the preceding kernel finishes.
         // Always safe: L2 is the coherence point, so a row the preceding
         // kernel still writes is read correctly after the wait below.  The
@@ -199,6 +220,12 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     pdl_wait();
     pdl_launch_dependents();
     if (!scan && !prefix) valid = min(Gm::TS, min(max(__ldg(a.local_len + b), 0), a.Tmax) - first);
+    if (scan && a.mode == 2) {
+        const int c = __ldcg(a.sel + ((size_t)b * a.Hq + h) * a.P + slot / a.nsub);
+        const int *so = a.seg_off + (size_t)h * (a.K1 + 1);
+        first = __ldg(so + c) + (slot % a.nsub) * Gm::CS;
+        valid = min(Gm::CS, __ldg(so + c + 1) - first);
+    }
     if (!early && tid == 0) issue(valid);
 
     if (scan) {
@@ -207,15 +234,15 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
         float nrl[RMT], nrh[RMT];
         const int src = 4 * gid + (gid >> 1);  // lane holding the diagonal entry of row gid
 #pragma unroll 1
-        for (int nt = 0; nt * 8 < a.B; ++nt) {
+        for (int nt = 0; nt * 8 < nq; ++nt) {
             const int bq = 8 * nt + gid;
             const uint32_t *qr = reinterpret_cast<const uint32_t *>(
-                a.q + ((size_t)min(bq, a.B - 1) * a.Hq + h) * D);
+                a.q + ((size_t)(qrow0 + min(bq, nq - 1)) * a.Hq + h) * D);
             uint32_t qb0[KS], qb1[KS];
 #pragma unroll
             for (int j = 0; j < KS; ++j) {
-                qb0[j] = bq < a.B ? __ldg(qr + 8 * j + quad) : 0u;
-                qb1[j] = bq < a.B ? __ldg(qr + 8 * j + 4 + quad) : 0u;
+                qb0[j] = bq < nq ? __ldg(qr + 8 * j + quad) : 0u;
+                qb1[j] = bq < nq ? __ldg(qr + 8 * j + 4 + quad) : 0u;
             }
             if (nt == 0 && !mbar_wait(bar, 0)) set_error(a.ws_err);
             float bs[2] = {kNegInf, kNegInf};
@@ -265,19 +292,19 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
                     if (better(os, oi, bs[e], bi[e])) { bs[e] = os; bi[e] = oi; }
                 }
                 const int bb = 8 * nt + 2 * quad + e;
-                if (gid == 0 && bb < a.B) wb[warp * a.B + bb] = make_float2(bs[e], __int_as_float(bi[e]));
+                if (gid == 0 && bb < nq) wb[warp * a.B + bb] = make_float2(bs[e], __int_as_float(bi[e]));
             }
         }
         __syncthreads();
 #pragma unroll 1
-        for (int bb = tid; bb < a.B; bb += kThreads) {
+        for (int bb = tid; bb < nq; bb += kThreads) {
             float bs = kNegInf;
             int bi = 0x7fffffff;
             for (int w = 0; w < kWarps; ++w) {
                 const float2 v = wb[w * a.B + bb];
                 if (better(v.x, __float_as_int(v.y), bs, bi)) { bs = v.x; bi = __float_as_int(v.y); }
             }
-            a.ws_srch[((size_t)bb * a.Hq + h) * a.nS + slot] = make_float2(bs, __int_as_float(bi));
+            a.ws_srch[((size_t)(qrow0 + bb) * a.Hq + h) * a.nS + slot] = make_float2(bs, __int_as_float(bi));
             if (bi != 0x7fffffff) {
                 // warm L2 with this unit's candidate state for the merge's gather
                 const __nv_bfloat16 *row = a.a_bar + ((size_t)h * a.K + bi) * D;
@@ -416,6 +443,57 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     }
 }
 
+// ---------------------------------------------------------- select kernel --
+//
+// Two-level search, first level: one CTA per (b, h) scores the K1
+// super-centres with the retrieval rule and keeps the P best (ties to the
+// smaller cluster index) for the centroid units.
+
+constexpr int kSelMaxK1 = 4096;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+asm_index_select(const Args a) {
+    constexpr int EPL = D / 32;
+    const int bh = blockIdx.x, h = bh % a.Hq;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __shared__ float sc[kSelMaxK1];
+    pdl_wait();
+    pdl_launch_dependents();
+    float qv[EPL];
+    load_vec<__nv_bfloat16, EPL>(a.q + (size_t)bh * D + lane * EPL, qv);
+    const __nv_bfloat16 *S = a.supers + (size_t)h * a.K1 * D;
+    for (int j = warp; j < a.K1; j += kWarps) {
+        float sv[EPL];
+        load_vec<__nv_bfloat16, EPL>(S + (size_t)j * D + lane * EPL, sv);
+        float dt = 0.f, nr = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            dt = fmaf(qv[e], sv[e], dt);
+            nr = fmaf(sv[e], sv[e], nr);
+        }
+        dt = warp_sum(dt);
+        nr = warp_sum(nr);
+        if (lane == 0) sc[j] = (a.metric == 0) ? dt - 0.5f * nr : (nr > 0.f ? dt / sqrtf(nr) : 0.f);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        for (int p = 0; p < a.P; ++p) {
+            float bs = kNegInf;
+            int bi = 0x7fffffff;
+            for (int j = lane; j < a.K1; j += 32)
+                if (better(sc[j], j, bs, bi)) { bs = sc[j]; bi = j; }
+            warp_argmax(bs, bi);
+            if (bi == 0x7fffffff) bi = 0;
+            if (lane == 0) {
+                a.sel[(size_t)bh * a.P + p] = bi;
+                sc[bi] = kNegInf;
+            }
+            __syncwarp();
+        }
+    }
+}
+
 // ----------------------------------------------------------- merge kernel --
 //
 // One CTA per (b, h) of SG x D threads: thread (sg, t) owns output dim t of
@@ -444,12 +522,13 @@ asm_decode_merge(const Args a) {
     __shared__ float so[kMergeMaxSG][D];
     __shared__ float sl[kMergeMaxSG];
     const int nslots = a.nP + a.nA;
+    const bool search = a.mode != 1;  // a memory lookup (flat or two-level) precedes the merge
     pdl_wait();
     pdl_launch_dependents();
     // ---- round 1: the centroid scores, the attention maxima, and each
     //      thread's first kMergeSlots partials
     float2 best = make_float2(kNegInf, __int_as_float(0x7fffffff));
-    if (a.mode == 0) {
+    if (search) {
         for (int s = tid; s < a.nS; s += NT) {
             const float2 v = __ldcg(a.ws_srch + (size_t)bh * a.nS + s);
             if (better(v.x, __float_as_int(v.y), best.x, __float_as_int(best.y))) best = v;
@@ -497,7 +576,7 @@ asm_decode_merge(const Args a) {
     const float M = sM;
     // ---- round 2: the retrieved state (issued before the weighted sums)
     float zb2 = kNegInf, ab = 0.f;
-    if (a.mode == 0 && sg == 0) {
+    if (search && sg == 0) {
         zb2 = __ldg(a.logz_bar + (size_t)h * a.K + idx) * kLog2e;
         ab = __bfloat162float(a.a_bar[((size_t)h * a.K + idx) * D + t]);
     }
@@ -540,12 +619,12 @@ asm_decode_merge(const Args a) {
     const float zl2 = (L > 0.f) ? M + lg2f(L) : kNegInf;
     const float loc = (L > 0.f) ? o / L : 0.f;
     float res, lse2;
-    if (a.mode == 0 && !(zb2 == kNegInf && zl2 == kNegInf)) {
+    if (search && !(zb2 == kNegInf && zl2 == kNegInf)) {
         const float m = fmaxf(zb2, zl2);
         const float eb = ex2f(zb2 - m), el = ex2f(zl2 - m);
         lse2 = m + lg2f(eb + el);
         res = (eb * ab + el * loc) / (eb + el);
-    } else if (a.mode == 0) {
+    } else if (search) {
         lse2 = kNegInf;
         res = 0.f;
     } else {
@@ -555,7 +634,7 @@ asm_decode_merge(const Args a) {
     a.out[(size_t)bh * D + t] = __float2bfloat16_rn(res);
     if (t == 0) {
         if (a.lse_out) a.lse_out[bh] = lse2 * kLn2;
-        if (a.idx_out && a.mode == 0) a.idx_out[bh] = idx;
+        if (a.idx_out && search) a.idx_out[bh] = idx;
     }
 }
 
@@ -567,16 +646,20 @@ bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uin
 
 namespace {
 struct TcWs {
-    size_t off_srch, off_ml, off_o, total;
+    size_t off_sel, off_srch, off_ml, off_o, total;
 };
 inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
-TcWs tc_ws_layout(int mode, int B, int Hq, int K, int Lp, int Tmax, int d) {
+// mode 0: flat search (K centres); 1: explicit prefix (Lp); 2: two-level
+// search with P kept clusters of at most max_seg members (K unused).
+TcWs tc_ws_layout(int mode, int B, int Hq, int K, int Lp, int Tmax, int d, int P = 0, int max_seg = 0) {
     const int CS = tc::kUnit / (2 * d), TS = tc::kUnit / (4 * d);
-    const size_t nS = mode == 0 ? (size_t)(K + CS - 1) / CS : 0;
+    const size_t nS = mode == 0 ? (size_t)(K + CS - 1) / CS
+                    : mode == 2 ? (size_t)P * ((max_seg + CS - 1) / CS) : 0;
     const size_t nP = mode == 1 ? (size_t)(Lp + TS - 1) / TS : 0;
     const size_t nA = (size_t)(Tmax + TS - 1) / TS;
     TcWs w;
-    w.off_srch = 256;  // word 0: device-side error code
+    w.off_sel = 256;  // word 0: device-side error code
+    w.off_srch = al256(w.off_sel + sizeof(int) * (size_t)B * Hq * (mode == 2 ? P : 0));
     w.off_ml = al256(w.off_srch + sizeof(float2) * (size_t)B * Hq * nS);
     w.off_o = al256(w.off_ml + sizeof(float2) * (size_t)B * Hq * (nP + nA));
     w.total = al256(w.off_o + sizeof(float) * (size_t)B * Hq * (nP + nA) * d);
@@ -589,7 +672,8 @@ cudaError_t tc_launch(tc::Args a, const void *centroids, const void *k_prefix, c
     using Gm = tc::Geo<D>;
     tc::Maps maps;
     memset(&maps, 0, sizeof(maps));
-    if (a.mode == 0 && !make_map_3d(&maps.c, centroids, D, a.K, a.Hq, Gm::CS)) return cudaErrorInvalidValue;
+    if ((a.mode == 0 || a.mode == 2) && !make_map_3d(&maps.c, centroids, D, a.K, a.Hq, Gm::CS))
+        return cudaErrorInvalidValue;
     if (a.Tmax > 0 && (!make_map_3d(&maps.k, k_cache, D, a.Tmax, (uint64_t)a.B * a.Hkv, Gm::TS) ||
                        !make_map_3d(&maps.v, v_cache, D, a.Tmax, (uint64_t)a.B * a.Hkv, Gm::TS)))
         return cudaErrorInvalidValue;
@@ -708,4 +792,66 @@ cudaError_t asm_decode_tc_launch(int mode, const void *q, const void *centroids,
     }
     if (d == 128) return tc_launch_g<128>(G, a, centroids, k_prefix, v_prefix, k_cache, v_cache, st);
     return tc_launch_g<64>(G, a, centroids, k_prefix, v_prefix, k_cache, v_cache, st);
+}
+
+size_t asm_decode_indexed_tc_ws_bytes(int B, int Hq, int P, int max_seg, int Tmax, int d) {
+    return asmk::tc_ws_layout(2, B, Hq, 0, 0, Tmax, d, P, max_seg).total;
+}
+
+// Two-level search decode: select kernel (kept clusters), units (members of
+// the kept clusters and the local tokens), merge.
+cudaError_t asm_decode_indexed_tc_launch(const void *q, const void *supers, const int32_t *seg_off, int K1, int P,
+                                         int max_seg, const void *centroids, const void *a_bar, const float *logz_bar,
+                                         const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
+                                         int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, void *out,
+                                         float *lse_out, int32_t *idx_out, void *ws, cudaStream_t st) {
+    using namespace asmk;
+    const TcWs w = tc_ws_layout(2, B, Hq, K, 0, Tmax, d, P, max_seg);
+    tc::Args a{};
+    a.q = (const __nv_bfloat16 *)q;
+    a.centroids = (const __nv_bfloat16 *)centroids;
+    a.k_cache = (const __nv_bfloat16 *)k_cache;
+    a.v_cache = (const __nv_bfloat16 *)v_cache;
+    a.a_bar = (const __nv_bfloat16 *)a_bar;
+    a.logz_bar = logz_bar;
+    a.local_len = local_len;
+    a.out = (__nv_bfloat16 *)out;
+    a.lse_out = lse_out;
+    a.idx_out = idx_out;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.K = K; a.Tmax = Tmax; a.Lp = 0;
+    a.qscale = scale * kLog2e;
+    a.metric = metric;
+    a.mode = 2;
+    a.flags = 0;
+    const int CS = tc::kUnit / (2 * d), TS = tc::kUnit / (4 * d);
+    a.K1 = K1;
+    a.P = P;
+    a.nsub = (max_seg + CS - 1) / CS;
+    a.nS = P * a.nsub;
+    a.nP = 0;
+    a.nA = (Tmax + TS - 1) / TS;
+    a.n_scan = B * Hq * a.nS;
+    a.seg_off = seg_off;
+    a.supers = (const __nv_bfloat16 *)supers;
+    char *base = static_cast<char *>(ws);
+    a.ws_err = reinterpret_cast<int *>(base);
+    a.sel = reinterpret_cast<int *>(base + w.off_sel);
+    a.ws_srch = reinterpret_cast<float2 *>(base + w.off_srch);
+    a.ws_ml = reinterpret_cast<float2 *>(base + w.off_ml);
+    a.ws_o = reinterpret_cast<float *>(base + w.off_o);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c0 = {};
+    c0.gridDim = dim3(B * Hq);
+    c0.blockDim = dim3(tc::kThreads);
+    c0.stream = st;
+    c0.attrs = attr;
+    c0.numAttrs = 1;
+    cudaError_t e = (d == 128) ? cudaLaunchKernelEx(&c0, tc::asm_index_select<128>, a)
+                               : cudaLaunchKernelEx(&c0, tc::asm_index_select<64>, a);
+    if (e != cudaSuccess) return e;
+    const int G = Hq / Hkv;
+    if (d == 128) return tc_launch_g<128>(G, a, centroids, nullptr, nullptr, k_cache, v_cache, st);
+    return tc_launch_g<64>(G, a, centroids, nullptr, nullptr, k_cache, v_cache, st);
 }

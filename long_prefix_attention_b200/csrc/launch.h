@@ -29,6 +29,19 @@ cudaError_t asm_decode_tc_launch(int mode, const void *q, const void *centroids,
                                  int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, void *out,
                                  float *lse_out, int32_t *idx_out, unsigned flags, void *ws, cudaStream_t st);
 
+// decode_tc.cu: two-level search decode (bf16)
+size_t asm_decode_indexed_tc_ws_bytes(int B, int Hq, int P, int max_seg, int Tmax, int d);
+cudaError_t asm_decode_indexed_tc_launch(const void *q, const void *supers, const int32_t *seg_off, int K1, int P,
+                                         int max_seg, const void *centroids, const void *a_bar, const float *logz_bar,
+                                         const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
+                                         int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, void *out,
+                                         float *lse_out, int32_t *idx_out, void *ws, cudaStream_t st);
+
+// index.cu: order a memory by cluster
+cudaError_t asm_index_reorder_launch(const int32_t *perm, int H, int K, int d, asm_dtype dt, const void *c,
+                                     const void *abar, const float *lz, void *c_out, void *abar_out, float *lz_out,
+                                     cudaStream_t st);
+
 // build_states.cu
 cudaError_t asm_build_states_launch(const void *q, const void *k, const void *v, int Hq, int Hkv,
                                     int N, int L, int d, float scale, asm_dtype dt,

@@ -202,6 +202,34 @@ def asm_flash_decode(q, k_prefix, v_prefix, k_cache, v_cache, local_len, scale: 
 
 # ---------------------------------------------------------------- helpers --
 
+def asm_index_reorder(perm, centroids, a_bar, logz_bar, centroids_ord, a_bar_ord, logz_bar_ord, stream=None):
+    """Lay a memory out by cluster: row i of head h <- row perm[h, i]."""
+    _contig(perm, centroids, a_bar, logz_bar, centroids_ord, a_bar_ord, logz_bar_ord)
+    H, K, d = centroids.shape
+    _check("asm_index_reorder", _lib.load().asm_index_reorder(
+        _p(perm), H, K, d, _dt(centroids), _p(centroids), _p(a_bar), _p(logz_bar), _p(centroids_ord),
+        _p(a_bar_ord), _p(logz_bar_ord), _stream(stream)))
+
+
+def asm_decode_indexed_workspace_size(B, Hq, Hkv, K1, P, max_seg, Tmax, d, dtype) -> int:
+    return int(_lib.load().asm_decode_indexed_workspace_size(B, Hq, Hkv, K1, P, max_seg, Tmax, d, _DT[dtype]))
+
+
+def asm_decode_step_indexed(q, supers, seg_off, P: int, max_seg: int, centroids, a_bar, logz_bar, k_cache,
+                            v_cache, local_len, scale: float, out, ws, lse_out=None, idx_out=None,
+                            metric: int = ASM_L2, stream=None):
+    """Decode step with the two-level search over a memory ordered by cluster."""
+    _contig(q, supers, seg_off, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, out, lse_out, idx_out)
+    B, Hq, d = q.shape
+    K1 = supers.shape[1]
+    K = centroids.shape[1]
+    Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    _check("asm_decode_step_indexed", _lib.load().asm_decode_step_indexed(
+        _p(q), _p(supers), _p(seg_off), K1, int(P), int(max_seg), _p(centroids), _p(a_bar), _p(logz_bar),
+        _p(k_cache), _p(v_cache), _p(local_len), B, Hq, Hkv, K, Tmax, d, float(scale), int(metric), _dt(q),
+        _p(out), _p(lse_out), _p(idx_out), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
 def alloc_workspace(nbytes: int, device, zero: bool = True) -> torch.Tensor:
     """A 256-byte-granular device buffer (zeroed: ready for decode calls)."""
     n = max(256, (int(nbytes) + 255) // 256 * 256)

@@ -106,3 +106,43 @@ def test_build_and_kmeans_validation(lib):
     # flash decode: nothing to attend
     assert lib.asm_flash_decode(P, P, P, 0, P, P, P, 1, 32, 8, 0, 128, 0.1, 1, P, NULL, P,
                                 1 << 30, None) == INVALID
+
+
+def indexed(lib, **kw):
+    a = dict(q=FAKE, s=FAKE, so=FAKE, K1=64, P=8, ms=40, c=FAKE, ab=FAKE, lz=FAKE, kc=FAKE, vc=FAKE, ll=FAKE, B=1,
+             Hq=32, Hkv=8, K=2048, Tmax=256, d=128, scale=0.088, metric=0, dt=1, out=FAKE, lse=NULL, idx=NULL,
+             ws=FAKE, wsb=1 << 30)
+    a.update(kw)
+    return lib.asm_decode_step_indexed(a["q"], a["s"], a["so"], a["K1"], a["P"], a["ms"], a["c"], a["ab"], a["lz"],
+                                       a["kc"], a["vc"], a["ll"], a["B"], a["Hq"], a["Hkv"], a["K"], a["Tmax"], a["d"],
+                                       a["scale"], a["metric"], a["dt"], a["out"], a["lse"], a["idx"], a["ws"],
+                                       a["wsb"], None)
+
+
+def test_indexed_decode_rejects_bad_arguments_before_any_launch(lib):
+    assert indexed(lib, P=0) == 1                 # no cluster kept
+    assert indexed(lib, P=65) == 1                # more kept than clusters
+    assert indexed(lib, K1=64, P=33) == 1         # more than 32 kept
+    assert indexed(lib, K1=5000, K=8192) == 1     # more than 4096 clusters
+    assert indexed(lib, ms=0) == 1                # empty largest cluster
+    assert indexed(lib, s=ODD) == 1               # misaligned super-centres
+    assert indexed(lib, dt=0) == 2                # fp32 storage: unsupported
+    assert indexed(lib, d=96) == 2                # head dim
+    assert indexed(lib, wsb=256) == 3             # workspace too small
+    need = lib.asm_decode_indexed_workspace_size(1, 32, 8, 64, 8, 40, 256, 128, 1)
+    assert need > 0 and indexed(lib, wsb=need - 16) == 3
+    assert lib.asm_decode_indexed_workspace_size(1, 32, 8, 64, 8, 40, 256, 128, 0) == 0  # fp32
+
+
+def test_index_reorder_rejects_bad_arguments(lib):
+    args = [FAKE, 4, 100, 128, 1, FAKE, FAKE, FAKE, ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000),
+            ctypes.c_void_p(0x40000), None]
+    bad = list(args)
+    bad[0] = NULL
+    assert lib.asm_index_reorder(*bad) == 1       # no permutation
+    bad = list(args)
+    bad[8] = FAKE
+    assert lib.asm_index_reorder(*bad) == 1       # output aliases its input
+    bad = list(args)
+    bad[3] = 80
+    assert lib.asm_index_reorder(*bad) == 2       # head dim
