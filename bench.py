@@ -9,7 +9,7 @@ streams its bytes from HBM); the 32 layer steps (two kernels each) are
 replayed from a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl asm|reference]
-    python bench.py --only states|assign|seed [--steps K] [--warmup W]
+    python bench.py --only states|assign|seed|lloyd|aggregate [--steps K] [--warmup W]
     python bench.py --sweep [--steps K] [--warmup W]
     python bench.py --index [--steps K] [--warmup W]
 
@@ -314,7 +314,9 @@ def run_stage(name, steps, warmup):
     """One build stage at the full build shape, `steps` timed launches (for
     profiling single kernels): states = one 4096-key block of the prefix
     (fresh states, no merge); assign = one Lloyd assignment against K
-    calibration points; seed = the whole k-means++ seeding."""
+    calibration points; lloyd = the 10 Lloyd rounds (assign + update);
+    aggregate = the Z-weighted aggregation; seed = the whole k-means++
+    seeding."""
     from long_prefix_attention_b200 import ops
     cfg = inputs.CONFIGS[3]
     bi = inputs.build_inputs(cfg)
@@ -336,6 +338,28 @@ def run_stage(name, steps, warmup):
         ws = ops.alloc_workspace(ops.asm_kmeans_workspace_size(H, N, d, K), "cuda")
         fn = lambda: ops.asm_kmeans_assign(x, cdt, assign, ws)
         flops = 2.0 * N * K * d * H
+    elif name in ("lloyd", "aggregate"):
+        g = torch.Generator().manual_seed(5)
+        init = torch.stack([torch.randperm(N, generator=g)[:K] for _ in range(H)]).to(torch.int32).cuda()
+        cen = torch.empty(H, K, d, dtype=torch.float32, device="cuda")
+        cdt = torch.empty(H, K, d, dtype=x.dtype, device="cuda")
+        assign = torch.empty(H, N, dtype=torch.int32, device="cuda")
+        counts = torch.empty(H, K, dtype=torch.int32, device="cuda")
+        perm = torch.empty(H, N, dtype=torch.int32, device="cuda")
+        seg = torch.empty(H, K + 1, dtype=torch.int32, device="cuda")
+        ws = ops.alloc_workspace(ops.asm_kmeans_workspace_size(H, N, d, K), "cuda")
+        iters = cfg["iters"]
+        if name == "lloyd":
+            fn = lambda: ops.asm_kmeans(x, init, iters, cen, cdt, assign, counts, perm, seg, ws)
+            flops = 2.0 * N * K * d * H * iters
+        else:
+            ops.asm_kmeans(x, init, 1, cen, cdt, assign, counts, perm, seg, ws)
+            a = torch.randn(H, N, d, device="cuda").to(x.dtype)
+            logz = torch.rand(H, N, device="cuda") * 5 + 5
+            a_bar = torch.empty(H, K, d, dtype=x.dtype, device="cuda")
+            lz_bar = torch.empty(H, K, dtype=torch.float32, device="cuda")
+            fn = lambda: ops.asm_aggregate(a, logz, perm, seg, a_bar, lz_bar)
+            flops = None
     else:
         u = bi["u"].cuda()
         init = torch.empty(H, K, dtype=torch.int32, device="cuda")
@@ -584,7 +608,7 @@ def main():
     ap.add_argument("--no-prefetch", action="store_true",
                     help="do not let a layer's kernel stream its (static) centroids before the "
                          "preceding kernel finishes")
-    ap.add_argument("--only", choices=["states", "assign", "seed"],
+    ap.add_argument("--only", choices=["states", "assign", "seed", "lloyd", "aggregate"],
                     help="time one build stage alone (single-kernel profiling) and exit")
     ap.add_argument("--index", action="store_true",
                     help="two-level (hierarchical) search against the flat search (time and recall) and exit")
