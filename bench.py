@@ -252,7 +252,49 @@ def cpu_decode_baseline(cfg, budget_s=12.0):
                       f"({dt:.1f} s of fp64 CPU work)"}
 
 
-def run_build(cfg):
+def cpu_build_baseline(cfg, bi):
+    """fp64 oracle of each build stage on the host cores, on bounded samples
+    of head 0 at the build shape, extrapolated to the whole build (all heads,
+    queries, rounds and Lloyd iterations): states over the full 16384-key
+    prefix for 192 queries, one assignment pass of 4096 points against the
+    8192 centres, 128 k-means++ rounds, and one head's aggregation."""
+    from oracle import asm_oracle as O
+    H, N, d = bi["q"].shape
+    K, iters = cfg["K"], cfg["iters"]
+    Hkv = bi["k"].shape[0]
+    q0 = O._f64(bi["q"][0:1])
+    k0, v0 = O._f64(bi["k"][0:1]), O._f64(bi["v"][0:1])
+    out = {}
+    t = time.perf_counter()
+    O.build_states(q0[:, :192], k0, v0, bi["scale"])
+    ts = time.perf_counter() - t
+    out["states_s"] = ts / 192 * N * H
+    x0 = q0[0]
+    t = time.perf_counter()
+    O.assign(x0[:4096], x0[:K])
+    ta = time.perf_counter() - t
+    out["lloyd_s"] = ta / 4096 * N * H * iters
+    u = O._f64(bi["u"][0:1, :128])
+    t = time.perf_counter()
+    O.kmeanspp_seed(q0, u)
+    tk = time.perf_counter() - t
+    out["kmeanspp_s"] = tk / 128 * K * H
+    lz = np.zeros(N)
+    asg = np.arange(N, dtype=np.int32) % K
+    t = time.perf_counter()
+    O.aggregate(x0, lz, asg, K)
+    tg = time.perf_counter() - t
+    out["aggregate_s"] = tg * H
+    total = sum(out.values())
+    return {"value": H * N / total, "unit": "queries/s", "cores": O.max_threads(), "kind": "oracle",
+            "extrapolated": True, "stage_s": out,
+            "sample": f"head 0 of the build shape: states of 192 queries over all 16384 keys ({ts:.1f} s), one "
+                      f"assignment pass of 4096 points against {K} centres ({ta:.1f} s), 128 k-means++ rounds "
+                      f"({tk:.1f} s), one head's aggregation ({tg:.1f} s); scaled to {H} heads, {N} queries, "
+                      f"{K} rounds and {iters} Lloyd iterations"}
+
+
+def run_build(cfg, with_cpu=True):
     """Full offline build at the 32/8-head, N=65536, L=16384, K=8192 shape."""
     from long_prefix_attention_b200 import ops
     bi = inputs.build_inputs(cfg)
@@ -298,8 +340,9 @@ def run_build(cfg):
     hbm, tf, tfs, src = peaks()
     states_flops = 4.0 * N * L * d * H
     assign_flops = 2.0 * N * K * d * H * iters
+    cpu = cpu_build_baseline(cfg, bi) if with_cpu else None
     return {
-        "workload": cfg["name"], "queries": H * N,
+        "workload": cfg["name"], "queries": H * N, "cpu_baseline": cpu,
         "value": H * N / (total / 1e3), "unit": "queries/s",
         "ms": {"states_4chunks": t[0], "kmeanspp_seed": t[1], "lloyd_10": t[2], "aggregate": t[3],
                "total": total},
@@ -679,7 +722,7 @@ def main():
     build = None
     if not args.no_build and rank == 0:
         try:
-            build = run_build(inputs.CONFIGS[3])
+            build = run_build(inputs.CONFIGS[3], with_cpu=not args.no_cpu and world == 1)
         except Exception as e:  # report, do not hide
             build = {"error": repr(e)}
     cpu = None
