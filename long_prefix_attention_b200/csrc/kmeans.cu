@@ -19,30 +19,75 @@ inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // ============================================================ k-means++ ===
 //
-// One launch per round.  Every block refreshes D2 for its slice of points
-// against the centre chosen in the previous round (fp64, exact for bf16
-// inputs) and publishes its slice sum; the last block of each head to arrive
-// (arrival counter, no waiting) scans the slice sums, finds the slice that
-// holds the threshold u * sum(D2) and the first index inside it whose running
-// sum exceeds the threshold, and records the pick for the next round.
+// One launch per round r.  The centre chosen in round r - 1 lowers D2_i =
+// min(D2_i, |x_i - c|^2) (fp64, exact for bf16 inputs and for the products of
+// fp32 inputs); the last block of each head to arrive (an arrival counter, no
+// waiting) refreshes the partial sums of the ranges whose D2 changed, finds
+// the range holding the threshold u * sum(D2) and the first point inside it
+// whose running sum exceeds the threshold, and records the pick.
+//
+// Exact pruning.  From round kSeedFirstGroup on, the points are grouped by the
+// chosen centre nearest to them (regrouped on a schedule as centres are
+// added).  Group g has anchor a_g (its centre) and radius R_g = max |x - a_g|
+// over its members; a piece (the part of a group inside one block's range of
+// positions) also keeps M = max sqrt(D2) over its members.  By the triangle
+// inequality every member has |x - c| >= |c - a_g| - R_g, so when
+// |c - a_g| > (R_g + M)(1 + 1e-12) no member's D2 can fall and the piece is
+// skipped; the margin covers the rounding of the fp64 distances, so the D2
+// values, and therefore the picks, are those of the unpruned update.
 
 constexpr int kSeedThreads = 256;
 constexpr int kSeedWarps = kSeedThreads / 32;
-constexpr int kSeedPts = 1024;  // points per block: 8 warps x 4 steps of 32 points
+constexpr int kSeedCh = 1024;        // positions per block
+constexpr int kSeedRange = 128;      // points per partial sum of D2
+constexpr int kSeedFirstGroup = 256; // first regrouping round
+constexpr double kSeedMargin = 1e-12;
 
 struct SeedWs {
-    size_t off_d2, off_bsum, off_cnt, off_taken, total;
+    size_t off_d2, off_mdp, off_rr, off_bsum, off_r2, off_near, off_perm, off_apos, off_gcnt, off_seg,
+        off_cur, off_pofs, off_dirty, off_taken, off_cnt, total;
 };
-SeedWs seed_ws(int H, int N) {
-    const int nblk = (N + kSeedPts - 1) / kSeedPts;
+SeedWs seed_ws(int H, int N, int K) {
+    const size_t h = (size_t)H, n = (size_t)N, k = (size_t)K;
+    const size_t nr = (n + kSeedRange - 1) / kSeedRange;
     SeedWs w;
     w.off_d2 = 0;
-    w.off_bsum = al256(w.off_d2 + sizeof(double) * (size_t)H * N);
-    w.off_cnt = al256(w.off_bsum + sizeof(double) * (size_t)H * nblk);
-    w.off_taken = al256(w.off_cnt + sizeof(int) * (size_t)H);
-    w.total = al256(w.off_taken + (size_t)H * N);
+    w.off_mdp = al256(w.off_d2 + sizeof(double) * h * n);
+    w.off_rr = al256(w.off_mdp + sizeof(double) * h * n);
+    w.off_bsum = al256(w.off_rr + sizeof(double) * h * n);
+    w.off_r2 = al256(w.off_bsum + sizeof(double) * h * nr);
+    w.off_near = al256(w.off_r2 + sizeof(double) * h * k);
+    w.off_perm = al256(w.off_near + sizeof(int) * h * n);
+    w.off_apos = al256(w.off_perm + sizeof(int) * h * n);
+    w.off_gcnt = al256(w.off_apos + sizeof(int) * h * n);
+    w.off_seg = al256(w.off_gcnt + sizeof(int) * h * k);
+    w.off_cur = al256(w.off_seg + sizeof(int) * h * (k + 1));
+    w.off_pofs = al256(w.off_cur + sizeof(int) * h * k);
+    w.off_dirty = al256(w.off_pofs + sizeof(uint16_t) * h * n);
+    w.off_taken = al256(w.off_dirty + h * nr);
+    w.off_cnt = al256(w.off_taken + h * n);
+    w.total = al256(w.off_cnt + sizeof(int) * h);
     return w;
 }
+
+struct SeedArgs {
+    const double *u;
+    int32_t *idx;           // [H][K] picks
+    double *d2;             // [H][N] D2 by point
+    double *mdp;            // [H][N] piece max of D2, at the piece's first position
+    double *rr;             // [H][N] R^2 of the group of each position
+    double *bsum;           // [H][NR] partial sums of D2 by range of points
+    double *r2;             // [H][G] group R^2 (regrouping scratch)
+    int32_t *near;          // [H][N] round of the nearest chosen centre
+    int32_t *perm;          // [H][N] point at each position (grouped order)
+    int32_t *apos;          // [H][N] anchor point of the group of each position
+    int32_t *gcnt, *seg, *cur;  // regrouping scratch: [H][G], [H][G+1], [H][G]
+    uint16_t *pofs;         // [H][N] offset of the piece's first position in its block
+    unsigned char *dirty;   // [H][NR] range touched this round
+    unsigned char *taken;   // [H][N] point already chosen
+    int *cnt;               // [H] arrival counters
+    int N, K, NR;
+};
 
 // Inclusive prefix sum over the block (fp64); every thread gets its value.
 __device__ __forceinline__ double block_scan_d(double v, double *sh) {
@@ -62,8 +107,7 @@ __device__ __forceinline__ double block_scan_d(double v, double *sh) {
 
 // D2 update geometry: a point is LPP lanes x 16 bytes; one 16-byte load per
 // lane covers PPL = 32 / LPP points, so a warp reads its 32 points with LPP
-// independent loads, all issued before any arithmetic (memory parallelism:
-// every round streams the whole of x from HBM).
+// independent loads, all issued before any arithmetic.
 template <typename T, int D>
 struct SeedGeo {
     static constexpr int E16 = 16 / (int)sizeof(T);   // elements per 16-byte load
@@ -89,115 +133,198 @@ __device__ __forceinline__ void widen16(const uint4 &u, double *out) {
     }
 }
 
+// |x_row - c|^2 (fp64) of 32 rows at once: lane j names row `row` (rows whose
+// bit in `mask` is clear are not read), lane l reads 16-byte chunk l % LPP of
+// rows i * PPL + l / LPP, and a transpose-reduction over the LPP lanes of a
+// row leaves in every lane the distance of row (l % LPP) * PPL + l / LPP.
+template <typename T, int D, bool STREAM>
+__device__ __forceinline__ double dist32(const T *__restrict__ xh, const double *cv, int row, unsigned mask,
+                                         int lane) {
+    using G = SeedGeo<T, D>;
+    const int sub = lane % G::LPP, grp = lane / G::LPP;
+    uint4 buf[G::LPP];
+#pragma unroll
+    for (int i = 0; i < G::LPP; ++i) {
+        const int q = i * G::PPL + grp;
+        const int src = __shfl_sync(0xffffffffu, row, q);
+        const uint4 *pp = reinterpret_cast<const uint4 *>(xh + (size_t)src * D + sub * G::E16);
+        buf[i] = ((mask >> q) & 1u) ? (STREAM ? __ldcs(pp) : __ldg(pp)) : make_uint4(0, 0, 0, 0);
+    }
+    double part[G::LPP];
+#pragma unroll
+    for (int i = 0; i < G::LPP; ++i) {
+        double xv[G::E16];
+        widen16<T>(buf[i], xv);
+        double acc = 0.0;
+#pragma unroll
+        for (int e = 0; e < G::E16; ++e) {
+            const double t = xv[e] - cv[e];
+            acc = fma(t, t, acc);
+        }
+        part[i] = acc;
+    }
+#pragma unroll
+    for (int n = G::LPP; n > 1; n >>= 1) {
+        const int half = n >> 1;
+        const bool up = (lane & half) != 0;
+#pragma unroll
+        for (int k = 0; k < half; ++k) {
+            const double send = up ? part[k] : part[k + half];
+            const double keep = up ? part[k + half] : part[k];
+            part[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+    }
+    return part[0];
+}
+
+// G = number of groups (0: no grouping yet, every point is updated).
 template <typename T, int D>
 __global__ void __launch_bounds__(kSeedThreads)
-kmeanspp_round(const T *__restrict__ x, int N, int K, int r, const double *__restrict__ u,
-               int32_t *idx, double *d2, double *bsum, int *cnt, unsigned char *taken) {
-    const int h = blockIdx.y, nblk = gridDim.x;
-    const T *xh = x + (size_t)h * N * D;
-    double *d2h = d2 + (size_t)h * N;
-    unsigned char *tk = taken + (size_t)h * N;
+kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G) {
+    using Gm = SeedGeo<T, D>;
+    const int h = blockIdx.y, N = s.N, K = s.K, NR = s.NR;
+    const size_t hN = (size_t)h * N;
+    const T *xh = x + hN * D;
+    double *d2h = s.d2 + hN;
+    unsigned char *tk = s.taken + hN;
+    unsigned char *dh = s.dirty + (size_t)h * NR;
+    __shared__ unsigned long long pmax[kSeedCh];  // piece max of D2 (bits), by first offset
+    __shared__ int list[kSeedCh];                 // piece first offsets / dirty ranges
+    __shared__ uint16_t lead[kSeedCh];            // piece first offset of each position
+    __shared__ unsigned char act[kSeedCh];        // piece is updated, by first offset
     __shared__ double sh[kSeedWarps];
-    __shared__ int last, pick_blk;
+    __shared__ int nlist, last, pick_blk;
     __shared__ double sh_base;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int p0 = blockIdx.x * kSeedPts;
-    const int p1 = min(N, p0 + kSeedPts);
+    const int p0 = blockIdx.x * kSeedCh;
+    const int p1 = min(N, p0 + kSeedCh);
 
-    double local = 0.0;
     if (r == 0) {
         // round 0: clear the state; the last block records floor(u * N)
         for (int i = p0 + tid; i < p1; i += kSeedThreads) {
             d2h[i] = __longlong_as_double(0x7ff0000000000000LL);  // +inf
             tk[i] = 0;
+            s.near[hN + i] = 0;
         }
+        for (int k = p0 / kSeedRange + tid; k < (p1 + kSeedRange - 1) / kSeedRange; k += kSeedThreads) dh[k] = 0;
     } else {
-        // D2_i = min(D2_i, |x_i - c|^2) in fp64 (exact products for bf16 and
-        // fp32 inputs): lane l reads 16-byte chunk (l % LPP) of points
-        // base + i * PPL + l / LPP, then a transpose-reduction over the LPP
-        // lanes of a point leaves one point's distance in every lane.
-        using G = SeedGeo<T, D>;
-        const int c = idx[(size_t)h * K + r - 1];
-        const int sub = lane % G::LPP, grp = lane / G::LPP;
-        double cv[G::E16];
-        widen16<T>(*reinterpret_cast<const uint4 *>(xh + (size_t)c * D + sub * G::E16), cv);
+        const int c = s.idx[(size_t)h * K + r - 1];
+        const int sub = lane % Gm::LPP;
+        double cv[Gm::E16];
+        widen16<T>(__ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + sub * Gm::E16)), cv);
+        const bool grouped = G > 0;
+        if (grouped) {
+            // the block's pieces, then the triangle test of each
+            if (tid == 0) nlist = 0;
+            __syncthreads();
+            const uint16_t *po = s.pofs + hN;
+            for (int o = tid; o < p1 - p0; o += kSeedThreads) {
+                const int f = po[p0 + o];
+                lead[o] = (uint16_t)f;
+                if (f == o) list[atomicAdd(&nlist, 1)] = o;
+            }
+            __syncthreads();
+            const int nl = nlist;
+            for (int j0 = warp * 32; j0 < nl; j0 += kSeedWarps * 32) {
+                const int j = j0 + lane;
+                const int o = j < nl ? list[j] : 0;
+                const int arow = j < nl ? __ldg(s.apos + hN + p0 + o) : 0;
+                const unsigned m = __ballot_sync(0xffffffffu, j < nl);
+                const double dc2 = dist32<T, D, false>(xh, cv, arow, m, lane);
+                const int q = (lane % Gm::LPP) * Gm::PPL + lane / Gm::LPP;  // the row this lane holds
+                const int oq = __shfl_sync(0xffffffffu, o, q);
+                if ((m >> q) & 1u) {
+                    const double R = sqrt(s.rr[hN + p0 + oq]);
+                    const double M = sqrt(s.mdp[hN + p0 + oq]);
+                    act[oq] = sqrt(dc2) > (R + M) * (1.0 + kSeedMargin) ? 0 : 1;
+                    pmax[oq] = 0ull;
+                }
+            }
+            __syncthreads();
+        }
+        // D2 update of the positions in updated pieces, 32 at a time per warp
         for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
-            uint4 buf[G::LPP];
-#pragma unroll
-            for (int i = 0; i < G::LPP; ++i) {
-                const int pt = base + i * G::PPL + grp;
-                buf[i] = pt < p1 ? __ldcs(reinterpret_cast<const uint4 *>(xh + (size_t)pt * D + sub * G::E16))
-                                 : make_uint4(0, 0, 0, 0);
-            }
-            double part[G::LPP];
-#pragma unroll
-            for (int i = 0; i < G::LPP; ++i) {
-                double xv[G::E16];
-                widen16<T>(buf[i], xv);
-                double acc = 0.0;
-#pragma unroll
-                for (int e = 0; e < G::E16; ++e) {
-                    const double t = xv[e] - cv[e];
-                    acc = fma(t, t, acc);
+            const int qp = base + lane;
+            const bool al = qp < p1 && (!grouped || act[lead[qp - p0]]);
+            const unsigned m = __ballot_sync(0xffffffffu, al);
+            if (m == 0u) continue;
+            const int pt = grouped ? (al ? s.perm[hN + qp] : 0) : qp;
+            const double dist = dist32<T, D, true>(xh, cv, pt, m, lane);
+            const int q = (lane % Gm::LPP) * Gm::PPL + lane / Gm::LPP;
+            const int i = __shfl_sync(0xffffffffu, pt, q);
+            if ((m >> q) & 1u) {
+                const double old = d2h[i];
+                const double nd = fmin(old, dist);
+                if (nd < old) {
+                    d2h[i] = nd;
+                    s.near[hN + i] = r - 1;
+                    dh[i / kSeedRange] = 1;
                 }
-                part[i] = acc;
-            }
-            // transpose-reduce over the LPP lanes of each point group
-#pragma unroll
-            for (int n = G::LPP; n > 1; n >>= 1) {
-                const int half = n >> 1;
-                const bool up = (lane & half) != 0;
-#pragma unroll
-                for (int k = 0; k < half; ++k) {
-                    const double send = up ? part[k] : part[k + half];
-                    const double keep = up ? part[k + half] : part[k];
-                    part[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-                }
-            }
-            const int i = base + sub * G::PPL + grp;
-            if (i < p1) {
-                const double nd = fmin(d2h[i], part[0]);
-                d2h[i] = nd;
-                local += nd;
+                if (grouped) atomicMax(&pmax[lead[base + q - p0]], (unsigned long long)__double_as_longlong(nd));
             }
         }
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) local += __shfl_xor_sync(0xffffffffu, local, m);
-        if (lane == 0) sh[warp] = local;
-        __syncthreads();
-        if (tid == 0) {
-            double t = 0.0;
-            for (int w = 0; w < kSeedWarps; ++w) t += sh[w];
-            bsum[(size_t)h * nblk + blockIdx.x] = t;
+        if (grouped) {
+            __syncthreads();
+            for (int j = tid; j < nlist; j += kSeedThreads) {
+                const int o = list[j];
+                if (act[o]) s.mdp[hN + p0 + o] = __longlong_as_double((long long)pmax[o]);
+            }
         }
     }
     __threadfence();
     __syncthreads();
     if (tid == 0) {
-        const int old = atomicAdd(&cnt[h], 1);
-        last = (old == nblk - 1);
+        const int old = atomicAdd(&s.cnt[h], 1);
+        last = (old == (int)gridDim.x - 1);
         __threadfence();
     }
     __syncthreads();
     if (!last) return;
 
     // ---------------- last block of head h: choose this round's centre
-    const double ur = u[(size_t)h * K + r];
+    const double ur = s.u[(size_t)h * K + r];
     if (r == 0) {
         if (tid == 0) {
             int pk = (int)floor(ur * (double)N);
             pk = min(max(pk, 0), N - 1);
-            idx[(size_t)h * K] = pk;
+            s.idx[(size_t)h * K] = pk;
             tk[pk] = 1;
-            cnt[h] = 0;
+            s.cnt[h] = 0;
         }
         return;
     }
-    // slice sums -> the slice holding the threshold u * sum(D2)
+    double *bs = s.bsum + (size_t)h * NR;
+    // refresh the sums of the ranges whose D2 changed (fixed order per range:
+    // lane-strided partials, then a butterfly, so every refresh is the same)
+    for (int k0 = 0; k0 < NR; k0 += kSeedThreads) {
+        if (tid == 0) nlist = 0;
+        __syncthreads();
+        const int k = k0 + tid;
+        if (k < NR && __ldcg(dh + k)) list[atomicAdd(&nlist, 1)] = k;
+        __syncthreads();
+        const int nd = nlist;
+        for (int j = warp; j < nd; j += kSeedWarps) {
+            const int kk = list[j];
+            const int q0 = kk * kSeedRange;
+            double v = 0.0;
+#pragma unroll
+            for (int e = 0; e < kSeedRange / 32; ++e) {
+                const int i = q0 + e * 32 + lane;
+                v += i < N ? __ldcg(d2h + i) : 0.0;
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+            if (lane == 0) {
+                bs[kk] = v;
+                dh[kk] = 0;
+            }
+        }
+        __syncthreads();
+    }
     double total = 0.0;
     {
         double v = 0.0;
-        for (int bb = tid; bb < nblk; bb += kSeedThreads) v += __ldcg(bsum + (size_t)h * nblk + bb);
+        for (int k = tid; k < NR; k += kSeedThreads) v += __ldcg(bs + k);
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
         __syncthreads();
@@ -208,57 +335,50 @@ kmeanspp_round(const T *__restrict__ x, int N, int K, int r, const double *__res
     if (total > 0.0) {
         const double thr = ur * total;
         if (tid == 0) pick_blk = 0x7fffffff;
-        // inclusive running sums of the slice sums, chunk by chunk; the first
-        // slice whose running sum exceeds thr holds the pick
+        // inclusive running sums of the range sums, chunk by chunk; the first
+        // range whose running sum exceeds thr holds the pick
         double carry = 0.0;
-        for (int c0 = 0; c0 < nblk; c0 += kSeedThreads) {
-            const int bb = c0 + tid;
-            const double v = bb < nblk ? __ldcg(bsum + (size_t)h * nblk + bb) : 0.0;
+        for (int c0 = 0; c0 < NR; c0 += kSeedThreads) {
+            const int kk = c0 + tid;
+            const double v = kk < NR ? __ldcg(bs + kk) : 0.0;
             const double inc = block_scan_d(v, sh) + carry;
             __syncthreads();
-            if (bb < nblk && inc > thr) atomicMin(&pick_blk, bb);
+            if (kk < NR && inc > thr) atomicMin(&pick_blk, kk);
             if (tid == kSeedThreads - 1) sh[0] = inc;  // carry into the next chunk
             __syncthreads();
             carry = sh[0];
-            if (bb == pick_blk) sh_base = inc - v;  // exclusive running sum of the slice
+            if (kk == pick_blk) sh_base = inc - v;  // exclusive running sum of the range
             __syncthreads();
         }
         int blk = pick_blk;
-        double base_run = blk != 0x7fffffff ? sh_base : 0.0;
-        if (blk == 0x7fffffff) {  // rounding put the threshold past the last sum
-            blk = nblk - 1;
-            base_run = -1.0;      // marks "take the last point with D2 > 0"
-        }
-        __syncthreads();
-        // inside the slice: the first point whose running sum exceeds thr
-        const int q0 = blk * kSeedPts, q1 = min(N, q0 + kSeedPts);
-        constexpr int PT = kSeedPts / kSeedThreads;  // points per thread (4)
-        double dv[PT];
-        double tsum = 0.0;
-#pragma unroll
-        for (int k = 0; k < PT; ++k) {
-            const int i = q0 + tid * PT + k;
-            dv[k] = i < q1 ? __ldcg(d2h + i) : 0.0;
-            tsum += dv[k];
-        }
-        const double inc = block_scan_d(tsum, sh);
+        const bool crossed = blk != 0x7fffffff;
+        const double base_run = crossed ? sh_base : 0.0;
         __syncthreads();
         if (tid == 0) pick_blk = 0x7fffffff;
         __syncthreads();
-        if (base_run >= 0.0) {
-            double run = base_run + inc - tsum;
-#pragma unroll
-            for (int k = 0; k < PT; ++k) {
-                run += dv[k];
-                if (run > thr) {
-                    atomicMin(&pick_blk, q0 + tid * PT + k);
-                    break;
-                }
+        if (crossed) {
+            // inside the range: the first point whose running sum exceeds thr
+            const int q0 = blk * kSeedRange;
+            const int i = q0 + tid;
+            const double dv = (tid < kSeedRange && i < N) ? __ldcg(d2h + i) : 0.0;
+            const double inc = block_scan_d(dv, sh);
+            if (tid < kSeedRange && i < N && base_run + inc > thr) atomicMin(&pick_blk, i);
+            __syncthreads();
+            if (pick_blk == 0x7fffffff) {
+                // rounding: the range's own running sum stayed at or below
+                // thr; take the range's last point with D2 > 0
+                if (tid == 0) pick_blk = -1;
+                __syncthreads();
+                if (tid < kSeedRange && i < N && dv > 0.0) atomicMax(&pick_blk, i);
+                __syncthreads();
+                if (tid == 0 && pick_blk < 0) pick_blk = 0x7fffffff;
+                __syncthreads();
             }
         }
-        __syncthreads();
         if (pick_blk == 0x7fffffff) {
-            // no point crossed thr by rounding: the last point with D2 > 0
+            // no range crossed thr (rounding with u near 1): the last point
+            // with D2 > 0
+            __syncthreads();
             if (tid == 0) pick_blk = -1;
             __syncthreads();
             for (int i = N - 1 - tid; i >= 0; i -= kSeedThreads) {
@@ -286,10 +406,42 @@ kmeanspp_round(const T *__restrict__ x, int N, int K, int r, const double *__res
     }
     if (tid == 0) {
         const int pk = pick_blk;
-        idx[(size_t)h * K + r] = pk;
+        s.idx[(size_t)h * K + r] = pk;
         tk[pk] = 1;
-        cnt[h] = 0;
+        s.cnt[h] = 0;
     }
+}
+
+// ---- regrouping (before round r, with G = r - 1 chosen centres applied)
+//
+// Group g holds the points whose nearest applied centre is centre g; its
+// radius is the largest of their D2 (D2 is exactly the distance to that
+// centre).  Counting sort: histogram and radius, exclusive scan, scatter of
+// the points with their piece offsets and group data.
+
+__global__ void seed_group_hist(const SeedArgs s, int G) {
+    const int h = blockIdx.y, i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= s.N) return;
+    const size_t hi = (size_t)h * s.N + i;
+    const int g = s.near[hi];
+    atomicAdd(&s.gcnt[(size_t)h * G + g], 1);
+    atomicMax(reinterpret_cast<unsigned long long *>(s.r2 + (size_t)h * G + g),
+              (unsigned long long)__double_as_longlong(s.d2[hi]));
+}
+
+__global__ void seed_group_scatter(const SeedArgs s, int G) {
+    const int h = blockIdx.y, i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= s.N) return;
+    const size_t hN = (size_t)h * s.N;
+    const int g = s.near[hN + i];
+    const int pos = atomicAdd(&s.cur[(size_t)h * G + g], 1);
+    const int cs = pos - pos % kSeedCh;
+    const double R2 = s.r2[(size_t)h * G + g];
+    s.perm[hN + pos] = i;
+    s.apos[hN + pos] = s.idx[(size_t)h * s.K + g];
+    s.rr[hN + pos] = R2;
+    s.mdp[hN + pos] = R2;
+    s.pofs[hN + pos] = (uint16_t)(max(s.seg[(size_t)h * (G + 1) + g], cs) - cs);
 }
 
 }  // namespace asmk
@@ -547,29 +699,67 @@ KmWs km_ws(int H, int N, int K) {
 using namespace asmk;
 
 size_t asm_kmeanspp_ws_bytes(int H, int N, int d, int K) {
-    (void)d; (void)K;
-    return seed_ws(H, N).total;
+    (void)d;
+    return seed_ws(H, N, K).total;
+}
+
+template <typename T, int D>
+static void seed_round(const T *x, const SeedArgs &s, int r, int G, int H, cudaStream_t st) {
+    dim3 grid((s.N + kSeedCh - 1) / kSeedCh, H);
+    kmeanspp_round<T, D><<<grid, kSeedThreads, 0, st>>>(x, s, r, G);
 }
 
 cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const double *u,
                                 asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st) {
-    SeedWs w = seed_ws(H, N);
+    const SeedWs w = seed_ws(H, N, K);
     char *b = static_cast<char *>(ws);
-    double *d2 = reinterpret_cast<double *>(b + w.off_d2);
-    double *bsum = reinterpret_cast<double *>(b + w.off_bsum);
-    int *cnt = reinterpret_cast<int *>(b + w.off_cnt);
-    unsigned char *taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
-    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int) * (size_t)H, st);
+    SeedArgs s{};
+    s.u = u;
+    s.idx = init_idx;
+    s.d2 = reinterpret_cast<double *>(b + w.off_d2);
+    s.mdp = reinterpret_cast<double *>(b + w.off_mdp);
+    s.rr = reinterpret_cast<double *>(b + w.off_rr);
+    s.bsum = reinterpret_cast<double *>(b + w.off_bsum);
+    s.r2 = reinterpret_cast<double *>(b + w.off_r2);
+    s.near = reinterpret_cast<int32_t *>(b + w.off_near);
+    s.perm = reinterpret_cast<int32_t *>(b + w.off_perm);
+    s.apos = reinterpret_cast<int32_t *>(b + w.off_apos);
+    s.gcnt = reinterpret_cast<int32_t *>(b + w.off_gcnt);
+    s.seg = reinterpret_cast<int32_t *>(b + w.off_seg);
+    s.cur = reinterpret_cast<int32_t *>(b + w.off_cur);
+    s.pofs = reinterpret_cast<uint16_t *>(b + w.off_pofs);
+    s.dirty = reinterpret_cast<unsigned char *>(b + w.off_dirty);
+    s.taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
+    s.cnt = reinterpret_cast<int *>(b + w.off_cnt);
+    s.N = N;
+    s.K = K;
+    s.NR = (N + kSeedRange - 1) / kSeedRange;
+    cudaError_t e = cudaMemsetAsync(s.cnt, 0, sizeof(int) * (size_t)H, st);
     if (e != cudaSuccess) return e;
-    dim3 grid((N + kSeedPts - 1) / kSeedPts, H);
+    const dim3 pgrid((N + 255) / 256, H);
+    int G = 0, next = kSeedFirstGroup;
     for (int r = 0; r < K; ++r) {
+        if (r == next) {
+            // regroup by the nearest of the r - 1 centres applied so far;
+            // then again each time the centres grow by a quarter of the
+            // largest power of two below r (at least 256 rounds apart)
+            G = r - 1;
+            if ((e = cudaMemsetAsync(s.gcnt, 0, sizeof(int) * (size_t)H * G, st)) != cudaSuccess) return e;
+            if ((e = cudaMemsetAsync(s.r2, 0, sizeof(double) * (size_t)H * G, st)) != cudaSuccess) return e;
+            seed_group_hist<<<pgrid, 256, 0, st>>>(s, G);
+            scan_kernel<<<H, 1024, 0, st>>>(s.gcnt, G, s.seg, s.cur);
+            seed_group_scatter<<<pgrid, 256, 0, st>>>(s, G);
+            int p2 = 1;
+            while (p2 * 2 <= r) p2 *= 2;
+            next = r + max(256, p2 / 4);
+        }
         if (dt == ASM_BF16) {
             using T = __nv_bfloat16;
-            if (d == 128) kmeanspp_round<T, 128><<<grid, kSeedThreads, 0, st>>>((const T *)x, N, K, r, u, init_idx, d2, bsum, cnt, taken);
-            else kmeanspp_round<T, 64><<<grid, kSeedThreads, 0, st>>>((const T *)x, N, K, r, u, init_idx, d2, bsum, cnt, taken);
+            if (d == 128) seed_round<T, 128>((const T *)x, s, r, G, H, st);
+            else seed_round<T, 64>((const T *)x, s, r, G, H, st);
         } else {
-            if (d == 128) kmeanspp_round<float, 128><<<grid, kSeedThreads, 0, st>>>((const float *)x, N, K, r, u, init_idx, d2, bsum, cnt, taken);
-            else kmeanspp_round<float, 64><<<grid, kSeedThreads, 0, st>>>((const float *)x, N, K, r, u, init_idx, d2, bsum, cnt, taken);
+            if (d == 128) seed_round<float, 128>((const float *)x, s, r, G, H, st);
+            else seed_round<float, 64>((const float *)x, s, r, G, H, st);
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

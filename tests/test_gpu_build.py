@@ -119,6 +119,32 @@ def test_kmeanspp_llama_build_config_prefix():
         np.testing.assert_array_equal(idx[h, :192], o[0])
 
 
+@pytest.mark.parametrize("dt,d,N,K", [("bf16", 128, 8192, 1024), ("f32", 64, 5000, 600),
+                                       ("bf16", 64, 3001, 520), ("f32", 128, 2500, 300)])
+def test_kmeanspp_pruned_rounds_match_the_oracle(dt, d, N, K):
+    """Past round 256 the D2 update skips groups of points that the triangle
+    inequality shows cannot move; the picks are those of the full update.
+    Clustered data (so that most groups are skipped), ragged N, both storage
+    types and head dims, several regroupings."""
+    x = inputs.mixture(inputs.BASE_SEED + 40 + d, "seed_q", 2, N, d, 48, 0.3, dt)
+    u = inputs.kmeanspp_uniforms(inputs.BASE_SEED + 41 + N, 2, K)
+    idx = gpu_seed(dev(x), dev(u))
+    np.testing.assert_array_equal(idx, O.kmeanspp_seed(x, u))
+    assert all(len(set(r.tolist())) == r.size for r in idx)
+
+
+def test_kmeanspp_duplicate_points_exhaust_the_distinct_ones():
+    """Fewer distinct points than centres: once every distinct point is
+    chosen, sum(D2) = 0 and the smallest unchosen index is taken, past the
+    regrouping rounds too."""
+    base = inputs.mixture(inputs.BASE_SEED + 42, "seed_q", 1, 200, 64, 8, 0.3, "f32")
+    x = base.repeat(1, 4, 1).contiguous()  # 800 points, 200 distinct
+    u = inputs.kmeanspp_uniforms(inputs.BASE_SEED + 43, 1, 700)
+    idx = gpu_seed(dev(x), dev(u))
+    np.testing.assert_array_equal(idx, O.kmeanspp_seed(x, u))
+    assert len(set(idx[0].tolist())) == 700
+
+
 def kmeans_buffers(H, N, d, K, dtype):
     c = torch.empty(H, K, d, dtype=torch.float32, device="cuda")
     cdt = torch.empty(H, K, d, dtype=dtype, device="cuda")
