@@ -111,7 +111,11 @@ asm_status asm_build_states(const void *q, const void *k, const void *v,
  *   u        [H, K]    fp64 uniform draws in [0, 1), one per round
  *   init_idx [H, K]    int32 output
  *   ws       asm_kmeanspp_workspace_size(H, N, d, K) bytes
- * Requires 1 <= K <= N.
+ * Requires 1 <= K <= N; N > 2^24 returns ASM_ERR_UNSUPPORTED.  The update
+ * skips groups of points that the triangle inequality shows cannot move (a
+ * work saving only: the D2 values and picks are those of the full update).
+ * One kernel launch per round, plus a regrouping (three small launches) on
+ * a schedule; the launches are queued on `stream` without synchronising.
  */
 size_t asm_kmeanspp_workspace_size(int H, int N, int d, int K);
 asm_status asm_kmeanspp_seed(const void *x, int H, int N, int d, int K,

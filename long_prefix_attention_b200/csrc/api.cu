@@ -84,7 +84,7 @@ asm_status asm_kmeanspp_seed(const void *x, int H, int N, int d, int K, const do
                              asm_dtype dt, int32_t *init_idx, void *ws, size_t ws_bytes,
                              cudaStream_t stream) {
     if (!dt_ok(dt) || H < 1 || N < 1 || K < 1 || K > N) return ASM_ERR_INVALID_ARG;
-    if (!d_ok(d)) return ASM_ERR_UNSUPPORTED;
+    if (!d_ok(d) || N > (1 << 24)) return ASM_ERR_UNSUPPORTED;
     if (!aligned(x, 16) || !aligned(u, 8) || !aligned(init_idx, 4)) return ASM_ERR_INVALID_ARG;
     if (!aligned(ws, 16) || ws_bytes < asm_kmeanspp_ws_bytes(H, N, d, K)) return ASM_ERR_WORKSPACE;
     return cuda_status(asm_kmeanspp_launch(x, H, N, d, K, u, dt, init_idx, ws, stream));

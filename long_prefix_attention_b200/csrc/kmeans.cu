@@ -6,6 +6,8 @@
 // cluster's queries).  Seeding is k-means++ (D^2 sampling) with the uniform
 // draws supplied by the caller.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -22,41 +24,51 @@ inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 // One launch per round r.  The centre chosen in round r - 1 lowers D2_i =
 // min(D2_i, |x_i - c|^2) (fp64, exact for bf16 inputs and for the products of
 // fp32 inputs); the last block of each head to arrive (an arrival counter, no
-// waiting) refreshes the partial sums of the ranges whose D2 changed, finds
-// the range holding the threshold u * sum(D2) and the first point inside it
-// whose running sum exceeds the threshold, and records the pick.
+// waiting) refreshes the partial sums of D2 that changed, finds where the
+// running sum first exceeds u * sum(D2) and records the pick.  The partial
+// sums form two levels, each summed in index order: S1 over 32 points and S2
+// over 32 consecutive S1.
 //
-// Exact pruning.  From round kSeedFirstGroup on, the points are grouped by the
+// Exact pruning.  From a regrouping round on, the points are grouped by the
 // chosen centre nearest to them (regrouped on a schedule as centres are
 // added).  Group g has anchor a_g (its centre) and radius R_g = max |x - a_g|
 // over its members; a piece (the part of a group inside one block's range of
-// positions) also keeps M = max sqrt(D2) over its members.  By the triangle
+// positions) also keeps M >= max sqrt(D2) over its members.  By the triangle
 // inequality every member has |x - c| >= |c - a_g| - R_g, so when
 // |c - a_g| > (R_g + M)(1 + 1e-12) no member's D2 can fall and the piece is
-// skipped; the margin covers the rounding of the fp64 distances, so the D2
-// values, and therefore the picks, are those of the unpruned update.
+// skipped; R_g and M are stored rounded up and the margin covers the rounding
+// of the fp64 distances, so the D2 values, and therefore the picks, are those
+// of the unpruned update.
+//
+// Rounds are chained by programmatic dependent launch: a round's blocks read
+// the grouping (static between regroupings) while the previous round ends.
 
 constexpr int kSeedThreads = 256;
 constexpr int kSeedWarps = kSeedThreads / 32;
-constexpr int kSeedCh = 1024;        // positions per block
-constexpr int kSeedRange = 128;      // points per partial sum of D2
-constexpr int kSeedFirstGroup = 256; // first regrouping round
+constexpr int kSeedChMin = 2048;     // positions per block: chosen at launch so
+constexpr int kSeedChMax = 8192;     // that the grid is one wave (multiple of 256)
+constexpr int kSeedS = 32;           // points per S1 sum, S1 sums per S2 sum
+constexpr int kSeedMaxN = 1 << 24;   // S2 dirty bits fit the block's 2 KB bitmap
 constexpr double kSeedMargin = 1e-12;
 
 struct SeedWs {
-    size_t off_d2, off_mdp, off_rr, off_bsum, off_r2, off_near, off_perm, off_apos, off_gcnt, off_seg,
+    size_t off_d2, off_bs1, off_bs2, off_r2, off_mdp, off_rr, off_near, off_perm, off_apos, off_gcnt, off_seg,
         off_cur, off_pofs, off_dirty, off_taken, off_cnt, total;
+    int nr1, nr2, dstride;
 };
 SeedWs seed_ws(int H, int N, int K) {
     const size_t h = (size_t)H, n = (size_t)N, k = (size_t)K;
-    const size_t nr = (n + kSeedRange - 1) / kSeedRange;
     SeedWs w;
+    w.nr1 = (N + kSeedS - 1) / kSeedS;
+    w.nr2 = (w.nr1 + kSeedS - 1) / kSeedS;
+    w.dstride = (w.nr1 + 7) & ~7;  // dirty flags are read 8 at a time
     w.off_d2 = 0;
-    w.off_mdp = al256(w.off_d2 + sizeof(double) * h * n);
-    w.off_rr = al256(w.off_mdp + sizeof(double) * h * n);
-    w.off_bsum = al256(w.off_rr + sizeof(double) * h * n);
-    w.off_r2 = al256(w.off_bsum + sizeof(double) * h * nr);
-    w.off_near = al256(w.off_r2 + sizeof(double) * h * k);
+    w.off_bs1 = al256(w.off_d2 + sizeof(double) * h * n);
+    w.off_bs2 = al256(w.off_bs1 + sizeof(double) * h * w.nr1);
+    w.off_r2 = al256(w.off_bs2 + sizeof(double) * h * w.nr2);
+    w.off_mdp = al256(w.off_r2 + sizeof(double) * h * k);
+    w.off_rr = al256(w.off_mdp + sizeof(float) * h * n);
+    w.off_near = al256(w.off_rr + sizeof(float) * h * n);
     w.off_perm = al256(w.off_near + sizeof(int) * h * n);
     w.off_apos = al256(w.off_perm + sizeof(int) * h * n);
     w.off_gcnt = al256(w.off_apos + sizeof(int) * h * n);
@@ -64,7 +76,7 @@ SeedWs seed_ws(int H, int N, int K) {
     w.off_cur = al256(w.off_seg + sizeof(int) * h * (k + 1));
     w.off_pofs = al256(w.off_cur + sizeof(int) * h * k);
     w.off_dirty = al256(w.off_pofs + sizeof(uint16_t) * h * n);
-    w.off_taken = al256(w.off_dirty + h * nr);
+    w.off_taken = al256(w.off_dirty + h * (size_t)w.dstride);
     w.off_cnt = al256(w.off_taken + h * n);
     w.total = al256(w.off_cnt + sizeof(int) * h);
     return w;
@@ -74,19 +86,19 @@ struct SeedArgs {
     const double *u;
     int32_t *idx;           // [H][K] picks
     double *d2;             // [H][N] D2 by point
-    double *mdp;            // [H][N] piece max of D2, at the piece's first position
-    double *rr;             // [H][N] R^2 of the group of each position
-    double *bsum;           // [H][NR] partial sums of D2 by range of points
+    double *bs1, *bs2;      // [H][NR1], [H][NR2] partial sums of D2
     double *r2;             // [H][G] group R^2 (regrouping scratch)
+    float *mdp;             // [H][N] piece bound M, at the piece's first position
+    float *rr;              // [H][N] R of the group of each position (rounded up)
     int32_t *near;          // [H][N] round of the nearest chosen centre
     int32_t *perm;          // [H][N] point at each position (grouped order)
     int32_t *apos;          // [H][N] anchor point of the group of each position
     int32_t *gcnt, *seg, *cur;  // regrouping scratch: [H][G], [H][G+1], [H][G]
     uint16_t *pofs;         // [H][N] offset of the piece's first position in its block
-    unsigned char *dirty;   // [H][NR] range touched this round
+    unsigned char *dirty;   // [H][DSTRIDE] S1 range touched this round
     unsigned char *taken;   // [H][N] point already chosen
     int *cnt;               // [H] arrival counters
-    int N, K, NR;
+    int N, K, NR1, NR2, DSTRIDE;
 };
 
 // Inclusive prefix sum over the block (fp64); every thread gets its value.
@@ -105,8 +117,18 @@ __device__ __forceinline__ double block_scan_d(double v, double *sh) {
     return v + off;
 }
 
-// D2 update geometry: a point is LPP lanes x 16 bytes; one 16-byte load per
-// lane covers PPL = 32 / LPP points, so a warp reads its 32 points with LPP
+// Inclusive prefix sum over the warp (fp64, fixed order).
+__device__ __forceinline__ double warp_scan_d(double v, int lane) {
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, v, m);
+        if (lane >= m) v += y;
+    }
+    return v;
+}
+
+// D2 geometry: a point is LPP lanes x 16 bytes; one 16-byte load per lane
+// covers PPL = 32 / LPP points, so a warp reads 32 points with LPP
 // independent loads, all issued before any arithmetic.
 template <typename T, int D>
 struct SeedGeo {
@@ -133,16 +155,13 @@ __device__ __forceinline__ void widen16(const uint4 &u, double *out) {
     }
 }
 
-// |x_row - c|^2 (fp64) of 32 rows at once: lane j names row `row` (rows whose
-// bit in `mask` is clear are not read), lane l reads 16-byte chunk l % LPP of
-// rows i * PPL + l / LPP, and a transpose-reduction over the LPP lanes of a
-// row leaves in every lane the distance of row (l % LPP) * PPL + l / LPP.
+// 32 rows at once: lane j names row `row`; rows whose bit in `mask` is clear
+// are not read.  Lane l loads 16-byte chunk l % LPP of rows i * PPL + l / LPP.
 template <typename T, int D, bool STREAM>
-__device__ __forceinline__ double dist32(const T *__restrict__ xh, const double *cv, int row, unsigned mask,
-                                         int lane) {
+__device__ __forceinline__ void load32(const T *__restrict__ xh, int row, unsigned mask, int lane,
+                                       uint4 (&buf)[SeedGeo<T, D>::LPP]) {
     using G = SeedGeo<T, D>;
     const int sub = lane % G::LPP, grp = lane / G::LPP;
-    uint4 buf[G::LPP];
 #pragma unroll
     for (int i = 0; i < G::LPP; ++i) {
         const int q = i * G::PPL + grp;
@@ -150,6 +169,14 @@ __device__ __forceinline__ double dist32(const T *__restrict__ xh, const double 
         const uint4 *pp = reinterpret_cast<const uint4 *>(xh + (size_t)src * D + sub * G::E16);
         buf[i] = ((mask >> q) & 1u) ? (STREAM ? __ldcs(pp) : __ldg(pp)) : make_uint4(0, 0, 0, 0);
     }
+}
+
+// |row - c|^2 (fp64) of the rows load32 read: a transpose-reduction over the
+// LPP lanes of a row leaves in lane l the distance of row
+// (l % LPP) * PPL + l / LPP (the row index seed_row gives).
+template <typename T, int D>
+__device__ __forceinline__ double dist32(const uint4 (&buf)[SeedGeo<T, D>::LPP], const double *cv, int lane) {
+    using G = SeedGeo<T, D>;
     double part[G::LPP];
 #pragma unroll
     for (int i = 0; i < G::LPP; ++i) {
@@ -176,28 +203,123 @@ __device__ __forceinline__ double dist32(const T *__restrict__ xh, const double 
     }
     return part[0];
 }
+// Widen the E16 elements of a 16-byte chunk to fp32 (exact).
+template <typename T>
+__device__ __forceinline__ void widen16f(const uint4 &u, float *out) {
+    if constexpr (sizeof(T) == 4) {
+        out[0] = __uint_as_float(u.x);
+        out[1] = __uint_as_float(u.y);
+        out[2] = __uint_as_float(u.z);
+        out[3] = __uint_as_float(u.w);
+    } else {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            out[2 * e] = __uint_as_float(w[e] << 16);
+            out[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+    }
+}
 
-// G = number of groups (0: no grouping yet, every point is updated).
+// dist32 in fp32 (same lane layout): each of the D terms and partial sums
+// is rounded once, so the result is at most (1 + 2^-24)^(D + 2) times the
+// exact squared distance.
 template <typename T, int D>
+__device__ __forceinline__ float dist32f(const uint4 (&buf)[SeedGeo<T, D>::LPP], const float *cv, int lane) {
+    using G = SeedGeo<T, D>;
+    float part[G::LPP];
+#pragma unroll
+    for (int i = 0; i < G::LPP; ++i) {
+        float xv[G::E16];
+        widen16f<T>(buf[i], xv);
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < G::E16; ++e) {
+            const float t = xv[e] - cv[e];
+            acc = fmaf(t, t, acc);
+        }
+        part[i] = acc;
+    }
+#pragma unroll
+    for (int n = G::LPP; n > 1; n >>= 1) {
+        const int half = n >> 1;
+        const bool up = (lane & half) != 0;
+#pragma unroll
+        for (int k = 0; k < half; ++k) {
+            const float send = up ? part[k] : part[k + half];
+            const float keep = up ? part[k + half] : part[k];
+            part[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+    }
+    return part[0];
+}
+template <typename T, int D>
+__device__ __forceinline__ int seed_row(int lane) {
+    using G = SeedGeo<T, D>;
+    return (lane % G::LPP) * G::PPL + lane / G::LPP;
+}
+
+// GROUPED: G > 0 groups (pruned update; pre = the grouping may be read before
+// the dependency wait, i.e. it was not just rebuilt).  Otherwise every point
+// is updated and each block writes the S1 and S2 sums of its own positions
+// (ch is then a multiple of the S2 range).
+template <typename T, int D, bool GROUPED>
 __global__ void __launch_bounds__(kSeedThreads)
-kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G) {
+kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G, int pre, int ch) {
     using Gm = SeedGeo<T, D>;
-    const int h = blockIdx.y, N = s.N, K = s.K, NR = s.NR;
+    const int h = blockIdx.y, N = s.N, K = s.K;
     const size_t hN = (size_t)h * N;
     const T *xh = x + hN * D;
     double *d2h = s.d2 + hN;
     unsigned char *tk = s.taken + hN;
-    unsigned char *dh = s.dirty + (size_t)h * NR;
-    __shared__ unsigned long long pmax[kSeedCh];  // piece max of D2 (bits), by first offset
-    __shared__ int list[kSeedCh];                 // piece first offsets / dirty ranges
-    __shared__ uint16_t lead[kSeedCh];            // piece first offset of each position
-    __shared__ unsigned char act[kSeedCh];        // piece is updated, by first offset
+    unsigned char *dh = s.dirty + (size_t)h * s.DSTRIDE;
+    // dynamic shared memory, ch positions: point at each position (then the
+    // dirty S1 ranges), piece bound M (float bits) by first offset, piece
+    // first offset of each position, piece first offsets, piece updated (then
+    // the S2 dirty bitmap)
+    extern __shared__ __align__(16) unsigned char seed_smem[];
+    int *pperm = reinterpret_cast<int *>(seed_smem);
+    unsigned *pmax = reinterpret_cast<unsigned *>(pperm + ch);
+    uint16_t *lead = reinterpret_cast<uint16_t *>(pmax + ch);
+    uint16_t *list = lead + ch;
+    unsigned char *act = reinterpret_cast<unsigned char *>(list + ch);
     __shared__ double sh[kSeedWarps];
+    __shared__ double s1own[GROUPED ? 1 : kSeedChMax / kSeedS];
     __shared__ int nlist, last, pick_blk;
     __shared__ double sh_base;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int p0 = blockIdx.x * kSeedCh;
-    const int p1 = min(N, p0 + kSeedCh);
+    const int p0 = blockIdx.x * ch;
+    const int p1 = min(N, p0 + ch);
+    constexpr bool grouped = GROUPED;
+
+    // ---- the block's pieces and the first 256 anchors (static data)
+    int nl = 0, ol = 0;
+    float Rl = 0.f;
+    unsigned am = 0u;
+    uint4 abuf[GROUPED ? Gm::LPP : 1];
+    auto stage = [&]() {
+        if (tid == 0) nlist = 0;
+        __syncthreads();
+        const uint16_t *po = s.pofs + hN;
+        for (int o = tid; o < p1 - p0; o += kSeedThreads) {
+            const int f = po[p0 + o];
+            lead[o] = (uint16_t)f;
+            pperm[o] = s.perm[hN + p0 + o];
+            if (f == o) list[atomicAdd(&nlist, 1)] = (uint16_t)o;
+        }
+        __syncthreads();
+        nl = nlist;
+        const int j = warp * 32 + lane;
+        const bool have = j < nl;
+        ol = have ? list[j] : 0;
+        Rl = have ? s.rr[hN + p0 + ol] : 0.f;
+        const int arow = have ? s.apos[hN + p0 + ol] : 0;
+        am = __ballot_sync(0xffffffffu, have);
+        if constexpr (GROUPED) load32<T, D, false>(xh, arow, am, lane, abuf);
+    };
+    if (grouped && pre) stage();
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (r == 0) {
         // round 0: clear the state; the last block records floor(u * N)
@@ -206,68 +328,99 @@ kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G) {
             tk[i] = 0;
             s.near[hN + i] = 0;
         }
-        for (int k = p0 / kSeedRange + tid; k < (p1 + kSeedRange - 1) / kSeedRange; k += kSeedThreads) dh[k] = 0;
+        for (int k = p0 / kSeedS + tid; k < (p1 + kSeedS - 1) / kSeedS; k += kSeedThreads) dh[k] = 0;
     } else {
+        if (grouped && !pre) stage();
         const int c = s.idx[(size_t)h * K + r - 1];
-        const int sub = lane % Gm::LPP;
+        const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + (lane % Gm::LPP) * Gm::E16));
         double cv[Gm::E16];
-        widen16<T>(__ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + sub * Gm::E16)), cv);
-        const bool grouped = G > 0;
-        if (grouped) {
-            // the block's pieces, then the triangle test of each
-            if (tid == 0) nlist = 0;
-            __syncthreads();
-            const uint16_t *po = s.pofs + hN;
-            for (int o = tid; o < p1 - p0; o += kSeedThreads) {
-                const int f = po[p0 + o];
-                lead[o] = (uint16_t)f;
-                if (f == o) list[atomicAdd(&nlist, 1)] = o;
-            }
-            __syncthreads();
-            const int nl = nlist;
-            for (int j0 = warp * 32; j0 < nl; j0 += kSeedWarps * 32) {
-                const int j = j0 + lane;
-                const int o = j < nl ? list[j] : 0;
-                const int arow = j < nl ? __ldg(s.apos + hN + p0 + o) : 0;
-                const unsigned m = __ballot_sync(0xffffffffu, j < nl);
-                const double dc2 = dist32<T, D, false>(xh, cv, arow, m, lane);
-                const int q = (lane % Gm::LPP) * Gm::PPL + lane / Gm::LPP;  // the row this lane holds
-                const int oq = __shfl_sync(0xffffffffu, o, q);
-                if ((m >> q) & 1u) {
-                    const double R = sqrt(s.rr[hN + p0 + oq]);
-                    const double M = sqrt(s.mdp[hN + p0 + oq]);
-                    act[oq] = sqrt(dc2) > (R + M) * (1.0 + kSeedMargin) ? 0 : 1;
-                    pmax[oq] = 0ull;
+        widen16<T>(craw, cv);
+        if constexpr (GROUPED) {
+            float cvf[Gm::E16];
+            widen16f<T>(craw, cvf);
+            // triangle test of each piece, 256 anchors per pass
+            const int q = seed_row<T, D>(lane);
+            for (int pass = 0; pass * kSeedThreads < nl; ++pass) {
+                if (pass > 0) {
+                    const int j = pass * kSeedThreads + warp * 32 + lane;
+                    const bool have = j < nl;
+                    ol = have ? list[j] : 0;
+                    Rl = have ? s.rr[hN + p0 + ol] : 0.f;
+                    const int arow = have ? s.apos[hN + p0 + ol] : 0;
+                    am = __ballot_sync(0xffffffffu, have);
+                    load32<T, D, false>(xh, arow, am, lane, abuf);
+                }
+                const float Ml = ((am >> lane) & 1u) ? s.mdp[hN + p0 + ol] : 0.f;
+                // fp32 distance, made a lower bound of the exact one by its
+                // rounding bound (1e-5 > (D + 2) 2^-24 relative for D <= 128)
+                const float dc2 = dist32f<T, D>(abuf, cvf, lane);
+                const int oq = __shfl_sync(0xffffffffu, ol, q);
+                const float Rq = __shfl_sync(0xffffffffu, Rl, q);
+                const float Mq = __shfl_sync(0xffffffffu, Ml, q);
+                if ((am >> q) & 1u) {
+                    const double lim = ((double)Rq + (double)Mq) * (1.0 + kSeedMargin);
+                    act[oq] = (double)dc2 * (1.0 - 1e-5) > lim * lim ? 0 : 1;
+                    pmax[oq] = 0u;
                 }
             }
             __syncthreads();
         }
         // D2 update of the positions in updated pieces, 32 at a time per warp
+        const int q = seed_row<T, D>(lane);
         for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
             const int qp = base + lane;
             const bool al = qp < p1 && (!grouped || act[lead[qp - p0]]);
             const unsigned m = __ballot_sync(0xffffffffu, al);
             if (m == 0u) continue;
-            const int pt = grouped ? (al ? s.perm[hN + qp] : 0) : qp;
-            const double dist = dist32<T, D, true>(xh, cv, pt, m, lane);
-            const int q = (lane % Gm::LPP) * Gm::PPL + lane / Gm::LPP;
+            const int pt = grouped ? (al ? pperm[qp - p0] : 0) : qp;
+            uint4 buf[Gm::LPP];
+            load32<T, D, true>(xh, pt, m, lane, buf);
             const int i = __shfl_sync(0xffffffffu, pt, q);
-            if ((m >> q) & 1u) {
-                const double old = d2h[i];
+            const bool mine = (m >> q) & 1u;
+            const double old = mine ? d2h[i] : 0.0;
+            const double dist = dist32<T, D>(buf, cv, lane);
+            if (mine) {
                 const double nd = fmin(old, dist);
                 if (nd < old) {
                     d2h[i] = nd;
                     s.near[hN + i] = r - 1;
-                    dh[i / kSeedRange] = 1;
+                    if (grouped) dh[i / kSeedS] = 1;
                 }
-                if (grouped) atomicMax(&pmax[lead[base + q - p0]], (unsigned long long)__double_as_longlong(nd));
+                if (grouped) atomicMax(&pmax[lead[base + q - p0]], __float_as_uint(__double2float_ru(sqrt(nd))));
             }
         }
+        __syncthreads();
         if (grouped) {
-            __syncthreads();
-            for (int j = tid; j < nlist; j += kSeedThreads) {
+            for (int j = tid; j < nl; j += kSeedThreads) {
                 const int o = list[j];
-                if (act[o]) s.mdp[hN + p0 + o] = __longlong_as_double((long long)pmax[o]);
+                if (act[o]) s.mdp[hN + p0 + o] = __uint_as_float(pmax[o]);
+            }
+        } else {
+            // the block's own S1 sums (index order), then its S2 sums
+            double *b1 = s.bs1 + (size_t)h * s.NR1;
+            const int k0 = p0 / kSeedS, k1 = (p1 + kSeedS - 1) / kSeedS;
+            for (int k = k0 + tid; k < k1; k += kSeedThreads) {
+                const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
+                double v = 0.0;
+                if (q1 - q0 == kSeedS) {
+                    double t[kSeedS];
+#pragma unroll
+                    for (int e = 0; e < kSeedS; ++e) t[e] = __ldcg(d2h + q0 + e);
+#pragma unroll
+                    for (int e = 0; e < kSeedS; ++e) v += t[e];
+                } else {
+                    for (int i2 = q0; i2 < q1; ++i2) v += __ldcg(d2h + i2);
+                }
+                b1[k] = v;
+                s1own[k - k0] = v;
+            }
+            __syncthreads();
+            const int m0 = k0 / kSeedS, m1 = (k1 + kSeedS - 1) / kSeedS;
+            for (int k2 = m0 + tid; k2 < m1; k2 += kSeedThreads) {
+                const int a0 = k2 * kSeedS, a1 = min(s.NR1, a0 + kSeedS);
+                double v = 0.0;
+                for (int k = a0; k < a1; ++k) v += s1own[k - k0];
+                s.bs2[(size_t)h * s.NR2 + k2] = v;
             }
         }
     }
@@ -293,38 +446,64 @@ kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G) {
         }
         return;
     }
-    double *bs = s.bsum + (size_t)h * NR;
-    // refresh the sums of the ranges whose D2 changed (fixed order per range:
-    // lane-strided partials, then a butterfly, so every refresh is the same)
-    for (int k0 = 0; k0 < NR; k0 += kSeedThreads) {
+    const int NR1 = s.NR1, NR2 = s.NR2;
+    double *b1 = s.bs1 + (size_t)h * NR1;
+    double *b2 = s.bs2 + (size_t)h * NR2;
+    // S1 sums of the ranges touched this round (each in index order), and
+    // the S2 sums over them
+    uint32_t *sd2 = reinterpret_cast<uint32_t *>(act);  // S2 dirty bitmap
+    int *dl = pperm;                                    // dirty S1 ranges
+    if constexpr (GROUPED) {
+    for (int i = tid; i < (NR2 + 31) / 32; i += kSeedThreads) sd2[i] = 0u;
+    for (int k0 = 0; k0 < NR1; k0 += kSeedThreads * 8) {
         if (tid == 0) nlist = 0;
         __syncthreads();
-        const int k = k0 + tid;
-        if (k < NR && __ldcg(dh + k)) list[atomicAdd(&nlist, 1)] = k;
+        const int kb = k0 + tid * 8;
+        if (kb < NR1) {
+            const uint2 f = __ldcg(reinterpret_cast<const uint2 *>(dh + kb));
+            const unsigned long long bits = (unsigned long long)f.x | ((unsigned long long)f.y << 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (((bits >> (8 * e)) & 0xffull) && kb + e < NR1) {
+                    const int k = kb + e;
+                    dl[atomicAdd(&nlist, 1)] = k;
+                    atomicOr(&sd2[k >> 10], 1u << ((k >> 5) & 31));
+                }
+        }
         __syncthreads();
         const int nd = nlist;
-        for (int j = warp; j < nd; j += kSeedWarps) {
-            const int kk = list[j];
-            const int q0 = kk * kSeedRange;
+        for (int j = tid; j < nd; j += kSeedThreads) {
+            const int k = dl[j];
+            const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
             double v = 0.0;
+            if (q1 - q0 == kSeedS) {
+                double t[kSeedS];
 #pragma unroll
-            for (int e = 0; e < kSeedRange / 32; ++e) {
-                const int i = q0 + e * 32 + lane;
-                v += i < N ? __ldcg(d2h + i) : 0.0;
-            }
+                for (int e = 0; e < kSeedS; ++e) t[e] = __ldcg(d2h + q0 + e);
 #pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-            if (lane == 0) {
-                bs[kk] = v;
-                dh[kk] = 0;
+                for (int e = 0; e < kSeedS; ++e) v += t[e];
+            } else {
+                for (int i = q0; i < q1; ++i) v += __ldcg(d2h + i);
             }
+            b1[k] = v;
+            dh[k] = 0;
         }
         __syncthreads();
     }
+    for (int k2 = tid; k2 < NR2; k2 += kSeedThreads) {
+        if ((sd2[k2 >> 5] >> (k2 & 31)) & 1u) {
+            const int k0 = k2 * kSeedS, k1 = min(NR1, k0 + kSeedS);
+            double v = 0.0;
+            for (int k = k0; k < k1; ++k) v += __ldcg(b1 + k);
+            b2[k2] = v;
+        }
+    }
+    }
+    __syncthreads();
     double total = 0.0;
     {
         double v = 0.0;
-        for (int k = tid; k < NR; k += kSeedThreads) v += __ldcg(bs + k);
+        for (int k = tid; k < NR2; k += kSeedThreads) v += __ldcg(b2 + k);
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
         __syncthreads();
@@ -335,47 +514,51 @@ kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G) {
     if (total > 0.0) {
         const double thr = ur * total;
         if (tid == 0) pick_blk = 0x7fffffff;
-        // inclusive running sums of the range sums, chunk by chunk; the first
-        // range whose running sum exceeds thr holds the pick
+        // the first S2 range whose running sum exceeds thr
         double carry = 0.0;
-        for (int c0 = 0; c0 < NR; c0 += kSeedThreads) {
+        for (int c0 = 0; c0 < NR2; c0 += kSeedThreads) {
             const int kk = c0 + tid;
-            const double v = kk < NR ? __ldcg(bs + kk) : 0.0;
+            const double v = kk < NR2 ? __ldcg(b2 + kk) : 0.0;
             const double inc = block_scan_d(v, sh) + carry;
             __syncthreads();
-            if (kk < NR && inc > thr) atomicMin(&pick_blk, kk);
+            if (kk < NR2 && inc > thr) atomicMin(&pick_blk, kk);
             if (tid == kSeedThreads - 1) sh[0] = inc;  // carry into the next chunk
             __syncthreads();
             carry = sh[0];
-            if (kk == pick_blk) sh_base = inc - v;  // exclusive running sum of the range
+            if (kk == pick_blk) sh_base = inc - v;  // exclusive running sum
             __syncthreads();
         }
-        int blk = pick_blk;
-        const bool crossed = blk != 0x7fffffff;
-        const double base_run = crossed ? sh_base : 0.0;
+        const int k2 = pick_blk;
+        const double base2 = sh_base;
         __syncthreads();
-        if (tid == 0) pick_blk = 0x7fffffff;
-        __syncthreads();
-        if (crossed) {
-            // inside the range: the first point whose running sum exceeds thr
-            const int q0 = blk * kSeedRange;
-            const int i = q0 + tid;
-            const double dv = (tid < kSeedRange && i < N) ? __ldcg(d2h + i) : 0.0;
-            const double inc = block_scan_d(dv, sh);
-            if (tid < kSeedRange && i < N && base_run + inc > thr) atomicMin(&pick_blk, i);
-            __syncthreads();
-            if (pick_blk == 0x7fffffff) {
-                // rounding: the range's own running sum stayed at or below
-                // thr; take the range's last point with D2 > 0
-                if (tid == 0) pick_blk = -1;
-                __syncthreads();
-                if (tid < kSeedRange && i < N && dv > 0.0) atomicMax(&pick_blk, i);
-                __syncthreads();
-                if (tid == 0 && pick_blk < 0) pick_blk = 0x7fffffff;
-                __syncthreads();
+        if (warp == 0) {
+            // then the S1 range, then the point; at either level, when
+            // rounding keeps the running sum at or below thr inside the
+            // chosen range, its last element with positive mass is taken
+            int pk = -1;
+            if (k2 != 0x7fffffff) {
+                const int k = k2 * kSeedS + lane;
+                const double v1 = k < NR1 ? __ldcg(b1 + k) : 0.0;
+                const double inc1 = warp_scan_d(v1, lane);
+                const unsigned cr1 = __ballot_sync(0xffffffffu, k < NR1 && base2 + inc1 > thr);
+                const unsigned pos1 = __ballot_sync(0xffffffffu, v1 > 0.0);
+                const int l1 = cr1 ? __ffs(cr1) - 1 : (pos1 ? 31 - __clz(pos1) : -1);
+                if (l1 >= 0) {
+                    const double b1x = base2 + __shfl_sync(0xffffffffu, inc1 - v1, l1);
+                    const bool exact1 = cr1 != 0u;
+                    const int i = (k2 * kSeedS + l1) * kSeedS + lane;
+                    const double v0 = i < N ? __ldcg(d2h + i) : 0.0;
+                    const double inc0 = warp_scan_d(v0, lane);
+                    const unsigned cr0 = exact1 ? __ballot_sync(0xffffffffu, i < N && b1x + inc0 > thr) : 0u;
+                    const unsigned pos0 = __ballot_sync(0xffffffffu, v0 > 0.0);
+                    const int l0 = cr0 ? __ffs(cr0) - 1 : (pos0 ? 31 - __clz(pos0) : -1);
+                    if (l0 >= 0) pk = (k2 * kSeedS + l1) * kSeedS + l0;
+                }
             }
+            if (lane == 0) pick_blk = pk;
         }
-        if (pick_blk == 0x7fffffff) {
+        __syncthreads();
+        if (pick_blk < 0) {
             // no range crossed thr (rounding with u near 1): the last point
             // with D2 > 0
             __syncthreads();
@@ -429,18 +612,18 @@ __global__ void seed_group_hist(const SeedArgs s, int G) {
               (unsigned long long)__double_as_longlong(s.d2[hi]));
 }
 
-__global__ void seed_group_scatter(const SeedArgs s, int G) {
+__global__ void seed_group_scatter(const SeedArgs s, int G, int ch) {
     const int h = blockIdx.y, i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= s.N) return;
     const size_t hN = (size_t)h * s.N;
     const int g = s.near[hN + i];
     const int pos = atomicAdd(&s.cur[(size_t)h * G + g], 1);
-    const int cs = pos - pos % kSeedCh;
-    const double R2 = s.r2[(size_t)h * G + g];
+    const int cs = pos - pos % ch;
+    const float R = __double2float_ru(sqrt(s.r2[(size_t)h * G + g]));
     s.perm[hN + pos] = i;
     s.apos[hN + pos] = s.idx[(size_t)h * s.K + g];
-    s.rr[hN + pos] = R2;
-    s.mdp[hN + pos] = R2;
+    s.rr[hN + pos] = R;
+    s.mdp[hN + pos] = R;
     s.pofs[hN + pos] = (uint16_t)(max(s.seg[(size_t)h * (G + 1) + g], cs) - cs);
 }
 
@@ -703,24 +886,102 @@ size_t asm_kmeanspp_ws_bytes(int H, int N, int d, int K) {
     return seed_ws(H, N, K).total;
 }
 
-template <typename T, int D>
-static void seed_round(const T *x, const SeedArgs &s, int r, int G, int H, cudaStream_t st) {
-    dim3 grid((s.N + kSeedCh - 1) / kSeedCh, H);
-    kmeanspp_round<T, D><<<grid, kSeedThreads, 0, st>>>(x, s, r, G);
+namespace {
+// dynamic shared memory of a grouped round (13 bytes per position)
+constexpr size_t seed_smem_bytes(int ch, bool grouped) { return grouped ? (size_t)13 * ch : 0; }
+
+// Positions per block: the smallest multiple of `step` (at least kSeedChMin)
+// for which every head's blocks fit the GPU in one wave, else kSeedChMax.
+template <typename T, int D, bool GROUPED>
+int seed_block_positions(int H, int N, cudaError_t *err) {
+    auto k = kmeanspp_round<T, D, GROUPED>;
+    constexpr int step = GROUPED ? 256 : kSeedS * kSeedS;
+    static bool attr = false;
+    if (!attr) {
+        *err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)seed_smem_bytes(kSeedChMax, GROUPED));
+        if (*err != cudaSuccess) return 0;
+        attr = true;
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+    for (int ch = kSeedChMin; ch <= kSeedChMax; ch += step) {
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kSeedThreads, seed_smem_bytes(ch, GROUPED)) !=
+            cudaSuccess)
+            break;
+        if ((long)H * ((N + ch - 1) / ch) <= (long)occ * sms) return ch;
+    }
+    (void)cudaGetLastError();
+    return kSeedChMax;
 }
+
+template <typename T, int D, bool GROUPED>
+cudaError_t seed_round(const T *x, const SeedArgs &s, int r, int G, int pre, int ch, int H, cudaStream_t st) {
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((s.N + ch - 1) / ch, H);
+    cfg.blockDim = dim3(kSeedThreads);
+    cfg.dynamicSmemBytes = seed_smem_bytes(ch, GROUPED);
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kmeanspp_round<T, D, GROUPED>, x, s, r, G, pre, ch);
+}
+
+template <typename T, int D>
+cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
+    const int chf = seed_block_positions<T, D, false>(H, s.N, &e);
+    if (e != cudaSuccess) return e;
+    const int chg = seed_block_positions<T, D, true>(H, s.N, &e);
+    if (e != cudaSuccess) return e;
+    const int N = s.N, K = s.K;
+    const dim3 pgrid((N + 255) / 256, H);
+    int G = 0, next = std::max(256, K / 8);
+    for (int r = 0; r < K; ++r) {
+        int pre = 1;
+        if (r == next) {
+            // regroup by the nearest of the r - 1 centres applied so far;
+            // then again each time the centres grow by a quarter of the
+            // largest power of two below r (at least 256 rounds apart)
+            G = r - 1;
+            pre = 0;
+            if ((e = cudaMemsetAsync(s.gcnt, 0, sizeof(int) * (size_t)H * G, st)) != cudaSuccess) return e;
+            if ((e = cudaMemsetAsync(s.r2, 0, sizeof(double) * (size_t)H * G, st)) != cudaSuccess) return e;
+            seed_group_hist<<<pgrid, 256, 0, st>>>(s, G);
+            scan_kernel<<<H, 1024, 0, st>>>(s.gcnt, G, s.seg, s.cur);
+            seed_group_scatter<<<pgrid, 256, 0, st>>>(s, G, chg);
+            int p2 = 1;
+            while (p2 * 2 <= r) p2 *= 2;
+            next = r + std::max(256, p2 / 4);
+        }
+        e = G > 0 ? seed_round<T, D, true>(x, s, r, G, pre, chg, H, st)
+                  : seed_round<T, D, false>(x, s, r, 0, 0, chf, H, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+}  // namespace
 
 cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const double *u,
                                 asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st) {
+    if (N > kSeedMaxN) return cudaErrorInvalidValue;
     const SeedWs w = seed_ws(H, N, K);
     char *b = static_cast<char *>(ws);
     SeedArgs s{};
     s.u = u;
     s.idx = init_idx;
     s.d2 = reinterpret_cast<double *>(b + w.off_d2);
-    s.mdp = reinterpret_cast<double *>(b + w.off_mdp);
-    s.rr = reinterpret_cast<double *>(b + w.off_rr);
-    s.bsum = reinterpret_cast<double *>(b + w.off_bsum);
+    s.bs1 = reinterpret_cast<double *>(b + w.off_bs1);
+    s.bs2 = reinterpret_cast<double *>(b + w.off_bs2);
     s.r2 = reinterpret_cast<double *>(b + w.off_r2);
+    s.mdp = reinterpret_cast<float *>(b + w.off_mdp);
+    s.rr = reinterpret_cast<float *>(b + w.off_rr);
     s.near = reinterpret_cast<int32_t *>(b + w.off_near);
     s.perm = reinterpret_cast<int32_t *>(b + w.off_perm);
     s.apos = reinterpret_cast<int32_t *>(b + w.off_apos);
@@ -733,38 +994,16 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
     s.cnt = reinterpret_cast<int *>(b + w.off_cnt);
     s.N = N;
     s.K = K;
-    s.NR = (N + kSeedRange - 1) / kSeedRange;
+    s.NR1 = w.nr1;
+    s.NR2 = w.nr2;
+    s.DSTRIDE = w.dstride;
     cudaError_t e = cudaMemsetAsync(s.cnt, 0, sizeof(int) * (size_t)H, st);
     if (e != cudaSuccess) return e;
-    const dim3 pgrid((N + 255) / 256, H);
-    int G = 0, next = kSeedFirstGroup;
-    for (int r = 0; r < K; ++r) {
-        if (r == next) {
-            // regroup by the nearest of the r - 1 centres applied so far;
-            // then again each time the centres grow by a quarter of the
-            // largest power of two below r (at least 256 rounds apart)
-            G = r - 1;
-            if ((e = cudaMemsetAsync(s.gcnt, 0, sizeof(int) * (size_t)H * G, st)) != cudaSuccess) return e;
-            if ((e = cudaMemsetAsync(s.r2, 0, sizeof(double) * (size_t)H * G, st)) != cudaSuccess) return e;
-            seed_group_hist<<<pgrid, 256, 0, st>>>(s, G);
-            scan_kernel<<<H, 1024, 0, st>>>(s.gcnt, G, s.seg, s.cur);
-            seed_group_scatter<<<pgrid, 256, 0, st>>>(s, G);
-            int p2 = 1;
-            while (p2 * 2 <= r) p2 *= 2;
-            next = r + max(256, p2 / 4);
-        }
-        if (dt == ASM_BF16) {
-            using T = __nv_bfloat16;
-            if (d == 128) seed_round<T, 128>((const T *)x, s, r, G, H, st);
-            else seed_round<T, 64>((const T *)x, s, r, G, H, st);
-        } else {
-            if (d == 128) seed_round<float, 128>((const float *)x, s, r, G, H, st);
-            else seed_round<float, 64>((const float *)x, s, r, G, H, st);
-        }
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+    if (dt == ASM_BF16) {
+        using T = __nv_bfloat16;
+        return d == 128 ? seed_all<T, 128>((const T *)x, s, H, st) : seed_all<T, 64>((const T *)x, s, H, st);
     }
-    return cudaSuccess;
+    return d == 128 ? seed_all<float, 128>((const float *)x, s, H, st) : seed_all<float, 64>((const float *)x, s, H, st);
 }
 
 size_t asm_kmeans_ws_bytes(int H, int N, int d, int K) {
