@@ -24,21 +24,24 @@ inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 // One launch per round r.  The centre chosen in round r - 1 lowers D2_i =
 // min(D2_i, |x_i - c|^2) (fp64, exact for bf16 inputs and for the products of
 // fp32 inputs); the last block of each head to arrive (an arrival counter, no
-// waiting) refreshes the partial sums of D2 that changed, finds where the
-// running sum first exceeds u * sum(D2) and records the pick.  The partial
-// sums form two levels, each summed in index order: S1 over 32 points and S2
-// over 32 consecutive S1.
+// waiting) brings the partial sums of D2 up to date, finds where the running
+// sum first exceeds u * sum(D2) and records the pick.  The partial sums form
+// two levels, each summed in index order: S1 over 32 points and S2 over 32
+// consecutive S1.
 //
 // Exact pruning.  From a regrouping round on, the points are grouped by the
 // chosen centre nearest to them (regrouped on a schedule as centres are
 // added).  Group g has anchor a_g (its centre) and radius R_g = max |x - a_g|
 // over its members; a piece (the part of a group inside one block's range of
 // positions) also keeps M >= max sqrt(D2) over its members.  By the triangle
-// inequality every member has |x - c| >= |c - a_g| - R_g, so when
-// |c - a_g| > (R_g + M)(1 + 1e-12) no member's D2 can fall and the piece is
-// skipped; R_g and M are stored rounded up and the margin covers the rounding
-// of the fp64 distances, so the D2 values, and therefore the picks, are those
-// of the unpruned update.
+// inequality every member has |x - c| >= |c - a_g| - R_g, so when a lower
+// bound of |c - a_g| exceeds R_g + M no member's D2 can fall and the piece is
+// skipped.  The lower bound comes from int8 copies of c and a_g with
+// power-of-two scales: |c - a| >= |c' - a'| - |c - c'| - |a - a'|, where
+// |c' - a'|^2 is formed from an exact integer dot product and the two
+// quantisation errors are computed exactly and rounded up.  R_g and M are
+// stored rounded up and the margins cover the fp64 rounding, so the D2
+// values, and therefore the picks, are those of the unpruned update.
 //
 // Rounds are chained by programmatic dependent launch: a round's blocks read
 // the grouping (static between regroupings) while the previous round ends.
@@ -46,36 +49,47 @@ inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 constexpr int kSeedThreads = 256;
 constexpr int kSeedWarps = kSeedThreads / 32;
 constexpr int kSeedChMin = 2048;     // positions per block: chosen at launch so
-constexpr int kSeedChMax = 8192;     // that the grid is one wave (multiple of 256)
+constexpr int kSeedChMax = 8192;     // that the grid is one wave
 constexpr int kSeedS = 32;           // points per S1 sum, S1 sums per S2 sum
 constexpr int kSeedMaxN = 1 << 24;   // S2 dirty bits fit the block's 2 KB bitmap
 constexpr double kSeedMargin = 1e-12;
+constexpr int kSeedScreen = 128;      // first round of the fp32 screen
 
 struct SeedWs {
-    size_t off_d2, off_bs1, off_bs2, off_r2, off_mdp, off_rr, off_near, off_perm, off_apos, off_gcnt, off_seg,
-        off_cur, off_pofs, off_dirty, off_taken, off_cnt, total;
-    int nr1, nr2, dstride;
+    size_t off_d2, off_bs1, off_bs2, off_r2, off_gs, off_ge, off_gr, off_gn, off_near, off_perm, off_gcnt, off_seg,
+        off_cur, off_pg, off_pm, off_plo, off_phi, off_pcnt, off_gq, off_dirty, off_taken, off_cnt, total;
+    int nr1, nr2, dstride, nbmax;
+    size_t cap;
 };
-SeedWs seed_ws(int H, int N, int K) {
+SeedWs seed_ws(int H, int N, int d, int K) {
     const size_t h = (size_t)H, n = (size_t)N, k = (size_t)K;
     SeedWs w;
     w.nr1 = (N + kSeedS - 1) / kSeedS;
     w.nr2 = (w.nr1 + kSeedS - 1) / kSeedS;
     w.dstride = (w.nr1 + 7) & ~7;  // dirty flags are read 8 at a time
+    w.nbmax = (N + kSeedChMin - 1) / kSeedChMin + 1;
+    // piece records of block b start at b * (ch + 1): at most N + N / ch + ch + 1
+    w.cap = n + (size_t)w.nbmax + kSeedChMax + 1;
     w.off_d2 = 0;
     w.off_bs1 = al256(w.off_d2 + sizeof(double) * h * n);
     w.off_bs2 = al256(w.off_bs1 + sizeof(double) * h * w.nr1);
     w.off_r2 = al256(w.off_bs2 + sizeof(double) * h * w.nr2);
-    w.off_mdp = al256(w.off_r2 + sizeof(double) * h * k);
-    w.off_rr = al256(w.off_mdp + sizeof(float) * h * n);
-    w.off_near = al256(w.off_rr + sizeof(float) * h * n);
+    w.off_gs = al256(w.off_r2 + sizeof(double) * h * k);
+    w.off_ge = al256(w.off_gs + sizeof(float) * h * k);
+    w.off_gr = al256(w.off_ge + sizeof(float) * h * k);
+    w.off_gn = al256(w.off_gr + sizeof(float) * h * k);
+    w.off_near = al256(w.off_gn + sizeof(int) * h * k);
     w.off_perm = al256(w.off_near + sizeof(int) * h * n);
-    w.off_apos = al256(w.off_perm + sizeof(int) * h * n);
-    w.off_gcnt = al256(w.off_apos + sizeof(int) * h * n);
+    w.off_gcnt = al256(w.off_perm + sizeof(int) * h * n);
     w.off_seg = al256(w.off_gcnt + sizeof(int) * h * k);
     w.off_cur = al256(w.off_seg + sizeof(int) * h * (k + 1));
-    w.off_pofs = al256(w.off_cur + sizeof(int) * h * k);
-    w.off_dirty = al256(w.off_pofs + sizeof(uint16_t) * h * n);
+    w.off_pg = al256(w.off_cur + sizeof(int) * h * k);
+    w.off_pm = al256(w.off_pg + sizeof(int) * h * w.cap);
+    w.off_plo = al256(w.off_pm + sizeof(float) * h * w.cap);
+    w.off_phi = al256(w.off_plo + sizeof(uint16_t) * h * w.cap);
+    w.off_pcnt = al256(w.off_phi + sizeof(uint16_t) * h * w.cap);
+    w.off_gq = al256(w.off_pcnt + sizeof(int) * h * (size_t)w.nbmax);
+    w.off_dirty = al256(w.off_gq + h * k * (size_t)d);
     w.off_taken = al256(w.off_dirty + h * (size_t)w.dstride);
     w.off_cnt = al256(w.off_taken + h * n);
     w.total = al256(w.off_cnt + sizeof(int) * h);
@@ -88,17 +102,21 @@ struct SeedArgs {
     double *d2;             // [H][N] D2 by point
     double *bs1, *bs2;      // [H][NR1], [H][NR2] partial sums of D2
     double *r2;             // [H][G] group R^2 (regrouping scratch)
-    float *mdp;             // [H][N] piece bound M, at the piece's first position
-    float *rr;              // [H][N] R of the group of each position (rounded up)
+    float *gs, *ge, *gr;    // [H][G] anchor scale, anchor quantisation error, R (rounded up)
+    int32_t *gn;            // [H][G] |int8 anchor|^2
+    int8_t *gq;             // [H][G][D] int8 anchor
     int32_t *near;          // [H][N] round of the nearest chosen centre
     int32_t *perm;          // [H][N] point at each position (grouped order)
-    int32_t *apos;          // [H][N] anchor point of the group of each position
     int32_t *gcnt, *seg, *cur;  // regrouping scratch: [H][G], [H][G+1], [H][G]
-    uint16_t *pofs;         // [H][N] offset of the piece's first position in its block
+    int32_t *pg;            // [H][CAP] piece records: group,
+    float *pm;              //   bound M (rounded up),
+    uint16_t *plo, *phi;    //   first and end offset in the block
+    int32_t *pcnt;          // [H][NBMAX] pieces of each block
     unsigned char *dirty;   // [H][DSTRIDE] S1 range touched this round
     unsigned char *taken;   // [H][N] point already chosen
     int *cnt;               // [H] arrival counters
-    int N, K, NR1, NR2, DSTRIDE;
+    int N, K, NR1, NR2, DSTRIDE, NBMAX;
+    size_t CAP;
 };
 
 // Inclusive prefix sum over the block (fp64); every thread gets its value.
@@ -203,6 +221,13 @@ __device__ __forceinline__ double dist32(const uint4 (&buf)[SeedGeo<T, D>::LPP],
     }
     return part[0];
 }
+template <typename T, int D>
+__device__ __forceinline__ int seed_row(int lane) {
+    using G = SeedGeo<T, D>;
+    return (lane % G::LPP) * G::PPL + lane / G::LPP;
+}
+
+
 // Widen the E16 elements of a 16-byte chunk to fp32 (exact).
 template <typename T>
 __device__ __forceinline__ void widen16f(const uint4 &u, float *out) {
@@ -221,9 +246,10 @@ __device__ __forceinline__ void widen16f(const uint4 &u, float *out) {
     }
 }
 
-// dist32 in fp32 (same lane layout): each of the D terms and partial sums
-// is rounded once, so the result is at most (1 + 2^-24)^(D + 2) times the
-// exact squared distance.
+
+// dist32 in fp32 (same lane layout): each of the D terms and partial sums is
+// rounded once, so the result is within (D + 2) 2^-24 < 1e-5 (D <= 128)
+// relative of the exact squared distance.
 template <typename T, int D>
 __device__ __forceinline__ float dist32f(const uint4 (&buf)[SeedGeo<T, D>::LPP], const float *cv, int lane) {
     using G = SeedGeo<T, D>;
@@ -253,188 +279,147 @@ __device__ __forceinline__ float dist32f(const uint4 (&buf)[SeedGeo<T, D>::LPP],
     }
     return part[0];
 }
-template <typename T, int D>
-__device__ __forceinline__ int seed_row(int lane) {
-    using G = SeedGeo<T, D>;
-    return (lane % G::LPP) * G::PPL + lane / G::LPP;
+
+// A point's D2 can fall only if its fp32 distance, lowered by its rounding
+// bound, is not above D2 (with the fp64 margin): otherwise the exact update
+// would leave D2 as it is.
+__device__ __forceinline__ bool seed_may_fall(float d32, double old) {
+    return !((double)d32 * (1.0 - 1e-5) > old * (1.0 + kSeedMargin));
 }
 
-// GROUPED: G > 0 groups (pruned update; pre = the grouping may be read before
-// the dependency wait, i.e. it was not just rebuilt).  Otherwise every point
-// is updated and each block writes the S1 and S2 sums of its own positions
-// (ch is then a multiple of the S2 range).
-template <typename T, int D, bool GROUPED>
-__global__ void __launch_bounds__(kSeedThreads)
-kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G, int pre, int ch) {
-    using Gm = SeedGeo<T, D>;
-    const int h = blockIdx.y, N = s.N, K = s.K;
-    const size_t hN = (size_t)h * N;
-    const T *xh = x + hN * D;
-    double *d2h = s.d2 + hN;
-    unsigned char *tk = s.taken + hN;
-    unsigned char *dh = s.dirty + (size_t)h * s.DSTRIDE;
-    // dynamic shared memory, ch positions: point at each position (then the
-    // dirty S1 ranges), piece bound M (float bits) by first offset, piece
-    // first offset of each position, piece first offsets, piece updated (then
-    // the S2 dirty bitmap)
-    extern __shared__ __align__(16) unsigned char seed_smem[];
-    int *pperm = reinterpret_cast<int *>(seed_smem);
-    unsigned *pmax = reinterpret_cast<unsigned *>(pperm + ch);
-    uint16_t *lead = reinterpret_cast<uint16_t *>(pmax + ch);
-    uint16_t *list = lead + ch;
-    unsigned char *act = reinterpret_cast<unsigned char *>(list + ch);
+// ---- int8 copies for the anchor test
+//
+// A row of D int8 is D / 16 lanes x 16 bytes; a warp covers 32 rows with
+// D / 16 loads per lane (the layout of load32 with 16-byte chunks of int8).
+template <int D>
+struct Q8 {
+    static constexpr int L8 = D / 16;  // lanes per row
+    static constexpr int R8 = 32 / L8;  // rows per load
+};
+template <int D>
+__device__ __forceinline__ int q8_row(int lane) {
+    return (lane % Q8<D>::L8) * Q8<D>::R8 + lane / Q8<D>::L8;
+}
+template <int D>
+__device__ __forceinline__ int q8_lane(int row) {
+    return (row % Q8<D>::R8) * Q8<D>::L8 + row / Q8<D>::R8;
+}
+
+// Power-of-two scale s with max|v| <= 127 s (1 for a zero vector).
+__device__ __forceinline__ float q8_scale(float amax) {
+    if (!(amax > 0.f)) return 1.f;
+    int e;
+    frexpf(amax * (1.0f / 127.0f) * (1.0f + 1e-6f), &e);
+    return ldexpf(1.0f, e);
+}
+__device__ __forceinline__ int q8_code(float v, float s) {
+    return max(-127, min(127, __float2int_rn(v / s)));
+}
+
+// Exact integer dot products of 32 int8 rows (loaded as by load32) with this
+// lane's 16-byte chunk of an int8 vector; the transpose-reduction leaves in
+// lane l the dot product of row q8_row(l).
+template <int D>
+__device__ __forceinline__ int dot32q(const uint4 (&buf)[Q8<D>::L8], const uint4 &qc, int lane) {
+    constexpr int L8 = Q8<D>::L8;
+    int part[L8];
+#pragma unroll
+    for (int i = 0; i < L8; ++i) {
+        int acc = __dp4a((int)buf[i].x, (int)qc.x, 0);
+        acc = __dp4a((int)buf[i].y, (int)qc.y, acc);
+        acc = __dp4a((int)buf[i].z, (int)qc.z, acc);
+        part[i] = __dp4a((int)buf[i].w, (int)qc.w, acc);
+    }
+#pragma unroll
+    for (int n = L8; n > 1; n >>= 1) {
+        const int half = n >> 1;
+        const bool up = (lane & half) != 0;
+#pragma unroll
+        for (int k = 0; k < half; ++k) {
+            const int send = up ? part[k] : part[k + half];
+            const int keep = up ? part[k + half] : part[k];
+            part[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+    }
+    return part[0];
+}
+
+// The int8 copy of a vector held by the warp, 16 elements per lane (lane l:
+// elements (l % L8) * 16 ..): its scale, this lane's codes, |codes|^2 and the
+// quantisation error |v - s codes| (fp64, rounded up to float).
+template <typename T, int D>
+__device__ __forceinline__ void q8_vector(const T *__restrict__ v, int lane, float &s, uint4 &codes, int &n2,
+                                          float &err) {
+    constexpr int L8 = Q8<D>::L8;
+    const int c0 = (lane % L8) * 16;
+    float f[16];
+    if constexpr (sizeof(T) == 2) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(v + c0));
+        const uint4 b = __ldg(reinterpret_cast<const uint4 *>(v + c0 + 8));
+        widen16f<T>(a, f);
+        widen16f<T>(b, f + 8);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) widen16f<T>(__ldg(reinterpret_cast<const uint4 *>(v + c0 + 4 * k)), f + 4 * k);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    s = q8_scale(amax);
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    int nn = 0;
+    double ee = 0.0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const int q = q8_code(f[e], s);
+        w[e >> 2] |= ((uint32_t)(q & 0xff)) << (8 * (e & 3));
+        nn += q * q;
+        const double dlt = (double)f[e] - (double)q * (double)s;
+        ee = fma(dlt, dlt, ee);
+    }
+    codes = make_uint4(w[0], w[1], w[2], w[3]);
+    // each chunk is held by R8 lanes: count lanes 0 .. L8 - 1 only
+    if (lane >= L8) {
+        nn = 0;
+        ee = 0.0;
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        nn += __shfl_xor_sync(0xffffffffu, nn, m);
+        ee += __shfl_xor_sync(0xffffffffu, ee, m);
+    }
+    n2 = nn;
+    err = __double2float_ru(sqrt(ee) * (1.0 + kSeedMargin));
+}
+
+// ---- arrival and pick (the last block of head h in round r)
+//
+// REFRESH: bring the S1 sums of the ranges flagged this round and the S2
+// sums above them up to date first.  dl (>= 2048 ints) and sd2 (>= 2048
+// bytes) are shared memory the block no longer needs.
+template <bool REFRESH>
+__device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r, int *dl, uint32_t *sd2) {
     __shared__ double sh[kSeedWarps];
-    __shared__ double s1own[GROUPED ? 1 : kSeedChMax / kSeedS];
     __shared__ int nlist, last, pick_blk;
     __shared__ double sh_base;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int p0 = blockIdx.x * ch;
-    const int p1 = min(N, p0 + ch);
-    constexpr bool grouped = GROUPED;
-
-    // ---- the block's pieces and the first 256 anchors (static data)
-    int nl = 0, ol = 0;
-    float Rl = 0.f;
-    unsigned am = 0u;
-    uint4 abuf[GROUPED ? Gm::LPP : 1];
-    auto stage = [&]() {
-        if (tid == 0) nlist = 0;
-        __syncthreads();
-        const uint16_t *po = s.pofs + hN;
-        for (int o = tid; o < p1 - p0; o += kSeedThreads) {
-            const int f = po[p0 + o];
-            lead[o] = (uint16_t)f;
-            pperm[o] = s.perm[hN + p0 + o];
-            if (f == o) list[atomicAdd(&nlist, 1)] = (uint16_t)o;
-        }
-        __syncthreads();
-        nl = nlist;
-        const int j = warp * 32 + lane;
-        const bool have = j < nl;
-        ol = have ? list[j] : 0;
-        Rl = have ? s.rr[hN + p0 + ol] : 0.f;
-        const int arow = have ? s.apos[hN + p0 + ol] : 0;
-        am = __ballot_sync(0xffffffffu, have);
-        if constexpr (GROUPED) load32<T, D, false>(xh, arow, am, lane, abuf);
-    };
-    if (grouped && pre) stage();
-    pdl_wait();
-    pdl_launch_dependents();
-
-    if (r == 0) {
-        // round 0: clear the state; the last block records floor(u * N)
-        for (int i = p0 + tid; i < p1; i += kSeedThreads) {
-            d2h[i] = __longlong_as_double(0x7ff0000000000000LL);  // +inf
-            tk[i] = 0;
-            s.near[hN + i] = 0;
-        }
-        for (int k = p0 / kSeedS + tid; k < (p1 + kSeedS - 1) / kSeedS; k += kSeedThreads) dh[k] = 0;
-    } else {
-        if (grouped && !pre) stage();
-        const int c = s.idx[(size_t)h * K + r - 1];
-        const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + (lane % Gm::LPP) * Gm::E16));
-        double cv[Gm::E16];
-        widen16<T>(craw, cv);
-        if constexpr (GROUPED) {
-            float cvf[Gm::E16];
-            widen16f<T>(craw, cvf);
-            // triangle test of each piece, 256 anchors per pass
-            const int q = seed_row<T, D>(lane);
-            for (int pass = 0; pass * kSeedThreads < nl; ++pass) {
-                if (pass > 0) {
-                    const int j = pass * kSeedThreads + warp * 32 + lane;
-                    const bool have = j < nl;
-                    ol = have ? list[j] : 0;
-                    Rl = have ? s.rr[hN + p0 + ol] : 0.f;
-                    const int arow = have ? s.apos[hN + p0 + ol] : 0;
-                    am = __ballot_sync(0xffffffffu, have);
-                    load32<T, D, false>(xh, arow, am, lane, abuf);
-                }
-                const float Ml = ((am >> lane) & 1u) ? s.mdp[hN + p0 + ol] : 0.f;
-                // fp32 distance, made a lower bound of the exact one by its
-                // rounding bound (1e-5 > (D + 2) 2^-24 relative for D <= 128)
-                const float dc2 = dist32f<T, D>(abuf, cvf, lane);
-                const int oq = __shfl_sync(0xffffffffu, ol, q);
-                const float Rq = __shfl_sync(0xffffffffu, Rl, q);
-                const float Mq = __shfl_sync(0xffffffffu, Ml, q);
-                if ((am >> q) & 1u) {
-                    const double lim = ((double)Rq + (double)Mq) * (1.0 + kSeedMargin);
-                    act[oq] = (double)dc2 * (1.0 - 1e-5) > lim * lim ? 0 : 1;
-                    pmax[oq] = 0u;
-                }
-            }
-            __syncthreads();
-        }
-        // D2 update of the positions in updated pieces, 32 at a time per warp
-        const int q = seed_row<T, D>(lane);
-        for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
-            const int qp = base + lane;
-            const bool al = qp < p1 && (!grouped || act[lead[qp - p0]]);
-            const unsigned m = __ballot_sync(0xffffffffu, al);
-            if (m == 0u) continue;
-            const int pt = grouped ? (al ? pperm[qp - p0] : 0) : qp;
-            uint4 buf[Gm::LPP];
-            load32<T, D, true>(xh, pt, m, lane, buf);
-            const int i = __shfl_sync(0xffffffffu, pt, q);
-            const bool mine = (m >> q) & 1u;
-            const double old = mine ? d2h[i] : 0.0;
-            const double dist = dist32<T, D>(buf, cv, lane);
-            if (mine) {
-                const double nd = fmin(old, dist);
-                if (nd < old) {
-                    d2h[i] = nd;
-                    s.near[hN + i] = r - 1;
-                    if (grouped) dh[i / kSeedS] = 1;
-                }
-                if (grouped) atomicMax(&pmax[lead[base + q - p0]], __float_as_uint(__double2float_ru(sqrt(nd))));
-            }
-        }
-        __syncthreads();
-        if (grouped) {
-            for (int j = tid; j < nl; j += kSeedThreads) {
-                const int o = list[j];
-                if (act[o]) s.mdp[hN + p0 + o] = __uint_as_float(pmax[o]);
-            }
-        } else {
-            // the block's own S1 sums (index order), then its S2 sums
-            double *b1 = s.bs1 + (size_t)h * s.NR1;
-            const int k0 = p0 / kSeedS, k1 = (p1 + kSeedS - 1) / kSeedS;
-            for (int k = k0 + tid; k < k1; k += kSeedThreads) {
-                const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
-                double v = 0.0;
-                if (q1 - q0 == kSeedS) {
-                    double t[kSeedS];
-#pragma unroll
-                    for (int e = 0; e < kSeedS; ++e) t[e] = __ldcg(d2h + q0 + e);
-#pragma unroll
-                    for (int e = 0; e < kSeedS; ++e) v += t[e];
-                } else {
-                    for (int i2 = q0; i2 < q1; ++i2) v += __ldcg(d2h + i2);
-                }
-                b1[k] = v;
-                s1own[k - k0] = v;
-            }
-            __syncthreads();
-            const int m0 = k0 / kSeedS, m1 = (k1 + kSeedS - 1) / kSeedS;
-            for (int k2 = m0 + tid; k2 < m1; k2 += kSeedThreads) {
-                const int a0 = k2 * kSeedS, a1 = min(s.NR1, a0 + kSeedS);
-                double v = 0.0;
-                for (int k = a0; k < a1; ++k) v += s1own[k - k0];
-                s.bs2[(size_t)h * s.NR2 + k2] = v;
-            }
-        }
-    }
+    const int N = s.N, K = s.K;
+    const size_t hN = (size_t)h * N;
+    double *d2h = s.d2 + hN;
+    unsigned char *tk = s.taken + hN;
+    unsigned char *dh = s.dirty + (size_t)h * s.DSTRIDE;
     __threadfence();
     __syncthreads();
     if (tid == 0) {
         const int old = atomicAdd(&s.cnt[h], 1);
-        last = (old == (int)gridDim.x - 1);
+        last = (old == (int)(gridDim.x - 1));
         __threadfence();
     }
     __syncthreads();
     if (!last) return;
 
-    // ---------------- last block of head h: choose this round's centre
     const double ur = s.u[(size_t)h * K + r];
     if (r == 0) {
         if (tid == 0) {
@@ -449,55 +434,53 @@ kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G, int pre,
     const int NR1 = s.NR1, NR2 = s.NR2;
     double *b1 = s.bs1 + (size_t)h * NR1;
     double *b2 = s.bs2 + (size_t)h * NR2;
-    // S1 sums of the ranges touched this round (each in index order), and
-    // the S2 sums over them
-    uint32_t *sd2 = reinterpret_cast<uint32_t *>(act);  // S2 dirty bitmap
-    int *dl = pperm;                                    // dirty S1 ranges
-    if constexpr (GROUPED) {
-    for (int i = tid; i < (NR2 + 31) / 32; i += kSeedThreads) sd2[i] = 0u;
-    for (int k0 = 0; k0 < NR1; k0 += kSeedThreads * 8) {
-        if (tid == 0) nlist = 0;
-        __syncthreads();
-        const int kb = k0 + tid * 8;
-        if (kb < NR1) {
-            const uint2 f = __ldcg(reinterpret_cast<const uint2 *>(dh + kb));
-            const unsigned long long bits = (unsigned long long)f.x | ((unsigned long long)f.y << 32);
+    if constexpr (REFRESH) {
+        // S1 sums of the ranges touched this round (each in index order),
+        // then the S2 sums over them
+        for (int i = tid; i < (NR2 + 31) / 32; i += kSeedThreads) sd2[i] = 0u;
+        for (int k0 = 0; k0 < NR1; k0 += kSeedThreads * 8) {
+            if (tid == 0) nlist = 0;
+            __syncthreads();
+            const int kb = k0 + tid * 8;
+            if (kb < NR1) {
+                const uint2 f = __ldcg(reinterpret_cast<const uint2 *>(dh + kb));
+                const unsigned long long bits = (unsigned long long)f.x | ((unsigned long long)f.y << 32);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (((bits >> (8 * e)) & 0xffull) && kb + e < NR1) {
-                    const int k = kb + e;
-                    dl[atomicAdd(&nlist, 1)] = k;
-                    atomicOr(&sd2[k >> 10], 1u << ((k >> 5) & 31));
-                }
-        }
-        __syncthreads();
-        const int nd = nlist;
-        for (int j = tid; j < nd; j += kSeedThreads) {
-            const int k = dl[j];
-            const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
-            double v = 0.0;
-            if (q1 - q0 == kSeedS) {
-                double t[kSeedS];
-#pragma unroll
-                for (int e = 0; e < kSeedS; ++e) t[e] = __ldcg(d2h + q0 + e);
-#pragma unroll
-                for (int e = 0; e < kSeedS; ++e) v += t[e];
-            } else {
-                for (int i = q0; i < q1; ++i) v += __ldcg(d2h + i);
+                for (int e = 0; e < 8; ++e)
+                    if (((bits >> (8 * e)) & 0xffull) && kb + e < NR1) {
+                        const int k = kb + e;
+                        dl[atomicAdd(&nlist, 1)] = k;
+                        atomicOr(&sd2[k >> 10], 1u << ((k >> 5) & 31));
+                    }
             }
-            b1[k] = v;
-            dh[k] = 0;
+            __syncthreads();
+            const int nd = nlist;
+            for (int j = tid; j < nd; j += kSeedThreads) {
+                const int k = dl[j];
+                const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
+                double v = 0.0;
+                if (q1 - q0 == kSeedS) {
+                    double t[kSeedS];
+#pragma unroll
+                    for (int e = 0; e < kSeedS; ++e) t[e] = __ldcg(d2h + q0 + e);
+#pragma unroll
+                    for (int e = 0; e < kSeedS; ++e) v += t[e];
+                } else {
+                    for (int i = q0; i < q1; ++i) v += __ldcg(d2h + i);
+                }
+                b1[k] = v;
+                dh[k] = 0;
+            }
+            __syncthreads();
         }
-        __syncthreads();
-    }
-    for (int k2 = tid; k2 < NR2; k2 += kSeedThreads) {
-        if ((sd2[k2 >> 5] >> (k2 & 31)) & 1u) {
-            const int k0 = k2 * kSeedS, k1 = min(NR1, k0 + kSeedS);
-            double v = 0.0;
-            for (int k = k0; k < k1; ++k) v += __ldcg(b1 + k);
-            b2[k2] = v;
+        for (int k2 = tid; k2 < NR2; k2 += kSeedThreads) {
+            if ((sd2[k2 >> 5] >> (k2 & 31)) & 1u) {
+                const int k0 = k2 * kSeedS, k1 = min(NR1, k0 + kSeedS);
+                double v = 0.0;
+                for (int k = k0; k < k1; ++k) v += __ldcg(b1 + k);
+                b2[k2] = v;
+            }
         }
-    }
     }
     __syncthreads();
     double total = 0.0;
@@ -595,12 +578,260 @@ kmeanspp_round(const T *__restrict__ x, const SeedArgs s, int r, int G, int pre,
     }
 }
 
+// ---- rounds before the first grouping: every point is updated, and each
+// block writes the S1 and S2 sums of its own positions (ch is a multiple of
+// the S2 range)
+// SCREEN: test each point first with the fp32 distance (worth it once few
+// points change per round; without it the kernel needs fewer registers).
+template <typename T, int D, bool SCREEN>
+__global__ void __launch_bounds__(kSeedThreads)
+kmeanspp_round_full(const T *__restrict__ x, const SeedArgs s, int r, int ch) {
+    using Gm = SeedGeo<T, D>;
+    const int h = blockIdx.y, N = s.N, K = s.K;
+    const size_t hN = (size_t)h * N;
+    const T *xh = x + hN * D;
+    double *d2h = s.d2 + hN;
+    __shared__ double s1own[kSeedChMax / kSeedS];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int p0 = blockIdx.x * ch;
+    const int p1 = min(N, p0 + ch);
+    pdl_wait();
+    pdl_launch_dependents();
+    if (r == 0) {
+        // round 0: clear the state; the last block records floor(u * N)
+        unsigned char *dh = s.dirty + (size_t)h * s.DSTRIDE;
+        for (int i = p0 + tid; i < p1; i += kSeedThreads) {
+            d2h[i] = __longlong_as_double(0x7ff0000000000000LL);  // +inf
+            s.taken[hN + i] = 0;
+            s.near[hN + i] = 0;
+        }
+        for (int k = p0 / kSeedS + tid; k < (p1 + kSeedS - 1) / kSeedS; k += kSeedThreads) dh[k] = 0;
+    } else {
+        const int c = s.idx[(size_t)h * K + r - 1];
+        const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + (lane % Gm::LPP) * Gm::E16));
+        double cv[Gm::E16];
+        float cvf[Gm::E16];
+        widen16<T>(craw, cv);
+        widen16f<T>(craw, cvf);
+        (void)cvf;
+        const int q = seed_row<T, D>(lane);
+        for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
+            const int qp = base + lane;
+            const unsigned m = __ballot_sync(0xffffffffu, qp < p1);
+            uint4 buf[Gm::LPP];
+            load32<T, D, true>(xh, qp, m, lane, buf);
+            const int i = base + q;
+            const bool mine = (m >> q) & 1u;
+            const double old = mine ? d2h[i] : 0.0;
+            // fp32 screen, then the exact distance where D2 may fall (the
+            // rows are read again, from cache, for the rare warps that need it)
+            if constexpr (SCREEN) {
+                const float d32 = dist32f<T, D>(buf, cvf, lane);  // every lane: it shuffles
+                const bool cand = mine && seed_may_fall(d32, old);
+                if (__any_sync(0xffffffffu, cand)) {
+                    uint4 buf2[Gm::LPP];
+                    load32<T, D, false>(xh, qp, m, lane, buf2);
+                    const double dist = dist32<T, D>(buf2, cv, lane);
+                    if (cand && dist < old) {
+                        d2h[i] = dist;
+                        s.near[hN + i] = r - 1;
+                    }
+                }
+            } else {
+                const double dist = dist32<T, D>(buf, cv, lane);
+                if (mine && dist < old) {
+                    d2h[i] = dist;
+                    s.near[hN + i] = r - 1;
+                }
+            }
+        }
+        __syncthreads();
+        // the block's own S1 sums (index order), then its S2 sums
+        double *b1 = s.bs1 + (size_t)h * s.NR1;
+        const int k0 = p0 / kSeedS, k1 = (p1 + kSeedS - 1) / kSeedS;
+        for (int k = k0 + tid; k < k1; k += kSeedThreads) {
+            const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
+            double v = 0.0;
+            if (q1 - q0 == kSeedS) {
+                double t[kSeedS];
+#pragma unroll
+                for (int e = 0; e < kSeedS; ++e) t[e] = __ldcg(d2h + q0 + e);
+#pragma unroll
+                for (int e = 0; e < kSeedS; ++e) v += t[e];
+            } else {
+                for (int i = q0; i < q1; ++i) v += __ldcg(d2h + i);
+            }
+            b1[k] = v;
+            s1own[k - k0] = v;
+        }
+        __syncthreads();
+        const int m0 = k0 / kSeedS, m1 = (k1 + kSeedS - 1) / kSeedS;
+        for (int k2 = m0 + tid; k2 < m1; k2 += kSeedThreads) {
+            const int a0 = k2 * kSeedS, a1 = min(s.NR1, a0 + kSeedS);
+            double v = 0.0;
+            for (int k = a0; k < a1; ++k) v += s1own[k - k0];
+            s.bs2[(size_t)h * s.NR2 + k2] = v;
+        }
+    }
+    seed_arrive_pick<false>(s, h, r, nullptr, nullptr);
+}
+
+// ---- grouped rounds (pruned update)
+//
+// pre = the grouping may be read before the dependency wait (it was not just
+// rebuilt).  Dynamic shared memory, ch positions: point at each position
+// (then the dirty S1 ranges), the active positions (piece << 16 | offset),
+// the piece bounds (float bits), the piece flags (then the S2 dirty bitmap).
+constexpr size_t seed_grouped_smem(int ch) { return (size_t)13 * ch + 16; }
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSeedThreads)
+kmeanspp_round_grouped(const T *__restrict__ x, const SeedArgs s, int r, int G, int pre, int ch) {
+    using Gm = SeedGeo<T, D>;
+    constexpr int L8 = Q8<D>::L8, R8 = Q8<D>::R8;
+    const int h = blockIdx.y, b = blockIdx.x, N = s.N, K = s.K;
+    const size_t hN = (size_t)h * N, hK = (size_t)h * K;
+    const T *xh = x + hN * D;
+    double *d2h = s.d2 + hN;
+    unsigned char *dh = s.dirty + (size_t)h * s.DSTRIDE;
+    extern __shared__ __align__(16) unsigned char seed_smem[];
+    int *pperm = reinterpret_cast<int *>(seed_smem);
+    uint32_t *alist = reinterpret_cast<uint32_t *>(pperm + ch);
+    uint32_t *pmax = alist + ch;
+    unsigned char *act = reinterpret_cast<unsigned char *>(pmax + ch + 1);
+    __shared__ int npc, na;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int p0 = b * ch;
+    const int p1 = min(N, p0 + ch);
+    const size_t rec = (size_t)h * s.CAP + (size_t)b * (ch + 1);
+    (void)G;
+
+    // ---- the block's pieces and the first 256 of them (static data)
+    int P = 0, gl = 0, lol = 0, hil = 0, nv = 0;
+    float Rv = 0.f, sv = 1.f, ev = 0.f;
+    uint4 abuf[L8];
+    auto fetch = [&](int pass) {
+        const int jl = pass * kSeedThreads + warp * 32 + lane;
+        const bool have = jl < P;
+        gl = have ? s.pg[rec + jl] : 0;
+        lol = have ? s.plo[rec + jl] : 0;
+        hil = have ? s.phi[rec + jl] : 0;
+        Rv = have ? s.gr[hK + gl] : 0.f;
+        sv = have ? s.gs[hK + gl] : 1.f;
+        ev = have ? s.ge[hK + gl] : 0.f;
+        nv = have ? s.gn[hK + gl] : 0;
+        const unsigned am = __ballot_sync(0xffffffffu, have);
+#pragma unroll
+        for (int i = 0; i < L8; ++i) {
+            const int row = i * R8 + lane / L8;
+            const int gi = __shfl_sync(0xffffffffu, gl, row);
+            abuf[i] = ((am >> row) & 1u)
+                          ? __ldg(reinterpret_cast<const uint4 *>(s.gq + (hK + gi) * D + (lane % L8) * 16))
+                          : make_uint4(0, 0, 0, 0);
+        }
+    };
+    auto stage = [&]() {
+        if (tid == 0) npc = s.pcnt[(size_t)h * s.NBMAX + b];
+        for (int o = tid; o < p1 - p0; o += kSeedThreads) pperm[o] = s.perm[hN + p0 + o];
+        __syncthreads();
+        P = npc;
+        fetch(0);
+    };
+    if (pre) stage();
+    pdl_wait();
+    pdl_launch_dependents();
+    if (!pre) stage();
+    if (tid == 0) na = 0;
+
+    const int c = s.idx[hK + r - 1];
+    const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + (lane % Gm::LPP) * Gm::E16));
+    double cv[Gm::E16];
+    float cvf[Gm::E16];
+    widen16<T>(craw, cv);
+    widen16f<T>(craw, cvf);
+    float sc, ec;
+    uint4 qc;
+    int nqc;
+    q8_vector<T, D>(xh + (size_t)c * D, lane, sc, qc, nqc, ec);
+    __syncthreads();  // na cleared
+
+    // triangle test of each piece, then its positions into the active list
+    for (int pass = 0; pass * kSeedThreads < P; ++pass) {
+        if (pass > 0) fetch(pass);
+        const int jl = pass * kSeedThreads + warp * 32 + lane;
+        const bool have = jl < P;
+        const float Mv = have ? s.pm[rec + jl] : 0.f;
+        const int dq = dot32q<D>(abuf, qc, lane);
+        const int dot = __shfl_sync(0xffffffffu, dq, q8_lane<D>(lane));  // this lane's piece
+        bool upd = false;
+        if (have) {
+            const double sa = sv, scd = sc;
+            const double dc2 = scd * scd * (double)nqc + sa * sa * (double)nv - 2.0 * scd * sa * (double)dot;
+            const double lb = sqrt(fmax(dc2, 0.0)) - (double)ec - (double)ev;
+            const double slack = 1e-7 * (scd * sqrt((double)nqc) + sa * sqrt((double)nv));
+            upd = !(lb > ((double)Rv + (double)Mv) * (1.0 + kSeedMargin) + slack);
+            act[jl] = upd ? 1 : 0;
+            if (upd) pmax[jl] = 0u;
+        }
+        unsigned bal = __ballot_sync(0xffffffffu, upd);
+        while (bal) {
+            const int src = __ffs(bal) - 1;
+            bal &= bal - 1;
+            const int lo = __shfl_sync(0xffffffffu, lol, src);
+            const int len = __shfl_sync(0xffffffffu, hil, src) - lo;
+            const uint32_t jj = (uint32_t)(pass * kSeedThreads + warp * 32 + src);
+            int start = 0;
+            if (lane == 0) start = atomicAdd(&na, len);
+            start = __shfl_sync(0xffffffffu, start, 0);
+            for (int t = lane; t < len; t += 32) alist[start + t] = (jj << 16) | (uint32_t)(lo + t);
+        }
+    }
+    __syncthreads();
+
+    // D2 update of the active positions, 32 at a time per warp
+    const int nact = na;
+    const int q = seed_row<T, D>(lane);
+    for (int base = warp * 32; base < nact; base += kSeedThreads) {
+        const int k = base + lane;
+        const bool al = k < nact;
+        const uint32_t e = al ? alist[k] : 0u;
+        const unsigned m = __ballot_sync(0xffffffffu, al);
+        const int pt = al ? pperm[e & 0xffffu] : 0;
+        uint4 buf[Gm::LPP];
+        load32<T, D, true>(xh, pt, m, lane, buf);
+        const int i = __shfl_sync(0xffffffffu, pt, q);
+        const uint32_t eq = __shfl_sync(0xffffffffu, e, q);
+        const bool mine = (m >> q) & 1u;
+        const double old = mine ? d2h[i] : 0.0;
+        // fp32 screen, then the exact distance where D2 may fall
+        const float d32 = dist32f<T, D>(buf, cvf, lane);  // every lane: it shuffles
+        const bool cand = mine && seed_may_fall(d32, old);
+        double nd = old;
+        if (__any_sync(0xffffffffu, cand)) {
+            uint4 buf2[Gm::LPP];
+            load32<T, D, false>(xh, pt, m, lane, buf2);
+            const double dist = dist32<T, D>(buf2, cv, lane);
+            if (cand && dist < old) {
+                nd = dist;
+                d2h[i] = nd;
+                s.near[hN + i] = r - 1;
+                dh[i / kSeedS] = 1;
+            }
+        }
+        if (mine) atomicMax(&pmax[eq >> 16], __float_as_uint(__double2float_ru(sqrt(nd))));
+    }
+    __syncthreads();
+    for (int j = tid; j < P; j += kSeedThreads)
+        if (act[j]) s.pm[rec + j] = __uint_as_float(pmax[j]);
+    seed_arrive_pick<true>(s, h, r, pperm, reinterpret_cast<uint32_t *>(act));
+}
+
 // ---- regrouping (before round r, with G = r - 1 chosen centres applied)
 //
 // Group g holds the points whose nearest applied centre is centre g; its
 // radius is the largest of their D2 (D2 is exactly the distance to that
-// centre).  Counting sort: histogram and radius, exclusive scan, scatter of
-// the points with their piece offsets and group data.
+// centre).  Counting sort (histogram and radius, exclusive scan, scatter),
+// the int8 copy of every anchor, then each block's piece records.
 
 __global__ void seed_group_hist(const SeedArgs s, int G) {
     const int h = blockIdx.y, i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -612,19 +843,92 @@ __global__ void seed_group_hist(const SeedArgs s, int G) {
               (unsigned long long)__double_as_longlong(s.d2[hi]));
 }
 
-__global__ void seed_group_scatter(const SeedArgs s, int G, int ch) {
+__global__ void seed_group_scatter(const SeedArgs s, int G) {
     const int h = blockIdx.y, i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= s.N) return;
     const size_t hN = (size_t)h * s.N;
     const int g = s.near[hN + i];
     const int pos = atomicAdd(&s.cur[(size_t)h * G + g], 1);
-    const int cs = pos - pos % ch;
-    const float R = __double2float_ru(sqrt(s.r2[(size_t)h * G + g]));
     s.perm[hN + pos] = i;
-    s.apos[hN + pos] = s.idx[(size_t)h * s.K + g];
-    s.rr[hN + pos] = R;
-    s.mdp[hN + pos] = R;
-    s.pofs[hN + pos] = (uint16_t)(max(s.seg[(size_t)h * (G + 1) + g], cs) - cs);
+}
+
+// One warp per group: int8 anchor, scale, |codes|^2, error and R.
+template <typename T, int D>
+__global__ void seed_group_anchor(const T *__restrict__ x, const SeedArgs s, int G) {
+    const int h = blockIdx.y, lane = threadIdx.x & 31;
+    const int g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (g >= G) return;
+    const size_t hK = (size_t)h * s.K;
+    const int ai = s.idx[hK + g];
+    float sc, err;
+    uint4 codes;
+    int n2;
+    q8_vector<T, D>(x + ((size_t)h * s.N + ai) * D, lane, sc, codes, n2, err);
+    if (lane < Q8<D>::L8) *reinterpret_cast<uint4 *>(s.gq + (hK + g) * D + lane * 16) = codes;
+    if (lane == 0) {
+        s.gs[hK + g] = sc;
+        s.ge[hK + g] = err;
+        s.gn[hK + g] = n2;
+        s.gr[hK + g] = __double2float_ru(sqrt(s.r2[(size_t)h * G + g]) * (1.0 + kSeedMargin));
+    }
+}
+
+// One block per range of ch positions: the non-empty parts of the groups
+// overlapping it, in group order, with M = R to start.
+__global__ void seed_group_pieces(const SeedArgs s, int G, int ch) {
+    const int h = blockIdx.y, b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int p0 = b * ch, p1 = min(s.N, p0 + ch);
+    const int *seg = s.seg + (size_t)h * (G + 1);
+    const size_t hK = (size_t)h * s.K;
+    const size_t rec = (size_t)h * s.CAP + (size_t)b * (ch + 1);
+    __shared__ int glo, ghi, base, wsum[kSeedWarps];
+    if (tid == 0) {
+        // last group starting at or before p0, and at or before p1 - 1
+        int lo = 0, hi = G - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (seg[mid] <= p0) lo = mid; else hi = mid - 1;
+        }
+        glo = lo;
+        lo = 0;
+        hi = G - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (seg[mid] <= p1 - 1) lo = mid; else hi = mid - 1;
+        }
+        ghi = lo;
+        base = 0;
+    }
+    __syncthreads();
+    for (int g0 = glo; g0 <= ghi; g0 += kSeedThreads) {
+        const int g = g0 + tid;
+        int lo = 0, hi = 0;
+        if (g <= ghi) {
+            lo = max(seg[g], p0);
+            hi = min(seg[g + 1], p1);
+        }
+        const bool v = g <= ghi && lo < hi;
+        const unsigned bl = __ballot_sync(0xffffffffu, v);
+        if (lane == 0) wsum[warp] = __popc(bl);
+        __syncthreads();
+        int off = base;
+        for (int w = 0; w < warp; ++w) off += wsum[w];
+        off += __popc(bl & ((1u << lane) - 1u));
+        if (v) {
+            s.pg[rec + off] = g;
+            s.plo[rec + off] = (uint16_t)(lo - p0);
+            s.phi[rec + off] = (uint16_t)(hi - p0);
+            s.pm[rec + off] = s.gr[hK + g];
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int t = 0;
+            for (int w = 0; w < kSeedWarps; ++w) t += wsum[w];
+            base += t;
+        }
+        __syncthreads();
+    }
+    if (tid == 0) s.pcnt[(size_t)h * s.NBMAX + b] = base;
 }
 
 }  // namespace asmk
@@ -882,66 +1186,58 @@ KmWs km_ws(int H, int N, int K) {
 using namespace asmk;
 
 size_t asm_kmeanspp_ws_bytes(int H, int N, int d, int K) {
-    (void)d;
-    return seed_ws(H, N, K).total;
+    return seed_ws(H, N, d, K).total;
 }
 
 namespace {
-// dynamic shared memory of a grouped round (13 bytes per position)
-constexpr size_t seed_smem_bytes(int ch, bool grouped) { return grouped ? (size_t)13 * ch : 0; }
-
 // Positions per block: the smallest multiple of `step` (at least kSeedChMin)
 // for which every head's blocks fit the GPU in one wave, else kSeedChMax.
-template <typename T, int D, bool GROUPED>
-int seed_block_positions(int H, int N, cudaError_t *err) {
-    auto k = kmeanspp_round<T, D, GROUPED>;
-    constexpr int step = GROUPED ? 256 : kSeedS * kSeedS;
-    static bool attr = false;
-    if (!attr) {
-        *err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)seed_smem_bytes(kSeedChMax, GROUPED));
-        if (*err != cudaSuccess) return 0;
-        attr = true;
-    }
+template <typename KERN>
+int seed_block_positions(KERN k, bool grouped, int step, int H, int N, cudaError_t *err) {
+    const size_t smax = grouped ? seed_grouped_smem(kSeedChMax) : 0;
+    *err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smax);
+    if (*err != cudaSuccess) return 0;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         sms = 148;
     for (int ch = kSeedChMin; ch <= kSeedChMax; ch += step) {
         int occ = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kSeedThreads, seed_smem_bytes(ch, GROUPED)) !=
-            cudaSuccess)
-            break;
+        const size_t sm = grouped ? seed_grouped_smem(ch) : 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kSeedThreads, sm) != cudaSuccess) break;
         if ((long)H * ((N + ch - 1) / ch) <= (long)occ * sms) return ch;
     }
     (void)cudaGetLastError();
     return kSeedChMax;
 }
 
-template <typename T, int D, bool GROUPED>
-cudaError_t seed_round(const T *x, const SeedArgs &s, int r, int G, int pre, int ch, int H, cudaStream_t st) {
+template <typename KERN, typename... Args>
+cudaError_t seed_launch(KERN k, dim3 grid, size_t smem, cudaStream_t st, Args... args) {
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((s.N + ch - 1) / ch, H);
+    cfg.gridDim = grid;
     cfg.blockDim = dim3(kSeedThreads);
-    cfg.dynamicSmemBytes = seed_smem_bytes(ch, GROUPED);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kmeanspp_round<T, D, GROUPED>, x, s, r, G, pre, ch);
+    return cudaLaunchKernelEx(&cfg, k, args...);
 }
 
 template <typename T, int D>
 cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
     cudaError_t e = cudaSuccess;
-    const int chf = seed_block_positions<T, D, false>(H, s.N, &e);
+    const int chf = seed_block_positions(kmeanspp_round_full<T, D, false>, false, kSeedS * kSeedS, H, s.N, &e);
     if (e != cudaSuccess) return e;
-    const int chg = seed_block_positions<T, D, true>(H, s.N, &e);
+    const int chs = seed_block_positions(kmeanspp_round_full<T, D, true>, false, kSeedS * kSeedS, H, s.N, &e);
+    if (e != cudaSuccess) return e;
+    const int chg = seed_block_positions(kmeanspp_round_grouped<T, D>, true, 256, H, s.N, &e);
     if (e != cudaSuccess) return e;
     const int N = s.N, K = s.K;
     const dim3 pgrid((N + 255) / 256, H);
+    const dim3 gfull((N + chf - 1) / chf, H), gscr((N + chs - 1) / chs, H), ggrp((N + chg - 1) / chg, H);
     int G = 0, next = std::max(256, K / 8);
     for (int r = 0; r < K; ++r) {
         int pre = 1;
@@ -955,13 +1251,16 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
             if ((e = cudaMemsetAsync(s.r2, 0, sizeof(double) * (size_t)H * G, st)) != cudaSuccess) return e;
             seed_group_hist<<<pgrid, 256, 0, st>>>(s, G);
             scan_kernel<<<H, 1024, 0, st>>>(s.gcnt, G, s.seg, s.cur);
-            seed_group_scatter<<<pgrid, 256, 0, st>>>(s, G, chg);
+            seed_group_scatter<<<pgrid, 256, 0, st>>>(s, G);
+            seed_group_anchor<T, D><<<dim3((G + 7) / 8, H), 256, 0, st>>>(x, s, G);
+            seed_group_pieces<<<ggrp, kSeedThreads, 0, st>>>(s, G, chg);
             int p2 = 1;
             while (p2 * 2 <= r) p2 *= 2;
             next = r + std::max(256, p2 / 4);
         }
-        e = G > 0 ? seed_round<T, D, true>(x, s, r, G, pre, chg, H, st)
-                  : seed_round<T, D, false>(x, s, r, 0, 0, chf, H, st);
+        if (G > 0) e = seed_launch(kmeanspp_round_grouped<T, D>, ggrp, seed_grouped_smem(chg), st, x, s, r, G, pre, chg);
+        else if (r < kSeedScreen) e = seed_launch(kmeanspp_round_full<T, D, false>, gfull, 0, st, x, s, r, chf);
+        else e = seed_launch(kmeanspp_round_full<T, D, true>, gscr, 0, st, x, s, r, chs);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
@@ -971,7 +1270,7 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
 cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const double *u,
                                 asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st) {
     if (N > kSeedMaxN) return cudaErrorInvalidValue;
-    const SeedWs w = seed_ws(H, N, K);
+    const SeedWs w = seed_ws(H, N, d, K);
     char *b = static_cast<char *>(ws);
     SeedArgs s{};
     s.u = u;
@@ -980,15 +1279,21 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
     s.bs1 = reinterpret_cast<double *>(b + w.off_bs1);
     s.bs2 = reinterpret_cast<double *>(b + w.off_bs2);
     s.r2 = reinterpret_cast<double *>(b + w.off_r2);
-    s.mdp = reinterpret_cast<float *>(b + w.off_mdp);
-    s.rr = reinterpret_cast<float *>(b + w.off_rr);
+    s.gs = reinterpret_cast<float *>(b + w.off_gs);
+    s.ge = reinterpret_cast<float *>(b + w.off_ge);
+    s.gr = reinterpret_cast<float *>(b + w.off_gr);
+    s.gn = reinterpret_cast<int32_t *>(b + w.off_gn);
+    s.gq = reinterpret_cast<int8_t *>(b + w.off_gq);
     s.near = reinterpret_cast<int32_t *>(b + w.off_near);
     s.perm = reinterpret_cast<int32_t *>(b + w.off_perm);
-    s.apos = reinterpret_cast<int32_t *>(b + w.off_apos);
     s.gcnt = reinterpret_cast<int32_t *>(b + w.off_gcnt);
     s.seg = reinterpret_cast<int32_t *>(b + w.off_seg);
     s.cur = reinterpret_cast<int32_t *>(b + w.off_cur);
-    s.pofs = reinterpret_cast<uint16_t *>(b + w.off_pofs);
+    s.pg = reinterpret_cast<int32_t *>(b + w.off_pg);
+    s.pm = reinterpret_cast<float *>(b + w.off_pm);
+    s.plo = reinterpret_cast<uint16_t *>(b + w.off_plo);
+    s.phi = reinterpret_cast<uint16_t *>(b + w.off_phi);
+    s.pcnt = reinterpret_cast<int32_t *>(b + w.off_pcnt);
     s.dirty = reinterpret_cast<unsigned char *>(b + w.off_dirty);
     s.taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
     s.cnt = reinterpret_cast<int *>(b + w.off_cnt);
@@ -997,6 +1302,8 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
     s.NR1 = w.nr1;
     s.NR2 = w.nr2;
     s.DSTRIDE = w.dstride;
+    s.NBMAX = w.nbmax;
+    s.CAP = w.cap;
     cudaError_t e = cudaMemsetAsync(s.cnt, 0, sizeof(int) * (size_t)H, st);
     if (e != cudaSuccess) return e;
     if (dt == ASM_BF16) {
