@@ -5,7 +5,9 @@ check and the benchmark's CPU-baseline leg may import this module.  It loads
 ``liboracle.so`` (built from ``asm_oracle.c`` by :func:`build`) with ctypes and
 marshals numpy arrays; every computation happens in the C file, in double
 precision, on the exact storage-dtype values the caller passes (bf16 inputs
-are upcast exactly).  Nothing here imports or calls the CUDA package.
+are upcast exactly), except the whitening functions, which are numpy in
+fp64 (with numpy's symmetric eigensolver as a library step).  Nothing here
+imports or calls the CUDA package.
 
 Method source: "Context Memorization for Efficient Long Context Generation"
 (gist.science summary of arXiv 2605.18226), section "Metodologia".
@@ -254,3 +256,47 @@ def full_attention(q, Kp, Vp, Kc, Vc, local_len, scale: float):
     _load().oracle_full_attention(_p(q), _p(Kp), _p(Vp), Lp, _p(Kc), _p(Vc), _p(ll), B, Hq,
                                   Hkv, Tmax, d, float(scale), _p(out), _p(lse))
     return out, lse
+
+
+# ------------------------------------------------------------ whitening ---
+#
+# "Context Memorization for Efficient Long Context Generation", Fase de
+# Inferencia Online, Recuperacion: retrieval may whiten the vectors first; the
+# pages give no recipe.  Reading: ZCA whitening from the calibration queries'
+# covariance, W = (C + eps I)^(-1/2) with C the (1/N) covariance of a head's
+# points and eps = eps_rel * trace(C) / d, applied as y = W (x - mu).
+
+
+def whitening(X, eps_rel: float = 1e-5):
+    """ZCA whitening of each head: X[H,N,d] -> mu[H,d], W[H,d,d] (symmetric)."""
+    X = _f64(X)
+    H, N, d = X.shape
+    mu = X.mean(axis=1)
+    W = np.empty((H, d, d))
+    for h in range(H):
+        Xc = X[h] - mu[h]
+        C = Xc.T @ Xc / N
+        eps = eps_rel * np.trace(C) / d
+        lam, V = np.linalg.eigh(C)
+        W[h] = (V * (lam + eps) ** -0.5) @ V.T
+    return mu, W
+
+
+def whiten(X, mu, W):
+    """y = W (x - mu) for every row of X[H,R,d] (W symmetric): (X - mu) @ W."""
+    X, mu, W = _f64(X), _f64(mu), _f64(W)
+    return np.einsum("hrd,hde->hre", X - mu[:, None, :], W)
+
+
+def decode_search(q, qs, C, Abar, logZbar, Kc, Vc, local_len, scale: float, metric: int = L2):
+    """One decode step whose centroid search uses qs[B,Hq,d] (for instance the
+    whitened queries against whitened centroids C) while the local attention
+    and the merge use q.  Returns (out, lse, idx, gap) as :func:`decode`."""
+    qs = _f64(qs)
+    B, Hq, _ = qs.shape
+    idx = np.zeros((B, Hq), dtype=np.int32)
+    gap = np.zeros((B, Hq))
+    for h in range(Hq):
+        idx[:, h], gap[:, h] = assign(qs[:, h], _f64(C)[h], metric)
+    out, lse, _, _ = decode(q, C, Abar, logZbar, Kc, Vc, local_len, scale, metric, idx_in=idx)
+    return out, lse, idx, gap

@@ -108,15 +108,17 @@ def test_kmeanspp_tiny_fp32_config_exact():
 
 
 def test_kmeanspp_llama_build_config_prefix():
-    """K = 8192 rounds on all 32 heads; the first 192 picks of two heads are
-    compared with the oracle (a pick depends only on earlier rounds)."""
+    """K = 8192 rounds on all 32 heads; picks compared with the oracle (a pick
+    depends only on earlier rounds): the first 2048 of head 0, which span the
+    pruned rounds from the first regrouping (round 1024) through four
+    regroupings, and the first 192 of head 31."""
     cfg = inputs.CONFIGS[3]
     bi = inputs.build_inputs(cfg)
     idx = gpu_seed(dev(bi["q"]), dev(bi["u"]))
     assert all(len(set(r.tolist())) == r.size for r in idx[[0, 31]])
-    for h in (0, 31):
-        o = O.kmeanspp_seed(bi["q"][h:h + 1], bi["u"][h:h + 1, :192])
-        np.testing.assert_array_equal(idx[h, :192], o[0])
+    for h, n in ((0, 2048), (31, 192)):
+        o = O.kmeanspp_seed(bi["q"][h:h + 1], bi["u"][h:h + 1, :n])
+        np.testing.assert_array_equal(idx[h, :n], o[0])
 
 
 @pytest.mark.parametrize("dt,d,N,K", [("bf16", 128, 8192, 1024), ("f32", 64, 5000, 600),

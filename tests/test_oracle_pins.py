@@ -441,3 +441,69 @@ def test_index_search_singleton_clusters_is_the_flat_search():
         np.testing.assert_array_equal(idx[:, h], flat)
         np.testing.assert_array_equal(sel[:, h, 0], flat)
         np.testing.assert_allclose(gs[:, h], gap)
+
+
+# ----------------------------------------------------------- whitening ---
+
+def test_whitening_diagonal_closed_form():
+    """Rows +-s_i e_i: mean 0 and covariance exactly diag(2 s_i^2 / N), so W
+    is diag((2 s_i^2 / N + eps)^-1/2) with eps = eps_rel * trace / d."""
+    d = 6
+    s = np.array([0.5, 1.0, 2.0, 3.0, 0.25, 1.5])
+    rows = np.concatenate([np.diag(s), -np.diag(s)])[None]  # N = 2d
+    N = 2 * d
+    mu, W = O.whitening(rows, eps_rel=1e-3)
+    var = 2 * s ** 2 / N
+    eps = 1e-3 * var.sum() / d
+    np.testing.assert_allclose(mu[0], 0.0, atol=1e-15)
+    np.testing.assert_allclose(W[0], np.diag((var + eps) ** -0.5), rtol=1e-12, atol=1e-12)
+
+
+def test_whitening_inverts_the_regularised_covariance():
+    """W is symmetric and W (C + eps I) W = I, C from numpy's own covariance."""
+    g = np.random.default_rng(3)
+    A = g.standard_normal((16, 16))
+    X = (g.standard_normal((2, 500, 16)) @ A) + 3.0
+    mu, W = O.whitening(X, eps_rel=1e-4)
+    for h in range(2):
+        C = np.cov(X[h], rowvar=False, bias=True)
+        eps = 1e-4 * np.trace(C) / 16
+        np.testing.assert_allclose(W[h], W[h].T, atol=1e-12)
+        np.testing.assert_allclose(W[h] @ (C + eps * np.eye(16)) @ W[h], np.eye(16), atol=1e-9)
+        np.testing.assert_allclose(mu[h], X[h].mean(0), atol=1e-12)
+
+
+def test_whitening_is_rotation_equivariant():
+    """ZCA (not PCA) whitening: rotating the data rotates W the same way."""
+    g = np.random.default_rng(4)
+    X = g.standard_normal((1, 400, 8)) @ g.standard_normal((8, 8))
+    Q, _ = np.linalg.qr(g.standard_normal((8, 8)))
+    _, W = O.whitening(X)
+    _, Wq = O.whitening(X @ Q)
+    np.testing.assert_allclose(Wq[0], Q.T @ W[0] @ Q, atol=1e-9)
+
+
+def test_whiten_gives_identity_covariance():
+    g = np.random.default_rng(5)
+    X = g.standard_normal((2, 1000, 12)) @ g.standard_normal((12, 12)) - 1.0
+    mu, W = O.whitening(X, eps_rel=0.0)
+    Y = O.whiten(X, mu, W)
+    for h in range(2):
+        np.testing.assert_allclose(Y[h].mean(0), 0.0, atol=1e-10)
+        np.testing.assert_allclose(np.cov(Y[h], rowvar=False, bias=True), np.eye(12), atol=1e-9)
+
+
+def test_decode_search_with_the_same_query_is_decode():
+    g = np.random.default_rng(6)
+    B, Hq, Hkv, d, K, T = 2, 4, 2, 16, 9, 5
+    q = g.standard_normal((B, Hq, d))
+    C = g.standard_normal((Hq, K, d))
+    Ab = g.standard_normal((Hq, K, d))
+    lz = g.uniform(5, 10, (Hq, K))
+    Kc = g.standard_normal((B, Hkv, T, d))
+    Vc = g.standard_normal((B, Hkv, T, d))
+    ll = np.array([T, 3], dtype=np.int32)
+    a = O.decode(q, C, Ab, lz, Kc, Vc, ll, 0.25)
+    b = O.decode_search(q, q, C, Ab, lz, Kc, Vc, ll, 0.25)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
