@@ -12,6 +12,7 @@ replayed from a CUDA graph.
     python bench.py --only states|assign|seed|lloyd|aggregate [--steps K] [--warmup W]
     python bench.py --sweep [--steps K] [--warmup W]
     python bench.py --index [--steps K] [--warmup W]
+    python bench.py --whiten [--steps K] [--warmup W]
 
 Prints ONE JSON line (rank 0).  `value` is decode query-heads/s over all
 ranks (each rank runs its own independent replica: weak scaling), timed with
@@ -645,6 +646,81 @@ def run_index(steps, warmup, Ps=(4, 8, 16)):
 
 # -------------------------------------------------------------------- main --
 
+def run_whiten(steps, warmup, layers=16):
+    """Whitened retrieval.  Build shape: the whitening of the 32 x 65536
+    calibration queries (fp64 moments and inverse square root) and their
+    transform.  LLaMA layer shape (K = 1024, T = 2048, B = 1): the decode step
+    with the whitened search (the query's transform, then the step searching
+    with it against whitened centres) against the plain step, `layers`
+    distinct layers per graph so every step streams from HBM."""
+    from long_prefix_attention_b200 import ops
+    bi = inputs.build_inputs(inputs.CONFIGS[3])
+    x = bi["q"].cuda()
+    H, N, d = x.shape
+    mu = torch.empty(H, d, dtype=torch.float32, device="cuda")
+    W = torch.empty(H, d, d, dtype=torch.float32, device="cuda")
+    ws = ops.alloc_workspace(ops.asm_whitening_workspace_size(H, d), "cuda")
+    y = torch.empty_like(x)
+
+    def ev_time(fn, n):
+        for _ in range(max(1, warmup // 4)):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    t_wh = ev_time(lambda: ops.asm_whitening(x, mu, W, ws), 3)
+    err = ops.asm_workspace_error(ws)
+    t_ap = ev_time(lambda: ops.asm_whiten(x, mu, W, y), 3)
+    del y, x
+    cfg = inputs.CONFIGS[1]
+    stack = DecodeStack(cfg, layers, inputs.BASE_SEED + 500)
+    for L in stack.layers:  # the memory's centres, whitened once with the heads' W
+        L["cw"] = torch.empty_like(L["centroids"])
+        ops.asm_whiten(L["centroids"], mu, W, L["cw"], layout="heads")
+        L["qs"] = torch.empty_like(L["q"])
+
+    def whitened_all():
+        for L in stack.layers:
+            ops.asm_whiten(L["q"], mu, W, L["qs"], layout="batch")
+            ops.asm_decode_step_search(L["q"], L["qs"], L["cw"], L["a_bar"], L["logz_bar"], L["k_cache"],
+                                       L["v_cache"], L["local_len"], L["scale"], L["out"], L["ws"])
+
+    def graph_of(fn):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
+    g_plain = graph_of(stack.launch_all)
+    g_wh = graph_of(whitened_all)
+    t_plain = time_steps(g_plain.replay, steps, warmup, 1) / steps / layers * 1e6
+    t_white = time_steps(g_wh.replay, steps, warmup, 1) / steps / layers * 1e6
+    print(json.dumps({
+        "whiten": "ZCA whitening of the calibration queries and the decode step with the whitened search",
+        "build": {"workload": inputs.CONFIGS[3]["name"], "whitening_ms": t_wh, "whitening_error": err,
+                  "moments_read_gbs": x_bytes(H, N, d) / (t_wh / 1e3) / 1e9, "transform_ms": t_ap,
+                  "transform_gbs": 2 * x_bytes(H, N, d) / (t_ap / 1e3) / 1e9},
+        "decode": {"workload": cfg["name"] + f" x {layers} layers", "plain_us_per_layer": t_plain,
+                   "whitened_search_us_per_layer": t_white, "steps": steps, "warmup": warmup}}))
+
+
+def x_bytes(H, N, d):
+    return H * N * d * 2
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -661,6 +737,8 @@ def main():
                     help="time one build stage alone (single-kernel profiling) and exit")
     ap.add_argument("--index", action="store_true",
                     help="two-level (hierarchical) search against the flat search (time and recall) and exit")
+    ap.add_argument("--whiten", action="store_true",
+                    help="whitening at the build shape and the decode step with the whitened search, and exit")
     ap.add_argument("--sweep", action="store_true",
                     help="decode over the 36-point B x K x T grid (and full attention at B=1) and exit")
     args = ap.parse_args()
@@ -672,6 +750,9 @@ def main():
         return
     if args.index:
         run_index(args.steps, args.warmup)
+        return
+    if args.whiten:
+        run_whiten(args.steps, args.warmup)
         return
     cfg = inputs.CONFIGS[1]
     world, rank, local = dist_setup(args.gpus)

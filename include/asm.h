@@ -345,13 +345,72 @@ asm_status asm_decode_step_indexed(const void *q, const void *supers,
                                    size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Whitened retrieval                                                       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The retrieval may whiten the vectors first ("Recuperacion" bullet of "Fase
+ * de Inferencia Online"; the pages give no recipe).  Reading: ZCA whitening
+ * from each head's calibration queries.  Build the clusters on the whitened
+ * queries (asm_whiten, then asm_kmeanspp_seed / asm_kmeans on the result);
+ * build the states from the original queries (asm_build_states) and aggregate
+ * them over those clusters (asm_aggregate); at decode, search with the
+ * whitened query against the whitened centres while the local attention uses
+ * the original query (asm_decode_step_search).
+ *
+ * asm_whitening -- per head h, from its N points x[h]:
+ *   mu[h] = mean of the points, C = (1/N) sum (x - mu)(x - mu)^T,
+ *   W[h]  = (C + eps I)^(-1/2), eps = eps_rel * trace(C) / d (symmetric).
+ *   x  [H, N, d] dt;  mu [H, d] fp32 output;  W [H, d, d] fp32 output.
+ *   ws asm_whitening_workspace_size(H, d) bytes; the error word (read with
+ *   asm_workspace_error) becomes ASM_ERR_TIMEOUT if the iteration for the
+ *   inverse square root has not converged after 100 steps.  That happens
+ *   for an exactly zero or a negative eigenvalue, which eps_rel > 0
+ *   excludes; a covariance singular only up to rounding has tiny positive
+ *   eigenvalues, and W then holds their (huge) inverse square roots, as the
+ *   exact definition does.  Use eps_rel > 0 for rank-deficient data.
+ * Moments in fp64, then a Newton-Schulz iteration in fp64 (two launches).
+ */
+size_t asm_whitening_workspace_size(int H, int d);
+asm_status asm_whitening(const void *x, int H, int N, int d, asm_dtype dt,
+                         float eps_rel, float *mu, float *W, void *ws,
+                         size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * asm_whiten -- y = W[h] (x - mu[h]) for R rows of every head h: row r of
+ * head h starts at element h * head_stride + r * row_stride of x (and of y
+ * with the y strides).  [H, N, d] points: strides (N d, d); decode queries
+ * [B, Hq, d] (H = Hq, R = B): strides (d, Hq d).  fp32 arithmetic, output
+ * rounded to dt.  x and y must not overlap.
+ */
+asm_status asm_whiten(const void *x, int H, int R, int d, asm_dtype dt,
+                      int64_t head_stride, int64_t row_stride, const float *mu,
+                      const float *W, void *y, int64_t y_head_stride,
+                      int64_t y_row_stride, cudaStream_t stream);
+
+/*
+ * asm_decode_step_search -- asm_decode_step whose centroid search uses
+ * q_search [B, Hq, d] (dt) in place of q; the local attention and the merge
+ * use q.  Same arguments, workspace and launches otherwise.
+ */
+asm_status asm_decode_step_search(const void *q, const void *q_search,
+                                  const void *centroids, const void *a_bar,
+                                  const float *logz_bar, const void *k_cache,
+                                  const void *v_cache, const int32_t *local_len,
+                                  int B, int Hq, int Hkv, int K, int Tmax, int d,
+                                  float scale, asm_metric metric, asm_dtype dt,
+                                  void *out, float *lse_out, int32_t *idx_out,
+                                  unsigned flags, void *ws, size_t ws_bytes,
+                                  cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Utilities                                                                */
 /* ------------------------------------------------------------------------ */
 
 /* Zero a decode / flash-decode / k-means workspace (counters, error word). */
 asm_status asm_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Error word of a decode / flash-decode / k-means workspace, copied to the host
+/* Error word of a decode / flash-decode / k-means / whitening workspace, copied to the host
  * pointer `code` (0 = no device-side error; otherwise ASM_ERR_TIMEOUT).
  * Synchronises `stream`. */
 asm_status asm_workspace_error(const void *ws, size_t ws_bytes, int *code,

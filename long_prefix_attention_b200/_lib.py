@@ -35,6 +35,11 @@ SIGNATURES = {
     "asm_decode_indexed_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I]),
     "asm_decode_step_indexed": (I, [P, P, P, I, I, I, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, P, P, P,
                                     SZ, P]),
+    "asm_whitening_workspace_size": (SZ, [I, I]),
+    "asm_whitening": (I, [P, I, I, I, I, F, P, P, P, SZ, P]),
+    "asm_whiten": (I, [P, I, I, I, I, ctypes.c_int64, ctypes.c_int64, P, P, P, ctypes.c_int64, ctypes.c_int64, P]),
+    "asm_decode_step_search": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, P, P, ctypes.c_uint, P,
+                                   SZ, P]),
     "asm_workspace_init": (I, [P, SZ, P]),
     "asm_workspace_error": (I, [P, SZ, ctypes.POINTER(ctypes.c_int), P]),
     "asm_status_string": (ctypes.c_char_p, [I]),

@@ -184,6 +184,57 @@ asm_status asm_decode_step(const void *q, const void *centroids, const void *a_b
                                          dt, out, lse_out, idx_out, flags, ws, num_sms(), stream));
 }
 
+asm_status asm_decode_step_search(const void *q, const void *q_search, const void *centroids, const void *a_bar,
+                                  const float *logz_bar, const void *k_cache, const void *v_cache,
+                                  const int32_t *local_len, int B, int Hq, int Hkv, int K, int Tmax, int d,
+                                  float scale, asm_metric metric, asm_dtype dt, void *out, float *lse_out,
+                                  int32_t *idx_out, unsigned flags, void *ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
+    if (!aligned(q_search, 16)) return ASM_ERR_INVALID_ARG;
+    if (!dt_ok(dt) || B < 1 || B > 4096 || K < 1 || Tmax < 0 || !(scale == scale)) return ASM_ERR_INVALID_ARG;
+    if (metric != ASM_L2 && metric != ASM_COSINE) return ASM_ERR_INVALID_ARG;
+    if ((flags & ~ASM_DECODE_PREFETCH_CENTROIDS) != 0) return ASM_ERR_INVALID_ARG;
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ASM_ERR_INVALID_ARG;
+    if (!d_ok(d) || !group_ok(Hq, Hkv)) return ASM_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(centroids, 16) || !aligned(a_bar, 16) || !aligned(logz_bar, 4) ||
+        !aligned(local_len, 4) || !aligned(out, 16))
+        return ASM_ERR_INVALID_ARG;
+    if (Tmax > 0 && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return ASM_ERR_INVALID_ARG;
+    if ((lse_out && !aligned(lse_out, 4)) || (idx_out && !aligned(idx_out, 4))) return ASM_ERR_INVALID_ARG;
+    if (!aligned(ws, 16) || ws_bytes < asm_decode_ws_bytes(0, B, Hq, Hkv, K, 0, Tmax, d, dt))
+        return ASM_ERR_WORKSPACE;
+    return cuda_status(asm_decode_launch(0, q, centroids, a_bar, logz_bar, nullptr, nullptr, 0, k_cache,
+                                         v_cache, local_len, B, Hq, Hkv, K, Tmax, d, scale, (int)metric,
+                                         dt, out, lse_out, idx_out, flags, ws, num_sms(), stream, q_search));
+}
+
+size_t asm_whitening_workspace_size(int H, int d) {
+    if (H < 1 || !d_ok(d)) return 0;
+    return asm_whitening_ws_bytes(H, d);
+}
+
+asm_status asm_whitening(const void *x, int H, int N, int d, asm_dtype dt, float eps_rel, float *mu, float *W,
+                         void *ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!dt_ok(dt) || H < 1 || N < 1 || !(eps_rel >= 0.f) || !(eps_rel < 1e30f)) return ASM_ERR_INVALID_ARG;
+    if (!d_ok(d)) return ASM_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(mu, 4) || !aligned(W, 4)) return ASM_ERR_INVALID_ARG;
+    if (!aligned(ws, 16) || ws_bytes < asm_whitening_ws_bytes(H, d)) return ASM_ERR_WORKSPACE;
+    return cuda_status(asm_whitening_launch(x, H, N, d, dt, eps_rel, mu, W, ws, stream));
+}
+
+asm_status asm_whiten(const void *x, int H, int R, int d, asm_dtype dt, int64_t head_stride, int64_t row_stride,
+                      const float *mu, const float *W, void *y, int64_t y_head_stride, int64_t y_row_stride,
+                      cudaStream_t stream) {
+    if (!dt_ok(dt) || H < 1 || R < 0) return ASM_ERR_INVALID_ARG;
+    if (!d_ok(d)) return ASM_ERR_UNSUPPORTED;
+    if (head_stride < 0 || row_stride < 0 || y_head_stride < 0 || y_row_stride < 0) return ASM_ERR_INVALID_ARG;
+    const size_t es = dt == ASM_BF16 ? 2 : 4;
+    if (!aligned(x, es) || !aligned(y, es) || !aligned(mu, 4) || !aligned(W, 4)) return ASM_ERR_INVALID_ARG;
+    if (R == 0) return ASM_OK;
+    return cuda_status(asm_whiten_launch(x, H, R, d, dt, (long long)head_stride, (long long)row_stride, mu, W, y,
+                                         (long long)y_head_stride, (long long)y_row_stride, stream));
+}
+
 asm_status asm_index_reorder(const int32_t *perm, int H, int K, int d, asm_dtype dt, const void *centroids,
                              const void *a_bar, const float *logz_bar, void *centroids_ord, void *a_bar_ord,
                              float *logz_bar_ord, cudaStream_t stream) {

@@ -74,6 +74,7 @@ struct DCfg {
 
 struct DecodeArgs {
     const void *q;
+    const void *qs;  // the queries of the centroid search (q unless given)
     const void *centroids;
     const void *a_bar;
     const float *logz_bar;
@@ -622,9 +623,9 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
                     for (int mt = 0; mt * 16 < a.B; ++mt) {
                         const int b0 = mt * 16 + gid, b1 = b0 + 8;
                         const uint32_t *q0 = reinterpret_cast<const uint32_t *>(
-                            (const T *)a.q + ((size_t)min(b0, a.B - 1) * a.Hq + x.h) * D);
+                            (const T *)a.qs + ((size_t)min(b0, a.B - 1) * a.Hq + x.h) * D);
                         const uint32_t *q1 = reinterpret_cast<const uint32_t *>(
-                            (const T *)a.q + ((size_t)min(b1, a.B - 1) * a.Hq + x.h) * D);
+                            (const T *)a.qs + ((size_t)min(b1, a.B - 1) * a.Hq + x.h) * D);
                         float dd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
                         for (int j = 0; j < C::KSTEPS; ++j) {
@@ -778,7 +779,7 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
                 const bool my_valid = (r0 + my_row) < x.valid;
                 for (int b = 0; b < a.B; ++b) {
                     float qv[C::EPL];
-                    load_vec<T, C::EPL>((const T *)a.q + ((size_t)b * a.Hq + x.h) * D + lane * C::EPL, qv);
+                    load_vec<T, C::EPL>((const T *)a.qs + ((size_t)b * a.Hq + x.h) * D + lane * C::EPL, qv);
                     float dp[C::CSW];
 #pragma unroll
                     for (int r = 0; r < C::CSW; ++r) {
@@ -1056,11 +1057,11 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
                               const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
                               int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, asm_dtype dt,
                               void *out, float *lse_out, int32_t *idx_out, unsigned flags, void *ws,
-                              int num_sms, cudaStream_t st) {
+                              int num_sms, cudaStream_t st, const void *q_search) {
     using namespace asmk;
     DecodeWs w = decode_ws_layout(mode, B, Hq, Hkv, K, Lp, Tmax, d, dt);
     DecodeArgs a{};
-    a.q = q; a.centroids = centroids; a.a_bar = a_bar; a.logz_bar = logz_bar;
+    a.q = q; a.qs = q_search ? q_search : q; a.centroids = centroids; a.a_bar = a_bar; a.logz_bar = logz_bar;
     a.k_prefix = k_prefix; a.v_prefix = v_prefix; a.k_cache = k_cache; a.v_cache = v_cache;
     a.local_len = local_len; a.out = out; a.lse_out = lse_out; a.idx_out = idx_out;
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.K = K; a.Tmax = Tmax; a.Lp = Lp;
@@ -1075,7 +1076,7 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
     if (dt == ASM_BF16)
         return asm_decode_tc_launch(mode, q, centroids, a_bar, logz_bar, k_prefix, v_prefix, Lp, k_cache, v_cache,
                                     local_len, B, Hq, Hkv, K, Tmax, d, scale, metric, out, lse_out, idx_out, flags,
-                                    ws, st);
+                                    ws, st, q_search);
     if (d == 128) return decode_launch_g<float, 128>(a, G, num_sms, st);
     return decode_launch_g<float, 64>(a, G, num_sms, st);
 }

@@ -54,6 +54,7 @@ struct Geo {
 
 struct Args {
     const __nv_bfloat16 *q;       // [B][Hq][D]
+    const __nv_bfloat16 *qs;      // [B][Hq][D] queries of the centroid search (q unless given)
     const __nv_bfloat16 *centroids;             // [Hq][K][D]
     const __nv_bfloat16 *k_cache, *v_cache;     // [B][Hkv][Tmax][D]
     const __nv_bfloat16 *k_prefix, *v_prefix;   // [Hkv][Lp][D]
@@ -237,7 +238,7 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
         for (int nt = 0; nt * 8 < nq; ++nt) {
             const int bq = 8 * nt + gid;
             const uint32_t *qr = reinterpret_cast<const uint32_t *>(
-                a.q + ((size_t)(qrow0 + min(bq, nq - 1)) * a.Hq + h) * D);
+                a.qs + ((size_t)(qrow0 + min(bq, nq - 1)) * a.Hq + h) * D);
             uint32_t qb0[KS], qb1[KS];
 #pragma unroll
             for (int j = 0; j < KS; ++j) {
@@ -461,7 +462,7 @@ asm_index_select(const Args a) {
     pdl_wait();
     pdl_launch_dependents();
     float qv[EPL];
-    load_vec<__nv_bfloat16, EPL>(a.q + (size_t)bh * D + lane * EPL, qv);
+    load_vec<__nv_bfloat16, EPL>(a.qs + (size_t)bh * D + lane * EPL, qv);
     const __nv_bfloat16 *S = a.supers + (size_t)h * a.K1 * D;
     for (int j = warp; j < a.K1; j += kWarps) {
         float sv[EPL];
@@ -740,11 +741,13 @@ cudaError_t asm_decode_tc_launch(int mode, const void *q, const void *centroids,
                                  const float *logz_bar, const void *k_prefix, const void *v_prefix, int Lp,
                                  const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
                                  int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, void *out,
-                                 float *lse_out, int32_t *idx_out, unsigned flags, void *ws, cudaStream_t st) {
+                                 float *lse_out, int32_t *idx_out, unsigned flags, void *ws, cudaStream_t st,
+                                 const void *q_search) {
     using namespace asmk;
     const TcWs w = tc_ws_layout(mode, B, Hq, K, Lp, Tmax, d);
     tc::Args a{};
     a.q = (const __nv_bfloat16 *)q;
+    a.qs = q_search ? (const __nv_bfloat16 *)q_search : a.q;
     a.centroids = (const __nv_bfloat16 *)centroids;
     a.k_cache = (const __nv_bfloat16 *)k_cache;
     a.v_cache = (const __nv_bfloat16 *)v_cache;
@@ -809,6 +812,7 @@ cudaError_t asm_decode_indexed_tc_launch(const void *q, const void *supers, cons
     const TcWs w = tc_ws_layout(2, B, Hq, K, 0, Tmax, d, P, max_seg);
     tc::Args a{};
     a.q = (const __nv_bfloat16 *)q;
+    a.qs = a.q;
     a.centroids = (const __nv_bfloat16 *)centroids;
     a.k_cache = (const __nv_bfloat16 *)k_cache;
     a.v_cache = (const __nv_bfloat16 *)v_cache;

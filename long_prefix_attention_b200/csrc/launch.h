@@ -17,7 +17,7 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
                               const int32_t *local_len, int B, int Hq, int Hkv, int K, int Tmax,
                               int d, float scale, int metric, asm_dtype dt, void *out,
                               float *lse_out, int32_t *idx_out, unsigned flags, void *ws,
-                              int num_sms, cudaStream_t st);
+                              int num_sms, cudaStream_t st, const void *q_search = nullptr);
 
 size_t asm_decode_ws_header_bytes(int B, int Hkv);
 
@@ -27,7 +27,8 @@ cudaError_t asm_decode_tc_launch(int mode, const void *q, const void *centroids,
                                  const float *logz_bar, const void *k_prefix, const void *v_prefix, int Lp,
                                  const void *k_cache, const void *v_cache, const int32_t *local_len, int B,
                                  int Hq, int Hkv, int K, int Tmax, int d, float scale, int metric, void *out,
-                                 float *lse_out, int32_t *idx_out, unsigned flags, void *ws, cudaStream_t st);
+                                 float *lse_out, int32_t *idx_out, unsigned flags, void *ws, cudaStream_t st,
+                                 const void *q_search = nullptr);
 
 // decode_tc.cu: two-level search decode (bf16)
 size_t asm_decode_indexed_tc_ws_bytes(int B, int Hq, int P, int max_seg, int Tmax, int d);
@@ -81,3 +82,11 @@ cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norm
 cudaError_t asm_aggregate_launch(const void *a, const float *logz, const int32_t *perm,
                                  const int32_t *seg_off, int H, int N, int d, int K, int zmode,
                                  asm_dtype dt, void *a_bar, float *logz_bar, cudaStream_t st);
+
+// whiten.cu: ZCA whitening (moments, inverse square root, row transform)
+size_t asm_whitening_ws_bytes(int H, int d);
+cudaError_t asm_whitening_launch(const void *x, int H, int N, int d, asm_dtype dt, float eps_rel, float *mu,
+                                 float *W, void *ws, cudaStream_t st);
+cudaError_t asm_whiten_launch(const void *x, int H, int R, int d, asm_dtype dt, long long sh_in, long long sr_in,
+                              const float *mu, const float *W, void *y, long long sh_out, long long sr_out,
+                              cudaStream_t st);

@@ -173,6 +173,59 @@ def asm_decode_step(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, 
         _p(idx_out), int(flags), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def asm_decode_step_search(q, q_search, centroids, a_bar, logz_bar, k_cache, v_cache, local_len,
+                           scale: float, out, ws, lse_out=None, idx_out=None, metric: int = ASM_L2,
+                           flags: int = 0, stream=None):
+    """asm_decode_step whose centroid search uses q_search[B,Hq,d] (e.g. the
+    whitened queries) while the local attention and the merge use q."""
+    _contig(q, q_search, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, out, lse_out, idx_out)
+    if q_search.shape != q.shape or q_search.dtype != q.dtype:
+        raise AsmError("asm_decode_step_search", ASM_ERR_INVALID_ARG)
+    B, Hq, d = q.shape
+    K = centroids.shape[1]
+    _, Hkv, Tmax, _ = k_cache.shape
+    _check("asm_decode_step_search", _lib.load().asm_decode_step_search(
+        _p(q), _p(q_search), _p(centroids), _p(a_bar), _p(logz_bar), _p(k_cache), _p(v_cache),
+        _p(local_len), B, Hq, Hkv, K, Tmax, d, float(scale), int(metric), _dt(q), _p(out), _p(lse_out),
+        _p(idx_out), int(flags), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def asm_whitening_workspace_size(H: int, d: int) -> int:
+    return int(_lib.load().asm_whitening_workspace_size(H, d))
+
+
+def asm_whitening(x, mu, W, ws, eps_rel: float = 1e-5, stream=None):
+    """ZCA whitening of each head of x[H,N,d]: mu[H,d] and W[H,d,d] (fp32)."""
+    _contig(x, mu, W)
+    H, N, d = x.shape
+    _check("asm_whitening", _lib.load().asm_whitening(
+        _p(x), H, N, d, _dt(x), float(eps_rel), _p(mu), _p(W), _p(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def asm_whiten(x, mu, W, y, layout: str | None = None, stream=None):
+    """y = W[h] (x - mu[h]) row by row.  layout "heads": x, y are [H, R, d]
+    (calibration points, centres); "batch": [R, H, d] (decode queries).  When
+    omitted it is inferred from which dimension equals H = mu.shape[0], and
+    must then be unambiguous."""
+    _contig(x, mu, W, y)
+    H, d = mu.shape
+    if x.shape != y.shape or x.dtype != y.dtype or x.dim() != 3 or x.shape[2] != d:
+        raise AsmError("asm_whiten", ASM_ERR_INVALID_ARG)
+    if layout is None:
+        if (x.shape[0] == H) == (x.shape[1] == H):
+            raise AsmError("asm_whiten", ASM_ERR_INVALID_ARG)
+        layout = "heads" if x.shape[0] == H else "batch"
+    if layout == "heads" and x.shape[0] == H:
+        R, sh, sr = x.shape[1], x.shape[1] * d, d
+    elif layout == "batch" and x.shape[1] == H:
+        R, sh, sr = x.shape[0], d, H * d
+    else:
+        raise AsmError("asm_whiten", ASM_ERR_INVALID_ARG)
+    _check("asm_whiten", _lib.load().asm_whiten(
+        _p(x), H, R, d, _dt(x), sh, sr, _p(mu), _p(W), _p(y), sh, sr, _stream(stream)))
+
+
 def asm_decode_step_noalloc(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len,
                             scale: float, out, lse_out=None, idx_out=None, metric: int = ASM_L2,
                             flags: int = 0, stream=None):

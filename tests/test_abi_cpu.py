@@ -146,3 +146,28 @@ def test_index_reorder_rejects_bad_arguments(lib):
     bad = list(args)
     bad[3] = 80
     assert lib.asm_index_reorder(*bad) == 2       # head dim
+
+
+def test_whitening_and_search_decode_reject_bad_arguments(lib):
+    P = FAKE
+    ws_need = lib.asm_whitening_workspace_size(32, 128)
+    assert ws_need > 0 and lib.asm_whitening_workspace_size(32, 96) == 0
+    # asm_whitening(x, H, N, d, dt, eps_rel, mu, W, ws, ws_bytes, stream)
+    assert lib.asm_whitening(P, 32, 65536, 96, 1, 1e-5, P, P, P, ws_need, None) == UNSUPPORTED
+    assert lib.asm_whitening(NULL, 32, 65536, 128, 1, 1e-5, P, P, P, ws_need, None) == INVALID
+    assert lib.asm_whitening(P, 32, 0, 128, 1, 1e-5, P, P, P, ws_need, None) == INVALID
+    assert lib.asm_whitening(P, 32, 100, 128, 1, -1.0, P, P, P, ws_need, None) == INVALID
+    assert lib.asm_whitening(P, 32, 100, 128, 1, float("nan"), P, P, P, ws_need, None) == INVALID
+    assert lib.asm_whitening(P, 32, 100, 128, 1, 1e-5, P, P, P, ws_need - 1, None) == WORKSPACE
+    # asm_whiten(x, H, R, d, dt, sh, sr, mu, W, y, ysh, ysr, stream)
+    assert lib.asm_whiten(P, 2, 10, 128, 1, 1280, -128, P, P, P, 1280, 128, None) == INVALID
+    assert lib.asm_whiten(P, 2, 10, 100, 1, 1000, 100, P, P, P, 1000, 100, None) == UNSUPPORTED
+    assert lib.asm_whiten(P, 2, 10, 128, 1, 1280, 128, P, P, NULL, 1280, 128, None) == INVALID
+    assert lib.asm_whiten(P, 2, 0, 128, 1, 1280, 128, P, P, P, 1280, 128, None) == 0  # nothing to do
+    # asm_decode_step_search: a missing search query is rejected first
+    assert lib.asm_decode_step_search(P, NULL, P, P, P, P, P, P, 1, 32, 8, 1024, 2048, 128, 0.088, 0, 1, P,
+                                      NULL, NULL, 0, P, 1 << 30, None) == INVALID
+    assert lib.asm_decode_step_search(P, ODD, P, P, P, P, P, P, 1, 32, 8, 1024, 2048, 128, 0.088, 0, 1, P,
+                                      NULL, NULL, 0, P, 1 << 30, None) == INVALID
+    assert lib.asm_decode_step_search(P, P, P, P, P, P, P, P, 1, 32, 8, 1024, 2048, 128, 0.088, 0, 1, P,
+                                      NULL, NULL, 0, P, 8, None) == WORKSPACE
