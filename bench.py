@@ -301,11 +301,33 @@ def cpu_build_baseline(cfg, bi):
                       f"{K} rounds and {iters} Lloyd iterations"}
 
 
-def run_build(cfg, with_cpu=True):
-    """Full offline build at the 32/8-head, N=65536, L=16384, K=8192 shape."""
+def build_head_shard(Hq, Hkv, world, rank):
+    """Query heads [h0, h1) that rank `rank` of `world` builds: whole KV groups
+    (the GQA heads sharing a KV head stay together), split as evenly as the
+    groups allow; a rank may get none when world > Hkv."""
+    G = Hq // Hkv
+    g0, g1 = rank * Hkv // world, (rank + 1) * Hkv // world
+    return g0 * G, g1 * G
+
+
+def run_build(cfg, with_cpu=True, world=1, rank=0):
+    """Full offline build at the 32/8-head, N=65536, L=16384, K=8192 shape.
+    With several ranks each builds its shard of the heads (heads are
+    independent: no data-path exchange); the job's time is the slowest
+    rank's, stage by stage."""
     from long_prefix_attention_b200 import ops
     bi = inputs.build_inputs(cfg)
-    x, k, v, u = bi["q"].cuda(), bi["k"].cuda(), bi["v"].cuda(), bi["u"].cuda()
+    Htot = bi["q"].shape[0]
+    h0, h1 = build_head_shard(Htot, bi["k"].shape[0], world, rank)
+    G = Htot // bi["k"].shape[0]
+    if h1 == h0:  # nothing to build on this rank: it only joins the timing
+        t = [0.0, 0.0, 0.0, 0.0]
+        for _ in range(2):
+            barrier(world)
+        t = [max_over_ranks(x, world) for x in t]
+        return None
+    x, u = bi["q"][h0:h1].cuda(), bi["u"][h0:h1].cuda()
+    k, v = bi["k"][h0 // G:h1 // G].cuda(), bi["v"][h0 // G:h1 // G].cuda()
     H, N, d = x.shape
     K, iters, L = cfg["K"], cfg["iters"], cfg["L"]
     chunks = cfg["chunks"]
@@ -327,6 +349,7 @@ def run_build(cfg, with_cpu=True):
     vc = [v[:, i * cl:(i + 1) * cl].contiguous() for i in range(chunks)]
 
     def stage_times():
+        barrier(world)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         ev[0].record()
         for i in range(chunks):
@@ -343,14 +366,16 @@ def run_build(cfg, with_cpu=True):
 
     stage_times()  # warm-up
     t = stage_times()
+    t = [max_over_ranks(x, world) for x in t]  # the slowest rank, stage by stage
     total = sum(t)
     hbm, tf, tfs, src = peaks()
-    states_flops = 4.0 * N * L * d * H
-    assign_flops = 2.0 * N * K * d * H * iters
+    states_flops = 4.0 * N * L * d * Htot
+    assign_flops = 2.0 * N * K * d * Htot * iters
     cpu = cpu_build_baseline(cfg, bi) if with_cpu else None
     return {
-        "workload": cfg["name"], "queries": H * N, "cpu_baseline": cpu,
-        "value": H * N / (total / 1e3), "unit": "queries/s",
+        "workload": cfg["name"], "queries": Htot * N, "cpu_baseline": cpu,
+        "ranks": world, "heads_per_rank": H,
+        "value": Htot * N / (total / 1e3), "unit": "queries/s",
         "ms": {"states_4chunks": t[0], "kmeanspp_seed": t[1], "lloyd_10": t[2], "aggregate": t[3],
                "total": total},
         "states_tflops": states_flops / (t[0] / 1e3) / 1e12,
@@ -806,9 +831,12 @@ def main():
     d2h = h2d
 
     build = None
-    if not args.no_build and rank == 0:
+    if not args.no_build:
+        # every rank builds its shard of the heads (the same collectives on
+        # every rank: barriers and the per-stage max over ranks)
         try:
-            build = run_build(inputs.CONFIGS[3], with_cpu=not args.no_cpu and world == 1)
+            build = run_build(inputs.CONFIGS[3], with_cpu=not args.no_cpu and world == 1, world=world,
+                              rank=rank)
         except Exception as e:  # report, do not hide
             build = {"error": repr(e)}
     cpu = None

@@ -60,3 +60,22 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(0.25, 1) == 0.25
     assert bench.job_throughput(10, 0.5, 1) == pytest.approx(20.0)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8, 12])
+def test_build_head_shards_cover_the_heads_in_whole_groups(world):
+    """The build leg's head shards: disjoint, in order, whole KV groups (the
+    G = 4 query heads of a KV head together), as even as the groups allow;
+    with more ranks than KV heads some ranks get none."""
+    sys.path.insert(0, ROOT)
+    import bench
+    Hq, Hkv = 32, 8
+    shards = [bench.build_head_shard(Hq, Hkv, world, r) for r in range(world)]
+    assert shards[0][0] == 0 and shards[-1][1] == Hq
+    for (a0, a1), (b0, b1) in zip(shards, shards[1:]):
+        assert a1 == b0
+    sizes = [h1 - h0 for h0, h1 in shards]
+    assert all(s % (Hq // Hkv) == 0 for s in sizes)
+    groups = [s // (Hq // Hkv) for s in sizes]
+    assert max(groups) - min(groups) <= 1
+    assert sum(s == 0 for s in sizes) == max(0, world - Hkv)
