@@ -320,11 +320,11 @@ def run_build(cfg, with_cpu=True, world=1, rank=0):
     Htot = bi["q"].shape[0]
     h0, h1 = build_head_shard(Htot, bi["k"].shape[0], world, rank)
     G = Htot // bi["k"].shape[0]
-    if h1 == h0:  # nothing to build on this rank: it only joins the timing
-        t = [0.0, 0.0, 0.0, 0.0]
+    if h1 == h0:  # nothing to build on this rank: it joins the same collectives
         for _ in range(2):
-            barrier(world)
-        t = [max_over_ranks(x, world) for x in t]
+            barrier(world)  # the two stage_times() calls
+        for _ in range(4):
+            max_over_ranks(0.0, world)  # the four stage maxima
         return None
     x, u = bi["q"][h0:h1].cuda(), bi["u"][h0:h1].cuda()
     k, v = bi["k"][h0 // G:h1 // G].cuda(), bi["v"][h0 // G:h1 // G].cuda()

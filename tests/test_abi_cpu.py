@@ -171,3 +171,19 @@ def test_whitening_and_search_decode_reject_bad_arguments(lib):
                                       NULL, NULL, 0, P, 1 << 30, None) == INVALID
     assert lib.asm_decode_step_search(P, P, P, P, P, P, P, P, 1, 32, 8, 1024, 2048, 128, 0.088, 0, 1, P,
                                       NULL, NULL, 0, P, 8, None) == WORKSPACE
+
+
+def test_whiten_binding_needs_an_unambiguous_layout():
+    """The Python binding infers [H, R, d] or [R, H, d] from mu's head count and
+    refuses to guess when both dimensions equal it (no library call is made)."""
+    import torch
+    from long_prefix_attention_b200 import ops
+    mu = torch.zeros(4, 64)
+    W = torch.zeros(4, 64, 64)
+    x = torch.zeros(4, 4, 64)
+    with pytest.raises(ops.AsmError):
+        ops.asm_whiten(x, mu, W, torch.zeros_like(x))
+    with pytest.raises(ops.AsmError):  # the named layout must match the shape
+        ops.asm_whiten(torch.zeros(5, 3, 64), mu, W, torch.zeros(5, 3, 64), layout="heads")
+    with pytest.raises(ops.AsmError):  # shape and dtype of y must match x
+        ops.asm_whiten(torch.zeros(4, 7, 64), mu, W, torch.zeros(4, 7, 64, dtype=torch.bfloat16))
