@@ -35,6 +35,7 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -73,7 +74,7 @@ def decode_bytes(B, Hq, Hkv, K, T, d, eb=2):
 class ClockSampler:
     def __init__(self, gpu_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"asm_bench_clocks_{os.getpid()}.csv")
         self.gpu = gpu_index
 
     def __enter__(self):
