@@ -810,7 +810,9 @@ def main():
         secs_rank = time_steps(stack.step, args.steps, max(3, args.warmup), world)
     value = job_throughput(stack.B * stack.Hq * args.layers * args.steps, secs_rank, world)
     secs = max_over_ranks(secs_rank, world)
-    launches = args.steps * args.layers * 2  # asm_decode_units + asm_decode_merge per layer
+    per_step_launches = stack.ops.asm_decode_step_launches(stack.B, stack.Hq, stack.Hkv, stack.K, stack.T,
+                                                           stack.d, torch.bfloat16)
+    launches = args.steps * args.layers * per_step_launches
     ms_per_step = secs * 1e3 / args.steps
     per_launch_s = secs / (args.steps * args.layers)  # one decode step (both kernels) of one layer
     bpl = stack.bytes_per_launch()

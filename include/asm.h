@@ -209,9 +209,10 @@ asm_status asm_aggregate(const void *a, const float *logz, const int32_t *perm,
  *   flags     0, or ASM_DECODE_PREFETCH_CENTROIDS
  *   ws        asm_decode_workspace_size(...) bytes, zeroed once by
  *             asm_workspace_init.
- * One kernel launch, with programmatic dependent launch enabled: the kernel
- * may start while the preceding kernel in `stream` finishes, and reads no
- * argument before that kernel has completed -- except, with
+ * One (fp32) or two (bf16) kernel launches, with programmatic dependent
+ * launch enabled: a kernel may start while the preceding kernel in `stream`
+ * finishes, and reads no argument before that kernel has completed --
+ * except, with
  * ASM_DECODE_PREFETCH_CENTROIDS, the `centroids` array, which it may start
  * streaming early.  Pass that flag only when the preceding kernel in the
  * stream does not write `centroids` (the memory is normally built once and
@@ -230,6 +231,15 @@ asm_status asm_decode_step(const void *q, const void *centroids,
                            void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * asm_decode_step_launches -- kernel launches one asm_decode_step (or
+ * asm_decode_step_search) call with these sizes makes, or -1 for sizes the
+ * call rejects or when no device is present: bf16 2 (split units, then a
+ * merge kernel), fp32 1 (streaming CTAs, merged by the last to finish).
+ */
+int asm_decode_step_launches(int B, int Hq, int Hkv, int K, int Tmax, int d,
+                             asm_dtype dt);
+
+/*
  * asm_decode_step_noalloc -- asm_decode_step without a caller workspace.
  * The paper has no counterpart: this is a convenience of the library.
  * It exists for callers that cannot allocate device memory at the point where
@@ -241,7 +251,9 @@ asm_status asm_decode_step(const void *q, const void *centroids,
  * holds it until the process exits).  Problems whose
  * asm_decode_workspace_size(...) exceeds 8 MiB are rejected with
  * ASM_ERR_WORKSPACE.  The call allocates and frees nothing.
- * Arguments, outputs and errors are those of asm_decode_step.
+ * Arguments, outputs and errors are those of asm_decode_step; every argument
+ * is checked before anything is enqueued.  A device-side timeout is recorded
+ * in the array's error word, which asm_decode_noalloc_error reads.
  * - The first call on a device looks up the array's device address for that
  *   device (with the device current); make that first call before any stream
  *   capture.
@@ -259,6 +271,16 @@ asm_status asm_decode_step_noalloc(const void *q, const void *centroids,
                                    asm_dtype dt, void *out, float *lse_out,
                                    int32_t *idx_out, unsigned flags,
                                    cudaStream_t stream);
+
+/*
+ * asm_decode_noalloc_error -- the error word of the built-in scratch of
+ * asm_decode_step_noalloc on the current device, copied to the host pointer
+ * `code`: 0, or ASM_ERR_TIMEOUT when a bounded device-side wait of the last
+ * asm_decode_step_noalloc call on this device gave up (its outputs are then
+ * not valid).  Each call clears the word when it starts, so this reports the
+ * most recent call.  Synchronises `stream`.
+ */
+asm_status asm_decode_noalloc_error(int *code, cudaStream_t stream);
 
 /*
  * asm_flash_decode -- the quantity the memory stands in for: decode attention

@@ -28,7 +28,9 @@ SIGNATURES = {
     "asm_aggregate": (I, [P, P, P, P, I, I, I, I, I, I, P, P, P]),
     "asm_decode_workspace_size": (SZ, [I, I, I, I, I, I, I]),
     "asm_decode_step": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, P, P, ctypes.c_uint, P, SZ, P]),
+    "asm_decode_step_launches": (I, [I, I, I, I, I, I, I]),
     "asm_decode_step_noalloc": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, P, P, ctypes.c_uint, P]),
+    "asm_decode_noalloc_error": (I, [ctypes.POINTER(ctypes.c_int), P]),
     "asm_flash_decode_workspace_size": (SZ, [I, I, I, I, I, I, I]),
     "asm_flash_decode": (I, [P, P, P, I, P, P, P, I, I, I, I, I, F, I, P, P, P, SZ, P]),
     "asm_index_reorder": (I, [P, I, I, I, I, P, P, P, P, P, P, P]),

@@ -29,18 +29,6 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxe
          "-I", INCLUDE, "-I", CSRC]
 
 
-def _cutlass_include() -> str | None:
-    """CUTLASS/CuTe headers vendored with the Python environment (header-only use)."""
-    import site
-    cands = []
-    for sp in site.getsitepackages() + [site.getusersitepackages()]:
-        cands.append(os.path.join(sp, "flashinfer", "data", "cutlass", "include"))
-    for c in cands:
-        if os.path.exists(os.path.join(c, "cute", "arch", "mma_sm100_desc.hpp")):
-            return c
-    return None
-
-
 def _headers() -> list[str]:
     return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         glob.glob(os.path.join(INCLUDE, "*.h"))
@@ -58,9 +46,6 @@ def build(force: bool = False, verbose: bool = False, jobs: int | None = None) -
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_mtime = max([os.path.getmtime(h) for h in _headers()] + [0.0])
     flags = list(FLAGS)
-    cut = _cutlass_include()
-    if cut:
-        flags += ["-isystem", cut, "-DASM_HAVE_CUTLASS=1"]
     objs, todo = [], []
     for s in srcs:
         o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")

@@ -161,12 +161,23 @@ size_t asm_decode_workspace_size(int B, int Hq, int Hkv, int K, int Tmax, int d,
     return asm_decode_ws_bytes(0, B, Hq, Hkv, K, 0, Tmax, d, dt);
 }
 
-asm_status asm_decode_step(const void *q, const void *centroids, const void *a_bar,
-                           const float *logz_bar, const void *k_cache, const void *v_cache,
-                           const int32_t *local_len, int B, int Hq, int Hkv, int K, int Tmax, int d,
-                           float scale, asm_metric metric, asm_dtype dt, void *out, float *lse_out,
-                           int32_t *idx_out, unsigned flags, void *ws, size_t ws_bytes,
-                           cudaStream_t stream) {
+int asm_decode_step_launches(int B, int Hq, int Hkv, int K, int Tmax, int d, asm_dtype dt) {
+    if (!dt_ok(dt) || B < 1 || B > 4096 || K < 1 || Tmax < 0 || !d_ok(d) || !group_ok(Hq, Hkv)) return -1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return -1;
+    }
+    return dt == ASM_F32 ? 1 : 2;
+}
+
+}  // extern "C"
+
+// Every check of asm_decode_step except the workspace's.
+asm_status asm_decode_check_args(const void *q, const void *centroids, const void *a_bar, const float *logz_bar,
+                                 const void *k_cache, const void *v_cache, const int32_t *local_len, int B, int Hq,
+                                 int Hkv, int K, int Tmax, int d, float scale, int metric, asm_dtype dt,
+                                 const void *out, const float *lse_out, const int32_t *idx_out, unsigned flags) {
     if (!dt_ok(dt) || B < 1 || B > 4096 || K < 1 || Tmax < 0 || !(scale == scale)) return ASM_ERR_INVALID_ARG;
     if (metric != ASM_L2 && metric != ASM_COSINE) return ASM_ERR_INVALID_ARG;
     if ((flags & ~ASM_DECODE_PREFETCH_CENTROIDS) != 0) return ASM_ERR_INVALID_ARG;
@@ -177,6 +188,20 @@ asm_status asm_decode_step(const void *q, const void *centroids, const void *a_b
         return ASM_ERR_INVALID_ARG;
     if (Tmax > 0 && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return ASM_ERR_INVALID_ARG;
     if ((lse_out && !aligned(lse_out, 4)) || (idx_out && !aligned(idx_out, 4))) return ASM_ERR_INVALID_ARG;
+    return ASM_OK;
+}
+
+extern "C" {
+
+asm_status asm_decode_step(const void *q, const void *centroids, const void *a_bar,
+                           const float *logz_bar, const void *k_cache, const void *v_cache,
+                           const int32_t *local_len, int B, int Hq, int Hkv, int K, int Tmax, int d,
+                           float scale, asm_metric metric, asm_dtype dt, void *out, float *lse_out,
+                           int32_t *idx_out, unsigned flags, void *ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+    const asm_status v = asm_decode_check_args(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, B, Hq,
+                                               Hkv, K, Tmax, d, scale, (int)metric, dt, out, lse_out, idx_out, flags);
+    if (v != ASM_OK) return v;
     if (!aligned(ws, 16) || ws_bytes < asm_decode_ws_bytes(0, B, Hq, Hkv, K, 0, Tmax, d, dt))
         return ASM_ERR_WORKSPACE;
     return cuda_status(asm_decode_launch(0, q, centroids, a_bar, logz_bar, nullptr, nullptr, 0, k_cache,

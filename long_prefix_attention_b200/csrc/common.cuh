@@ -203,10 +203,12 @@ __device__ __forceinline__ int ld_cg(const int *p) { return __ldcg(p); }
 // ------------------------------------------- warp-level tensor-core MMA ----
 namespace asmk {
 
-// D += A * B for one m16n8k16 tile, bf16 inputs, fp32 accumulation.
+// D += A * B for one m16n8k16 tile, bf16 inputs, fp32 accumulation.  It
+// reads and writes registers only, so the compiler may interleave
+// independent accumulation chains.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

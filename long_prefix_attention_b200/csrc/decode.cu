@@ -1,4 +1,4 @@
-// decode.cu -- fused ASM decode step and the full-attention flash-decode.
+// decode.cu -- fp32 ASM decode step and full-attention flash-decode.
 //
 // "Context Memorization for Efficient Long Context Generation", Metodologia,
 // "Fase de Inferencia Online": each query head retrieves the nearest memory
@@ -12,11 +12,9 @@
 // (flash-decode mode instead has, per (b,g), [prefix K/V units][local units]).
 // CTA i owns the contiguous unit range [i*upc, (i+1)*upc), one CTA per SM.
 // A producer warp streams the units through a ring of shared-memory stages
-// (bf16: 3-D TMA tensor loads with 128-byte swizzling; fp32: 1-D bulk
-// copies), completing on mbarrier transaction counts; four consumer warps
-// process each unit -- bf16 on tensor cores with warp-level m16n8k16 MMAs
-// (q.c and |c|^2 from the same ldmatrix fragments, then q.k and p.v), fp32 on
-// CUDA cores.  Consecutive units of one key (a head for centroid scans, a
+// with 1-D bulk copies, completing on mbarrier transaction counts; four
+// consumer warps process each unit on CUDA cores in fp32 (the bf16 storage
+// type runs in decode_tc.cu).  Consecutive units of one key (a head for centroid scans, a
 // (b,g) pair for attention) are reduced in registers and written as ONE
 // partial per CTA run, into the slot of the run's first unit.  Each CTA then
 // adds the run length to the (b,g) arrival counter; the CTA that completes a
@@ -26,15 +24,14 @@
 // resets the counter for the next call.  No CTA ever waits for another.
 //
 // Launched with programmatic dependent launch: every thread waits for the
-// preceding grid before reading inputs; with ASM_DECODE_PREFETCH_CENTROIDS
-// the producer may stream the first centroid units before that wait.
+// preceding grid before reading inputs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
 
-#include <type_traits>
+#include <algorithm>
 
 #include "common.cuh"
 #include "launch.h"
@@ -48,28 +45,17 @@ constexpr int kDecodeStages = 8;
 
 template <typename T, int D, int G>
 struct DCfg {
-    static constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;
-    static constexpr int EPL = D / 32;                         // dims per lane (CUDA-core path)
+    static constexpr int EPL = D / 32;                         // dims per lane
     static constexpr int ROWB = D * (int)sizeof(T);            // bytes per row
     static constexpr int CS = kUnitBytes / ROWB;               // centroid rows / unit
     static constexpr int TS = kUnitBytes / (2 * ROWB);         // tokens / unit
-    // CUDA-core path
     static constexpr int TSW = (32 / G) < TS ? (32 / G) : TS;  // tokens / warp step
     static constexpr int NV = G * TSW;                         // values reduced / step
     static constexpr int R = 32 / NV;                          // lanes per value
     static constexpr int NTG = TS / TSW;                       // token groups / unit
     static constexpr int CSW = CS / kDecodeConsumerWarps;      // centroid rows / warp
-    // tensor-core path (bf16)
-    static constexpr int HALVES = D / 64;                      // 128-byte column halves
-    static constexpr int TW = TS / kDecodeConsumerWarps;       // tokens / warp / unit (8 or 16)
-    static constexpr int NTS = TW / 8;                         // S n-tiles / warp
-    static constexpr int RB = CS / kDecodeConsumerWarps / 16;  // 16-row scan blocks / warp
-    static constexpr int KSTEPS = D / 16;
-    static constexpr int NTO = D / 8;                          // O n-tiles
     static_assert(NV <= 32 && (NV & (NV - 1)) == 0, "NV");
     static_assert(CSW >= 1 && CSW <= 32 && (CSW & (CSW - 1)) == 0, "CSW");
-    static_assert(!TC || (TW == 8 || TW == 16), "TW");
-    static_assert(!TC || G <= 8, "G");
 };
 
 struct DecodeArgs {
@@ -105,12 +91,6 @@ struct DecodeArgs {
     float *ws_o;      // [B][Hq][nP+nA][D] unnormalised outputs
     int *ws_cnt;      // [B][Hkv] arrival counters (self-resetting)
     int *ws_err;
-};
-
-// TMA descriptors (bf16 path): centroids [Hq][K][D], caches [B*Hkv][Tmax][D],
-// prefix [Hkv][Lp][D]; boxes of 64 columns (128 bytes) x unit rows.
-struct DecodeMaps {
-    CUtensorMap c, k, v, kp, vp;
 };
 
 // n / d for 0 <= n < 2^31 and d >= 1, from a float reciprocal and an exact fix-up.
@@ -332,7 +312,7 @@ __device__ __noinline__ void combine(const DecodeArgs &a, int b, int g, int warp
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
-decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
+decode_kernel(const DecodeArgs a) {
     using C = DCfg<T, D, G>;
     constexpr int S = kDecodeStages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -366,23 +346,6 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
     }
     __syncthreads();
 
-    // Units issued before the dependency wait: leading centroid units only,
-    // and only when the caller allows it (the memory is not written by the
-    // preceding kernel).
-    int pre = 0;
-    if constexpr (C::TC) {
-        if (warp == kDecodeConsumerWarps && lane == 0 && (a.flags & 1)) {
-            for (; pre < min(n_units, S); ++pre) {
-                const Unit x = decode_unit<T, D, G>(a, u_begin + pre, nullptr);
-                if (x.kind != 0) break;
-                unsigned char *dst = stage_buf + (size_t)pre * kUnitBytes;
-                mbar_arrive_expect_tx(&full[pre], C::CS * C::ROWB);
-#pragma unroll
-                for (int hf = 0; hf < C::HALVES; ++hf)
-                    tma_load_3d(dst + hf * C::CS * 128, &maps.c, 64 * hf, x.first, x.h, &full[pre]);
-            }
-        }
-    }
     pdl_wait();
     pdl_launch_dependents();
     const int *lens = a.local_len;
@@ -393,7 +356,7 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
             // start fetching the row lengths the local units of this range need
             asm volatile("prefetch.global.L1 [%0];" ::"l"(lens));
             asm volatile("prefetch.global.L1 [%0];" ::"l"(lens + (a.B - 1)));
-            for (int i = pre; i < n_units; ++i) {
+            for (int i = 0; i < n_units; ++i) {
                 const int s = i % S;
                 if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) set_error(a.ws_err);
                 const Unit x = decode_unit<T, D, G>(a, u_begin + i, lens);
@@ -402,46 +365,26 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
                     mbar_arrive(&full[s]);
                     continue;
                 }
-                if constexpr (C::TC) {
-                    if (x.kind == 0) {
-                        mbar_arrive_expect_tx(&full[s], C::CS * C::ROWB);
-#pragma unroll
-                        for (int hf = 0; hf < C::HALVES; ++hf)
-                            tma_load_3d(dst + hf * C::CS * 128, &maps.c, 64 * hf, x.first, x.h, &full[s]);
-                    } else {
-                        mbar_arrive_expect_tx(&full[s], 2 * C::TS * C::ROWB);
-                        const CUtensorMap *mk = x.prefix ? &maps.kp : &maps.k;
-                        const CUtensorMap *mv = x.prefix ? &maps.vp : &maps.v;
-                        const int c2 = x.prefix ? x.g : x.b * a.Hkv + x.g;
-#pragma unroll
-                        for (int hf = 0; hf < C::HALVES; ++hf) {
-                            tma_load_3d(dst + hf * C::TS * 128, mk, 64 * hf, x.first, c2, &full[s]);
-                            tma_load_3d(dst + kUnitBytes / 2 + hf * C::TS * 128, mv, 64 * hf, x.first, c2,
-                                        &full[s]);
-                        }
-                    }
+                const uint32_t rb = (uint32_t)x.valid * C::ROWB;
+                if (x.kind == 0) {
+                    const char *src = (const char *)a.centroids + ((size_t)x.h * a.K + x.first) * C::ROWB;
+                    mbar_arrive_expect_tx(&full[s], rb);
+                    bulk_g2s(dst, src, rb, &full[s]);
                 } else {
-                    const uint32_t rb = (uint32_t)x.valid * C::ROWB;
-                    if (x.kind == 0) {
-                        const char *src = (const char *)a.centroids + ((size_t)x.h * a.K + x.first) * C::ROWB;
-                        mbar_arrive_expect_tx(&full[s], rb);
-                        bulk_g2s(dst, src, rb, &full[s]);
+                    size_t off;
+                    const char *kb, *vb;
+                    if (x.prefix) {
+                        off = ((size_t)x.g * a.Lp + x.first) * C::ROWB;
+                        kb = (const char *)a.k_prefix;
+                        vb = (const char *)a.v_prefix;
                     } else {
-                        size_t off;
-                        const char *kb, *vb;
-                        if (x.prefix) {
-                            off = ((size_t)x.g * a.Lp + x.first) * C::ROWB;
-                            kb = (const char *)a.k_prefix;
-                            vb = (const char *)a.v_prefix;
-                        } else {
-                            off = (((size_t)x.b * a.Hkv + x.g) * a.Tmax + x.first) * C::ROWB;
-                            kb = (const char *)a.k_cache;
-                            vb = (const char *)a.v_cache;
-                        }
-                        mbar_arrive_expect_tx(&full[s], 2 * rb);
-                        bulk_g2s(dst, kb + off, rb, &full[s]);
-                        bulk_g2s(dst + kUnitBytes / 2, vb + off, rb, &full[s]);
+                        off = (((size_t)x.b * a.Hkv + x.g) * a.Tmax + x.first) * C::ROWB;
+                        kb = (const char *)a.k_cache;
+                        vb = (const char *)a.v_cache;
                     }
+                    mbar_arrive_expect_tx(&full[s], 2 * rb);
+                    bulk_g2s(dst, kb + off, rb, &full[s]);
+                    bulk_g2s(dst + kUnitBytes / 2, vb + off, rb, &full[s]);
                 }
             }
             // Drain: every issued copy has landed before the CTA may exit.
@@ -452,17 +395,12 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
     }
 
     // ---------------------------------------------------- consumer warps
-    const int gid = lane >> 2, quad = lane & 3;
     int cur_key = -1;
     Unit run{};
     int run_len = 0;
-    // CUDA-core attention state: (m, l, o) per head of the group, lanes = dims
+    // attention state: (m, l, o) per head of the group, lanes = dims
     float m_run[G], l_run[G], o_run[G][C::EPL];
     float qreg[G][C::EPL];
-    // tensor-core attention state: row gid (= head of the group), O fragments
-    float tm_run = kNegInf, tl_run = 0.f;
-    float to[C::NTO][4];
-    uint32_t qa0[C::KSTEPS], qa2[C::KSTEPS];
 
     auto flush = [&](const Unit &rx, int len) {
         // Publish this CTA's partial of the run's key, then count arrivals.
@@ -479,29 +417,15 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
                 a.ws_srch[((size_t)b * a.Hq + rx.h) * a.nS + rx.slot] = make_float2(bs, __int_as_float(bi));
             }
         } else {
-            if constexpr (C::TC) {
-                if (gid < G) {
-                    if (quad == 0) {
-                        flush_m[warp * G + gid] = tm_run;
-                        flush_l[warp * G + gid] = tl_run;
-                    }
 #pragma unroll
-                    for (int c = 0; c < C::NTO; ++c) {
-                        flush_o[(warp * G + gid) * D + 8 * c + 2 * quad] = to[c][0];
-                        flush_o[(warp * G + gid) * D + 8 * c + 2 * quad + 1] = to[c][1];
-                    }
+            for (int h = 0; h < G; ++h) {
+                if (lane == 0) {
+                    flush_m[warp * G + h] = m_run[h];
+                    flush_l[warp * G + h] = l_run[h];
                 }
-            } else {
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    if (lane == 0) {
-                        flush_m[warp * G + h] = m_run[h];
-                        flush_l[warp * G + h] = l_run[h];
-                    }
-#pragma unroll
-                    for (int e = 0; e < C::EPL; ++e)
-                        flush_o[(warp * G + h) * D + lane * C::EPL + e] = o_run[h][e];
-                }
+                for (int e = 0; e < C::EPL; ++e)
+                    flush_o[(warp * G + h) * D + lane * C::EPL + e] = o_run[h][e];
             }
             consumer_sync();
             const int nslots = a.nP + a.nA;
@@ -552,31 +476,16 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
                 for (int b = lane; b < a.B; b += 32)
                     best[warp * a.B + b] = make_float2(kNegInf, __int_as_float(0x7fffffff));
             } else {
-                if constexpr (C::TC) {
-                    tm_run = kNegInf;
-                    tl_run = 0.f;
 #pragma unroll
-                    for (int c = 0; c < C::NTO; ++c) to[c][0] = to[c][1] = to[c][2] = to[c][3] = 0.f;
-                    // A fragments of the group's queries: row gid = head gid of the group
-                    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
-                        (const T *)a.q + ((size_t)x.b * a.Hq + x.g * G + min(gid, G - 1)) * D);
+                for (int h = 0; h < G; ++h) {
+                    m_run[h] = kNegInf;
+                    l_run[h] = 0.f;
+                    float qv[C::EPL];
+                    load_vec<T, C::EPL>((const T *)a.q + ((size_t)x.b * a.Hq + x.g * G + h) * D + lane * C::EPL, qv);
 #pragma unroll
-                    for (int j = 0; j < C::KSTEPS; ++j) {
-                        qa0[j] = gid < G ? __ldg(qrow + 8 * j + quad) : 0u;
-                        qa2[j] = gid < G ? __ldg(qrow + 8 * j + 4 + quad) : 0u;
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        m_run[h] = kNegInf;
-                        l_run[h] = 0.f;
-                        float qv[C::EPL];
-                        load_vec<T, C::EPL>((const T *)a.q + ((size_t)x.b * a.Hq + x.g * G + h) * D + lane * C::EPL, qv);
-#pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) {
-                            o_run[h][e] = 0.f;
-                            qreg[h][e] = qv[e] * a.qscale;
-                        }
+                    for (int e = 0; e < C::EPL; ++e) {
+                        o_run[h][e] = 0.f;
+                        qreg[h][e] = qv[e] * a.qscale;
                     }
                 }
             }
@@ -586,285 +495,115 @@ decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
         if (!mbar_wait(&full[s], (i / S) & 1)) set_error(a.ws_err);
         const unsigned char *buf = stage_buf + (size_t)s * kUnitBytes;
 
-        if constexpr (C::TC) {
-            const uint32_t sbuf = smem_addr(buf);
-            if (x.kind == 0) {
-                // -------- centroid scan on tensor cores: 16-row blocks, all rows b
+        if (x.kind == 0) {
+            // ---------------- centroid scan (CUDA cores): CSW rows per warp
+            const int r0 = warp * C::CSW;
+            float nrm[C::CSW];
+            float cf[C::CSW][C::EPL];
 #pragma unroll
-                for (int rb = 0; rb < C::RB; ++rb) {
-                    const int r0 = (warp * C::RB + rb) * 16;
-                    if (r0 >= x.valid) break;
-                    uint32_t bf[C::KSTEPS][2][2];  // [k-step][n-tile][lo/hi]
+            for (int r = 0; r < C::CSW; ++r) {
+                if (r0 + r < x.valid) {
+                    load_vec<T, C::EPL>(reinterpret_cast<const T *>(buf + (size_t)(r0 + r) * C::ROWB) + lane * C::EPL, cf[r]);
+                } else {
 #pragma unroll
-                    for (int j = 0; j < C::KSTEPS; ++j) {
-                        const int i4 = lane >> 3;
-                        const int row = r0 + 8 * (i4 >> 1) + (lane & 7);
-                        const int col = 16 * j + 8 * (i4 & 1);
-                        const uint32_t addr = sbuf + (col >> 6) * (C::CS * 128) + swz128(row, (col & 63) >> 3);
-                        ldsm_x4(addr, bf[j][0][0], bf[j][0][1], bf[j][1][0], bf[j][1][1]);
-                    }
-                    // |c|^2 as the diagonal of C C^T (same fragments as A and B)
-                    float dn[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                    for (int j = 0; j < C::KSTEPS; ++j)
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt)
-                            mma_bf16_16816(dn[nt], bf[j][0][0], bf[j][1][0], bf[j][0][1], bf[j][1][1],
-                                           bf[j][nt][0], bf[j][nt][1]);
-                    const float diag0 = dn[0][gid & 1], diag1 = dn[1][2 + (gid & 1)];
-                    float nrm[2][2];
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int rr = 2 * quad + e;
-                            nrm[nt][e] = __shfl_sync(0xffffffffu, nt == 0 ? diag0 : diag1, 4 * rr + (rr >> 1));
-                        }
-                    for (int mt = 0; mt * 16 < a.B; ++mt) {
-                        const int b0 = mt * 16 + gid, b1 = b0 + 8;
-                        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(
-                            (const T *)a.qs + ((size_t)min(b0, a.B - 1) * a.Hq + x.h) * D);
-                        const uint32_t *q1 = reinterpret_cast<const uint32_t *>(
-                            (const T *)a.qs + ((size_t)min(b1, a.B - 1) * a.Hq + x.h) * D);
-                        float dd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                        for (int j = 0; j < C::KSTEPS; ++j) {
-                            const uint32_t a0 = b0 < a.B ? __ldg(q0 + 8 * j + quad) : 0u;
-                            const uint32_t a1 = b1 < a.B ? __ldg(q1 + 8 * j + quad) : 0u;
-                            const uint32_t a2 = b0 < a.B ? __ldg(q0 + 8 * j + 4 + quad) : 0u;
-                            const uint32_t a3 = b1 < a.B ? __ldg(q1 + 8 * j + 4 + quad) : 0u;
-#pragma unroll
-                            for (int nt = 0; nt < 2; ++nt)
-                                mma_bf16_16816(dd[nt], a0, a1, a2, a3, bf[j][nt][0], bf[j][nt][1]);
-                        }
-#pragma unroll
-                        for (int hr = 0; hr < 2; ++hr) {  // rows b0 (hr 0) and b1
-                            float bs = kNegInf;
-                            int bi = 0x7fffffff;
-#pragma unroll
-                            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int rloc = r0 + 8 * nt + 2 * quad + e;
-                                    const float dot = dd[nt][2 * hr + e];
-                                    const float nr = nrm[nt][e];
-                                    float sc = (a.metric == 0) ? dot - 0.5f * nr
-                                                               : (nr > 0.f ? dot / sqrtf(nr) : 0.f);
-                                    int ci = x.first + rloc;
-                                    if (rloc >= x.valid) { sc = kNegInf; ci = 0x7fffffff; }
-                                    if (better(sc, ci, bs, bi)) { bs = sc; bi = ci; }
-                                }
-#pragma unroll
-                            for (int m = 1; m <= 2; m <<= 1) {
-                                const float os = __shfl_xor_sync(0xffffffffu, bs, m);
-                                const int oi = __shfl_xor_sync(0xffffffffu, bi, m);
-                                if (better(os, oi, bs, bi)) { bs = os; bi = oi; }
-                            }
-                            const int bb = hr ? b1 : b0;
-                            if (quad == 0 && bb < a.B) {
-                                const float2 cur = best[warp * a.B + bb];
-                                if (better(bs, bi, cur.x, __float_as_int(cur.y)))
-                                    best[warp * a.B + bb] = make_float2(bs, __int_as_float(bi));
-                            }
-                        }
-                    }
+                    for (int e = 0; e < C::EPL; ++e) cf[r][e] = 0.f;
                 }
-            } else {
-                // -------- attention on tensor cores: TW tokens per warp
-                const int t0 = warp * C::TW;
-                if (t0 < x.valid) {
-                    float sf[C::NTS][4];
+                float t = 0.f;
 #pragma unroll
-                    for (int nt = 0; nt < C::NTS; ++nt) sf[nt][0] = sf[nt][1] = sf[nt][2] = sf[nt][3] = 0.f;
+                for (int e = 0; e < C::EPL; ++e) t = fmaf(cf[r][e], cf[r][e], t);
+                nrm[r] = t;
+            }
+            const float nr = transpose_reduce<C::CSW>(nrm, lane);
+            const int my_row = lane / (32 / C::CSW);
+            const int my_c = x.first + r0 + my_row;
+            const bool my_valid = (r0 + my_row) < x.valid;
+            for (int b = 0; b < a.B; ++b) {
+                float qv[C::EPL];
+                load_vec<T, C::EPL>((const T *)a.qs + ((size_t)b * a.Hq + x.h) * D + lane * C::EPL, qv);
+                float dp[C::CSW];
 #pragma unroll
-                    for (int j = 0; j < C::KSTEPS; j += 2) {
+                for (int r = 0; r < C::CSW; ++r) {
+                    float t = 0.f;
 #pragma unroll
-                        for (int nt = 0; nt < C::NTS; ++nt) {
-                            const int i4 = lane >> 3;
-                            const int row = t0 + 8 * nt + (lane & 7);
-                            const int col = 16 * (j + (i4 >> 1)) + 8 * (i4 & 1);
-                            const uint32_t addr = sbuf + (col >> 6) * (C::TS * 128) + swz128(row, (col & 63) >> 3);
-                            uint32_t b0, b1, b2, b3;
-                            ldsm_x4(addr, b0, b1, b2, b3);
-                            mma_bf16_16816(sf[nt], qa0[j], 0u, qa2[j], 0u, b0, b1);
-                            mma_bf16_16816(sf[nt], qa0[j + 1], 0u, qa2[j + 1], 0u, b2, b3);
-                        }
-                    }
-                    // online softmax for row gid (head), base-2 logits
-                    float p[C::NTS][2];
-                    float mx = kNegInf;
-#pragma unroll
-                    for (int nt = 0; nt < C::NTS; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int tok = t0 + 8 * nt + 2 * quad + e;
-                            p[nt][e] = tok < x.valid ? sf[nt][e] * a.qscale : kNegInf;
-                            mx = fmaxf(mx, p[nt][e]);
-                        }
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float mnew = fmaxf(tm_run, mx);
-                    const float alpha = (mnew == kNegInf) ? 1.f : exp2f(tm_run - mnew);
-                    float rs = 0.f;
-#pragma unroll
-                    for (int nt = 0; nt < C::NTS; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            p[nt][e] = (p[nt][e] == kNegInf) ? 0.f : exp2f(p[nt][e] - mnew);
-                            rs += p[nt][e];
-                        }
-                    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-                    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-                    tl_run = tl_run * alpha + rs;
-                    tm_run = mnew;
-#pragma unroll
-                    for (int c = 0; c < C::NTO; ++c) {
-                        to[c][0] *= alpha;
-                        to[c][1] *= alpha;
-                    }
-                    const uint32_t pa0 = pack_bf16(p[0][0], p[0][1]);
-                    const uint32_t pa2 = C::NTS == 2 ? pack_bf16(p[C::NTS - 1][0], p[C::NTS - 1][1]) : 0u;
-                    const uint32_t vbase = sbuf + kUnitBytes / 2;
-                    if constexpr (C::NTS == 1) {
-#pragma unroll
-                        for (int c = 0; c < C::NTO; c += 4) {
-                            const int i4 = lane >> 3;
-                            const int row = t0 + (lane & 7);
-                            const int col = 8 * (c + i4);
-                            const uint32_t addr = vbase + (col >> 6) * (C::TS * 128) + swz128(row, (col & 63) >> 3);
-                            uint32_t v0, v1, v2, v3;
-                            ldsm_x4_t(addr, v0, v1, v2, v3);
-                            mma_bf16_16816(to[c], pa0, 0u, 0u, 0u, v0, 0u);
-                            mma_bf16_16816(to[c + 1], pa0, 0u, 0u, 0u, v1, 0u);
-                            mma_bf16_16816(to[c + 2], pa0, 0u, 0u, 0u, v2, 0u);
-                            mma_bf16_16816(to[c + 3], pa0, 0u, 0u, 0u, v3, 0u);
-                        }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < C::NTO; c += 2) {
-                            const int i4 = lane >> 3;
-                            const int row = t0 + 8 * (i4 & 1) + (lane & 7);
-                            const int col = 8 * (c + (i4 >> 1));
-                            const uint32_t addr = vbase + (col >> 6) * (C::TS * 128) + swz128(row, (col & 63) >> 3);
-                            uint32_t v0, v1, v2, v3;
-                            ldsm_x4_t(addr, v0, v1, v2, v3);
-                            mma_bf16_16816(to[c], pa0, 0u, pa2, 0u, v0, v1);
-                            mma_bf16_16816(to[c + 1], pa0, 0u, pa2, 0u, v2, v3);
-                        }
-                    }
+                    for (int e = 0; e < C::EPL; ++e) t = fmaf(qv[e], cf[r][e], t);
+                    dp[r] = t;
+                }
+                const float dot = transpose_reduce<C::CSW>(dp, lane);
+                float sc = (a.metric == 0) ? dot - 0.5f * nr : (nr > 0.f ? dot / sqrtf(nr) : 0.f);
+                int ci = my_c;
+                if (!my_valid) { sc = kNegInf; ci = 0x7fffffff; }
+                warp_argmax(sc, ci);
+                if (lane == 0) {
+                    const float2 cur = best[warp * a.B + b];
+                    if (better(sc, ci, cur.x, __float_as_int(cur.y)))
+                        best[warp * a.B + b] = make_float2(sc, __int_as_float(ci));
                 }
             }
         } else {
-            if (x.kind == 0) {
-                // ---------------- centroid scan (CUDA cores): CSW rows per warp
-                const int r0 = warp * C::CSW;
-                float nrm[C::CSW];
-                float cf[C::CSW][C::EPL];
+            // ---------------- attention (CUDA cores): warps take token groups
+            const unsigned char *kb = buf;
+            const unsigned char *vb = buf + kUnitBytes / 2;
+            for (int tg = warp; tg < C::NTG; tg += kDecodeConsumerWarps) {
+                const int t0 = tg * C::TSW;
+                if (t0 >= x.valid) break;
+                float part[C::NV];
 #pragma unroll
-                for (int r = 0; r < C::CSW; ++r) {
-                    if (r0 + r < x.valid) {
-                        load_vec<T, C::EPL>(reinterpret_cast<const T *>(buf + (size_t)(r0 + r) * C::ROWB) + lane * C::EPL, cf[r]);
+                for (int t = 0; t < C::TSW; ++t) {
+                    float kf[C::EPL];
+                    if (t0 + t < x.valid) {
+                        load_vec<T, C::EPL>(reinterpret_cast<const T *>(kb + (size_t)(t0 + t) * C::ROWB) + lane * C::EPL, kf);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) cf[r][e] = 0.f;
+                        for (int e = 0; e < C::EPL; ++e) kf[e] = 0.f;
                     }
-                    float t = 0.f;
-#pragma unroll
-                    for (int e = 0; e < C::EPL; ++e) t = fmaf(cf[r][e], cf[r][e], t);
-                    nrm[r] = t;
-                }
-                const float nr = transpose_reduce<C::CSW>(nrm, lane);
-                const int my_row = lane / (32 / C::CSW);
-                const int my_c = x.first + r0 + my_row;
-                const bool my_valid = (r0 + my_row) < x.valid;
-                for (int b = 0; b < a.B; ++b) {
-                    float qv[C::EPL];
-                    load_vec<T, C::EPL>((const T *)a.qs + ((size_t)b * a.Hq + x.h) * D + lane * C::EPL, qv);
-                    float dp[C::CSW];
-#pragma unroll
-                    for (int r = 0; r < C::CSW; ++r) {
-                        float t = 0.f;
-#pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) t = fmaf(qv[e], cf[r][e], t);
-                        dp[r] = t;
-                    }
-                    const float dot = transpose_reduce<C::CSW>(dp, lane);
-                    float sc = (a.metric == 0) ? dot - 0.5f * nr : (nr > 0.f ? dot / sqrtf(nr) : 0.f);
-                    int ci = my_c;
-                    if (!my_valid) { sc = kNegInf; ci = 0x7fffffff; }
-                    warp_argmax(sc, ci);
-                    if (lane == 0) {
-                        const float2 cur = best[warp * a.B + b];
-                        if (better(sc, ci, cur.x, __float_as_int(cur.y)))
-                            best[warp * a.B + b] = make_float2(sc, __int_as_float(ci));
-                    }
-                }
-            } else {
-                // ---------------- attention (CUDA cores): warps take token groups
-                const unsigned char *kb = buf;
-                const unsigned char *vb = buf + kUnitBytes / 2;
-                for (int tg = warp; tg < C::NTG; tg += kDecodeConsumerWarps) {
-                    const int t0 = tg * C::TSW;
-                    if (t0 >= x.valid) break;
-                    float part[C::NV];
-#pragma unroll
-                    for (int t = 0; t < C::TSW; ++t) {
-                        float kf[C::EPL];
-                        if (t0 + t < x.valid) {
-                            load_vec<T, C::EPL>(reinterpret_cast<const T *>(kb + (size_t)(t0 + t) * C::ROWB) + lane * C::EPL, kf);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < C::EPL; ++e) kf[e] = 0.f;
-                        }
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            float acc = 0.f;
-#pragma unroll
-                            for (int e = 0; e < C::EPL; ++e) acc = fmaf(qreg[h][e], kf[e], acc);
-                            part[h * C::TSW + t] = acc;
-                        }
-                    }
-                    float sv = transpose_reduce<C::NV>(part, lane);
-                    const int vidx = lane / C::R;
-                    const int my_t = vidx % C::TSW;
-                    if (t0 + my_t >= x.valid) sv = kNegInf;
-                    float mx = sv;
-#pragma unroll
-                    for (int m = 16 / G; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-                    float mnew[G], alpha[G];
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        const float mh = __shfl_sync(0xffffffffu, mx, h * (32 / G));
-                        mnew[h] = fmaxf(m_run[h], mh);
-                        alpha[h] = (mnew[h] == kNegInf) ? 1.f : exp2f(m_run[h] - mnew[h]);
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < C::EPL; ++e) acc = fmaf(qreg[h][e], kf[e], acc);
+                        part[h * C::TSW + t] = acc;
                     }
-                    const int my_h = vidx / C::TSW;
-                    float mh_l = mnew[0];
+                }
+                float sv = transpose_reduce<C::NV>(part, lane);
+                const int vidx = lane / C::R;
+                const int my_t = vidx % C::TSW;
+                if (t0 + my_t >= x.valid) sv = kNegInf;
+                float mx = sv;
 #pragma unroll
-                    for (int h = 1; h < G; ++h) if (my_h == h) mh_l = mnew[h];
-                    const float p = (sv == kNegInf) ? 0.f : exp2f(sv - mh_l);
-                    float ps = p;
+                for (int m = 16 / G; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+                float mnew[G], alpha[G];
 #pragma unroll
-                    for (int m = 16 / G; m >= C::R; m >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
+                for (int h = 0; h < G; ++h) {
+                    const float mh = __shfl_sync(0xffffffffu, mx, h * (32 / G));
+                    mnew[h] = fmaxf(m_run[h], mh);
+                    alpha[h] = (mnew[h] == kNegInf) ? 1.f : exp2f(m_run[h] - mnew[h]);
+                }
+                const int my_h = vidx / C::TSW;
+                float mh_l = mnew[0];
+#pragma unroll
+                for (int h = 1; h < G; ++h) if (my_h == h) mh_l = mnew[h];
+                const float p = (sv == kNegInf) ? 0.f : exp2f(sv - mh_l);
+                float ps = p;
+#pragma unroll
+                for (int m = 16 / G; m >= C::R; m >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float sh = __shfl_sync(0xffffffffu, ps, h * (32 / G));
+                    l_run[h] = l_run[h] * alpha[h] + sh;
+                    m_run[h] = mnew[h];
+#pragma unroll
+                    for (int e = 0; e < C::EPL; ++e) o_run[h][e] *= alpha[h];
+                }
+#pragma unroll
+                for (int t = 0; t < C::TSW; ++t) {
+                    if (t0 + t >= x.valid) break;
+                    float vf[C::EPL];
+                    load_vec<T, C::EPL>(reinterpret_cast<const T *>(vb + (size_t)(t0 + t) * C::ROWB) + lane * C::EPL, vf);
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        const float sh = __shfl_sync(0xffffffffu, ps, h * (32 / G));
-                        l_run[h] = l_run[h] * alpha[h] + sh;
-                        m_run[h] = mnew[h];
+                        const float ph = __shfl_sync(0xffffffffu, p, (h * C::TSW + t) * C::R);
 #pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) o_run[h][e] *= alpha[h];
-                    }
-#pragma unroll
-                    for (int t = 0; t < C::TSW; ++t) {
-                        if (t0 + t >= x.valid) break;
-                        float vf[C::EPL];
-                        load_vec<T, C::EPL>(reinterpret_cast<const T *>(vb + (size_t)(t0 + t) * C::ROWB) + lane * C::EPL, vf);
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            const float ph = __shfl_sync(0xffffffffu, p, (h * C::TSW + t) * C::R);
-#pragma unroll
-                            for (int e = 0; e < C::EPL; ++e) o_run[h][e] = fmaf(ph, vf[e], o_run[h][e]);
-                        }
+                        for (int e = 0; e < C::EPL; ++e) o_run[h][e] = fmaf(ph, vf[e], o_run[h][e]);
                     }
                 }
             }
@@ -969,21 +708,6 @@ template <typename T, int D, int G>
 static cudaError_t decode_launch_t(DecodeArgs a, int num_sms, cudaStream_t st) {
     using C = DCfg<T, D, G>;
     decode_geometry<T, D, G>(a, num_sms);
-    DecodeMaps maps;
-    memset(&maps, 0, sizeof(maps));
-    if constexpr (C::TC) {
-        if (a.mode == 0 && !make_map_3d(&maps.c, a.centroids, D, a.K, a.Hq, C::CS)) return cudaErrorInvalidValue;
-        if (a.Tmax > 0) {
-            if (!make_map_3d(&maps.k, a.k_cache, D, a.Tmax, (uint64_t)a.B * a.Hkv, C::TS) ||
-                !make_map_3d(&maps.v, a.v_cache, D, a.Tmax, (uint64_t)a.B * a.Hkv, C::TS))
-                return cudaErrorInvalidValue;
-        }
-        if (a.mode == 1 && a.Lp > 0) {
-            if (!make_map_3d(&maps.kp, a.k_prefix, D, a.Lp, a.Hkv, C::TS) ||
-                !make_map_3d(&maps.vp, a.v_prefix, D, a.Lp, a.Hkv, C::TS))
-                return cudaErrorInvalidValue;
-        }
-    }
     const int grid = (a.U + a.upc - 1) / a.upc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -1007,7 +731,7 @@ static cudaError_t decode_launch_t(DecodeArgs a, int num_sms, cudaStream_t st) {
     }
     cfg.blockDim = dim3(kDecodeThreads);
     cfg.dynamicSmemBytes = smem;
-    return cudaLaunchKernelEx(&cfg, kern, a, maps);
+    return cudaLaunchKernelEx(&cfg, kern, a);
     }
 }
 
@@ -1081,8 +805,7 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
     return decode_launch_g<float, 64>(a, G, num_sms, st);
 }
 
-// Bytes at the start of a decode workspace that must be zero before a call:
-// the error word and the (b, g) arrival counters.
-size_t asm_decode_ws_header_bytes(int B, int Hkv) {
+size_t asm_decode_ws_header_bytes(int B, int Hkv, asm_dtype dt) {
+    if (dt == ASM_BF16) return 256;  // the bf16 kernels keep no counters: only the error word
     return align256(256 + sizeof(int) * (size_t)B * Hkv);
 }

@@ -52,14 +52,32 @@ extern "C" asm_status asm_decode_step_noalloc(const void *q, const void *centroi
                                               int Hq, int Hkv, int K, int Tmax, int d, float scale,
                                               asm_metric metric, asm_dtype dt, void *out, float *lse_out,
                                               int32_t *idx_out, unsigned flags, cudaStream_t stream) {
+    // every argument is checked before anything touches the stream
+    const asm_status v = asm_decode_check_args(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, B, Hq,
+                                               Hkv, K, Tmax, d, scale, (int)metric, dt, out, lse_out, idx_out, flags);
+    if (v != ASM_OK) return v;
     const size_t need = asm_decode_workspace_size(B, Hq, Hkv, K, Tmax, d, dt);
     if (need == 0) return ASM_ERR_INVALID_ARG;
     if (need > kNoAllocScratchBytes) return ASM_ERR_WORKSPACE;  // beyond the fixed scratch
     void *ws = scratch_on_current_device();
     if (ws == nullptr) return ASM_ERR_CUDA;
-    // The array keeps the previous call's contents: clear the error word and
-    // the arrival counters, which must start at zero.
-    if (cudaMemsetAsync(ws, 0, asm_decode_ws_header_bytes(B, Hkv), stream) != cudaSuccess) return ASM_ERR_CUDA;
+    // The array keeps the previous call's contents: clear the error word (and
+    // for fp32 the arrival counters), which must start at zero.
+    if (cudaMemsetAsync(ws, 0, asm_decode_ws_header_bytes(B, Hkv, dt), stream) != cudaSuccess) return ASM_ERR_CUDA;
     return asm_decode_step(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, B, Hq, Hkv, K, Tmax, d,
                            scale, metric, dt, out, lse_out, idx_out, flags, ws, kNoAllocScratchBytes, stream);
+}
+
+// The error word of the built-in scratch on the current device: the device-side
+// status of the last asm_decode_step_noalloc call there.
+extern "C" asm_status asm_decode_noalloc_error(int *code, cudaStream_t stream) {
+    if (code == nullptr) return ASM_ERR_INVALID_ARG;
+    void *ws = scratch_on_current_device();
+    if (ws == nullptr) return ASM_ERR_CUDA;
+    int v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return ASM_ERR_CUDA;
+    *code = v;
+    return ASM_OK;
 }

@@ -40,6 +40,7 @@ namespace tc {
 constexpr int kUnit = 32768;     // bytes per unit
 constexpr int kWarps = 4;        // compute warps per unit CTA
 constexpr int kThreads = kWarps * 32;
+constexpr int kScanFmaRows = 2;  // query rows up to which centroid units scan on CUDA cores
 
 template <int D>
 struct Geo {
@@ -95,6 +96,80 @@ __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
     return y;
 }
 
+// s += lo^2 + hi^2 of a packed bf16 pair.
+__device__ __forceinline__ float sq2(uint32_t x, float s) {
+    const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xffff0000u);
+    return fmaf(hi, hi, fmaf(lo, lo, s));
+}
+
+// Centroid scan on CUDA cores for a few query rows: one centroid row per
+// lane, read as 16-byte chunks of the 128-byte-swizzled tile (four
+// wavefronts per warp-wide read, the minimum for 512 bytes), the query rows
+// in fp32 shared memory (broadcast reads).  |c|^2 and <q_b, c> in fp32; the
+// warp's best (score, index) per query row goes to wbw[b].
+template <int D>
+__device__ __forceinline__ void scan_fma(const unsigned char *tile, const float *sq, int nq, int metric,
+                                         int first, int valid, int warp, int lane, float2 *wbw) {
+    using Gm = Geo<D>;
+    constexpr int RPL = Gm::CS / (kWarps * 32);  // rows per lane
+    constexpr int CH = D / 8;                     // 16-byte chunks per row
+    float bs[kScanFmaRows];
+    int bi[kScanFmaRows];
+#pragma unroll
+    for (int b = 0; b < kScanFmaRows; ++b) {
+        bs[b] = kNegInf;
+        bi[b] = 0x7fffffff;
+    }
+#pragma unroll
+    for (int rr = 0; rr < RPL; ++rr) {
+        const int r = (warp * RPL + rr) * 32 + lane;
+        float nrm = 0.f, dot[kScanFmaRows];
+#pragma unroll
+        for (int b = 0; b < kScanFmaRows; ++b) dot[b] = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < CH; ++c) {
+            const int half = c >> 3, cc = c & 7;
+            const uint4 v = *reinterpret_cast<const uint4 *>(tile + half * (Gm::CS * 128) + r * 128 +
+                                                             ((cc ^ (r & 7)) << 4));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            float x[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                x[2 * k] = __uint_as_float(w[k] << 16);
+                x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) nrm = fmaf(x[k], x[k], nrm);
+#pragma unroll
+            for (int b = 0; b < kScanFmaRows; ++b) {
+                if (b < nq) {
+                    const float4 q0 = *reinterpret_cast<const float4 *>(sq + b * D + c * 8);
+                    const float4 q1 = *reinterpret_cast<const float4 *>(sq + b * D + c * 8 + 4);
+                    float t = dot[b];
+                    t = fmaf(x[0], q0.x, t); t = fmaf(x[1], q0.y, t); t = fmaf(x[2], q0.z, t);
+                    t = fmaf(x[3], q0.w, t); t = fmaf(x[4], q1.x, t); t = fmaf(x[5], q1.y, t);
+                    t = fmaf(x[6], q1.z, t); t = fmaf(x[7], q1.w, t);
+                    dot[b] = t;
+                }
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < kScanFmaRows; ++b) {
+            if (b >= nq) break;
+            float sc = (metric == 0) ? dot[b] - 0.5f * nrm : (nrm > 0.f ? dot[b] / sqrtf(nrm) : 0.f);
+            int ci = first + r;
+            if (r >= valid) { sc = kNegInf; ci = 0x7fffffff; }
+            if (better(sc, ci, bs[b], bi[b])) { bs[b] = sc; bi[b] = ci; }
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < kScanFmaRows; ++b) {
+        if (b >= nq) break;
+        warp_argmax(bs[b], bi[b]);
+        if (lane == 0) wbw[b] = make_float2(bs[b], __int_as_float(bi[b]));
+    }
+}
+
 // ------------------------------------------------------------ unit kernel --
 
 template <int D, int G>
@@ -109,6 +184,8 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     float *wm = wo + kWarps * G * D;                      // [W][G]
     float *wl = wm + kWarps * G;                          // [W][G]
     float2 *wb = reinterpret_cast<float2 *>(wl + kWarps * G);  // [W][B]
+    float *sq = reinterpret_cast<float *>(                   // [kScanFmaRows][D], 16-byte aligned
+        (reinterpret_cast<uintptr_t>(wb + kWarps * a.B) + 15) & ~(uintptr_t)15);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, quad = lane & 3, i4 = lane >> 3;
@@ -229,11 +306,22 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     }
     if (!early && tid == 0) issue(valid);
 
-    if (scan) {
-        // ------------------------------------------- centroid unit
+    if (scan && nq <= kScanFmaRows) {
+        // ------------------------------- centroid unit, few query rows: CUDA cores
+        for (int i = tid; i < nq * (D / 4); i += kThreads) {
+            const int bq = i / (D / 4), c4 = i - bq * (D / 4);
+            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(a.qs + ((size_t)(qrow0 + bq) * a.Hq + h) * D) + c4);
+            *reinterpret_cast<float4 *>(sq + bq * D + 4 * c4) =
+                make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                            __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+        }
+        __syncthreads();
+        if (!mbar_wait(bar, 0)) set_error(a.ws_err);
+        scan_fma<D>(tile, sq, nq, a.metric, first, valid, warp, lane, wb + warp * a.B);
+    } else if (scan) {
+        // ------------------------------- centroid unit, more query rows: tensor cores
         constexpr int KS = Gm::KS, RMT = Gm::RMT;
         float nrl[RMT], nrh[RMT];
-        const int src = 4 * gid + (gid >> 1);  // lane holding the diagonal entry of row gid
 #pragma unroll 1
         for (int nt = 0; nt * 8 < nq; ++nt) {
             const int bq = 8 * nt + gid;
@@ -252,24 +340,32 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
             for (int mt = 0; mt < RMT; ++mt) {
                 const int r0 = (warp * RMT + mt) * 16;
                 const int row = r0 + 8 * (i4 & 1) + (lane & 7);
-                float dd[4] = {0.f, 0.f, 0.f, 0.f};
-                float dn0[4] = {0.f, 0.f, 0.f, 0.f}, dn1[4] = {0.f, 0.f, 0.f, 0.f};
+                float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+                float sl = 0.f, sh = 0.f;
 #pragma unroll
                 for (int j = 0; j < KS; ++j) {
                     const int col = 16 * j + 8 * (i4 >> 1);
                     uint32_t a0, a1, a2, a3;
                     ldsm_x4(sbuf + (col >> 6) * (Gm::CS * 128) + swz128(row, (col & 63) >> 3), a0, a1, a2, a3);
-                    mma_bf16_16816(dd, a0, a1, a2, a3, qb0[j], qb1[j]);
+                    if (j & 1) mma_bf16_16816(d1, a0, a1, a2, a3, qb0[j], qb1[j]);
+                    else       mma_bf16_16816(d0, a0, a1, a2, a3, qb0[j], qb1[j]);
                     if (nt == 0) {
-                        // the same fragments as B operands give C C^T (rows 0-7 / 8-15)
-                        mma_bf16_16816(dn0, a0, a1, a2, a3, a0, a2);
-                        mma_bf16_16816(dn1, a0, a1, a2, a3, a1, a3);
+                        // |c|^2 of rows gid (a0, a2) and gid + 8 (a1, a3), this lane's columns
+                        sl = sq2(a2, sq2(a0, sl));
+                        sh = sq2(a3, sq2(a1, sh));
                     }
                 }
                 if (nt == 0) {
-                    nrl[mt] = __shfl_sync(0xffffffffu, dn0[gid & 1], src);
-                    nrh[mt] = __shfl_sync(0xffffffffu, dn1[2 + (gid & 1)], src);
+                    sl += __shfl_xor_sync(0xffffffffu, sl, 1);
+                    sh += __shfl_xor_sync(0xffffffffu, sh, 1);
+                    sl += __shfl_xor_sync(0xffffffffu, sl, 2);
+                    sh += __shfl_xor_sync(0xffffffffu, sh, 2);
+                    nrl[mt] = sl;
+                    nrh[mt] = sh;
                 }
+                float dd[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) dd[k] = d0[k] + d1[k];
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {
                     const int rloc = r0 + gid + 8 * hr;
@@ -296,6 +392,8 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
                 if (gid == 0 && bb < nq) wb[warp * a.B + bb] = make_float2(bs[e], __int_as_float(bi[e]));
             }
         }
+    }
+    if (scan) {
         __syncthreads();
 #pragma unroll 1
         for (int bb = tid; bb < nq; bb += kThreads) {
@@ -683,7 +781,7 @@ cudaError_t tc_launch(tc::Args a, const void *centroids, const void *k_prefix, c
         return cudaErrorInvalidValue;
     const int units = a.n_scan + a.B * a.Hkv * ((a.ext_prefix ? 0 : a.nP) + a.nA);
     const size_t smem = 1024 + tc::kUnit + 16 + sizeof(float) * tc::kWarps * G * (D + 2) +
-                        sizeof(float2) * tc::kWarps * a.B;
+                        sizeof(float2) * tc::kWarps * a.B + 16 + sizeof(float) * tc::kScanFmaRows * D;
     auto k1 = tc::asm_decode_units<D, G>;
     static size_t k1_smem = 0;
     if (smem > k1_smem) {

@@ -19,7 +19,15 @@ cudaError_t asm_decode_launch(int mode, const void *q, const void *centroids, co
                               float *lse_out, int32_t *idx_out, unsigned flags, void *ws,
                               int num_sms, cudaStream_t st, const void *q_search = nullptr);
 
-size_t asm_decode_ws_header_bytes(int B, int Hkv);
+// Bytes at the start of a decode workspace that must be zero before a call:
+// the error word, and for fp32 the (b, g) arrival counters.
+size_t asm_decode_ws_header_bytes(int B, int Hkv, asm_dtype dt);
+
+// api.cu: every argument check of asm_decode_step except the workspace's
+asm_status asm_decode_check_args(const void *q, const void *centroids, const void *a_bar, const float *logz_bar,
+                                 const void *k_cache, const void *v_cache, const int32_t *local_len, int B, int Hq,
+                                 int Hkv, int K, int Tmax, int d, float scale, int metric, asm_dtype dt,
+                                 const void *out, const float *lse_out, const int32_t *idx_out, unsigned flags);
 
 // decode_tc.cu: the bf16 path (split units on tensor cores, then a merge kernel)
 size_t asm_decode_tc_ws_bytes(int mode, int B, int Hq, int K, int Lp, int Tmax, int d);

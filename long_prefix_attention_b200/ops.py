@@ -143,6 +143,11 @@ def asm_decode_workspace_size(B, Hq, Hkv, K, Tmax, d, dtype) -> int:
     return int(_lib.load().asm_decode_workspace_size(B, Hq, Hkv, K, Tmax, d, _DT[dtype]))
 
 
+def asm_decode_step_launches(B, Hq, Hkv, K, Tmax, d, dtype) -> int:
+    """Kernel launches of one asm_decode_step with these sizes on the current device."""
+    return int(_lib.load().asm_decode_step_launches(B, Hq, Hkv, K, Tmax, d, _DT[dtype]))
+
+
 def asm_flash_decode_workspace_size(B, Hq, Hkv, Lp, Tmax, d, dtype) -> int:
     return int(_lib.load().asm_flash_decode_workspace_size(B, Hq, Hkv, Lp, Tmax, d, _DT[dtype]))
 
@@ -238,6 +243,13 @@ def asm_decode_step_noalloc(q, centroids, a_bar, logz_bar, k_cache, v_cache, loc
         _p(q), _p(centroids), _p(a_bar), _p(logz_bar), _p(k_cache), _p(v_cache), _p(local_len),
         B, Hq, Hkv, K, Tmax, d, float(scale), int(metric), _dt(q), _p(out), _p(lse_out),
         _p(idx_out), int(flags), _stream(stream)))
+
+
+def asm_decode_noalloc_error(stream=None) -> int:
+    """Device-side status of the last asm_decode_step_noalloc call on the current device."""
+    code = ctypes.c_int(0)
+    _check("asm_decode_noalloc_error", _lib.load().asm_decode_noalloc_error(ctypes.byref(code), _stream(stream)))
+    return code.value
 
 
 def asm_flash_decode(q, k_prefix, v_prefix, k_cache, v_cache, local_len, scale: float, out, ws,

@@ -141,6 +141,95 @@ def test_decode_counters_reset_across_calls():
     assert torch.equal(out1, out5)
 
 
+# ------------------------------------------- LLaMA-like KV-head counts --
+#
+# 8 or more KV heads (the LLaMA-3.1-8B layer has 8): every group size and
+# head dim, ragged and empty local windows, partial centroid tiles, the
+# largest batch, long windows and the longest batch-1 window of the sweep.
+
+def fused_case(B, G, d, K, T, local_len=None, Hkv=8, seed=11):
+    return small_case("bf16", B=B, Hq=G * Hkv, Hkv=Hkv, K=K, T=T, d=d, local_len=local_len, seed=seed)
+
+
+def assert_two_launches(ins):
+    B, Hq, d = ins["q"].shape
+    K = ins["centroids"].shape[1]
+    _, Hkv, T, _ = ins["k_cache"].shape
+    assert ops.asm_decode_step_launches(B, Hq, Hkv, K, T, d, torch.bfloat16) == 2
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_decode_llama_heads_shapes(d, G):
+    ins = fused_case(5, G, d, K=300, T=200, local_len=[200, 0, 1, 129, 64], seed=G * d + 1)
+    assert_two_launches(ins)
+    check_decode(ins, calls=2)
+
+
+@pytest.mark.parametrize("B,K,T,lens", [
+    (1, 1, 0, None),                  # no local cache, one centre
+    (1, 129, 1, None),                # one token; a partial second centroid tile
+    (64, 1000, 70, "ragged"),         # a large batch with ragged rows, some empty
+    (33, 4097, 65, None),             # an odd batch; a one-row last centroid unit
+    (2, 5000, 3000, [3000, 1500]),    # long windows: many partials per row
+])
+def test_decode_llama_heads_edges(B, K, T, lens):
+    if lens == "ragged":
+        lens = [(7 * b) % (T + 1) for b in range(B)]
+    ins = fused_case(B, 4, 128, K=K, T=T, local_len=lens, seed=B + K)
+    assert_two_launches(ins)
+    check_decode(ins)
+
+
+@pytest.mark.parametrize("Hkv,G", [(16, 2), (32, 1)])
+def test_decode_llama_heads_more_kv_heads(Hkv, G):
+    ins = fused_case(3, G, 128, K=700, T=150, local_len=[150, 77, 0], Hkv=Hkv, seed=Hkv)
+    assert_two_launches(ins)
+    check_decode(ins)
+
+
+def test_decode_llama_heads_long_window_b1():
+    """The longest batch-1 window of the throughput sweep: K = 8192, T = 32768."""
+    ins = inputs.decode_inputs(inputs.CONFIGS[1], seed=inputs.BASE_SEED + 77, B=1, K=8192, T=32768)
+    assert_two_launches(ins)
+    check_decode(ins)
+
+
+def test_decode_llama_heads_cosine_prefetch_and_repeat():
+    ins = fused_case(3, 4, 128, K=900, T=333, local_len=[333, 5, 200], seed=5)
+    check_decode(ins, metric=ops.ASM_COSINE, flags=ops.ASM_DECODE_PREFETCH_CENTROIDS)
+    # nothing carries over between calls: one call and five calls agree bit for bit
+    out1, lse1, idx1 = run_decode(ins, calls=1)
+    out5, lse5, idx5 = run_decode(ins, calls=5, flags=ops.ASM_DECODE_PREFETCH_CENTROIDS)
+    assert torch.equal(out1, out5) and torch.equal(lse1, lse5) and torch.equal(idx1, idx5)
+
+
+def test_decode_llama_heads_search_query():
+    """asm_decode_step_search: the search uses its own query, the local
+    attention and the merge use q."""
+    ins = fused_case(2, 4, 128, K=500, T=100, seed=9)
+    qs_ins = fused_case(2, 4, 128, K=500, T=100, seed=10)
+    q, qs = dev(ins["q"]), dev(qs_ins["q"])
+    C, Ab, lz = dev(ins["centroids"]), dev(ins["a_bar"]), dev(ins["logz_bar"])
+    kc, vc, ll = dev(ins["k_cache"]), dev(ins["v_cache"]), dev(ins["local_len"])
+    B, Hq, d = q.shape
+    ws = ops.alloc_workspace(ops.asm_decode_workspace_size(B, Hq, 8, 500, 100, d, q.dtype), "cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device="cuda")
+    idx = torch.empty(B, Hq, dtype=torch.int32, device="cuda")
+    ops.asm_decode_step_search(q, qs, C, Ab, lz, kc, vc, ll, ins["scale"], out, ws, lse_out=lse, idx_out=idx)
+    torch.cuda.synchronize()
+    assert ops.asm_workspace_error(ws) == 0
+    _, _, s_idx, s_gap = O.decode(qs_ins["q"], ins["centroids"], ins["a_bar"], ins["logz_bar"],
+                                  ins["k_cache"], ins["v_cache"], ins["local_len"], ins["scale"])
+    g_idx = host(idx).numpy()
+    check_indices(g_idx, s_idx, s_gap)
+    o_out, o_lse, _, _ = O.decode(ins["q"], ins["centroids"], ins["a_bar"], ins["logz_bar"], ins["k_cache"],
+                                  ins["v_cache"], ins["local_len"], ins["scale"], idx_in=g_idx)
+    assert max_abs(f64(out), o_out) <= TOL[torch.bfloat16]
+    assert max_abs(f64(lse), o_lse) <= TOL[torch.bfloat16]
+
+
 # ------------------------------------------------------------ flash decode --
 
 def run_flash(q, kp, vp, kc, vc, ll, scale):
