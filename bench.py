@@ -125,8 +125,29 @@ class ClockSampler:
 
 # ------------------------------------------------------------- distributed --
 
+def torchrun_argv(n_gpus, argv, port):
+    """The command that runs this script as `n_gpus` ranks on this node (one
+    per GPU), bounded by `timeout` well above the process group's own."""
+    return ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n_gpus}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+            os.path.abspath(__file__)] + list(argv)
+
+
+def launcher_world():
+    """WORLD_SIZE set by a launcher (torchrun), or 0 when started directly."""
+    return int(os.environ.get("WORLD_SIZE", "0"))
+
+
+def check_world(n_gpus, world):
+    """--gpus N must be the launcher's world size: a mismatch is refused, not
+    silently measured on another number of GPUs."""
+    if world != n_gpus:
+        raise SystemExit(f"bench.py: --gpus {n_gpus} but the launcher started {world} rank(s)")
+
+
 def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    world = launcher_world() or 1
+    check_world(n_gpus, world)
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
@@ -222,6 +243,9 @@ class DecodeStack:
 
 
 def time_steps(fn, steps, warmup, world):
+    """Seconds for exactly `steps` calls of fn after `warmup` untimed ones,
+    CUDA events on the current stream, a barrier and a synchronize on both
+    sides (this rank's time; the job's is the max over ranks)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -747,6 +771,131 @@ def x_bytes(H, N, d):
     return H * N * d * 2
 
 
+# ----------------------------------------------------------------- traffic --
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per layer step,
+# summed over the step's two kernels (mean of 8 layer steps of one ncu
+# capture of this benchmark), with the digest of the kernel source they were
+# taken on: a changed kernel reports null until it is measured again.
+TRAFFIC = {
+    "llama31-8b-layer-decode-K1024-T2048-B1": {  # units 16 936 992 + merge 585 120
+        "bytes": 17522112, "source": "14a39ab15a4f2c84"},
+    "llama31-8b-layer-decode-K8192-T4096-B16": {  # units 356 002 880 + merge 17 530 816
+        "bytes": 373533696, "source": "14a39ab15a4f2c84"},
+}
+TRAFFIC_SOURCE = os.path.join(ROOT, "long_prefix_attention_b200", "csrc", "decode_tc.cu")
+
+
+def source_digest(path):
+    import hashlib
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(key):
+    rec = TRAFFIC.get(key)
+    if rec is None or rec["source"] != source_digest(TRAFFIC_SOURCE):
+        return None
+    return rec["bytes"]
+
+
+# ------------------------------------------------------------- JSON line --
+
+def decode_line(value, ms_per_step, world, steps, warmup, config, roofline, e2e, launches, clocks,
+                cpu=None, build=None, extra=None):
+    """The benchmark's JSON line (rank 0 prints it)."""
+    line = {
+        "metric": METRIC, "value": value, "unit": "query-heads/s", "n_gpus": world,
+        "steps": steps, "warmup": warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config,
+        "hbm_gbs": roofline["achieved"], "hbm_frac_of_8tbs": roofline["achieved"] / NOMINAL_HBM_GBS,
+        "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+        "cpu_baseline": cpu, "build": build,
+    }
+    if extra:
+        line.update(extra)
+    return line
+
+
+def decode_roofline(bytes_per_launch, us_per_launch, peak, peak_src, traffic, kernel):
+    achieved = bytes_per_launch / (us_per_launch * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": traffic, "kernel": kernel, "bytes_per_launch": bytes_per_launch,
+            "us_per_launch": us_per_launch, "peak_source": f"{peak_src} HBM copy"}
+
+
+def run_decode_large(cfg, layers, steps, warmup, world, rank, hbm, src):
+    """The largest single-GPU decode configuration (K = 8192, T = 4096, B = 16,
+    where the search is a [16 x 128] x [128 x 8192] product per head): the
+    same 32-layer graph as the headline, inputs generated on the device."""
+    from long_prefix_attention_b200 import ops
+    B, K, T = cfg["B"], cfg["K"], cfg["T"]
+    Hq, Hkv, d = cfg["Hq"], cfg["Hkv"], cfg["d"]
+    bufs = []
+    for l in range(layers):
+        L = inputs.decode_layer_device(cfg, replica_seed_base(rank) + 500 + l, B, K, T)
+        L["out"] = torch.empty_like(L["q"])
+        L["ws"] = ops.alloc_workspace(ops.asm_decode_workspace_size(B, Hq, Hkv, K, T, d, L["q"].dtype), "cuda")
+        bufs.append(L)
+
+    def run_all():
+        for L in bufs:
+            ops.asm_decode_step(L["q"], L["centroids"], L["a_bar"], L["logz_bar"], L["k_cache"], L["v_cache"],
+                                L["local_len"], L["scale"], L["out"], L["ws"], flags=1)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        run_all()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_all()
+    secs = max_over_ranks(time_steps(g.replay, steps, max(3, warmup), world), world)
+    del g
+    per = secs / (steps * layers)
+    byt = decode_bytes(B, Hq, Hkv, K, T, d)
+    err = max(ops.asm_workspace_error(L["ws"]) for L in bufs)
+    launches = ops.asm_decode_step_launches(B, Hq, Hkv, K, T, d, torch.bfloat16)
+    out = {"workload": cfg["name"] + f" x {layers} layers", "K": K, "local_len": T, "batch": B,
+           "value": B * Hq * layers * steps * world / secs, "unit": "query-heads/s",
+           "ms_per_step": secs * 1e3 / steps, "gpu_launches": steps * layers * launches,
+           "device_error_word": err,
+           "roofline": decode_roofline(byt, per * 1e6, hbm, src, recorded_traffic(cfg["name"]),
+                                       "asm_decode_step = asm_decode_units<128,4> + asm_decode_merge<128>")}
+    del bufs
+    torch.cuda.empty_cache()
+    return out
+
+
+def build_rooflines(build, tf, hbm, src):
+    """Each build stage against the roofline that bounds it: the states and
+    the assignment on the bf16 tensor peak (flops of the definition), the
+    aggregation on the HBM copy rate (one read of the member states, logZ and
+    the member lists, one write of the cluster states); the seeding is K
+    dependent rounds and is reported as time per round."""
+    cfg = inputs.CONFIGS[3]
+    H, N, d, K, L, iters = cfg["Hq"], cfg["N"], cfg["d"], cfg["K"], cfg["L"], cfg["iters"]
+    ms = build["ms"]
+    states = 4.0 * N * L * d * H / (ms["states_4chunks"] / 1e3) / 1e12
+    lloyd = 2.0 * N * K * d * H * iters / (ms["lloyd_10"] / 1e3) / 1e12
+    agg_bytes = H * N * (d * 2 + 4 + 4) + H * K * (d * 2 + 4)
+    agg = agg_bytes / (ms["aggregate"] / 1e3) / 1e9
+    return {
+        "states": {"bound": "tensor", "achieved": states, "peak": tf, "unit": "TFLOP/s", "frac": states / tf,
+                   "peak_source": f"{src} bf16", "flops": 4.0 * N * L * d * H},
+        "lloyd": {"bound": "tensor", "achieved": lloyd, "peak": tf, "unit": "TFLOP/s", "frac": lloyd / tf,
+                  "peak_source": f"{src} bf16", "flops": 2.0 * N * K * d * H * iters,
+                  "note": "assignment flops over the 10 rounds, update included in the time"},
+        "aggregate": {"bound": "hbm", "achieved": agg, "peak": hbm, "unit": "GB/s", "frac": agg / hbm,
+                      "peak_source": f"{src} HBM copy", "bytes": agg_bytes},
+        "kmeanspp_seed": {"bound": "sequential rounds", "rounds": K,
+                          "us_per_round": ms["kmeanspp_seed"] * 1e3 / K},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -756,6 +905,7 @@ def main():
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--no-build", action="store_true", help="skip the offline-build measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--no-large", action="store_true", help="skip the K=8192/T=4096/B=16 decode entry")
     ap.add_argument("--no-prefetch", action="store_true",
                     help="do not let a layer's kernel stream its (static) centroids before the "
                          "preceding kernel finishes")
@@ -767,6 +917,8 @@ def main():
                     help="whitening at the build shape and the decode step with the whitened search, and exit")
     ap.add_argument("--sweep", action="store_true",
                     help="decode over the 36-point B x K x T grid (and full attention at B=1) and exit")
+    ap.add_argument("--decode-large", action="store_true",
+                    help="only the K=8192/T=4096/B=16 decode entry (one GPU), printed as its own line")
     args = ap.parse_args()
     if args.only:
         run_stage(args.only, args.steps, args.warmup)
@@ -780,17 +932,28 @@ def main():
     if args.whiten:
         run_whiten(args.steps, args.warmup)
         return
+    if args.decode_large:
+        torch.cuda.set_device(0)
+        hbm, _, _, src = peaks()
+        print(json.dumps(run_decode_large(inputs.CONFIGS[2], args.layers, args.steps, max(3, args.warmup), 1, 0,
+                                          hbm, src)))
+        return
+    if args.gpus > 1 and launcher_world() == 0:
+        # started directly: run as N ranks, one per GPU, and hand back their status
+        with __import__("socket").socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        sys.exit(subprocess.call(torchrun_argv(args.gpus, sys.argv[1:], port)))
     cfg = inputs.CONFIGS[1]
-    world, rank, local = dist_setup(args.gpus)
-    hbm, tf, tfs, peak_src = peaks()
-    config = {"workload": cfg["name"] + f" x {args.layers} layers", "layers": args.layers,
-              "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "d": cfg["d"], "K": cfg["K"], "local_len": cfg["T"],
-              "batch": cfg["B"], "l2": f"inputs larger than L2: {args.layers} distinct layer buffers",
-              "parallelism": f"replicas x{world}"}
-
     if args.impl == "reference":
-        if rank != 0:
+        # the fp64 oracle on the host cores: rank 0 alone (the others exit without work)
+        world = launcher_world() or 1
+        check_world(args.gpus, world)
+        if int(os.environ.get("RANK", "0")) != 0:
             return
+        config = {"workload": cfg["name"] + f" x {args.layers} layers", "layers": args.layers,
+                  "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "d": cfg["d"], "K": cfg["K"], "local_len": cfg["T"],
+                  "batch": cfg["B"], "parallelism": f"replicas x{world}"}
         cb = cpu_decode_baseline(cfg, budget_s=max(3.0, min(20.0, 0.05 * args.steps)))
         line = {"metric": METRIC, "value": cb["value"], "unit": "query-heads/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "impl": "reference",
@@ -802,12 +965,19 @@ def main():
         print(json.dumps(line))
         return
 
+    world, rank, local = dist_setup(args.gpus)
+    hbm, tf, tfs, peak_src = peaks()
+    config = {"workload": cfg["name"] + f" x {args.layers} layers", "layers": args.layers,
+              "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "d": cfg["d"], "K": cfg["K"], "local_len": cfg["T"],
+              "batch": cfg["B"], "l2": f"inputs larger than L2: {args.layers} distinct layer buffers",
+              "parallelism": f"replicas x{world}"}
     flags = 0 if args.no_prefetch else 1  # ASM_DECODE_PREFETCH_CENTROIDS
     config["prefetch_centroids"] = bool(flags)
     stack = DecodeStack(cfg, args.layers, seed_base=replica_seed_base(rank), flags=flags)
     stack.capture()
+    warmup = max(3, args.warmup)
     with ClockSampler(local) as clk:
-        secs_rank = time_steps(stack.step, args.steps, max(3, args.warmup), world)
+        secs_rank = time_steps(stack.step, args.steps, warmup, world)
     value = job_throughput(stack.B * stack.Hq * args.layers * args.steps, secs_rank, world)
     secs = max_over_ranks(secs_rank, world)
     per_step_launches = stack.ops.asm_decode_step_launches(stack.B, stack.Hq, stack.Hkv, stack.K, stack.T,
@@ -815,23 +985,45 @@ def main():
     launches = args.steps * args.layers * per_step_launches
     ms_per_step = secs * 1e3 / args.steps
     per_launch_s = secs / (args.steps * args.layers)  # one decode step (both kernels) of one layer
-    bpl = stack.bytes_per_launch()
-    achieved = bpl / per_launch_s / 1e9
+    roofline = decode_roofline(stack.bytes_per_launch(), per_launch_s * 1e6, hbm, peak_src,
+                               recorded_traffic(cfg["name"]),
+                               "asm_decode_step = asm_decode_units<128,4> + asm_decode_merge<128>")
 
-    # end to end: per-step queries H2D from pinned memory, outputs D2H
+    # end to end through the public API: every step copies that step's queries
+    # from pinned host memory and reads its outputs back.  "graph": the layer
+    # steps replayed from the captured CUDA graph; "eager": asm_decode_step
+    # called layer by layer (host-side validation and launch every call).
     qh_host = stack.q_all.cpu().pin_memory()
     out_host = torch.empty_like(qh_host).pin_memory()
 
-    def e2e_step():
-        # one host-to-device copy of every layer's queries, the graph, one copy back
+    def e2e_graph():
         stack.q_all.copy_(qh_host, non_blocking=True)
         stack.graph.replay()
         out_host.copy_(stack.out_all, non_blocking=True)
 
-    e2e_secs = max_over_ranks(time_steps(e2e_step, max(10, args.steps // 4), 3, world), world)
+    def e2e_eager():
+        stack.q_all.copy_(qh_host, non_blocking=True)
+        stack.launch_all()
+        out_host.copy_(stack.out_all, non_blocking=True)
+
     e2e_steps = max(10, args.steps // 4)
+    e2e_secs = max_over_ranks(time_steps(e2e_graph, e2e_steps, 3, world), world)
+    eager_secs = max_over_ranks(time_steps(e2e_eager, e2e_steps, 3, world), world)
     h2d = qh_host[0].numel() * qh_host.element_size() * args.layers
     d2h = h2d
+    units = stack.B * stack.Hq * args.layers * e2e_steps * world
+    e2e = {"value": units / e2e_secs, "unit": "query-heads/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "path": "CUDA graph of the layer steps between the two copies",
+           "eager_value": units / eager_secs,
+           "eager_path": "asm_decode_step called per layer (validation and launches every call)"}
+
+    large = None
+    if not args.no_large:
+        try:
+            large = run_decode_large(inputs.CONFIGS[2], args.layers, max(5, args.steps // 10), warmup, world,
+                                     rank, hbm, peak_src)
+        except Exception as e:  # report, do not hide
+            large = {"error": repr(e)}
 
     build = None
     if not args.no_build:
@@ -840,6 +1032,8 @@ def main():
         try:
             build = run_build(inputs.CONFIGS[3], with_cpu=not args.no_cpu and world == 1, world=world,
                               rank=rank)
+            if build is not None:
+                build["roofline"] = build_rooflines(build, tf, hbm, peak_src)
         except Exception as e:  # report, do not hide
             build = {"error": repr(e)}
     cpu = None
@@ -847,24 +1041,8 @@ def main():
         cpu = cpu_decode_baseline(cfg)
 
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "query-heads/s", "n_gpus": world,
-            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": config,
-            "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": None,
-                         "kernel": "asm_decode_step = asm_decode_units<128,4> + asm_decode_merge<128>",
-                         "bytes_per_launch": bpl, "us_per_launch": per_launch_s * 1e6,
-                         "peak_source": f"{peak_src} HBM copy"},
-            "e2e": {"value": stack.B * stack.Hq * args.layers * e2e_steps * world / e2e_secs,
-                    "unit": "query-heads/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches,
-            "clocks": clk.summary(),
-            "cpu_baseline": cpu,
-            "build": build,
-        }
+        line = decode_line(value, ms_per_step, world, args.steps, warmup, config, roofline, e2e, launches,
+                           clk.summary(), cpu=cpu, build=build, extra={"decode_large": large})
         print(json.dumps(line))
     if world > 1:
         stack.graph = None

@@ -37,7 +37,11 @@ def _worker(rank, world, port, out):
         seeds = [None] * world
         dist.all_gather_object(seeds, seed)
         bench.barrier(world)
-        out[rank] = (mx, thr, seeds)
+        # the line rank 0 prints: whole-job throughput, the slowest rank's time, N ranks
+        roof = bench.decode_roofline(16_801_920, 11.0, 6543.4, "measured", None, "k")
+        line = bench.decode_line(thr, mx * 1e3 / 10, world, 10, 3, {"workload": "w"}, roof,
+                                 {"value": thr}, 10 * 32 * 2, {"sm_mhz": None})
+        out[rank] = (mx, thr, seeds, line["n_gpus"], line["value"])
     finally:
         dist.destroy_process_group()
 
@@ -49,10 +53,30 @@ def test_two_gloo_ranks_max_time_and_job_throughput():
         mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
         res = dict(out)
     for r in range(world):
-        mx, thr, seeds = res[r]
+        mx, thr, seeds, n_gpus, value = res[r]
         assert mx == pytest.approx(1.5)                  # max over ranks
         assert thr == pytest.approx(1000 * world / 1.5)  # all ranks' units over the slowest time
         assert len(set(seeds)) == world                  # independent replicas
+        assert n_gpus == world and value == pytest.approx(thr)
+
+
+def test_gpus_flag_is_honoured():
+    """`--gpus N` runs N ranks: started directly it re-launches itself under
+    torchrun with N processes on 127.0.0.1; under a launcher the launcher's
+    world size must be N, else the run is refused rather than measured on
+    another number of GPUs."""
+    sys.path.insert(0, ROOT)
+    import bench
+    cmd = bench.torchrun_argv(4, ["--gpus", "4", "--steps", "20"], 29123)
+    assert "--nproc-per-node=4" in cmd and "torch.distributed.run" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1" and "29123" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "20"] and cmd[-5].endswith("bench.py")
+    assert cmd[:3] == ["timeout", "-k", "60"]
+    bench.check_world(2, 2)
+    with pytest.raises(SystemExit):
+        bench.check_world(2, 1)
+    with pytest.raises(SystemExit):
+        bench.check_world(1, 8)
 
 
 def test_single_rank_is_identity():
