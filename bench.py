@@ -327,12 +327,9 @@ def cpu_build_baseline(cfg, bi):
 
 
 def build_head_shard(Hq, Hkv, world, rank):
-    """Query heads [h0, h1) that rank `rank` of `world` builds: whole KV groups
-    (the GQA heads sharing a KV head stay together), split as evenly as the
-    groups allow; a rank may get none when world > Hkv."""
-    G = Hq // Hkv
-    g0, g1 = rank * Hkv // world, (rank + 1) * Hkv // world
-    return g0 * G, g1 * G
+    """Query heads [h0, h1) that rank `rank` of `world` builds (whole KV groups)."""
+    from long_prefix_attention_b200 import sharding
+    return sharding.head_shard(Hq, Hkv, world, rank)
 
 
 def run_build(cfg, with_cpu=True, world=1, rank=0):

@@ -101,6 +101,23 @@ asm_status asm_build_states(const void *q, const void *k, const void *v,
                             cudaStream_t stream);
 
 /*
+ * asm_merge_states -- merge a second set of attention states into a first,
+ * row by row, by the online-softmax identity ("Eficiencia" bullet: the
+ * states of a long prefix's chunks are combined by the identity; with the
+ * chunks encoded on several GPUs, the gathered chunk states are folded with
+ * this call in chunk order):
+ *   z = ln(e^z_acc + e^z_in),  a_acc = e^(z_acc - z) a_acc + e^(z_in - z) a_in
+ * The empty state (0, -inf) is the identity; a_acc is rounded to dt.
+ *   a_acc  [R, d] dt   in/out     logz_acc [R] fp32 in/out
+ *   a_in   [R, d] dt              logz_in  [R] fp32
+ * R rows (for example heads x queries).  The two sets must not overlap
+ * (ASM_ERR_INVALID_ARG).  No workspace; one kernel launch, HBM-bound.
+ */
+asm_status asm_merge_states(void *a_acc, float *logz_acc, const void *a_in,
+                            const float *logz_in, int64_t R, int d,
+                            asm_dtype dt, cudaStream_t stream);
+
+/*
  * asm_kmeanspp_seed -- k-means++ initial centres of every head's points
  * (the clustering of the "Agrupamiento" bullet; seeding by D^2 sampling,
  * Arthur & Vassilvitskii 2007).  Round 0 takes point floor(u[h,0] * N); round

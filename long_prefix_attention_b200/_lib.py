@@ -19,6 +19,7 @@ SZ = ctypes.c_size_t
 # name -> (restype, argtypes); mirrors include/asm.h
 SIGNATURES = {
     "asm_build_states": (I, [P, P, P, I, I, I, I, I, F, I, I, P, P, P]),
+    "asm_merge_states": (I, [P, P, P, P, ctypes.c_int64, I, I, P]),
     "asm_kmeanspp_workspace_size": (SZ, [I, I, I, I]),
     "asm_kmeanspp_seed": (I, [P, I, I, I, I, P, I, P, P, SZ, P]),
     "asm_kmeans_assign": (I, [P, P, I, I, I, I, I, I, P, P, SZ, P]),

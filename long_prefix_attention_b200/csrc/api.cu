@@ -75,6 +75,22 @@ asm_status asm_build_states(const void *q, const void *k, const void *v, int Hq,
                                                a, logz, num_sms(), stream));
 }
 
+asm_status asm_merge_states(void *a_acc, float *logz_acc, const void *a_in, const float *logz_in, int64_t R,
+                            int d, asm_dtype dt, cudaStream_t stream) {
+    if (!dt_ok(dt) || R < 0) return ASM_ERR_INVALID_ARG;
+    if (!d_ok(d)) return ASM_ERR_UNSUPPORTED;
+    if (R == 0) return ASM_OK;
+    if (!aligned(a_acc, 16) || !aligned(a_in, 16) || !aligned(logz_acc, 4) || !aligned(logz_in, 4))
+        return ASM_ERR_INVALID_ARG;
+    // the two sets must not overlap (the accumulator is written in place)
+    const size_t es = dt == ASM_BF16 ? 2 : 4, ab = (size_t)R * d * es, zb = (size_t)R * sizeof(float);
+    const char *pa = static_cast<const char *>(a_acc), *pb = static_cast<const char *>(a_in);
+    const char *za = reinterpret_cast<const char *>(logz_acc), *zb2 = reinterpret_cast<const char *>(logz_in);
+    if ((pa < pb + ab && pb < pa + ab) || (za < zb2 + zb && zb2 < za + zb)) return ASM_ERR_INVALID_ARG;
+    return cuda_status(asm_merge_states_launch(a_acc, logz_acc, a_in, logz_in, (long long)R, d, dt, num_sms(),
+                                               stream));
+}
+
 size_t asm_kmeanspp_workspace_size(int H, int N, int d, int K) {
     if (H < 1 || N < 1 || K < 1) return 0;
     return asm_kmeanspp_ws_bytes(H, N, d, K);

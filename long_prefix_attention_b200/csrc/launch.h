@@ -86,6 +86,10 @@ cudaError_t asm_kmeans_update_launch(const void *x, const int32_t *assign, int H
 cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, int H, int N, int K,
                                  int metric, int32_t *assign, int *err, cudaStream_t st);
 
+// merge.cu: online-softmax merge of two state arrays, row by row
+cudaError_t asm_merge_states_launch(void *a, float *z, const void *a2, const float *z2, long long R, int d,
+                                    asm_dtype dt, int num_sms, cudaStream_t st);
+
 // aggregate.cu
 cudaError_t asm_aggregate_launch(const void *a, const float *logz, const int32_t *perm,
                                  const int32_t *seg_off, int H, int N, int d, int K, int zmode,

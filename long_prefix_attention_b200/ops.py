@@ -80,6 +80,20 @@ def asm_build_states(q, k, v, scale: float, a, logz, accumulate: bool = False, s
         _p(a), _p(logz), _stream(stream)))
 
 
+def asm_merge_states(a_acc, logz_acc, a_in, logz_in, stream=None):
+    """Fold the states (a_in, logz_in) into (a_acc, logz_acc) by the
+    online-softmax identity, row by row (any leading shape, d innermost)."""
+    _contig(a_acc, logz_acc, a_in, logz_in)
+    if a_acc.shape != a_in.shape or logz_acc.shape != logz_in.shape or a_acc.dtype != a_in.dtype:
+        raise AsmError("asm_merge_states", ASM_ERR_INVALID_ARG)
+    d = a_acc.shape[-1]
+    R = a_acc.numel() // d
+    if logz_acc.numel() != R:
+        raise AsmError("asm_merge_states", ASM_ERR_INVALID_ARG)
+    _check("asm_merge_states", _lib.load().asm_merge_states(
+        _p(a_acc), _p(logz_acc), _p(a_in), _p(logz_in), R, d, _dt(a_acc), _stream(stream)))
+
+
 def asm_kmeanspp_workspace_size(H: int, N: int, d: int, K: int) -> int:
     return int(_lib.load().asm_kmeanspp_workspace_size(H, N, d, K))
 

@@ -103,3 +103,83 @@ def test_build_head_shards_cover_the_heads_in_whole_groups(world):
     groups = [s // (Hq // Hkv) for s in sizes]
     assert max(groups) - min(groups) <= 1
     assert sum(s == 0 for s in sizes) == max(0, world - Hkv)
+
+
+# ------------------------------------------------ build split over ranks --
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 5, 8, 12])
+def test_chunk_and_head_shards_cover_the_work_once(world):
+    """Every prefix chunk is encoded by exactly one rank, in contiguous runs
+    in rank order (so the gathered states arrive in chunk order); every head
+    is built by exactly one rank, in whole KV groups."""
+    sys.path.insert(0, ROOT)
+    from long_prefix_attention_b200 import sharding
+    for n_chunks in (1, 3, 4, 7, 16):
+        runs = [sharding.chunk_shard(n_chunks, world, r) for r in range(world)]
+        covered = [c for c0, c1 in runs for c in range(c0, c1)]
+        assert covered == list(range(n_chunks))
+        assert all(c0 <= c1 for c0, c1 in runs)
+    heads = [h for r in range(world) for h in range(*sharding.head_shard(32, 8, world, r))]
+    assert heads == list(range(32))
+
+
+def _split_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        sys.path.insert(0, ROOT)
+        import numpy as np
+        from long_prefix_attention_b200 import inputs, sharding
+        from oracle import asm_oracle as O
+        cfg = dict(inputs.CONFIGS[0])
+        bi = inputs.build_inputs(cfg, N=96, L=200, K=4)
+        Hq, N, d = bi["q"].shape
+        bounds = [0, 37, 80, 81, 150, 200]  # five uneven chunks, one of a single key
+        kc = [bi["k"][:, b0:b1] for b0, b1 in zip(bounds, bounds[1:])]
+        vc = [bi["v"][:, b0:b1] for b0, b1 in zip(bounds, bounds[1:])]
+
+        def encode(q, k, v, s, a, z, acc):  # the oracle's states as the payload
+            oa, oz = O.build_states(q, k, v, s, A=a.numpy() if acc else None,
+                                    logZ=z.numpy() if acc else None, accumulate=acc)
+            a.copy_(torch.from_numpy(oa))
+            z.copy_(torch.from_numpy(oz))
+
+        seen = []
+
+        def merge(a, z, a_in, z_in):  # the oracle's merge, row by row, recording the order
+            seen.append(float(z_in.sum()))
+            A, Z, Ai, Zi = a.numpy().reshape(-1, d), z.numpy().reshape(-1), a_in.numpy().reshape(-1, d), \
+                z_in.numpy().reshape(-1)
+            for i in range(Z.size):
+                m, zz = O.merge(A[i], Z[i], Ai[i], Zi[i])
+                A[i], Z[i] = m, zz
+
+        a = torch.zeros(Hq, N, d, dtype=torch.float64)
+        z = torch.zeros(Hq, N, dtype=torch.float64)
+        sharding.build_states_split(bi["q"], kc, vc, bi["scale"], a, z, encode=encode, merge=merge)
+        # what each rank gathered: its own states, in rank order
+        own = [None] * world
+        c0, c1 = sharding.chunk_shard(len(kc), world, rank)
+        dist.all_gather_object(own, (c0, c1))
+        ref_a, ref_z = O.build_states(bi["q"], bi["k"], bi["v"], bi["scale"])
+        out[rank] = (float(np.abs(a.numpy() - ref_a).max()), float(np.abs(z.numpy() - ref_z).max()), own, seen)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_prefix_chunks_split_over_gloo_ranks_fold_to_the_single_pass(world):
+    """Each rank encodes its run of the five prefix chunks, the ranks
+    all-gather their states and fold them in chunk order: the result equals
+    the single-pass oracle state over the whole prefix on every rank."""
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_split_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+        res = dict(out)
+    for r in range(world):
+        ea, ez, runs, seen = res[r]
+        assert ea < 1e-12 and ez < 1e-12
+        assert [c for c0, c1 in runs for c in range(c0, c1)] == list(range(5))  # chunk order = rank order
+        assert len(seen) == world - 1                                           # one merge per other rank
