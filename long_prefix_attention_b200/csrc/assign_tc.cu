@@ -5,19 +5,25 @@
 // arg-min over centroids is the arg-max of <x, c> - |c|^2 / 2 (cosine: the
 // arg-max of <x, c> / |c|), so the work is a dense X C^T contraction (bf16
 // in, fp32 accumulate) followed by a row-wise arg-max with a per-column term.
+// For L2 the term rides on the contraction: a ninth K=16 step multiplies a
+// constant tile of ones by three bf16 parts of -|c|^2 / 2 per centre (their
+// sum is the fp32 value to within 2^-24 of it), so the accumulator already
+// holds <x, c> - |c|^2 / 2 and the epilogue is the arg-max alone (with the
+// term applied by the CUDA cores the epilogue, not the MMA, set the pace).
 //
 // One CTA owns 256 points of one head (two M=128 halves that share every
 // centroid tile, which halves the L2 -> shared traffic per flop) and sweeps
 // all K centroids in tiles of 128.  Warp roles:
 //   warp 0     producer: TMA of the 256x128 point tile once, then the 128x128
-//              centroid tiles (128-byte swizzle, 4 stages); its lanes copy the
-//              tile's |c|^2 (or |c|) into a 4-deep shared ring;
+//              centroid tiles (128-byte swizzle, 4 stages) with, for L2, the
+//              128x16 tile of bias parts (32-byte swizzle); for cosine its
+//              lanes copy the tile's |c| into a 4-deep shared ring;
 //   warp 1     allocates 512 TMEM columns and one lane issues tcgen05.mma
-//              (M=128, N=128, K=16 x 8, both halves) into two ping-pong
-//              accumulator pairs, committing to mbarriers;
+//              (M=128, N=128, K=16 x 8 (+1 for L2), both halves) into two
+//              ping-pong accumulator pairs, committing to mbarriers;
 //   warps 2-9  epilogue: warp w reads TMEM lane quarter w%4 of one half,
-//              folds the per-column term and keeps a running arg-max (ties
-//              go to the smaller index) while the next tile is multiplied.
+//              (cosine: divides by |c|) and keeps a running arg-max (ties go
+//              to the smaller index) while the next tile is multiplied.
 // Every wait is bounded; a timeout sets the workspace error word to 5.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -44,10 +50,13 @@ constexpr uint32_t kTmemCols = 512;   // 2 buffers x 2 halves x 128 fp32 columns
 constexpr int kSub = 128 * 128;       // one 128-row x 64-column swizzled box (16 KB)
 constexpr int kABytes = 4 * kSub;     // [half][k-half]
 constexpr int kBBytes = 2 * kSub;     // [k-half]
+constexpr int kEBytes = 128 * 32;     // 128 rows x 16 columns, 32-byte swizzle (the bias step)
 
 struct Smem {
     unsigned char a[kABytes];
     unsigned char b[kStages][kBBytes];
+    unsigned char be[kStages][kEBytes];  // bias parts of the centroid tile (L2)
+    unsigned char ae[kEBytes];           // the ones they multiply (L2)
     float bias[kBias][kN];
     uint64_t a_full, b_full[kStages], b_empty[kStages], acc_full[2], acc_empty[2];
     uint64_t bias_full[kBias], bias_empty[kBias];
@@ -59,6 +68,12 @@ struct Smem {
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// The same for 32-byte rows (K = 16 bf16) with the 32-byte swizzle: 8-row
+// groups 256 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
 }
 
 // D[tmem] (+)= A * B^T, bf16 operands from shared memory, fp32 accumulator
@@ -93,37 +108,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 struct Maps {
-    CUtensorMap x, c;
+    CUtensorMap x, c, e;
 };
 
-// Three-input maximum and paired fp32 fused multiply-add (sm_100).
+// Three-input maximum (sm_100).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float m;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
     return m;
 }
-__device__ __forceinline__ void fma2(float a0, float a1, float b, float c0, float c1, float &d0, float &d1) {
-    uint64_t d;
-    asm("{\n .reg .b64 a, b, c;\n mov.b64 a, {%1, %2};\n mov.b64 b, {%3, %3};\n mov.b64 c, {%4, %5};\n"
-        " fma.rn.f32x2 %0, a, b, c;\n}\n"
-        : "=l"(d) : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
-}
 
 // Fold 32 accumulator columns (global centre indices col0 ..) into the
 // running arg-max; only the first `nv` of them are real centres (FULL: all).
+// L2: the accumulator is the score; cosine: divided by |c| from `bias`.
 template <int METRIC, bool FULL>
 __device__ __forceinline__ void fold32(const uint32_t (&r)[32], const float *bias, int col0, int nv,
                                        float &best, int &bidx) {
     float v[32];
 #pragma unroll
     for (int k = 0; k < 32; k += 4) {
-        const float4 bn = *reinterpret_cast<const float4 *>(bias + k);
         if (METRIC == 0) {
-            // acc - |c|^2 / 2, two columns per instruction (the product is exact)
-            fma2(bn.x, bn.y, -0.5f, __uint_as_float(r[k]), __uint_as_float(r[k + 1]), v[k], v[k + 1]);
-            fma2(bn.z, bn.w, -0.5f, __uint_as_float(r[k + 2]), __uint_as_float(r[k + 3]), v[k + 2], v[k + 3]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[k + u] = __uint_as_float(r[k + u]);
         } else {
+            const float4 bn = *reinterpret_cast<const float4 *>(bias + k);
             const float bb[4] = {bn.x, bn.y, bn.z, bn.w};   // the term holds |c|
 #pragma unroll
             for (int u = 0; u < 4; ++u) v[k + u] = bb[u] > 0.f ? __uint_as_float(r[k + u]) / bb[u] : 0.f;
@@ -177,6 +185,16 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
         }
         fence_mbar_init();
     }
+    if (METRIC == 0) {
+        // the ones of the bias step: columns 0-2 of each 16-byte half of every
+        // 32-byte row (both halves alike, so the swizzle leaves them in place);
+        // the tensor cores read them through the async proxy
+        for (int i = tid; i < kEBytes / 16; i += kThreads) {
+            const uint32_t one = 0x3F80u;  // bf16 1.0
+            reinterpret_cast<uint4 *>(sm.ae)[i] = make_uint4(one | (one << 16), one, 0u, 0u);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_addr(&sm.tmem_base)), "r"(kTmemCols));
@@ -201,10 +219,12 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
             const int s = t % kStages, r = t % kBias;
             if (lane == 0) {
                 if (t >= kStages) ok &= mbar_wait(&sm.b_empty[s], ((t / kStages) - 1) & 1);
-                mbar_arrive_expect_tx(&sm.b_full[s], kBBytes);
+                mbar_arrive_expect_tx(&sm.b_full[s], kBBytes + (METRIC == 0 ? kEBytes : 0));
                 tma_load_3d(sm.b[s], &maps.c, 0, t * kN, h, &sm.b_full[s]);
                 tma_load_3d(sm.b[s] + kSub, &maps.c, 64, t * kN, h, &sm.b_full[s]);
+                if (METRIC == 0) tma_load_3d(sm.be[s], &maps.e, 0, t * kN, h, &sm.b_full[s]);
             }
+            if (METRIC == 0) continue;
             if (t >= kBias) ok &= mbar_wait(&sm.bias_empty[r], ((t / kBias) - 1) & 1);
 #pragma unroll
             for (int u = 0; u < kN / 32; ++u) {
@@ -240,6 +260,9 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
                         const uint64_t bd = sdesc_sw128(b_base + koff);
                         umma_bf16(tmem + (uint32_t)((b * 2 + m) * kN), ad, bd, idesc, j > 0 ? 1u : 0u);
                     }
+                    if (METRIC == 0)  // + 1 x (-|c|^2 / 2), in three bf16 parts
+                        umma_bf16(tmem + (uint32_t)((b * 2 + m) * kN), sdesc_sw32(smem_addr(sm.ae)),
+                                  sdesc_sw32(smem_addr(sm.be[s])), idesc, 1u);
                 }
                 umma_commit(&sm.b_empty[s]);   // the centroid stage is free once these MMAs finish
                 umma_commit(&sm.acc_full[b]);  // and the accumulator pair is ready for the epilogue
@@ -257,7 +280,7 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
         for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1, r = t % kBias;
             ok &= mbar_wait(&sm.acc_full[b], (t >> 1) & 1);
-            ok &= mbar_wait(&sm.bias_full[r], (t / kBias) & 1);
+            if (METRIC == 1) ok &= mbar_wait(&sm.bias_full[r], (t / kBias) & 1);
             tc_fence_after();
             const int nv = min(kN, K - t * kN);
             const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((b * 2 + m) * kN);
@@ -280,7 +303,7 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&sm.acc_empty[b]);
-                mbar_arrive(&sm.bias_empty[r]);
+                if (METRIC == 1) mbar_arrive(&sm.bias_empty[r]);
             }
         }
         if (p0 + row < N) assign[(size_t)h * N + p0 + row] = bidx;
@@ -297,16 +320,20 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
 }  // namespace atc
 
 bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows);
+bool make_map_rows16(CUtensorMap *m, const void *base, uint64_t d1, uint64_t d2, uint32_t rows);
 
 }  // namespace asmk
 
-// bf16, d = 128.  `norms` [H, K] holds |c|^2 of the stored (bf16) centres.
-cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, int H, int N, int K, int metric,
-                                 int32_t *assign, int *err, cudaStream_t st) {
+// bf16, d = 128.  `norms` [H, K] holds |c|^2 of the stored (bf16) centres
+// (the cosine term); `bias` [H, K, 16] bf16 the three parts of -|c|^2 / 2
+// in columns 0-2 and zeros (the L2 term; unused for cosine).
+cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, const void *bias, int H, int N,
+                                 int K, int metric, int32_t *assign, int *err, cudaStream_t st) {
     using namespace asmk;
     atc::Maps maps;
     memset(&maps, 0, sizeof(maps));
-    if (!make_map_3d(&maps.x, x, atc::kD, N, H, atc::kMH) || !make_map_3d(&maps.c, c, atc::kD, K, H, atc::kN))
+    if (!make_map_3d(&maps.x, x, atc::kD, N, H, atc::kMH) || !make_map_3d(&maps.c, c, atc::kD, K, H, atc::kN) ||
+        (metric == 0 && !make_map_rows16(&maps.e, bias, K, H, atc::kN)))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(atc::Smem) + 1024;
     auto kern = metric == 0 ? atc::assign_tc_kernel<0> : atc::assign_tc_kernel<1>;

@@ -686,6 +686,20 @@ bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uin
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map [d2][d1][16]: a box of the 16 columns (one 32-byte row,
+// 32-byte swizzle) x `rows` rows x 1.
+bool make_map_rows16(CUtensorMap *m, const void *base, uint64_t d1, uint64_t d2, uint32_t rows) {
+    auto fn = encode_fn();
+    if (!fn || base == nullptr || d1 == 0 || d2 == 0) return false;
+    cuuint64_t dims[3] = {16, d1, d2};
+    cuuint64_t strides[2] = {32, 32 * d1};
+    cuuint32_t box[3] = {16, rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T, int D, int G>
 static void decode_geometry(DecodeArgs &a, int workers) {
     using C = DCfg<T, D, G>;

@@ -949,9 +949,12 @@ __global__ void kmeans_init(const T *__restrict__ x, int N, int K, const int32_t
     centroids_dt[((size_t)h * K + c) * D + e] = v;
 }
 
-// |c|^2 of every storage-dtype centre (fp32), one warp per centre.
+// |c|^2 of every storage-dtype centre (fp32), one warp per centre; with
+// `bias`, also the row [hi, mid, lo, 0 x 13] (bf16) whose first three parts
+// sum to -|c|^2 / 2: each part rounds what the earlier ones leave (the
+// differences are exact in fp32), so the sum is within 2^-24 of the value.
 template <typename T, int D>
-__global__ void centroid_norms(const T *__restrict__ c, int HK, float *norms) {
+__global__ void centroid_norms(const T *__restrict__ c, int HK, float *norms, __nv_bfloat16 *bias) {
     constexpr int EPL = D / 32;
     const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (w >= HK) return;
@@ -962,6 +965,19 @@ __global__ void centroid_norms(const T *__restrict__ c, int HK, float *norms) {
     for (int e = 0; e < EPL; ++e) s = fmaf(f[e], f[e], s);
     s = warp_sum(s);
     if (lane == 0) norms[w] = s;
+    if (bias != nullptr && lane < 2) {
+        uint4 row = make_uint4(0u, 0u, 0u, 0u);
+        if (lane == 0) {
+            const float b = -0.5f * s;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(b);
+            const float r1 = b - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+            row.x = (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(mid) << 16);
+            row.y = (uint32_t)__bfloat16_as_ushort(lo);
+        }
+        reinterpret_cast<uint4 *>(bias + (size_t)w * 16)[lane] = row;
+    }
 }
 
 // ================================================================ assign ===
@@ -1169,14 +1185,15 @@ __global__ void means_kernel(const T *__restrict__ x, const int32_t *__restrict_
 // (5 = a tensor-core wait timed out), the |c|^2 of every centre, and the
 // scatter cursors.
 struct KmWs {
-    size_t off_norm, off_cursor, total;
+    size_t off_norm, off_cursor, off_bias, total;
 };
 KmWs km_ws(int H, int N, int K) {
     (void)N;
     KmWs w;
     w.off_norm = 256;
     w.off_cursor = al256(w.off_norm + sizeof(float) * (size_t)H * K);
-    w.total = al256(w.off_cursor + sizeof(int) * (size_t)H * K);
+    w.off_bias = al256(w.off_cursor + sizeof(int) * (size_t)H * K);   // [H][K][16] bf16
+    w.total = al256(w.off_bias + 32 * (size_t)H * K);
     return w;
 }
 
@@ -1341,20 +1358,23 @@ cudaError_t asm_kmeans_assign_launch(const void *x, const void *centroids_dt, in
     (void)num_sms;
     KmWs w = km_ws(H, N, K);
     float *norms = reinterpret_cast<float *>(static_cast<char *>(ws) + w.off_norm);
+    const bool tc = dt == ASM_BF16 && d == 128;
+    __nv_bfloat16 *bias = (tc && metric == 0)
+                              ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + w.off_bias) : nullptr;
     const int HK = H * K;
     const int nb = (HK * 32 + 255) / 256;
     if (dt == ASM_BF16) {
         using T = __nv_bfloat16;
-        if (d == 128) centroid_norms<T, 128><<<nb, 256, 0, st>>>((const T *)centroids_dt, HK, norms);
-        else centroid_norms<T, 64><<<nb, 256, 0, st>>>((const T *)centroids_dt, HK, norms);
+        if (d == 128) centroid_norms<T, 128><<<nb, 256, 0, st>>>((const T *)centroids_dt, HK, norms, bias);
+        else centroid_norms<T, 64><<<nb, 256, 0, st>>>((const T *)centroids_dt, HK, norms, nullptr);
     } else {
-        if (d == 128) centroid_norms<float, 128><<<nb, 256, 0, st>>>((const float *)centroids_dt, HK, norms);
-        else centroid_norms<float, 64><<<nb, 256, 0, st>>>((const float *)centroids_dt, HK, norms);
+        if (d == 128) centroid_norms<float, 128><<<nb, 256, 0, st>>>((const float *)centroids_dt, HK, norms, nullptr);
+        else centroid_norms<float, 64><<<nb, 256, 0, st>>>((const float *)centroids_dt, HK, norms, nullptr);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (dt == ASM_BF16 && d == 128)
-        return asm_assign_tc_launch(x, centroids_dt, norms, H, N, K, metric, assign, static_cast<int *>(ws), st);
+    if (tc)
+        return asm_assign_tc_launch(x, centroids_dt, norms, bias, H, N, K, metric, assign, static_cast<int *>(ws), st);
     dim3 grid((N + kAsP - 1) / kAsP, H);
     if (dt == ASM_BF16) {
         using T = __nv_bfloat16;

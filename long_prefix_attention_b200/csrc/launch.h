@@ -83,8 +83,8 @@ cudaError_t asm_kmeans_update_launch(const void *x, const int32_t *assign, int H
                                      cudaStream_t st);
 
 // assign_tc.cu: bf16, d = 128 assignment on tcgen05; `err` is the workspace error word
-cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, int H, int N, int K,
-                                 int metric, int32_t *assign, int *err, cudaStream_t st);
+cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, const void *bias, int H, int N,
+                                 int K, int metric, int32_t *assign, int *err, cudaStream_t st);
 
 // merge.cu: online-softmax merge of two state arrays, row by row
 cudaError_t asm_merge_states_launch(void *a, float *z, const void *a2, const float *z2, long long R, int d,
