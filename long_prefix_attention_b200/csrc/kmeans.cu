@@ -394,13 +394,94 @@ __device__ __forceinline__ void q8_vector(const T *__restrict__ v, int lane, flo
     err = __double2float_ru(sqrt(ee) * (1.0 + kSeedMargin));
 }
 
+// The refresh with every S1 and S2 sum of the head cached in shared memory
+// (s1c [NR1], s2c [NR2]): one round of loads brings the flags and all sums,
+// the flagged S1 sums are recomputed from D2 and the S2 sums above them from
+// the cache.  Out of line: inlined into the round kernel, it changed the code
+// of the update loop before it and slowed that by more than it saves.
+__device__ __noinline__ void seed_refresh_cached(double *b1, double *b2, unsigned char *dh, const double *d2h, int N,
+                                                 int NR1, int NR2, int *dl, uint32_t *sd2, double *s1c, double *s2c,
+                                                 int *nlist) {
+    const int tid = threadIdx.x;
+    // one round of loads: the flags, every S1 sum and every S2 sum
+    uint2 f[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int kb = (i * kSeedThreads + tid) * 8;
+        f[i] = kb < NR1 ? __ldcg(reinterpret_cast<const uint2 *>(dh + kb)) : make_uint2(0u, 0u);
+    }
+    // (every load issued before the first store: the stores go through a
+    // generic pointer that could alias them)
+    constexpr int kS1PerThread = 16;  // NR1 <= 2 * 8 * kSeedThreads
+    double t1[kS1PerThread];
+#pragma unroll
+    for (int i = 0; i < kS1PerThread; ++i) {
+        const int k = i * kSeedThreads + tid;
+        t1[i] = k < NR1 ? __ldcg(b1 + k) : 0.0;
+    }
+    const double t2 = tid < NR2 ? __ldcg(b2 + tid) : 0.0;
+#pragma unroll
+    for (int i = 0; i < kS1PerThread; ++i) {
+        const int k = i * kSeedThreads + tid;
+        if (k < NR1) s1c[k] = t1[i];
+    }
+    if (tid < NR2) s2c[tid] = t2;
+    for (int i = tid; i < (NR2 + 31) / 32; i += kSeedThreads) sd2[i] = 0u;
+    if (tid == 0) *nlist = 0;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int kb = (i * kSeedThreads + tid) * 8;
+        const unsigned long long bits = (unsigned long long)f[i].x | ((unsigned long long)f[i].y << 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (((bits >> (8 * e)) & 0xffull) && kb + e < NR1) {
+                const int k = kb + e;
+                dl[atomicAdd(nlist, 1)] = k;
+                atomicOr(&sd2[k >> 10], 1u << ((k >> 5) & 31));
+            }
+    }
+    __syncthreads();
+    const int nd = *nlist;
+    for (int j = tid; j < nd; j += kSeedThreads) {
+        const int k = dl[j];
+        const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
+        double v = 0.0;
+        if (q1 - q0 == kSeedS) {
+            double t[kSeedS];
+#pragma unroll
+            for (int e = 0; e < kSeedS; ++e) t[e] = __ldcg(d2h + q0 + e);
+#pragma unroll
+            for (int e = 0; e < kSeedS; ++e) v += t[e];
+        } else {
+            for (int i = q0; i < q1; ++i) v += __ldcg(d2h + i);
+        }
+        b1[k] = v;
+        s1c[k] = v;
+        dh[k] = 0;
+    }
+    __syncthreads();
+    if (tid < NR2 && ((sd2[tid >> 5] >> (tid & 31)) & 1u)) {
+        const int k0 = tid * kSeedS, k1 = min(NR1, k0 + kSeedS);
+        double v = 0.0;
+        for (int k = k0; k < k1; ++k) v += s1c[k];
+        b2[tid] = v;
+        s2c[tid] = v;
+    }
+}
+
 // ---- arrival and pick (the last block of head h in round r)
 //
 // REFRESH: bring the S1 sums of the ranges flagged this round and the S2
 // sums above them up to date first.  dl (>= 2048 ints) and sd2 (>= 2048
-// bytes) are shared memory the block no longer needs.
+// bytes) are shared memory the block no longer needs.  With a shared-memory
+// cache of `cache_n` doubles that holds every S1 and S2 sum of the head, the
+// sums are loaded once, together with the flags, and the refresh and the
+// scans read them from there (the same values in the same order, so the same
+// pick, with fewer dependent trips to L2).
 template <bool REFRESH>
-__device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r, int *dl, uint32_t *sd2) {
+__device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r, int *dl, uint32_t *sd2,
+                                                 double *cache = nullptr, int cache_n = 0) {
     __shared__ double sh[kSeedWarps];
     __shared__ int nlist, last, pick_blk;
     __shared__ double sh_base;
@@ -434,7 +515,14 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
     const int NR1 = s.NR1, NR2 = s.NR2;
     double *b1 = s.bs1 + (size_t)h * NR1;
     double *b2 = s.bs2 + (size_t)h * NR2;
-    if constexpr (REFRESH) {
+    // cached: every S1 and S2 sum in shared memory (at most two flag words of
+    // 8 ranges per thread, one scan chunk of S2 sums)
+    const bool cached = REFRESH && cache != nullptr && NR1 + NR2 <= cache_n && NR1 <= 2 * 8 * kSeedThreads &&
+                        NR2 <= kSeedThreads;
+    double *s1c = cache, *s2c = cached ? cache + NR1 : nullptr;
+    if (cached) {
+        seed_refresh_cached(b1, b2, dh, d2h, N, NR1, NR2, dl, sd2, s1c, s2c, &nlist);
+    } else if constexpr (REFRESH) {
         // S1 sums of the ranges touched this round (each in index order),
         // then the S2 sums over them
         for (int i = tid; i < (NR2 + 31) / 32; i += kSeedThreads) sd2[i] = 0u;
@@ -483,10 +571,12 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
         }
     }
     __syncthreads();
+    auto get1 = [&](int k) { return cached ? s1c[k] : __ldcg(b1 + k); };
+    auto get2 = [&](int k) { return cached ? s2c[k] : __ldcg(b2 + k); };
     double total = 0.0;
     {
         double v = 0.0;
-        for (int k = tid; k < NR2; k += kSeedThreads) v += __ldcg(b2 + k);
+        for (int k = tid; k < NR2; k += kSeedThreads) v += get2(k);
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
         __syncthreads();
@@ -501,7 +591,7 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
         double carry = 0.0;
         for (int c0 = 0; c0 < NR2; c0 += kSeedThreads) {
             const int kk = c0 + tid;
-            const double v = kk < NR2 ? __ldcg(b2 + kk) : 0.0;
+            const double v = kk < NR2 ? get2(kk) : 0.0;
             const double inc = block_scan_d(v, sh) + carry;
             __syncthreads();
             if (kk < NR2 && inc > thr) atomicMin(&pick_blk, kk);
@@ -521,7 +611,7 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
             int pk = -1;
             if (k2 != 0x7fffffff) {
                 const int k = k2 * kSeedS + lane;
-                const double v1 = k < NR1 ? __ldcg(b1 + k) : 0.0;
+                const double v1 = k < NR1 ? get1(k) : 0.0;
                 const double inc1 = warp_scan_d(v1, lane);
                 const unsigned cr1 = __ballot_sync(0xffffffffu, k < NR1 && base2 + inc1 > thr);
                 const unsigned pos1 = __ballot_sync(0xffffffffu, v1 > 0.0);
@@ -823,7 +913,8 @@ kmeanspp_round_grouped(const T *__restrict__ x, const SeedArgs s, int r, int G, 
     __syncthreads();
     for (int j = tid; j < P; j += kSeedThreads)
         if (act[j]) s.pm[rec + j] = __uint_as_float(pmax[j]);
-    seed_arrive_pick<true>(s, h, r, pperm, reinterpret_cast<uint32_t *>(act));
+    // the piece lists (alist, pmax: 8 ch bytes) hold the S1 and S2 sums in the pick
+    seed_arrive_pick<true>(s, h, r, pperm, reinterpret_cast<uint32_t *>(act), reinterpret_cast<double *>(alist), ch);
 }
 
 // ---- regrouping (before round r, with G = r - 1 chosen centres applied)
