@@ -179,9 +179,12 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *tile = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(tile + kUnit);
-    float *wo = reinterpret_cast<float *>(bar + 2);       // [W][G][D]
-    float *wm = wo + kWarps * G * D;                      // [W][G]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(tile + kUnit);  // [2]: the unit's two halves
+    // [W][G][D] attention partials of the warps: over the K half of the tile,
+    // which every warp has read (barrier) before any writes here
+    float *wo = reinterpret_cast<float *>(tile);
+    static_assert(kWarps * G * D * sizeof(float) <= kUnit / 2, "partials fit the K half");
+    float *wm = reinterpret_cast<float *>(bar + 2);       // [W][G]
     float *wl = wm + kWarps * G;                          // [W][G]
     float2 *wb = reinterpret_cast<float2 *>(wl + kWarps * G);  // [W][B]
     float *sq = reinterpret_cast<float *>(                   // [kScanFmaRows][D], 16-byte aligned
@@ -240,29 +243,38 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
 
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bar + 1, 1);
         fence_mbar_init();
     }
     __syncthreads();
+    // Two barriers, so that compute starts on the first half of a unit while
+    // the second lands: the column halves of a centroid tile (d = 128; at
+    // d = 64 the whole tile is the first half), or the K and V of a token tile.
     auto issue = [&](int vrows) {
         if (scan && vrows > 0) {
-            mbar_arrive_expect_tx(bar, Gm::CS * Gm::ROWB);
 #pragma unroll
-            for (int hf = 0; hf < Gm::HALVES; ++hf)
-                tma_load_3d(tile + hf * Gm::CS * 128, &maps.c, 64 * hf, first, h, bar);
+            for (int hf = 0; hf < Gm::HALVES; ++hf) {
+                mbar_arrive_expect_tx(bar + hf, Gm::CS * 128);
+                tma_load_3d(tile + hf * Gm::CS * 128, &maps.c, 64 * hf, first, h, bar + hf);
+            }
+            if (Gm::HALVES == 1) mbar_arrive(bar + 1);
         } else if (scan) {
             mbar_arrive(bar);  // a unit past its cluster's members: nothing to load
+            mbar_arrive(bar + 1);
         } else if (vrows > 0) {
-            mbar_arrive_expect_tx(bar, 2 * Gm::TS * Gm::ROWB);
             const CUtensorMap *mk = prefix ? &maps.kp : &maps.k;
             const CUtensorMap *mv = prefix ? &maps.vp : &maps.v;
             const int c2 = prefix ? g : b * a.Hkv + g;
+            mbar_arrive_expect_tx(bar, Gm::TS * Gm::ROWB);
+            mbar_arrive_expect_tx(bar + 1, Gm::TS * Gm::ROWB);
 #pragma unroll
-            for (int hf = 0; hf < Gm::HALVES; ++hf) {
-                tma_load_3d(tile + hf * Gm::TS * 128, mk, 64 * hf, first, c2, bar);
-                tma_load_3d(tile + kUnit / 2 + hf * Gm::TS * 128, mv, 64 * hf, first, c2, bar);
-            }
+            for (int hf = 0; hf < Gm::HALVES; ++hf) tma_load_3d(tile + hf * Gm::TS * 128, mk, 64 * hf, first, c2, bar);
+#pragma unroll
+            for (int hf = 0; hf < Gm::HALVES; ++hf)
+                tma_load_3d(tile + kUnit / 2 + hf * Gm::TS * 128, mv, 64 * hf, first, c2, bar + 1);
         } else {
             mbar_arrive(bar);
+            mbar_arrive(bar + 1);
         }
     };
     // static centroids may stream before the dependency wait (caller's choice)
@@ -316,7 +328,7 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
                             __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
         }
         __syncthreads();
-        if (!mbar_wait(bar, 0)) set_error(a.ws_err);
+        if (!mbar_wait(bar, 0) || !mbar_wait(bar + 1, 0)) set_error(a.ws_err);
         scan_fma<D>(tile, sq, nq, a.metric, first, valid, warp, lane, wb + warp * a.B);
     } else if (scan) {
         // ------------------------------- centroid unit, more query rows: tensor cores
@@ -344,6 +356,7 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
                 float sl = 0.f, sh = 0.f;
 #pragma unroll
                 for (int j = 0; j < KS; ++j) {
+                    if (j == KS / 2 && nt == 0 && mt == 0 && !mbar_wait(bar + 1, 0)) set_error(a.ws_err);
                     const int col = 16 * j + 8 * (i4 >> 1);
                     uint32_t a0, a1, a2, a3;
                     ldsm_x4(sbuf + (col >> 6) * (Gm::CS * 128) + swz128(row, (col & 63) >> 3), a0, a1, a2, a3);
@@ -488,6 +501,9 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
         pb0[kk] = movm_t(pack_bf16(sf[kk][0], sf[kk][1]));
         pb1[kk] = movm_t(pack_bf16(sf[kk][2], sf[kk][3]));
     }
+    // every warp is done with K (its half becomes the partials), and V is here
+    __syncthreads();
+    if (!mbar_wait(bar + 1, 0)) set_error(a.ws_err);
     const uint32_t vbase = sbuf + kUnit / 2;
 #pragma unroll
     for (int md = 0; md < NMD; ++md) {
@@ -780,7 +796,7 @@ cudaError_t tc_launch(tc::Args a, const void *centroids, const void *k_prefix, c
                                     !make_map_3d(&maps.vp, v_prefix, D, a.Lp, a.Hkv, Gm::TS)))
         return cudaErrorInvalidValue;
     const int units = a.n_scan + a.B * a.Hkv * ((a.ext_prefix ? 0 : a.nP) + a.nA);
-    const size_t smem = 1024 + tc::kUnit + 16 + sizeof(float) * tc::kWarps * G * (D + 2) +
+    const size_t smem = 1024 + tc::kUnit + 16 + sizeof(float) * tc::kWarps * G * 2 +
                         sizeof(float2) * tc::kWarps * a.B + 16 + sizeof(float) * tc::kScanFmaRows * D;
     auto k1 = tc::asm_decode_units<D, G>;
     static size_t k1_smem = 0;
