@@ -173,7 +173,7 @@ __device__ __forceinline__ void scan_fma(const unsigned char *tile, const float 
 // ------------------------------------------------------------ unit kernel --
 
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 6)  // six CTAs per SM (shared memory allows six)
 asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
     using Gm = Geo<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -344,6 +344,13 @@ asm_decode_units(const Args a, const __grid_constant__ Maps maps) {
             for (int j = 0; j < KS; ++j) {
                 qb0[j] = bq < nq ? __ldg(qr + 8 * j + quad) : 0u;
                 qb1[j] = bq < nq ? __ldg(qr + 8 * j + 4 + quad) : 0u;
+            }
+            // the next n-tile's query rows into L1 while this one multiplies
+            constexpr int QL = D * 2 / 128;  // 128-byte lines per query row
+            if ((nt + 1) * 8 < nq && lane < 8 * QL) {
+                const int rn = min(8 * (nt + 1) + lane / QL, nq - 1);
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(a.qs + ((size_t)(qrow0 + rn) * a.Hq + h) * D +
+                                                               (lane % QL) * 64));
             }
             if (nt == 0 && !mbar_wait(bar, 0)) set_error(a.ws_err);
             float bs[2] = {kNegInf, kNegInf};
