@@ -775,10 +775,10 @@ def x_bytes(H, N, d):
 # capture of this benchmark), with the digest of the kernel source they were
 # taken on: a changed kernel reports null until it is measured again.
 TRAFFIC = {
-    "llama31-8b-layer-decode-K1024-T2048-B1": {  # units 16 936 992 + merge 585 120
-        "bytes": 17522112, "source": "14a39ab15a4f2c84"},
-    "llama31-8b-layer-decode-K8192-T4096-B16": {  # units 356 002 880 + merge 17 530 816
-        "bytes": 373533696, "source": "14a39ab15a4f2c84"},
+    "llama31-8b-layer-decode-K1024-T2048-B1": {  # units 16 943 680 + merge 585 216
+        "bytes": 17528896, "source": "f4eb5d7dc4ecd911"},
+    "llama31-8b-layer-decode-K8192-T4096-B16": {  # units 356 772 736 + merge 17 530 624
+        "bytes": 374303360, "source": "f4eb5d7dc4ecd911"},
 }
 TRAFFIC_SOURCE = os.path.join(ROOT, "long_prefix_attention_b200", "csrc", "decode_tc.cu")
 
