@@ -57,7 +57,7 @@ constexpr int kSeedScreen = 128;      // first round of the fp32 screen
 
 struct SeedWs {
     size_t off_d2, off_bs1, off_bs2, off_r2, off_gs, off_ge, off_gr, off_gn, off_near, off_perm, off_gcnt, off_seg,
-        off_cur, off_pg, off_pm, off_plo, off_phi, off_pcnt, off_gq, off_dirty, off_taken, off_cnt, total;
+        off_cur, off_pg, off_pm, off_plo, off_phi, off_pcnt, off_gq, off_dirty, off_taken, off_cnt, off_ctr, total;
     int nr1, nr2, dstride, nbmax;
     size_t cap;
 };
@@ -92,7 +92,8 @@ SeedWs seed_ws(int H, int N, int d, int K) {
     w.off_dirty = al256(w.off_gq + h * k * (size_t)d);
     w.off_taken = al256(w.off_dirty + h * (size_t)w.dstride);
     w.off_cnt = al256(w.off_taken + h * n);
-    w.total = al256(w.off_cnt + sizeof(int) * h);
+    w.off_ctr = al256(w.off_cnt + sizeof(int) * h);
+    w.total = al256(w.off_ctr + sizeof(int) * (size_t)K);
     return w;
 }
 
@@ -115,6 +116,7 @@ struct SeedArgs {
     unsigned char *dirty;   // [H][DSTRIDE] S1 range touched this round
     unsigned char *taken;   // [H][N] point already chosen
     int *cnt;               // [H] arrival counters
+    int *ctr;               // [K] work counters of the rounds with dynamic chunks
     int N, K, NR1, NR2, DSTRIDE, NBMAX;
     size_t CAP;
 };
@@ -470,7 +472,7 @@ __device__ __noinline__ void seed_refresh_cached(double *b1, double *b2, unsigne
     }
 }
 
-// ---- arrival and pick (the last block of head h in round r)
+// ---- arrival and pick (the last of the `arrivals` arrivals of head h in round r)
 //
 // REFRESH: bring the S1 sums of the ranges flagged this round and the S2
 // sums above them up to date first.  dl (>= 2048 ints) and sd2 (>= 2048
@@ -480,8 +482,8 @@ __device__ __noinline__ void seed_refresh_cached(double *b1, double *b2, unsigne
 // scans read them from there (the same values in the same order, so the same
 // pick, with fewer dependent trips to L2).
 template <bool REFRESH>
-__device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r, int *dl, uint32_t *sd2,
-                                                 double *cache = nullptr, int cache_n = 0) {
+__device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r, int arrivals, int *dl,
+                                                 uint32_t *sd2, double *cache = nullptr, int cache_n = 0) {
     __shared__ double sh[kSeedWarps];
     __shared__ int nlist, last, pick_blk;
     __shared__ double sh_base;
@@ -495,7 +497,7 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
     __syncthreads();
     if (tid == 0) {
         const int old = atomicAdd(&s.cnt[h], 1);
-        last = (old == (int)(gridDim.x - 1));
+        last = (old == arrivals - 1);
         __threadfence();
     }
     __syncthreads();
@@ -669,20 +671,92 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
 }
 
 // ---- rounds before the first grouping: every point is updated, and each
-// block writes the S1 and S2 sums of its own positions (ch is a multiple of
-// the S2 range)
+// range of positions [p0, p1) (a multiple of the S2 range, or the tail) gets
+// its S1 and S2 sums written by the block that updated it.
 // SCREEN: test each point first with the fp32 distance (worth it once few
 // points change per round; without it the kernel needs fewer registers).
 template <typename T, int D, bool SCREEN>
-__global__ void __launch_bounds__(kSeedThreads)
-kmeanspp_round_full(const T *__restrict__ x, const SeedArgs s, int r, int ch) {
+__device__ __forceinline__ void seed_full_range(const T *__restrict__ x, const SeedArgs &s, int h, int r, int p0,
+                                                int p1, double *s1own) {
     using Gm = SeedGeo<T, D>;
-    const int h = blockIdx.y, N = s.N, K = s.K;
+    const int N = s.N, K = s.K;
     const size_t hN = (size_t)h * N;
     const T *xh = x + hN * D;
     double *d2h = s.d2 + hN;
-    __shared__ double s1own[kSeedChMax / kSeedS];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = s.idx[(size_t)h * K + r - 1];
+    const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + (lane % Gm::LPP) * Gm::E16));
+    double cv[Gm::E16];
+    float cvf[Gm::E16];
+    widen16<T>(craw, cv);
+    widen16f<T>(craw, cvf);
+    (void)cvf;
+    const int q = seed_row<T, D>(lane);
+    double *b1 = s.bs1 + (size_t)h * s.NR1;
+    const int k0 = p0 / kSeedS, k1 = (p1 + kSeedS - 1) / kSeedS;
+    for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
+        const int qp = base + lane;
+        const unsigned m = __ballot_sync(0xffffffffu, qp < p1);
+        uint4 buf[Gm::LPP];
+        load32<T, D, true>(xh, qp, m, lane, buf);
+        const int i = base + q;
+        const bool mine = (m >> q) & 1u;
+        const double old = mine ? d2h[i] : 0.0;
+        double fin = old;  // the point's D2 after this round (0 past p1)
+        // fp32 screen, then the exact distance where D2 may fall (the
+        // rows are read again, from cache, for the rare warps that need it)
+        if constexpr (SCREEN) {
+            const float d32 = dist32f<T, D>(buf, cvf, lane);  // every lane: it shuffles
+            const bool cand = mine && seed_may_fall(d32, old);
+            if (__any_sync(0xffffffffu, cand)) {
+                uint4 buf2[Gm::LPP];
+                load32<T, D, false>(xh, qp, m, lane, buf2);
+                const double dist = dist32<T, D>(buf2, cv, lane);
+                if (cand && dist < old) {
+                    d2h[i] = dist;
+                    s.near[hN + i] = r - 1;
+                    fin = dist;
+                }
+            }
+        } else {
+            const double dist = dist32<T, D>(buf, cv, lane);
+            if (mine && dist < old) {
+                d2h[i] = dist;
+                s.near[hN + i] = r - 1;
+                fin = dist;
+            }
+        }
+        // the S1 sum of these 32 points (base is a multiple of 32), in index
+        // order from the registers: point j is in lane (j % PPL) LPP + j / PPL
+        double v = 0.0;
+#pragma unroll
+        for (int j = 0; j < kSeedS; ++j)
+            v += __shfl_sync(0xffffffffu, fin, (j % Gm::PPL) * Gm::LPP + j / Gm::PPL);
+        if (lane == 0) {
+            b1[base / kSeedS] = v;
+            s1own[base / kSeedS - k0] = v;
+        }
+    }
+    __syncthreads();
+    const int m0 = k0 / kSeedS, m1 = (k1 + kSeedS - 1) / kSeedS;
+    for (int k2 = m0 + tid; k2 < m1; k2 += kSeedThreads) {
+        const int a0 = k2 * kSeedS, a1 = min(s.NR1, a0 + kSeedS);
+        double v = 0.0;
+        for (int k = a0; k < a1; ++k) v += s1own[k - k0];
+        s.bs2[(size_t)h * s.NR2 + k2] = v;
+    }
+}
+
+// One block per range of ch positions of head blockIdx.y (round 0 clears
+// the state).
+template <typename T, int D, bool SCREEN>
+__global__ void __launch_bounds__(kSeedThreads)
+kmeanspp_round_full(const T *__restrict__ x, const SeedArgs s, int r, int ch) {
+    const int h = blockIdx.y, N = s.N;
+    const size_t hN = (size_t)h * N;
+    double *d2h = s.d2 + hN;
+    __shared__ double s1own[kSeedChMax / kSeedS];
+    const int tid = threadIdx.x;
     const int p0 = blockIdx.x * ch;
     const int p1 = min(N, p0 + ch);
     pdl_wait();
@@ -697,73 +771,40 @@ kmeanspp_round_full(const T *__restrict__ x, const SeedArgs s, int r, int ch) {
         }
         for (int k = p0 / kSeedS + tid; k < (p1 + kSeedS - 1) / kSeedS; k += kSeedThreads) dh[k] = 0;
     } else {
-        const int c = s.idx[(size_t)h * K + r - 1];
-        const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + (lane % Gm::LPP) * Gm::E16));
-        double cv[Gm::E16];
-        float cvf[Gm::E16];
-        widen16<T>(craw, cv);
-        widen16f<T>(craw, cvf);
-        (void)cvf;
-        const int q = seed_row<T, D>(lane);
-        for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
-            const int qp = base + lane;
-            const unsigned m = __ballot_sync(0xffffffffu, qp < p1);
-            uint4 buf[Gm::LPP];
-            load32<T, D, true>(xh, qp, m, lane, buf);
-            const int i = base + q;
-            const bool mine = (m >> q) & 1u;
-            const double old = mine ? d2h[i] : 0.0;
-            // fp32 screen, then the exact distance where D2 may fall (the
-            // rows are read again, from cache, for the rare warps that need it)
-            if constexpr (SCREEN) {
-                const float d32 = dist32f<T, D>(buf, cvf, lane);  // every lane: it shuffles
-                const bool cand = mine && seed_may_fall(d32, old);
-                if (__any_sync(0xffffffffu, cand)) {
-                    uint4 buf2[Gm::LPP];
-                    load32<T, D, false>(xh, qp, m, lane, buf2);
-                    const double dist = dist32<T, D>(buf2, cv, lane);
-                    if (cand && dist < old) {
-                        d2h[i] = dist;
-                        s.near[hN + i] = r - 1;
-                    }
-                }
-            } else {
-                const double dist = dist32<T, D>(buf, cv, lane);
-                if (mine && dist < old) {
-                    d2h[i] = dist;
-                    s.near[hN + i] = r - 1;
-                }
-            }
-        }
-        __syncthreads();
-        // the block's own S1 sums (index order), then its S2 sums
-        double *b1 = s.bs1 + (size_t)h * s.NR1;
-        const int k0 = p0 / kSeedS, k1 = (p1 + kSeedS - 1) / kSeedS;
-        for (int k = k0 + tid; k < k1; k += kSeedThreads) {
-            const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
-            double v = 0.0;
-            if (q1 - q0 == kSeedS) {
-                double t[kSeedS];
-#pragma unroll
-                for (int e = 0; e < kSeedS; ++e) t[e] = __ldcg(d2h + q0 + e);
-#pragma unroll
-                for (int e = 0; e < kSeedS; ++e) v += t[e];
-            } else {
-                for (int i = q0; i < q1; ++i) v += __ldcg(d2h + i);
-            }
-            b1[k] = v;
-            s1own[k - k0] = v;
-        }
-        __syncthreads();
-        const int m0 = k0 / kSeedS, m1 = (k1 + kSeedS - 1) / kSeedS;
-        for (int k2 = m0 + tid; k2 < m1; k2 += kSeedThreads) {
-            const int a0 = k2 * kSeedS, a1 = min(s.NR1, a0 + kSeedS);
-            double v = 0.0;
-            for (int k = a0; k < a1; ++k) v += s1own[k - k0];
-            s.bs2[(size_t)h * s.NR2 + k2] = v;
-        }
+        seed_full_range<T, D, SCREEN>(x, s, h, r, p0, p1, s1own);
     }
-    seed_arrive_pick<false>(s, h, r, nullptr, nullptr);
+    seed_arrive_pick<false>(s, h, r, gridDim.x, nullptr, nullptr);
+}
+
+// The same rounds (r >= 1) with the work handed out dynamically: the grid is
+// the blocks that fit the GPU at once, and each block takes the next S2 range
+// of positions (1024; head-major order) from the round's counter until none
+// is left.  A static split left blocks idle while others still worked (the
+// blocks of one round ended 76-136 us after its start; their fp64 rechecks
+// and their SM's share differ), and each head now waits only for its last
+// range.  The block that completes a head's last range picks for it.
+template <typename T, int D, bool SCREEN>
+__global__ void __launch_bounds__(kSeedThreads)
+kmeanspp_round_full_dyn(const T *__restrict__ x, const SeedArgs s, int r, int H) {
+    constexpr int kChunk = kSeedS * kSeedS;
+    __shared__ double s1own[kSeedS];
+    __shared__ int next_item;
+    const int N = s.N, nch = (N + kChunk - 1) / kChunk, total = nch * H;
+    pdl_wait();
+    pdl_launch_dependents();
+    if (threadIdx.x == 0) next_item = atomicAdd(&s.ctr[r], 1);
+    __syncthreads();
+    int it = next_item;
+    while (it < total) {
+        __syncthreads();  // every thread has read next_item
+        // the following range, in flight while this one is updated
+        if (threadIdx.x == 0) next_item = atomicAdd(&s.ctr[r], 1);
+        const int h = it / nch, p0 = (it - h * nch) * kChunk;
+        seed_full_range<T, D, SCREEN>(x, s, h, r, p0, min(N, p0 + kChunk), s1own);
+        seed_arrive_pick<false>(s, h, r, nch, nullptr, nullptr);
+        __syncthreads();
+        it = next_item;
+    }
 }
 
 // ---- grouped rounds (pruned update)
@@ -914,7 +955,8 @@ kmeanspp_round_grouped(const T *__restrict__ x, const SeedArgs s, int r, int G, 
     for (int j = tid; j < P; j += kSeedThreads)
         if (act[j]) s.pm[rec + j] = __uint_as_float(pmax[j]);
     // the piece lists (alist, pmax: 8 ch bytes) hold the S1 and S2 sums in the pick
-    seed_arrive_pick<true>(s, h, r, pperm, reinterpret_cast<uint32_t *>(act), reinterpret_cast<double *>(alist), ch);
+    seed_arrive_pick<true>(s, h, r, gridDim.x, pperm, reinterpret_cast<uint32_t *>(act),
+                           reinterpret_cast<double *>(alist), ch);
 }
 
 // ---- regrouping (before round r, with G = r - 1 chosen centres applied)
@@ -1319,6 +1361,17 @@ int seed_block_positions(KERN k, bool grouped, int step, int H, int N, cudaError
     return kSeedChMax;
 }
 
+// Blocks of kernel k (kSeedThreads, no dynamic shared memory) resident on the GPU at once.
+template <typename KERN>
+int seed_resident(KERN k, cudaError_t *err) {
+    int occ = 0, dev = 0, sms = 0;
+    if ((*err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kSeedThreads, 0)) != cudaSuccess ||
+        (*err = cudaGetDevice(&dev)) != cudaSuccess ||
+        (*err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return 0;
+    return std::max(1, occ * sms);
+}
+
 template <typename KERN, typename... Args>
 cudaError_t seed_launch(KERN k, dim3 grid, size_t smem, cudaStream_t st, Args... args) {
     cudaLaunchAttribute at[1];
@@ -1339,13 +1392,18 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
     cudaError_t e = cudaSuccess;
     const int chf = seed_block_positions(kmeanspp_round_full<T, D, false>, false, kSeedS * kSeedS, H, s.N, &e);
     if (e != cudaSuccess) return e;
-    const int chs = seed_block_positions(kmeanspp_round_full<T, D, true>, false, kSeedS * kSeedS, H, s.N, &e);
+    // rounds 1 .. the first grouping: as many blocks as fit the GPU at once,
+    // taking S2 ranges of positions dynamically
+    const int items = H * ((s.N + kSeedS * kSeedS - 1) / (kSeedS * kSeedS));
+    const int rdf = std::min(items, seed_resident(kmeanspp_round_full_dyn<T, D, false>, &e));
+    if (e != cudaSuccess) return e;
+    const int rds = std::min(items, seed_resident(kmeanspp_round_full_dyn<T, D, true>, &e));
     if (e != cudaSuccess) return e;
     const int chg = seed_block_positions(kmeanspp_round_grouped<T, D>, true, 256, H, s.N, &e);
     if (e != cudaSuccess) return e;
     const int N = s.N, K = s.K;
     const dim3 pgrid((N + 255) / 256, H);
-    const dim3 gfull((N + chf - 1) / chf, H), gscr((N + chs - 1) / chs, H), ggrp((N + chg - 1) / chg, H);
+    const dim3 gfull((N + chf - 1) / chf, H), ggrp((N + chg - 1) / chg, H);
     int G = 0, next = std::max(256, K / 8);
     for (int r = 0; r < K; ++r) {
         int pre = 1;
@@ -1367,8 +1425,9 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
             next = r + std::max(256, p2 / 4);
         }
         if (G > 0) e = seed_launch(kmeanspp_round_grouped<T, D>, ggrp, seed_grouped_smem(chg), st, x, s, r, G, pre, chg);
-        else if (r < kSeedScreen) e = seed_launch(kmeanspp_round_full<T, D, false>, gfull, 0, st, x, s, r, chf);
-        else e = seed_launch(kmeanspp_round_full<T, D, true>, gscr, 0, st, x, s, r, chs);
+        else if (r == 0) e = seed_launch(kmeanspp_round_full<T, D, false>, gfull, 0, st, x, s, r, chf);
+        else if (r < kSeedScreen) e = seed_launch(kmeanspp_round_full_dyn<T, D, false>, dim3(rdf), 0, st, x, s, r, H);
+        else e = seed_launch(kmeanspp_round_full_dyn<T, D, true>, dim3(rds), 0, st, x, s, r, H);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
@@ -1405,6 +1464,7 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
     s.dirty = reinterpret_cast<unsigned char *>(b + w.off_dirty);
     s.taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
     s.cnt = reinterpret_cast<int *>(b + w.off_cnt);
+    s.ctr = reinterpret_cast<int *>(b + w.off_ctr);
     s.N = N;
     s.K = K;
     s.NR1 = w.nr1;
@@ -1413,6 +1473,7 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
     s.NBMAX = w.nbmax;
     s.CAP = w.cap;
     cudaError_t e = cudaMemsetAsync(s.cnt, 0, sizeof(int) * (size_t)H, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s.ctr, 0, sizeof(int) * (size_t)K, st);
     if (e != cudaSuccess) return e;
     if (dt == ASM_BF16) {
         using T = __nv_bfloat16;
