@@ -449,6 +449,29 @@ asm_status asm_decode_step_search(const void *q, const void *q_search,
 /* Zero a decode / flash-decode / k-means workspace (counters, error word). */
 asm_status asm_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * asm_wait_spin_limit -- how many unsuccessful mbarrier try_wait polls any
+ * wait in the library's kernels makes before it gives up, sets the error
+ * word to ASM_ERR_TIMEOUT and lets its CTA finish.
+ */
+uint32_t asm_wait_spin_limit(void);
+
+/*
+ * asm_wait_selftest -- run the give-up path of a bounded wait on purpose: one
+ * CTA waits on an mbarrier that nothing arrives at, `polls` try_wait polls
+ * (0: the library's own bounded wait, asm_wait_spin_limit() polls), then
+ * completes the barrier's phase itself.  No copy is in flight and no tensor
+ * memory is held, so the context stays usable.
+ *   ws          >= 256 bytes, 16-byte aligned: its error word (read with
+ *               asm_workspace_error) is cleared, then set to ASM_ERR_TIMEOUT
+ *               when the wait gives up
+ *   elapsed_ns  host: how long the wait took (device %globaltimer)
+ * Synchronises `stream`.  ASM_ERR_INVALID_ARG for polls < 0, a short or
+ * misaligned ws, or a null elapsed_ns.
+ */
+asm_status asm_wait_selftest(int polls, void *ws, size_t ws_bytes, uint64_t *elapsed_ns,
+                             cudaStream_t stream);
+
 /* Error word of a decode / flash-decode / k-means / whitening workspace, copied to the host
  * pointer `code` (0 = no device-side error; otherwise ASM_ERR_TIMEOUT).
  * Synchronises `stream`. */

@@ -45,6 +45,8 @@ SIGNATURES = {
                                    SZ, P]),
     "asm_workspace_init": (I, [P, SZ, P]),
     "asm_workspace_error": (I, [P, SZ, ctypes.POINTER(ctypes.c_int), P]),
+    "asm_wait_spin_limit": (ctypes.c_uint32, []),
+    "asm_wait_selftest": (I, [I, P, SZ, ctypes.POINTER(ctypes.c_uint64), P]),
     "asm_status_string": (ctypes.c_char_p, [I]),
     "asm_last_cuda_error": (ctypes.c_char_p, []),
     "asm_version": (ctypes.c_char_p, []),

@@ -349,6 +349,22 @@ asm_status asm_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream) {
     return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, stream));
 }
 
+uint32_t asm_wait_spin_limit(void) { return asm_wait_spin_limit_value(); }
+
+asm_status asm_wait_selftest(int polls, void *ws, size_t ws_bytes, uint64_t *elapsed_ns, cudaStream_t stream) {
+    if (polls < 0 || !aligned(ws, 16) || ws_bytes < 256 || elapsed_ns == nullptr) return ASM_ERR_INVALID_ARG;
+    char *b = static_cast<char *>(ws);
+    unsigned long long *dev_ns = reinterpret_cast<unsigned long long *>(b + 8);
+    cudaError_t e = cudaMemsetAsync(ws, 0, 16, stream);
+    if (e == cudaSuccess) e = asm_selftest_wait_launch(polls, reinterpret_cast<int *>(b), dev_ns, stream);
+    unsigned long long v = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&v, dev_ns, sizeof(v), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    *elapsed_ns = v;
+    return ASM_OK;
+}
+
 asm_status asm_workspace_error(const void *ws, size_t ws_bytes, int *code, cudaStream_t stream) {
     if (!aligned(ws, 16) || ws_bytes < 256 || code == nullptr) return ASM_ERR_INVALID_ARG;
     int v = 0;

@@ -14,8 +14,11 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // Bounded spins: a wait that has not completed after this many polls gives
-// up and raises ASM_ERR_TIMEOUT in the caller's error word.
-constexpr uint32_t kSpinLimit = 1u << 22;
+// up and raises ASM_ERR_TIMEOUT in the caller's error word.  A poll of an
+// mbarrier that does not complete suspends the thread for about 4 us on
+// this part (measured by the timeout self-test), so the bound is about one
+// second, thousands of times any wait of a working kernel.
+constexpr uint32_t kSpinLimit = 1u << 18;
 
 // ---------------------------------------------------------------- dtypes --
 

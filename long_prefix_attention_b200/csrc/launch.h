@@ -87,6 +87,8 @@ cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norm
                                  int K, int metric, int32_t *assign, int *err, cudaStream_t st);
 
 // merge.cu: online-softmax merge of two state arrays, row by row
+cudaError_t asm_selftest_wait_launch(int polls, int *err, unsigned long long *elapsed_ns, cudaStream_t st);
+uint32_t asm_wait_spin_limit_value();
 cudaError_t asm_merge_states_launch(void *a, float *z, const void *a2, const float *z2, long long R, int d,
                                     asm_dtype dt, int num_sms, cudaStream_t st);
 

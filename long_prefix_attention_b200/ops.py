@@ -178,6 +178,21 @@ def asm_workspace_error(ws, stream=None) -> int:
     return code.value
 
 
+def asm_wait_spin_limit() -> int:
+    """Unsuccessful try_wait polls after which any library wait gives up."""
+    return int(_lib.load().asm_wait_spin_limit())
+
+
+def asm_wait_selftest(polls: int, ws, stream=None) -> int:
+    """Run a bounded wait that nothing completes (polls try_wait polls, 0 =
+    the library's own bound); returns its duration in ns.  The workspace's
+    error word then holds ASM_ERR_TIMEOUT (read with asm_workspace_error)."""
+    ns = ctypes.c_uint64(0)
+    _check("asm_wait_selftest", _lib.load().asm_wait_selftest(
+        int(polls), _p(ws), ws.numel() * ws.element_size(), ctypes.byref(ns), _stream(stream)))
+    return int(ns.value)
+
+
 def asm_decode_step(q, centroids, a_bar, logz_bar, k_cache, v_cache, local_len, scale: float,
                     out, ws, lse_out=None, idx_out=None, metric: int = ASM_L2, flags: int = 0,
                     stream=None):
