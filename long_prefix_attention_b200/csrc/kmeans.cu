@@ -54,10 +54,16 @@ constexpr int kSeedS = 32;           // points per S1 sum, S1 sums per S2 sum
 constexpr int kSeedMaxN = 1 << 24;   // S2 dirty bits fit the block's 2 KB bitmap
 constexpr double kSeedMargin = 1e-12;
 constexpr int kSeedScreen = 128;      // first round of the fp32 screen
+// Record of the centre a round picked, for the next round: its row (up to
+// 512 bytes), its int8 codes (up to 128 bytes, at 512) and scale, |codes|^2
+// and quantisation error (at 640).
+constexpr int kSeedCenBytes = 1024;
+constexpr int kSeedCenCodes = 512, kSeedCenScal = 640;
 
 struct SeedWs {
     size_t off_d2, off_bs1, off_bs2, off_r2, off_gs, off_ge, off_gr, off_gn, off_near, off_perm, off_gcnt, off_seg,
-        off_cur, off_pg, off_pm, off_plo, off_phi, off_pcnt, off_gq, off_dirty, off_taken, off_cnt, off_ctr, total;
+        off_cur, off_pg, off_pm, off_plo, off_phi, off_pcnt, off_gq, off_dirty, off_taken, off_cnt, off_ctr, off_cen,
+        total;
     int nr1, nr2, dstride, nbmax;
     size_t cap;
 };
@@ -93,7 +99,8 @@ SeedWs seed_ws(int H, int N, int d, int K) {
     w.off_taken = al256(w.off_dirty + h * (size_t)w.dstride);
     w.off_cnt = al256(w.off_taken + h * n);
     w.off_ctr = al256(w.off_cnt + sizeof(int) * h);
-    w.total = al256(w.off_ctr + sizeof(int) * (size_t)K);
+    w.off_cen = al256(w.off_ctr + sizeof(int) * (size_t)K);
+    w.total = al256(w.off_cen + kSeedCenBytes * h);
     return w;
 }
 
@@ -117,6 +124,7 @@ struct SeedArgs {
     unsigned char *taken;   // [H][N] point already chosen
     int *cnt;               // [H] arrival counters
     int *ctr;               // [K] work counters of the rounds with dynamic chunks
+    unsigned char *cen;     // [H][kSeedCenBytes] the last chosen centre (see seed_write_centre)
     int N, K, NR1, NR2, DSTRIDE, NBMAX;
     size_t CAP;
 };
@@ -396,6 +404,31 @@ __device__ __forceinline__ void q8_vector(const T *__restrict__ v, int lane, flo
     err = __double2float_ru(sqrt(ee) * (1.0 + kSeedMargin));
 }
 
+// Warp-wide: write the record of centre pk of a head (its row, then the int8
+// copy the anchor test uses) for the next round, which then reads one record
+// instead of the centre's index and then its row.  Out of line, like the
+// refresh below, so that the round kernels' own code stays as it was.
+template <typename T, int D>
+__device__ __noinline__ void seed_write_centre(const T *__restrict__ xh, int pk, unsigned char *rec, int lane) {
+    constexpr int L8 = Q8<D>::L8, U = 16 * (int)sizeof(T) / 16;  // uint4 per lane's 16 elements
+    float sc, ec;
+    uint4 qc;
+    int n2;
+    q8_vector<T, D>(xh + (size_t)pk * D, lane, sc, qc, n2, ec);
+    if (lane < L8) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(xh + (size_t)pk * D + lane * 16);
+        uint4 *dst = reinterpret_cast<uint4 *>(rec) + lane * U;
+#pragma unroll
+        for (int k = 0; k < U; ++k) dst[k] = __ldg(src + k);
+        reinterpret_cast<uint4 *>(rec + kSeedCenCodes)[lane] = qc;
+    }
+    if (lane == 0) {
+        reinterpret_cast<float *>(rec + kSeedCenScal)[0] = sc;
+        reinterpret_cast<int *>(rec + kSeedCenScal)[1] = n2;
+        reinterpret_cast<float *>(rec + kSeedCenScal)[2] = ec;
+    }
+}
+
 // The refresh with every S1 and S2 sum of the head cached in shared memory
 // (s1c [NR1], s2c [NR2]): one round of loads brings the flags and all sums,
 // the flagged S1 sums are recomputed from D2 and the S2 sums above them from
@@ -481,9 +514,10 @@ __device__ __noinline__ void seed_refresh_cached(double *b1, double *b2, unsigne
 // sums are loaded once, together with the flags, and the refresh and the
 // scans read them from there (the same values in the same order, so the same
 // pick, with fewer dependent trips to L2).
-template <bool REFRESH>
-__device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r, int arrivals, int *dl,
-                                                 uint32_t *sd2, double *cache = nullptr, int cache_n = 0) {
+template <bool REFRESH, typename T, int D>
+__device__ __forceinline__ void seed_arrive_pick(const T *__restrict__ x, const SeedArgs &s, int h, int r,
+                                                 int arrivals, int *dl, uint32_t *sd2, double *cache = nullptr,
+                                                 int cache_n = 0) {
     __shared__ double sh[kSeedWarps];
     __shared__ int nlist, last, pick_blk;
     __shared__ double sh_base;
@@ -504,13 +538,18 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
     if (!last) return;
 
     const double ur = s.u[(size_t)h * K + r];
+    const T *xh = x + hN * D;
+    unsigned char *rec = s.cen + (size_t)h * kSeedCenBytes;
     if (r == 0) {
-        if (tid == 0) {
+        if (warp == 0) {
             int pk = (int)floor(ur * (double)N);
             pk = min(max(pk, 0), N - 1);
-            s.idx[(size_t)h * K] = pk;
-            tk[pk] = 1;
-            s.cnt[h] = 0;
+            if (lane == 0) {
+                s.idx[(size_t)h * K] = pk;
+                tk[pk] = 1;
+                s.cnt[h] = 0;
+            }
+            seed_write_centre<T, D>(xh, pk, rec, lane);
         }
         return;
     }
@@ -623,6 +662,12 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
                     const bool exact1 = cr1 != 0u;
                     const int i = (k2 * kSeedS + l1) * kSeedS + lane;
                     const double v0 = i < N ? __ldcg(d2h + i) : 0.0;
+                    if (i < N) {
+                        // the candidates' rows into L1, for the centre record
+#pragma unroll
+                        for (int ln = 0; ln < D * (int)sizeof(T) / 128; ++ln)
+                            asm volatile("prefetch.global.L1 [%0];" ::"l"(xh + (size_t)i * D + ln * (128 / sizeof(T))));
+                    }
                     const double inc0 = warp_scan_d(v0, lane);
                     const unsigned cr0 = exact1 ? __ballot_sync(0xffffffffu, i < N && b1x + inc0 > thr) : 0u;
                     const unsigned pos0 = __ballot_sync(0xffffffffu, v0 > 0.0);
@@ -662,11 +707,14 @@ __device__ __forceinline__ void seed_arrive_pick(const SeedArgs &s, int h, int r
         if (tid == 0 && pick_blk == 0x7fffffff) pick_blk = 0;
         __syncthreads();
     }
-    if (tid == 0) {
+    if (warp == 0) {
         const int pk = pick_blk;
-        s.idx[(size_t)h * K + r] = pk;
-        tk[pk] = 1;
-        s.cnt[h] = 0;
+        if (lane == 0) {
+            s.idx[(size_t)h * K + r] = pk;
+            tk[pk] = 1;
+            s.cnt[h] = 0;
+        }
+        seed_write_centre<T, D>(xh, pk, rec, lane);
     }
 }
 
@@ -684,8 +732,8 @@ __device__ __forceinline__ void seed_full_range(const T *__restrict__ x, const S
     const T *xh = x + hN * D;
     double *d2h = s.d2 + hN;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = s.idx[(size_t)h * K + r - 1];
-    const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + (lane % Gm::LPP) * Gm::E16));
+    // the previous round's centre, from its record
+    const uint4 craw = __ldcg(reinterpret_cast<const uint4 *>(s.cen + (size_t)h * kSeedCenBytes) + lane % Gm::LPP);
     double cv[Gm::E16];
     float cvf[Gm::E16];
     widen16<T>(craw, cv);
@@ -693,6 +741,7 @@ __device__ __forceinline__ void seed_full_range(const T *__restrict__ x, const S
     (void)cvf;
     const int q = seed_row<T, D>(lane);
     double *b1 = s.bs1 + (size_t)h * s.NR1;
+    (void)K;
     const int k0 = p0 / kSeedS, k1 = (p1 + kSeedS - 1) / kSeedS;
     for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
         const int qp = base + lane;
@@ -773,7 +822,7 @@ kmeanspp_round_full(const T *__restrict__ x, const SeedArgs s, int r, int ch) {
     } else {
         seed_full_range<T, D, SCREEN>(x, s, h, r, p0, p1, s1own);
     }
-    seed_arrive_pick<false>(s, h, r, gridDim.x, nullptr, nullptr);
+    seed_arrive_pick<false, T, D>(x, s, h, r, gridDim.x, nullptr, nullptr);
 }
 
 // The same rounds (r >= 1) with the work handed out dynamically: the grid is
@@ -801,7 +850,7 @@ kmeanspp_round_full_dyn(const T *__restrict__ x, const SeedArgs s, int r, int H)
         if (threadIdx.x == 0) next_item = atomicAdd(&s.ctr[r], 1);
         const int h = it / nch, p0 = (it - h * nch) * kChunk;
         seed_full_range<T, D, SCREEN>(x, s, h, r, p0, min(N, p0 + kChunk), s1own);
-        seed_arrive_pick<false>(s, h, r, nch, nullptr, nullptr);
+        seed_arrive_pick<false, T, D>(x, s, h, r, nch, nullptr, nullptr);
         __syncthreads();
         it = next_item;
     }
@@ -874,16 +923,17 @@ kmeanspp_round_grouped(const T *__restrict__ x, const SeedArgs s, int r, int G, 
     if (!pre) stage();
     if (tid == 0) na = 0;
 
-    const int c = s.idx[hK + r - 1];
-    const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)c * D + (lane % Gm::LPP) * Gm::E16));
+    // the previous round's centre and its int8 copy, from its record
+    const unsigned char *cenr = s.cen + (size_t)h * kSeedCenBytes;
+    const uint4 craw = __ldcg(reinterpret_cast<const uint4 *>(cenr) + lane % Gm::LPP);
     double cv[Gm::E16];
     float cvf[Gm::E16];
     widen16<T>(craw, cv);
     widen16f<T>(craw, cvf);
-    float sc, ec;
-    uint4 qc;
-    int nqc;
-    q8_vector<T, D>(xh + (size_t)c * D, lane, sc, qc, nqc, ec);
+    const uint4 qc = __ldcg(reinterpret_cast<const uint4 *>(cenr + kSeedCenCodes) + lane % L8);
+    const float sc = __ldcg(reinterpret_cast<const float *>(cenr + kSeedCenScal));
+    const int nqc = __ldcg(reinterpret_cast<const int *>(cenr + kSeedCenScal) + 1);
+    const float ec = __ldcg(reinterpret_cast<const float *>(cenr + kSeedCenScal) + 2);
     __syncthreads();  // na cleared
 
     // triangle test of each piece, then its positions into the active list
@@ -955,7 +1005,7 @@ kmeanspp_round_grouped(const T *__restrict__ x, const SeedArgs s, int r, int G, 
     for (int j = tid; j < P; j += kSeedThreads)
         if (act[j]) s.pm[rec + j] = __uint_as_float(pmax[j]);
     // the piece lists (alist, pmax: 8 ch bytes) hold the S1 and S2 sums in the pick
-    seed_arrive_pick<true>(s, h, r, gridDim.x, pperm, reinterpret_cast<uint32_t *>(act),
+    seed_arrive_pick<true, T, D>(x, s, h, r, gridDim.x, pperm, reinterpret_cast<uint32_t *>(act),
                            reinterpret_cast<double *>(alist), ch);
 }
 
@@ -1465,6 +1515,7 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
     s.taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
     s.cnt = reinterpret_cast<int *>(b + w.off_cnt);
     s.ctr = reinterpret_cast<int *>(b + w.off_ctr);
+    s.cen = reinterpret_cast<unsigned char *>(b + w.off_cen);
     s.N = N;
     s.K = K;
     s.NR1 = w.nr1;
