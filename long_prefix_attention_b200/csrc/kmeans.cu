@@ -63,10 +63,21 @@ constexpr int kSeedCenCodes = 512, kSeedCenScal = 640;
 struct SeedWs {
     size_t off_d2, off_bs1, off_bs2, off_r2, off_gs, off_ge, off_gr, off_gn, off_near, off_perm, off_gcnt, off_seg,
         off_cur, off_pg, off_pm, off_plo, off_phi, off_pcnt, off_gq, off_dirty, off_taken, off_cnt, off_ctr, off_cen,
-        total;
-    int nr1, nr2, dstride, nbmax;
+        off_skey, off_anc, off_aws, total;
+    int nr1, nr2, dstride, nbmax, anchors;
     size_t cap;
 };
+// Anchors of the static groups that prune the rounds before the first
+// grouping by chosen centres (0: none).  Every (N / A)-th point is an anchor;
+// each point joins its nearest anchor (tensor-core assignment), so the
+// groups need the bf16 d = 128 assignment kernel and enough rounds before
+// the first regrouping (from round 2 to max(256, K / 8)) to pay for
+// themselves.
+int seed_static_anchors(int N, int d, int K) {
+    if (d != 128 || K < 512 || N < 8192) return 0;
+    return std::min(4096, std::min(K / 2, N / 16));
+}
+
 SeedWs seed_ws(int H, int N, int d, int K) {
     const size_t h = (size_t)H, n = (size_t)N, k = (size_t)K;
     SeedWs w;
@@ -100,7 +111,13 @@ SeedWs seed_ws(int H, int N, int d, int K) {
     w.off_cnt = al256(w.off_taken + h * n);
     w.off_ctr = al256(w.off_cnt + sizeof(int) * h);
     w.off_cen = al256(w.off_ctr + sizeof(int) * (size_t)K);
-    w.total = al256(w.off_cen + kSeedCenBytes * h);
+    // the static anchor groups of the early rounds (bf16, d = 128 only)
+    w.anchors = seed_static_anchors(N, d, K);
+    const size_t a = (size_t)w.anchors;
+    w.off_skey = al256(w.off_cen + kSeedCenBytes * h);
+    w.off_anc = al256(w.off_skey + (a ? sizeof(int) * h * n : 0));
+    w.off_aws = al256(w.off_anc + 2 * h * a * (size_t)d);
+    w.total = al256(w.off_aws + (a ? asm_kmeans_ws_bytes(H, N, d, w.anchors) : 0));
     return w;
 }
 
@@ -125,6 +142,10 @@ struct SeedArgs {
     int *cnt;               // [H] arrival counters
     int *ctr;               // [K] work counters of the rounds with dynamic chunks
     unsigned char *cen;     // [H][kSeedCenBytes] the last chosen centre (see seed_write_centre)
+    int32_t *skey;          // [H][N] nearest static anchor of each point
+    void *anc;              // [H][A][D] the static anchors' rows
+    void *aws;              // workspace of the assignment to the anchors
+    int A;                  // static anchors (0: none)
     int N, K, NR1, NR2, DSTRIDE, NBMAX;
     size_t CAP;
 };
@@ -1026,23 +1047,98 @@ __global__ void seed_group_hist(const SeedArgs s, int G) {
               (unsigned long long)__double_as_longlong(s.d2[hi]));
 }
 
-__global__ void seed_group_scatter(const SeedArgs s, int G) {
+// key: the group of each point ([H][N]: the nearest chosen centre, or the
+// nearest static anchor)
+__global__ void seed_group_scatter(const SeedArgs s, int G, const int32_t *__restrict__ key) {
     const int h = blockIdx.y, i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= s.N) return;
     const size_t hN = (size_t)h * s.N;
-    const int g = s.near[hN + i];
+    const int g = key[hN + i];
     const int pos = atomicAdd(&s.cur[(size_t)h * G + g], 1);
     s.perm[hN + pos] = i;
 }
 
-// One warp per group: int8 anchor, scale, |codes|^2, error and R.
+// Static groups: the anchors' rows (point j N / A of each head), gathered
+// for the assignment.
 template <typename T, int D>
-__global__ void seed_group_anchor(const T *__restrict__ x, const SeedArgs s, int G) {
+__global__ void seed_gather_anchors(const T *__restrict__ x, const SeedArgs s) {
+    const int h = blockIdx.y, j = blockIdx.x, A = s.A;
+    const int ai = (int)((long long)j * s.N / A);
+    const T *src = x + ((size_t)h * s.N + ai) * D;
+    T *dst = static_cast<T *>(s.anc) + ((size_t)h * A + j) * D;
+    for (int e = threadIdx.x; e < D; e += blockDim.x) dst[e] = src[e];
+}
+
+// |row - its anchor|^2 (fp64) of the 32 rows load32 read into buf, whose
+// anchors' rows (loaded the same way) are in abuf: lane l ends with row
+// seed_row(l).
+template <typename T, int D>
+__device__ __forceinline__ double dist32_pair(const uint4 (&buf)[SeedGeo<T, D>::LPP],
+                                              const uint4 (&abuf)[SeedGeo<T, D>::LPP], int lane) {
+    using G = SeedGeo<T, D>;
+    double part[G::LPP];
+#pragma unroll
+    for (int i = 0; i < G::LPP; ++i) {
+        double xv[G::E16], av[G::E16];
+        widen16<T>(buf[i], xv);
+        widen16<T>(abuf[i], av);
+        double acc = 0.0;
+#pragma unroll
+        for (int e = 0; e < G::E16; ++e) {
+            const double t = xv[e] - av[e];
+            acc = fma(t, t, acc);
+        }
+        part[i] = acc;
+    }
+#pragma unroll
+    for (int n = G::LPP; n > 1; n >>= 1) {
+        const int half = n >> 1;
+        const bool up = (lane & half) != 0;
+#pragma unroll
+        for (int k = 0; k < half; ++k) {
+            const double send = up ? part[k] : part[k + half];
+            const double keep = up ? part[k + half] : part[k];
+            part[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+    }
+    return part[0];
+}
+
+// Static groups: member counts and R^2 = the largest |x - anchor|^2 (fp64)
+// of each group, 32 points per warp.
+template <typename T, int D>
+__global__ void seed_group_hist_static(const T *__restrict__ x, const SeedArgs s) {
+    const int h = blockIdx.y, N = s.N, A = s.A, lane = threadIdx.x & 31;
+    const int base = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32;
+    if (base >= N) return;
+    const size_t hN = (size_t)h * N;
+    const T *xh = x + hN * D;
+    const int i = base + lane;
+    const unsigned m = __ballot_sync(0xffffffffu, i < N);
+    const int g = i < N ? s.skey[hN + i] : 0;
+    const int ai = (int)((long long)g * N / A);
+    uint4 buf[SeedGeo<T, D>::LPP], abuf[SeedGeo<T, D>::LPP];
+    load32<T, D, true>(xh, i, m, lane, buf);
+    load32<T, D, false>(xh, ai, m, lane, abuf);
+    const double d2 = dist32_pair<T, D>(buf, abuf, lane);
+    const int q = seed_row<T, D>(lane);
+    const int gq = __shfl_sync(0xffffffffu, g, q);  // this lane's distance is point base + q's
+    if ((m >> q) & 1u) {
+        atomicAdd(&s.gcnt[(size_t)h * A + gq], 1);
+        atomicMax(reinterpret_cast<unsigned long long *>(s.r2 + (size_t)h * A + gq),
+                  (unsigned long long)__double_as_longlong(d2));
+    }
+}
+
+// One warp per group: int8 anchor, scale, |codes|^2, error and R.  The
+// anchor is chosen centre g, or with static groups the point g N / G.
+template <typename T, int D>
+__global__ void seed_group_anchor(const T *__restrict__ x, const SeedArgs s, int G, int is_static) {
     const int h = blockIdx.y, lane = threadIdx.x & 31;
     const int g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (g >= G) return;
     const size_t hK = (size_t)h * s.K;
-    const int ai = s.idx[hK + g];
+    const int ai = is_static ? (int)((long long)g * s.N / G) : s.idx[hK + g];
     float sc, err;
     uint4 codes;
     int n2;
@@ -1057,8 +1153,11 @@ __global__ void seed_group_anchor(const T *__restrict__ x, const SeedArgs s, int
 }
 
 // One block per range of ch positions: the non-empty parts of the groups
-// overlapping it, in group order, with M = R to start.
-__global__ void seed_group_pieces(const SeedArgs s, int G, int ch) {
+// overlapping it, in group order, with M = R to start (centre groups: R is
+// the largest sqrt(D2) of the group), or M = +inf (static groups, whose
+// radius says nothing of D2: the first round over them visits every piece
+// and records its M).
+__global__ void seed_group_pieces(const SeedArgs s, int G, int ch, int is_static) {
     const int h = blockIdx.y, b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int p0 = b * ch, p1 = min(s.N, p0 + ch);
     const int *seg = s.seg + (size_t)h * (G + 1);
@@ -1101,7 +1200,7 @@ __global__ void seed_group_pieces(const SeedArgs s, int G, int ch) {
             s.pg[rec + off] = g;
             s.plo[rec + off] = (uint16_t)(lo - p0);
             s.phi[rec + off] = (uint16_t)(hi - p0);
-            s.pm[rec + off] = s.gr[hK + g];
+            s.pm[rec + off] = is_static ? __int_as_float(0x7f800000) : s.gr[hK + g];
         }
         __syncthreads();
         if (tid == 0) {
@@ -1455,8 +1554,29 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
     const dim3 pgrid((N + 255) / 256, H);
     const dim3 gfull((N + chf - 1) / chf, H), ggrp((N + chg - 1) / chg, H);
     int G = 0, next = std::max(256, K / 8);
+    const int sstart = std::max(2, next / 3);
     for (int r = 0; r < K; ++r) {
         int pre = 1;
+        if (r == sstart && s.A > 0 && next > sstart) {
+            // static groups for the last two thirds of the rounds before the
+            // first regrouping (earlier, most points still move each round
+            // and the full update is cheaper): each point joins its nearest
+            // of A anchors (every (N / A)-th point); R is the exact largest
+            // distance to the anchor, M starts at +inf
+            const int A = s.A;
+            G = A;
+            pre = 0;
+            seed_gather_anchors<T, D><<<dim3(A, H), 128, 0, st>>>(x, s);
+            if ((e = asm_kmeans_assign_launch(x, s.anc, H, N, D, A, 0, ASM_BF16, s.skey, s.aws, 0, st)) != cudaSuccess)
+                return e;
+            if ((e = cudaMemsetAsync(s.gcnt, 0, sizeof(int) * (size_t)H * A, st)) != cudaSuccess) return e;
+            if ((e = cudaMemsetAsync(s.r2, 0, sizeof(double) * (size_t)H * A, st)) != cudaSuccess) return e;
+            seed_group_hist_static<T, D><<<dim3((N + 255) / 256, H), 256, 0, st>>>(x, s);
+            scan_kernel<<<H, 1024, 0, st>>>(s.gcnt, A, s.seg, s.cur);
+            seed_group_scatter<<<pgrid, 256, 0, st>>>(s, A, s.skey);
+            seed_group_anchor<T, D><<<dim3((A + 7) / 8, H), 256, 0, st>>>(x, s, A, 1);
+            seed_group_pieces<<<ggrp, kSeedThreads, 0, st>>>(s, A, chg, 1);
+        }
         if (r == next) {
             // regroup by the nearest of the r - 1 centres applied so far;
             // then again each time the centres grow by a quarter of the
@@ -1467,9 +1587,9 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
             if ((e = cudaMemsetAsync(s.r2, 0, sizeof(double) * (size_t)H * G, st)) != cudaSuccess) return e;
             seed_group_hist<<<pgrid, 256, 0, st>>>(s, G);
             scan_kernel<<<H, 1024, 0, st>>>(s.gcnt, G, s.seg, s.cur);
-            seed_group_scatter<<<pgrid, 256, 0, st>>>(s, G);
-            seed_group_anchor<T, D><<<dim3((G + 7) / 8, H), 256, 0, st>>>(x, s, G);
-            seed_group_pieces<<<ggrp, kSeedThreads, 0, st>>>(s, G, chg);
+            seed_group_scatter<<<pgrid, 256, 0, st>>>(s, G, s.near);
+            seed_group_anchor<T, D><<<dim3((G + 7) / 8, H), 256, 0, st>>>(x, s, G, 0);
+            seed_group_pieces<<<ggrp, kSeedThreads, 0, st>>>(s, G, chg, 0);
             int p2 = 1;
             while (p2 * 2 <= r) p2 *= 2;
             next = r + std::max(256, p2 / 4);
@@ -1516,6 +1636,10 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
     s.cnt = reinterpret_cast<int *>(b + w.off_cnt);
     s.ctr = reinterpret_cast<int *>(b + w.off_ctr);
     s.cen = reinterpret_cast<unsigned char *>(b + w.off_cen);
+    s.A = (dt == ASM_BF16) ? w.anchors : 0;
+    s.skey = reinterpret_cast<int32_t *>(b + w.off_skey);
+    s.anc = b + w.off_anc;
+    s.aws = b + w.off_aws;
     s.N = N;
     s.K = K;
     s.NR1 = w.nr1;
