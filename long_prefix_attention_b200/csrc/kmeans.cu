@@ -71,8 +71,8 @@ struct SeedWs {
 // grouping by chosen centres (0: none).  Every (N / A)-th point is an anchor;
 // each point joins its nearest anchor (tensor-core assignment), so the
 // groups need the bf16 d = 128 assignment kernel and enough rounds before
-// the first regrouping (from round 2 to max(256, K / 8)) to pay for
-// themselves.
+// the first regrouping to pay for themselves.  At the build shape 4096
+// anchors gave 239.7 ms of seeding, 2048 and 8192 both 246.8.
 int seed_static_anchors(int N, int d, int K) {
     if (d != 128 || K < 512 || N < 8192) return 0;
     return std::min(4096, std::min(K / 2, N / 16));
@@ -1553,16 +1553,20 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
     const int N = s.N, K = s.K;
     const dim3 pgrid((N + 255) / 256, H);
     const dim3 gfull((N + chf - 1) / chf, H), ggrp((N + chg - 1) / chg, H);
-    int G = 0, next = std::max(256, K / 8);
-    const int sstart = std::max(2, next / 3);
+    // first regrouping by centres at 3K/16 (at least 256); static groups from
+    // a third of max(256, K/8) (measured at the build shape: regrouping at
+    // 1024, 1280, 1536, 1792 or 2048 gave 239.8, 232.1, 229.0, 229.9 and
+    // 231.9 ms; static groups from round 256, 341 or 448: 230.6, 229.0, 229.5)
+    int G = 0, next = std::max(256, (3 * K) / 16);
+    const int sstart = std::max(2, std::max(256, K / 8) / 3);
     for (int r = 0; r < K; ++r) {
         int pre = 1;
         if (r == sstart && s.A > 0 && next > sstart) {
-            // static groups for the last two thirds of the rounds before the
-            // first regrouping (earlier, most points still move each round
-            // and the full update is cheaper): each point joins its nearest
-            // of A anchors (every (N / A)-th point); R is the exact largest
-            // distance to the anchor, M starts at +inf
+            // static groups until the first regrouping by centres (earlier,
+            // most points still move each round and the full update is
+            // cheaper): each point joins its nearest of A anchors (every
+            // (N / A)-th point); R is the exact largest distance to the
+            // anchor, M starts at +inf
             const int A = s.A;
             G = A;
             pre = 0;
