@@ -131,8 +131,11 @@ asm_status asm_merge_states(void *a_acc, float *logz_acc, const void *a_in,
  * Requires 1 <= K <= N; N > 2^24 returns ASM_ERR_UNSUPPORTED.  The update
  * skips groups of points that the triangle inequality shows cannot move (a
  * work saving only: the D2 values and picks are those of the full update).
- * One kernel launch per round, plus a regrouping (three small launches) on
- * a schedule; the launches are queued on `stream` without synchronising.
+ * The groups are, first, the points nearest to each of a fixed set of
+ * anchor points (bf16, d = 128, from a third of max(256, K/8) rounds), then
+ * the points nearest to each chosen centre (from 3K/16 rounds, regrouped on
+ * a schedule).  One kernel launch per round, plus a few launches at each
+ * regrouping; all are queued on `stream` without synchronising.
  */
 size_t asm_kmeanspp_workspace_size(int H, int N, int d, int K);
 asm_status asm_kmeanspp_seed(const void *x, int H, int N, int d, int K,
