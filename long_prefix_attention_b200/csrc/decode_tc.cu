@@ -646,7 +646,6 @@ asm_decode_merge(const Args a) {
     const int nslots = a.nP + a.nA;
     const bool search = a.mode != 1;  // a memory lookup (flat or two-level) precedes the merge
     pdl_wait();
-    pdl_launch_dependents();
     // ---- round 1: the centroid scores, the attention maxima, and each
     //      thread's first kMergeSlots partials
     float2 best = make_float2(kNegInf, __int_as_float(0x7fffffff));
@@ -696,6 +695,10 @@ asm_decode_merge(const Args a) {
     }
     const int idx = sidx;
     const float M = sM;
+    // The next kernel may start now: its prefetch stream (the next step's
+    // units warm L2 before their dependency wait) then queues behind this
+    // kernel's first round of loads instead of ahead of them.
+    pdl_launch_dependents();
     // ---- round 2: the retrieved state (issued before the weighted sums)
     float zb2 = kNegInf, ab = 0.f;
     if (search && sg == 0) {
