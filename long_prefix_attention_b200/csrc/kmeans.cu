@@ -1559,6 +1559,11 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
     // 231.9 ms; static groups from round 256, 341 or 448: 230.6, 229.0, 229.5)
     int G = 0, next = std::max(256, (3 * K) / 16);
     const int sstart = std::max(2, std::max(256, K / 8) / 3);
+    // no regrouping after round K/4: more groups mean more pieces to test in
+    // every round, which cost more than the finer groups save (last
+    // regrouping at 1792, 2048, 2560, 3072, 4096 or 7168: 220.2, 219.1,
+    // 220.4, 221.6, 224.5 and 228.8 ms)
+    const int last = std::max(next, K / 4);
     for (int r = 0; r < K; ++r) {
         int pre = 1;
         if (r == sstart && s.A > 0 && next > sstart) {
@@ -1584,7 +1589,8 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
         if (r == next) {
             // regroup by the nearest of the r - 1 centres applied so far;
             // then again each time the centres grow by a quarter of the
-            // largest power of two below r (at least 256 rounds apart)
+            // largest power of two below r (at least 256 rounds apart), up
+            // to round `last`
             G = r - 1;
             pre = 0;
             if ((e = cudaMemsetAsync(s.gcnt, 0, sizeof(int) * (size_t)H * G, st)) != cudaSuccess) return e;
@@ -1596,7 +1602,7 @@ cudaError_t seed_all(const T *x, SeedArgs &s, int H, cudaStream_t st) {
             seed_group_pieces<<<ggrp, kSeedThreads, 0, st>>>(s, G, chg, 0);
             int p2 = 1;
             while (p2 * 2 <= r) p2 *= 2;
-            next = r + std::max(256, p2 / 4);
+            next = r >= last ? K : r + std::max(256, p2 / 4);
         }
         if (G > 0) e = seed_launch(kmeanspp_round_grouped<T, D>, ggrp, seed_grouped_smem(chg), st, x, s, r, G, pre, chg);
         else if (r == 0) e = seed_launch(kmeanspp_round_full<T, D, false>, gfull, 0, st, x, s, r, chf);
