@@ -130,12 +130,16 @@ def test_kmeanspp_llama_build_config_prefix():
 
 
 @pytest.mark.parametrize("dt,d,N,K", [("bf16", 128, 8192, 1024), ("f32", 64, 5000, 600),
-                                       ("bf16", 64, 3001, 520), ("f32", 128, 2500, 300)])
+                                       ("bf16", 64, 3001, 520), ("f32", 128, 2500, 300),
+                                       ("bf16", 128, 9001, 600)])
 def test_kmeanspp_pruned_rounds_match_the_oracle(dt, d, N, K):
-    """Past round 256 the D2 update skips groups of points that the triangle
+    """From round 256 the D2 update skips groups of points that the triangle
     inequality shows cannot move; the picks are those of the full update.
     Clustered data (so that most groups are skipped), ragged N, both storage
-    types and head dims, several regroupings."""
+    types and head dims, several regroupings.  The bf16 d = 128 cases with
+    N >= 8192 and K >= 512 also run the static anchor groups before round
+    256 (K = 1024: 512 anchors from round 85; N = 9001, K = 600: 300 anchors,
+    ragged, from round 85)."""
     x = inputs.mixture(inputs.BASE_SEED + 40 + d, "seed_q", 2, N, d, 48, 0.3, dt)
     u = inputs.kmeanspp_uniforms(inputs.BASE_SEED + 41 + N, 2, K)
     idx = gpu_seed(dev(x), dev(u))
