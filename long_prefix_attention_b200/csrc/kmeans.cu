@@ -72,7 +72,8 @@ struct SeedWs {
 // each point joins its nearest anchor (tensor-core assignment), so the
 // groups need the bf16 d = 128 assignment kernel and enough rounds before
 // the first regrouping to pay for themselves.  At the build shape 4096
-// anchors gave 239.7 ms of seeding, 2048 and 8192 both 246.8.
+// anchors gave 228.8 ms of seeding, 3072 235.6 and 6144 228.9 (earlier, with
+// the first regrouping at round 1024: 4096 239.7, 2048 and 8192 246.8).
 int seed_static_anchors(int N, int d, int K) {
     if (d != 128 || K < 512 || N < 8192) return 0;
     return std::min(4096, std::min(K / 2, N / 16));
