@@ -861,7 +861,7 @@ def run_decode_large(cfg, layers, steps, warmup, world, rank, hbm, src):
            "ms_per_step": secs * 1e3 / steps, "gpu_launches": steps * layers * launches,
            "device_error_word": err,
            "roofline": decode_roofline(byt, per * 1e6, hbm, src, recorded_traffic(cfg["name"]),
-                                       "asm_decode_step = asm_decode_units<128,4> + asm_decode_merge<128>")}
+                                       "asm_decode_step = asm_decode_units<128,4> + asm_decode_merge<128,32>")}
     del bufs
     torch.cuda.empty_cache()
     return out
@@ -984,7 +984,7 @@ def main():
     per_launch_s = secs / (args.steps * args.layers)  # one decode step (both kernels) of one layer
     roofline = decode_roofline(stack.bytes_per_launch(), per_launch_s * 1e6, hbm, peak_src,
                                recorded_traffic(cfg["name"]),
-                               "asm_decode_step = asm_decode_units<128,4> + asm_decode_merge<128>")
+                               "asm_decode_step = asm_decode_units<128,4> + asm_decode_merge<128,16>")
 
     # end to end through the public API: every step copies that step's queries
     # from pinned host memory and reads its outputs back.  "graph": the layer

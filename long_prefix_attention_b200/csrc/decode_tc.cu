@@ -619,18 +619,19 @@ asm_index_select(const Args a) {
 // ----------------------------------------------------------- merge kernel --
 //
 // One CTA per (b, h) of SG x D threads: thread (sg, t) owns output dim t of
-// the attention partials sg, sg + SG, ...; it keeps kMergeSlots of them in
-// flight per round.  SG grows with the partial count (1 for up to 32 partials,
-// up to 8 for 256 and more), so a long local window or prefix does not turn
-// the merge into a serial loop.
+// the attention partials sg, sg + SG, ...; it keeps SLOTS of them in flight
+// per round.  SG grows with the partial count (16 or 32 partials per
+// thread, up to SG = 8), so a long local window or prefix does not turn the
+// merge into a serial loop.
 
-constexpr int kMergeSlots = 32;  // partial rows a thread keeps in flight
+constexpr int kMergeSlots = 32;  // partial rows a thread keeps in flight per round (at most)
 constexpr int kMergeMaxSG = 8;   // slot groups per CTA (up to 8 x D threads)
 constexpr int kMergeSml = 2048;  // (m, l) pairs staged in shared memory
 
-template <int D>
+template <int D, int SLOTS>
 __global__ void __launch_bounds__(kMergeMaxSG * D)
 asm_decode_merge(const Args a) {
+    static_assert(SLOTS <= kMergeSlots, "slots per round");
     const int bh = blockIdx.x;
     const int b = bh / a.Hq, h = bh - b * a.Hq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -647,7 +648,7 @@ asm_decode_merge(const Args a) {
     const bool search = a.mode != 1;  // a memory lookup (flat or two-level) precedes the merge
     pdl_wait();
     // ---- round 1: the centroid scores, the attention maxima, and each
-    //      thread's first kMergeSlots partials
+    //      thread's first SLOTS partials
     float2 best = make_float2(kNegInf, __int_as_float(0x7fffffff));
     if (search) {
         for (int s = tid; s < a.nS; s += NT) {
@@ -657,9 +658,9 @@ asm_decode_merge(const Args a) {
     }
     const float2 *mlp = a.ws_ml + (size_t)bh * nslots;
     const float *op = a.ws_o + (size_t)bh * nslots * D + t;
-    float ov[kMergeSlots];
+    float ov[SLOTS];
 #pragma unroll
-    for (int k = 0; k < kMergeSlots; ++k) {
+    for (int k = 0; k < SLOTS; ++k) {
         const int s = sg + SG * k;
         ov[k] = s < nslots ? __ldcg(op + (size_t)s * D) : 0.f;
     }
@@ -707,17 +708,17 @@ asm_decode_merge(const Args a) {
     }
     float L = 0.f, o = 0.f;
     if (M != kNegInf) {
-        for (int k0 = 0;; k0 += kMergeSlots) {
+        for (int k0 = 0;; k0 += SLOTS) {
             if (k0 > 0) {
                 if (sg + SG * k0 >= nslots) break;
 #pragma unroll
-                for (int k = 0; k < kMergeSlots; ++k) {
+                for (int k = 0; k < SLOTS; ++k) {
                     const int s = sg + SG * (k0 + k);
                     ov[k] = s < nslots ? __ldcg(op + (size_t)s * D) : 0.f;
                 }
             }
 #pragma unroll
-            for (int k = 0; k < kMergeSlots; ++k) {
+            for (int k = 0; k < SLOTS; ++k) {
                 const int s = sg + SG * (k0 + k);
                 if (s >= nslots) break;
                 const float2 ml = s < kMergeSml ? sml[s] : __ldcg(mlp + s);
@@ -727,7 +728,7 @@ asm_decode_merge(const Args a) {
                     o = fmaf(w, ov[k], o);
                 }
             }
-            if (sg + SG * (k0 + kMergeSlots) >= nslots) break;
+            if (sg + SG * (k0 + SLOTS) >= nslots) break;
         }
     }
     // slot groups meet in shared memory
@@ -830,16 +831,24 @@ cudaError_t tc_launch(tc::Args a, const void *centroids, const void *k_prefix, c
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t c2 = {};
-    // slot groups of the merge: one per 32 partials, at most kMergeMaxSG
+    // slot groups of the merge, at most kMergeMaxSG
     const int nslots = a.nP + a.nA;
     int sg = 1;
-    while (sg < tc::kMergeMaxSG && sg * tc::kMergeSlots < nslots) sg *= 2;
+    // With few (b, h) pairs (at most 128 merge CTAs) and partials that fit
+    // one round at 16 per thread, each thread takes 16, so the CTAs grow and
+    // each thread's dependent chain of weighted sums is short (LLaMA layer,
+    // B = 1: 9.6 against 10.3 us per step); otherwise 32 per round, so that
+    // the CTAs stay small or the rounds few.
+    const bool short_rounds = a.B * a.Hq <= 128 && nslots <= 16 * tc::kMergeMaxSG;
+    const int per = short_rounds ? 16 : tc::kMergeSlots;
+    while (sg < tc::kMergeMaxSG && sg * per < nslots) sg *= 2;
     c2.gridDim = dim3(a.B * a.Hq);
     c2.blockDim = dim3(sg * D);
     c2.stream = st;
     c2.attrs = attr;
     c2.numAttrs = 1;
-    return cudaLaunchKernelEx(&c2, tc::asm_decode_merge<D>, a);
+    return short_rounds ? cudaLaunchKernelEx(&c2, tc::asm_decode_merge<D, 16>, a)
+                        : cudaLaunchKernelEx(&c2, tc::asm_decode_merge<D, tc::kMergeSlots>, a);
 }
 
 template <int D>
