@@ -775,10 +775,10 @@ def x_bytes(H, N, d):
 # capture of this benchmark), with the digest of the kernel source they were
 # taken on: a changed kernel reports null until it is measured again.
 TRAFFIC = {
-    "llama31-8b-layer-decode-K1024-T2048-B1": {  # units 16 943 424 + merge 585 696
-        "bytes": 17529120, "source": "7597e35a875e3520"},
-    "llama31-8b-layer-decode-K8192-T4096-B16": {  # units 356 926 720 + merge 17 531 776
-        "bytes": 374458496, "source": "7597e35a875e3520"},
+    "llama31-8b-layer-decode-K1024-T2048-B1": {  # units 16 943 872 + merge 577 504
+        "bytes": 17521376, "source": "34fb8ab3bad75454"},
+    "llama31-8b-layer-decode-K8192-T4096-B16": {  # units 356 988 672 + merge 17 535 872
+        "bytes": 374524544, "source": "34fb8ab3bad75454"},
 }
 TRAFFIC_SOURCE = os.path.join(ROOT, "long_prefix_attention_b200", "csrc", "decode_tc.cu")
 
