@@ -230,6 +230,111 @@ void oracle_kmeanspp_seed(const double *X, int H, int N, int d, int K,
 }
 
 /*
+ * Batched k-means++ seeding (the batched seeding of k-means|| by Bahmani et
+ * al. 2012, without its final reclustering; the pages leave the seeding
+ * open).  Rounds draw up to b centres at once from the same D2 distribution
+ * and only then update D2, so K centres take about K / b rounds instead of K.
+ *   u[U]: uniform draws in [0,1), consumed in order (draw p uses u[p % U]).
+ *   round 0: the point floor(u[0] * N).
+ *   round r >= 1, with m centres chosen: nb = min(b, K - m) draws; draw j
+ *            takes the smallest i whose running sum of D2 (index order)
+ *            exceeds u_j * sum(D2), or the last point with D2 > 0 if none
+ *            does; if sum(D2) == 0, draw j takes the j-th smallest index not
+ *            yet chosen.  A draw equal to an earlier draw of the same round
+ *            is dropped.  The kept draws are appended in draw order, then
+ *            D2_i = min(D2_i, |x_i - c|^2) over them.
+ *   after ceil((K - 1) / b) + 16 rounds the remaining centres, if any, are
+ *   the smallest indices not yet chosen.
+ * With b = 1 this is oracle_kmeanspp_seed with u[r] for round r.
+ */
+static void kmeanspp_batched_one(const double *X, int N, int d, int K, int b,
+                                 const double *u, int U, int32_t *idx)
+{
+    double *D2 = (double *)malloc(sizeof(double) * (size_t)N);
+    unsigned char *taken = (unsigned char *)calloc((size_t)N, 1);
+    int32_t *batch = (int32_t *)malloc(sizeof(int32_t) * (size_t)(b > 0 ? b : 1));
+    int i, j, q, m = 0, p = 0, round, cap = (K - 1 + b - 1) / b + 16;
+    for (i = 0; i < N; i++) D2[i] = INFINITY;
+    {
+        int first = (int)floor(u[p % U] * (double)N);
+        p++;
+        if (first >= N) first = N - 1;
+        if (first < 0) first = 0;
+        idx[m++] = first;
+        taken[first] = 1;
+        for (i = 0; i < N; i++) {
+            double t = sqdist(X + (size_t)i * d, X + (size_t)first * d, d);
+            if (t < D2[i]) D2[i] = t;
+        }
+    }
+    for (round = 1; m < K && round <= cap; round++) {
+        int nb = K - m < b ? K - m : b, kept = 0;
+        double total = 0.0;
+        for (i = 0; i < N; i++) total += D2[i];
+        for (j = 0; j < nb; j++) {
+            int pick = -1;
+            double uj = u[p % U];
+            p++;
+            if (total > 0.0) {
+                double thr = uj * total, run = 0.0;
+                int last_pos = -1;
+                for (i = 0; i < N; i++) {
+                    run += D2[i];
+                    if (D2[i] > 0.0) last_pos = i;
+                    if (run > thr) {
+                        pick = i;
+                        break;
+                    }
+                }
+                if (pick < 0) pick = last_pos;
+            } else {
+                int seen = 0;
+                for (i = 0; i < N; i++)
+                    if (!taken[i]) {
+                        if (seen == j) {
+                            pick = i;
+                            break;
+                        }
+                        seen++;
+                    }
+                if (pick < 0) pick = 0;
+            }
+            for (q = 0; q < kept; q++)
+                if (batch[q] == pick) break;
+            if (q == kept) batch[kept++] = pick;
+        }
+        for (q = 0; q < kept; q++) {
+            idx[m++] = batch[q];
+            taken[batch[q]] = 1;
+        }
+        for (i = 0; i < N; i++)
+            for (q = 0; q < kept; q++) {
+                double t = sqdist(X + (size_t)i * d, X + (size_t)batch[q] * d, d);
+                if (t < D2[i]) D2[i] = t;
+            }
+    }
+    for (i = 0; m < K && i < N; i++)
+        if (!taken[i]) {
+            idx[m++] = i;
+            taken[i] = 1;
+        }
+    free(D2);
+    free(taken);
+    free(batch);
+}
+
+/* X[H,N,d], u[H,U] -> idx[H,K] (batched seeding, b draws per round). */
+void oracle_kmeanspp_seed_batched(const double *X, int H, int N, int d, int K,
+                                  int b, const double *u, int U, int32_t *idx)
+{
+    int h;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (h = 0; h < H; h++)
+        kmeanspp_batched_one(X + (size_t)h * N * d, N, d, K, b, u + (size_t)h * U, U,
+                             idx + (size_t)h * K);
+}
+
+/*
  * Nearest centre of each point ("Agrupamiento" bullet for k-means; the
  * "Recuperacion" bullet for the decode-time lookup).
  *   metric 0 (L2):     argmin_c |x - c|^2, computed as the squared distance.

@@ -58,6 +58,7 @@ def _load():
         lib.oracle_merge.argtypes = [P, D, P, D, I, P, P]
         lib.oracle_build_states.argtypes = [P, P, P, I, I, I, I, I, D, I, P, P]
         lib.oracle_kmeanspp_seed.argtypes = [P, I, I, I, I, P, P]
+        lib.oracle_kmeanspp_seed_batched.argtypes = [P, I, I, I, I, I, P, I, P]
         lib.oracle_assign.argtypes = [P, P, I, I, I, I, P, P]
         lib.oracle_update.argtypes = [P, P, I, I, I, P, P, P]
         lib.oracle_round_storage.argtypes = [P, ctypes.c_long, I, P]
@@ -138,6 +139,17 @@ def kmeanspp_seed(X, u):
     K = u.shape[1]
     idx = np.zeros((H, K), dtype=np.int32)
     _load().oracle_kmeanspp_seed(_p(X), H, N, d, K, _p(u), _p(idx))
+    return idx
+
+
+def kmeanspp_seed_batched(X, u, K: int, b: int):
+    """Batched k-means++ seed indices [H,K] of X[H,N,d]: up to b draws per
+    round from the same D2 distribution (uniform draws u[H,U], in order)."""
+    X, u = _f64(X), _f64(u)
+    H, N, d = X.shape
+    U = u.shape[1]
+    idx = np.zeros((H, K), dtype=np.int32)
+    _load().oracle_kmeanspp_seed_batched(_p(X), H, N, d, int(K), int(b), _p(u), U, _p(idx))
     return idx
 
 

@@ -186,6 +186,71 @@ def test_kmeanspp_all_duplicate_points():
     assert idx.tolist() == [3, 0, 1, 2]
 
 
+# ------------------------------------------------- batched k-means++ ------
+
+@pytest.mark.parametrize("dup", [False, True])
+def test_kmeanspp_batched_one_draw_per_round_is_kmeanspp(dup):
+    """b = 1: one draw per round, D2 updated after each, is k-means++ itself
+    (clustered points, and points repeated so that sum(D2) reaches 0)."""
+    g = np.random.default_rng(31 + dup)
+    base = g.standard_normal((2, 40, 6))
+    X = np.concatenate([base, base], axis=1) if dup else g.standard_normal((2, 80, 6))
+    K = 60
+    u = g.random((2, K))
+    np.testing.assert_array_equal(O.kmeanspp_seed_batched(X, u, K, 1), O.kmeanspp_seed(X, u))
+
+
+def test_kmeanspp_batched_hand_case_with_a_repeated_draw():
+    """Four points on a line at 0, 1, 10, 11, K = 3, two draws per round.
+    Round 0: u = 0 takes point 0; D2 = 0, 1, 100, 121 (sum 222).  Round 1:
+    both draws are 0.5 -> thresholds 111: the running sums 0, 1, 101, 222
+    first exceed it at point 3, twice, so the second draw is dropped.  D2
+    becomes 0, 1, 1, 0 (sum 2).  Round 2 (one centre left): u = 0.75 ->
+    threshold 1.5, first exceeded at point 2 (running sum 2)."""
+    X = np.array([[[0.0], [1.0], [10.0], [11.0]]])
+    u = np.array([[0.0, 0.5, 0.5, 0.75]])
+    assert O.kmeanspp_seed_batched(X, u, 3, 2)[0].tolist() == [0, 3, 2]
+
+
+def test_kmeanspp_batched_all_duplicates_take_the_smallest_unchosen():
+    """Six equal points: round 0 takes floor(0.6 * 6) = 3, then sum(D2) = 0 and
+    the three draws of round 1 take the 1st, 2nd and 3rd smallest unchosen
+    indices."""
+    X = np.ones((1, 6, 4))
+    u = np.array([[0.6, 0.9, 0.1, 0.5]])
+    assert O.kmeanspp_seed_batched(X, u, 4, 3)[0].tolist() == [3, 0, 1, 2]
+
+
+def test_kmeanspp_batched_k_equals_n_is_a_permutation():
+    g = np.random.default_rng(33)
+    N = 50
+    X = g.standard_normal((1, N, 3))
+    u = g.random((1, 2 * N))
+    idx = O.kmeanspp_seed_batched(X, u, N, 8)[0]
+    assert idx[0] == int(u[0, 0] * N)
+    assert sorted(idx.tolist()) == list(range(N))
+
+
+def test_kmeanspp_batched_first_round_draws_follow_d2():
+    """All draws of round 1 come from the same D2 distribution (the round-0
+    centre's): over a fine grid of u, the picks of each draw position hit
+    point i in proportion to D2_i (repeats within a round dropped only when
+    two draws hit the same point, which a grid of distinct u spreads out)."""
+    g = np.random.default_rng(34)
+    N, d, M, b = 9, 3, 4000, 4
+    X = g.standard_normal((N, d))
+    first = 4
+    D2 = cdist(X, X[first:first + 1], "sqeuclidean")[:, 0]
+    p = D2 / D2.sum()
+    grid = (np.arange(M) + 0.5) / M
+    # case m: K = b + 1, so round 1 makes b draws, all equal to grid[m]: they
+    # hit the same point and the round keeps one, the inverse CDF of grid[m]
+    u = np.concatenate([np.full((M, 1), (first + 0.5) / N), np.repeat(grid[:, None], b, axis=1)], axis=1)
+    picks = O.kmeanspp_seed_batched(np.broadcast_to(X, (M, N, d)), u, b + 1, b)[:, 1]
+    counts = np.bincount(picks, minlength=N)
+    np.testing.assert_allclose(counts / M, p, atol=2.0 / M)
+
+
 # ---------------------------------------------------------------- assign ----
 
 @pytest.mark.parametrize("metric", [O.L2, O.COSINE])
