@@ -138,6 +138,38 @@ asm_status asm_merge_states(void *a_acc, float *logz_acc, const void *a_in,
  * regrouping; all are queued on `stream` without synchronising.
  */
 size_t asm_kmeanspp_workspace_size(int H, int N, int d, int K);
+
+/*
+ * asm_kmeanspp_seed_batched -- batched k-means++ seeding: each round draws
+ * up to `batch` centres from the same D2 distribution and only then updates
+ * D2 (the batched seeding of k-means||, Bahmani et al. 2012, without its
+ * reclustering), so K centres take about K / batch rounds instead of K.  It
+ * changes the seeds: with batch = 1 it is asm_kmeanspp_seed.
+ *   round 0: point floor(u[h,0] * N).  Round r: nb = min(batch, K - m) draws
+ *   (m centres chosen), draw j taking the smallest i whose running sum of D2
+ *   (index order) exceeds u_j * sum(D2) (the last point with D2 > 0 if
+ *   rounding leaves none; the j-th smallest unchosen index if sum(D2) = 0); a
+ *   draw equal to an earlier one of the same round is dropped; the kept
+ *   draws are appended in draw order; then D2_i = min(D2_i, |x_i - c|^2)
+ *   over them.  After ceil((K - 1) / batch) + 16 rounds any remaining
+ *   centres are the smallest unchosen indices.  D2 is exact fp64 to the
+ *   centre the tensor-core (bf16, d = 128) or CUDA-core assignment finds
+ *   nearest among the round's centres.
+ *   x        [H, N, d] dt   points
+ *   u        [H, U]    fp64 uniform draws in [0, 1), consumed in order
+ *                           (draw p of a head uses u[h, p % U])
+ *   init_idx [H, K]    int32 output
+ *   ws       asm_kmeanspp_batched_workspace_size(H, N, d, K, batch) bytes;
+ *            its word 0 is the error word (asm_workspace_error)
+ * Requires 1 <= K <= N, 1 <= batch <= 256, U >= 1; N > 2^21 returns
+ * ASM_ERR_UNSUPPORTED.  Four launches per round; synchronises `stream`
+ * once, after about K / batch rounds, to see whether repeated draws left
+ * any head short.
+ */
+size_t asm_kmeanspp_batched_workspace_size(int H, int N, int d, int K, int batch);
+asm_status asm_kmeanspp_seed_batched(const void *x, int H, int N, int d, int K, int batch,
+                                     const double *u, int U, asm_dtype dt, int32_t *init_idx,
+                                     void *ws, size_t ws_bytes, cudaStream_t stream);
 asm_status asm_kmeanspp_seed(const void *x, int H, int N, int d, int K,
                              const double *u, asm_dtype dt, int32_t *init_idx,
                              void *ws, size_t ws_bytes, cudaStream_t stream);

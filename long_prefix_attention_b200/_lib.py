@@ -22,6 +22,8 @@ SIGNATURES = {
     "asm_merge_states": (I, [P, P, P, P, ctypes.c_int64, I, I, P]),
     "asm_kmeanspp_workspace_size": (SZ, [I, I, I, I]),
     "asm_kmeanspp_seed": (I, [P, I, I, I, I, P, I, P, P, SZ, P]),
+    "asm_kmeanspp_batched_workspace_size": (SZ, [I, I, I, I, I]),
+    "asm_kmeanspp_seed_batched": (I, [P, I, I, I, I, I, P, I, I, P, P, SZ, P]),
     "asm_kmeans_assign": (I, [P, P, I, I, I, I, I, I, P, P, SZ, P]),
     "asm_kmeans_update": (I, [P, P, I, I, I, I, I, P, P, P, P, P, P, SZ, P]),
     "asm_kmeans_workspace_size": (SZ, [I, I, I, I]),

@@ -106,6 +106,21 @@ asm_status asm_kmeanspp_seed(const void *x, int H, int N, int d, int K, const do
     return cuda_status(asm_kmeanspp_launch(x, H, N, d, K, u, dt, init_idx, ws, stream));
 }
 
+size_t asm_kmeanspp_batched_workspace_size(int H, int N, int d, int K, int batch) {
+    if (H < 1 || N < 1 || K < 1 || batch < 1 || batch > 256 || !d_ok(d)) return 0;
+    return asm_kmeanspp_batched_ws_bytes(H, N, d, K, batch);
+}
+
+asm_status asm_kmeanspp_seed_batched(const void *x, int H, int N, int d, int K, int batch, const double *u,
+                                     int U, asm_dtype dt, int32_t *init_idx, void *ws, size_t ws_bytes,
+                                     cudaStream_t stream) {
+    if (!dt_ok(dt) || H < 1 || N < 1 || K < 1 || K > N || batch < 1 || U < 1) return ASM_ERR_INVALID_ARG;
+    if (!d_ok(d) || batch > 256 || N > (1 << 21)) return ASM_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(u, 8) || !aligned(init_idx, 4)) return ASM_ERR_INVALID_ARG;
+    if (!aligned(ws, 16) || ws_bytes < asm_kmeanspp_batched_ws_bytes(H, N, d, K, batch)) return ASM_ERR_WORKSPACE;
+    return cuda_status(asm_kmeanspp_batched_launch(x, H, N, d, K, batch, u, U, dt, init_idx, ws, stream));
+}
+
 size_t asm_kmeans_workspace_size(int H, int N, int d, int K) {
     if (H < 1 || N < 1 || K < 1) return 0;
     return asm_kmeans_ws_bytes(H, N, d, K);

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <vector>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -1214,6 +1215,296 @@ __global__ void seed_group_pieces(const SeedArgs s, int G, int ch, int is_static
     if (tid == 0) s.pcnt[(size_t)h * s.NBMAX + b] = base;
 }
 
+// ================================================ batched k-means++ seeding ==
+//
+// Up to b draws per round from one D2 distribution, repeats within a round
+// dropped, then one D2 update with all the round's centres (the batched
+// seeding of k-means||, Bahmani et al. 2012, without its reclustering): about
+// K / b rounds instead of K.  A round is four launches: the pick (one CTA per
+// head: the draws' inverse-CDF searches over the S2 / S1 / point sums), the
+// norms and the nearest-centre assignment of every point to the round's
+// centres (the tensor-core assignment for bf16, d = 128), and the update
+// (D2 = min(D2, exact fp64 distance to the assigned centre) and the S1 / S2
+// sums of each 1024-position range, in index order).  Heads that have all K
+// centres skip their work.
+
+struct BSeedArgs {
+    const double *u;        // [H][U] draws
+    int32_t *idx;           // [H][K] picks
+    double *d2;             // [H][N]
+    double *bs1, *bs2;      // [H][NR1], [H][NR2] sums of D2 (index order)
+    unsigned char *taken;   // [H][N]
+    int *st;                // [H][4]: centres chosen, draws used, kept this round
+    int32_t *key;           // [H][N] nearest centre of the round
+    void *cb;               // [H][B][D] the round's centres (storage type)
+    int *err;
+    int N, K, B, U, NR1, NR2;
+};
+
+// Round 0: the point floor(u * N) of each head, and D2 to it.
+template <typename T, int D>
+__global__ void __launch_bounds__(kSeedThreads)
+bseed_first(const T *__restrict__ x, const BSeedArgs a) {
+    using Gm = SeedGeo<T, D>;
+    const int h = blockIdx.y, N = a.N, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const size_t hN = (size_t)h * N;
+    const T *xh = x + hN * D;
+    int first = (int)floor(a.u[(size_t)h * a.U] * (double)N);
+    first = min(max(first, 0), N - 1);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        a.idx[(size_t)h * a.K] = first;
+        a.taken[hN + first] = 1;
+        a.st[4 * h] = 1;
+        a.st[4 * h + 1] = 1;
+        a.st[4 * h + 2] = 0;
+    }
+    const uint4 craw = __ldg(reinterpret_cast<const uint4 *>(xh + (size_t)first * D + (lane % Gm::LPP) * Gm::E16));
+    double cv[Gm::E16];
+    widen16<T>(craw, cv);
+    const int q = seed_row<T, D>(lane);
+    const int base = (blockIdx.x * kSeedWarps + warp) * 32;
+    if (base >= N) return;
+    const int i = base + lane;
+    const unsigned m = __ballot_sync(0xffffffffu, i < N);
+    uint4 buf[Gm::LPP];
+    load32<T, D, true>(xh, i, m, lane, buf);
+    const double dist = dist32<T, D>(buf, cv, lane);
+    if ((m >> q) & 1u) a.d2[hN + base + q] = dist;
+}
+
+// S1 sums (32 points) and S2 sums (32 S1 sums) of every head, index order.
+__global__ void __launch_bounds__(kSeedThreads)
+bseed_sums(const BSeedArgs a) {
+    const int h = blockIdx.y, N = a.N;
+    const double *d2h = a.d2 + (size_t)h * N;
+    __shared__ double s1[kSeedThreads];
+    const int k = blockIdx.x * kSeedThreads + threadIdx.x;  // S1 range
+    double v = 0.0;
+    if (k < a.NR1) {
+        const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
+        for (int i = q0; i < q1; ++i) v += __ldcg(d2h + i);
+        a.bs1[(size_t)h * a.NR1 + k] = v;
+    }
+    s1[threadIdx.x] = v;
+    __syncthreads();
+    if (threadIdx.x < kSeedThreads / kSeedS) {
+        const int k2 = blockIdx.x * (kSeedThreads / kSeedS) + threadIdx.x;
+        if (k2 < a.NR2) {
+            double w = 0.0;
+            const int k0 = k2 * kSeedS, k1 = min(a.NR1, k0 + kSeedS);
+            for (int kk = k0; kk < k1; ++kk) w += s1[kk - blockIdx.x * kSeedThreads];
+            a.bs2[(size_t)h * a.NR2 + k2] = w;
+        }
+    }
+}
+
+constexpr int kBSeedMaxB = kSeedThreads;        // draws per round (one per thread)
+constexpr int kBSeedMaxNR2 = 2048;              // S2 prefix in shared memory (N <= 2^21)
+
+// Inverse CDF of one draw (threshold thr in (0, total)): the S2 range whose
+// prefix first exceeds thr, then the S1 range, then the point, each a running
+// sum in index order from the range's base; where rounding keeps a range's
+// running sum at or below thr, its last element with positive mass is taken.
+__device__ int bseed_search(const BSeedArgs &a, int h, const double *P2, double thr) {
+    const int NR1 = a.NR1, NR2 = a.NR2, N = a.N;
+    const double *b1 = a.bs1 + (size_t)h * NR1;
+    const double *b2 = a.bs2 + (size_t)h * NR2;
+    const double *d2h = a.d2 + (size_t)h * N;
+    int lo = 0, hi = NR2;  // first k2 with P2[k2] > thr (NR2 if none)
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (P2[mid] > thr) hi = mid; else lo = mid + 1;
+    }
+    int k2 = lo;
+    bool exact = k2 < NR2;
+    if (!exact) {  // the last S2 range with positive mass
+        k2 = NR2 - 1;
+        while (k2 > 0 && !(__ldcg(b2 + k2) > 0.0)) --k2;
+    }
+    double run = k2 > 0 ? P2[k2 - 1] : 0.0;
+    const int s0 = k2 * kSeedS, s1 = min(NR1, s0 + kSeedS);
+    double t[kSeedS];
+#pragma unroll
+    for (int e = 0; e < kSeedS; ++e) t[e] = s0 + e < s1 ? __ldcg(b1 + s0 + e) : 0.0;
+    int k1 = -1, lastpos = -1;
+#pragma unroll
+    for (int e = 0; e < kSeedS; ++e) {
+        if (k1 < 0 && s0 + e < s1) {
+            if (t[e] > 0.0) lastpos = e;
+            if (exact && run + t[e] > thr) k1 = e; else run += t[e];
+        }
+    }
+    if (k1 < 0) {
+        exact = false;
+        k1 = lastpos < 0 ? 0 : lastpos;
+    }
+    const int q0 = (s0 + k1) * kSeedS, q1 = min(N, q0 + kSeedS);
+#pragma unroll
+    for (int e = 0; e < kSeedS; ++e) t[e] = q0 + e < q1 ? __ldcg(d2h + q0 + e) : 0.0;
+    int pick = -1;
+    lastpos = -1;
+#pragma unroll
+    for (int e = 0; e < kSeedS; ++e) {
+        if (pick < 0 && q0 + e < q1) {
+            if (t[e] > 0.0) lastpos = e;
+            if (exact && run + t[e] > thr) pick = e; else run += t[e];
+        }
+    }
+    if (pick < 0) pick = lastpos < 0 ? 0 : lastpos;
+    return q0 + pick;
+}
+
+// One CTA per head: the round's draws, repeats dropped, the kept centres
+// appended to the picks and gathered for the assignment (the unused slots
+// repeat the first kept centre, which changes no minimum).
+template <typename T, int D>
+__global__ void __launch_bounds__(kSeedThreads)
+bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
+    const int h = blockIdx.x, N = a.N, K = a.K, B = a.B, tid = threadIdx.x;
+    const size_t hN = (size_t)h * N;
+    __shared__ double P2[kBSeedMaxNR2];
+    __shared__ int picks[kBSeedMaxB], keep[kBSeedMaxB], pos[kBSeedMaxB], slotpick[kBSeedMaxB], nkept;
+    __shared__ double total_s;
+    int *st = a.st + 4 * h;
+    const int m = st[0], p = st[1];
+    if (m >= K) {
+        if (tid == 0) st[2] = 0;
+        return;
+    }
+    const int nb = min(B, K - m);
+    for (int k = tid; k < a.NR2; k += kSeedThreads) P2[k] = __ldcg(a.bs2 + (size_t)h * a.NR2 + k);
+    __syncthreads();
+    if (tid == 0) {
+        double r = 0.0;
+        for (int k = 0; k < a.NR2; ++k) {
+            r += P2[k];
+            P2[k] = r;
+        }
+        total_s = r;
+    }
+    __syncthreads();
+    const double total = total_s;
+    for (int j = tid; j < nb; j += kSeedThreads) {
+        const double uj = a.u[(size_t)h * a.U + (p + j) % a.U];
+        int pick;
+        if (total > 0.0) {
+            pick = bseed_search(a, h, P2, uj * total);
+        } else {
+            // every remaining point coincides with a centre: the j-th
+            // smallest index not yet chosen
+            pick = 0;
+            int seen = 0;
+            for (int i = 0; i < N; ++i)
+                if (!a.taken[hN + i]) {
+                    if (seen == j) {
+                        pick = i;
+                        break;
+                    }
+                    ++seen;
+                }
+        }
+        picks[j] = pick;
+    }
+    __syncthreads();
+    for (int j = tid; j < nb; j += kSeedThreads) {
+        int k = 1;
+        for (int j2 = 0; j2 < j; ++j2)
+            if (picks[j2] == picks[j]) k = 0;
+        keep[j] = k;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int c = 0;
+        for (int j = 0; j < nb; ++j) {
+            pos[j] = c;
+            c += keep[j];
+        }
+        nkept = c;
+        st[0] = m + c;
+        st[1] = p + nb;
+        st[2] = c;
+    }
+    __syncthreads();
+    for (int j = tid; j < nb; j += kSeedThreads)
+        if (keep[j]) {
+            a.idx[(size_t)h * K + m + pos[j]] = picks[j];
+            a.taken[hN + picks[j]] = 1;
+            slotpick[pos[j]] = picks[j];
+        }
+    __syncthreads();
+    // the round's centres, then copies of the first one
+    const int kept = nkept;
+    constexpr int C16 = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
+    uint4 *cbh = reinterpret_cast<uint4 *>(static_cast<T *>(a.cb) + (size_t)h * B * D);
+    for (int w = tid; w < B * C16; w += kSeedThreads) {
+        const int slot = w / C16, c = w - slot * C16;
+        const int src = slot < kept ? slotpick[slot] : picks[0];
+        cbh[w] = __ldg(reinterpret_cast<const uint4 *>(x + (hN + src) * D) + c);
+    }
+}
+
+// D2 = min(D2, |x - the assigned centre of the round|^2) (exact fp64), then
+// the S1 and S2 sums of this 1024-position range from the registers.
+template <typename T, int D>
+__global__ void __launch_bounds__(kSeedThreads)
+bseed_update(const T *__restrict__ x, const BSeedArgs a) {
+    using Gm = SeedGeo<T, D>;
+    const int h = blockIdx.y, N = a.N, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (a.st[4 * h + 2] == 0) return;  // no centre this round: D2 and sums stand
+    const size_t hN = (size_t)h * N;
+    const T *xh = x + hN * D;
+    const T *cbh = static_cast<const T *>(a.cb) + (size_t)h * a.B * D;
+    double *d2h = a.d2 + hN;
+    __shared__ double s1own[kSeedS];
+    const int p0 = blockIdx.x * kSeedS * kSeedS, p1 = min(N, p0 + kSeedS * kSeedS);
+    const int q = seed_row<T, D>(lane);
+    for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
+        const int i = base + lane;
+        const unsigned m = __ballot_sync(0xffffffffu, i < p1);
+        const int c = i < p1 ? min(max(a.key[hN + i], 0), a.B - 1) : 0;  // in range even after a give-up
+        uint4 buf[Gm::LPP], abuf[Gm::LPP];
+        load32<T, D, true>(xh, i, m, lane, buf);
+        load32<T, D, false>(cbh, c, m, lane, abuf);
+        const double dist = dist32_pair<T, D>(buf, abuf, lane);
+        const bool mine = (m >> q) & 1u;
+        double fin = mine ? d2h[base + q] : 0.0;
+        if (mine && dist < fin) {
+            fin = dist;
+            d2h[base + q] = dist;
+        }
+        double v = 0.0;
+#pragma unroll
+        for (int j = 0; j < kSeedS; ++j)
+            v += __shfl_sync(0xffffffffu, fin, (j % Gm::PPL) * Gm::LPP + j / Gm::PPL);
+        if (lane == 0) {
+            a.bs1[(size_t)h * a.NR1 + base / kSeedS] = v;
+            s1own[(base - p0) / kSeedS] = v;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int k0 = p0 / kSeedS, k1 = (p1 + kSeedS - 1) / kSeedS;
+        double v = 0.0;
+        for (int k = k0; k < k1; ++k) v += s1own[k - k0];
+        a.bs2[(size_t)h * a.NR2 + blockIdx.x] = v;
+    }
+}
+
+// After the last round: heads still short of K take the smallest indices not
+// yet chosen.
+__global__ void bseed_fill(const BSeedArgs a) {
+    const int h = blockIdx.x;
+    if (threadIdx.x != 0) return;
+    int m = a.st[4 * h];
+    const size_t hN = (size_t)h * a.N;
+    for (int i = 0; m < a.K && i < a.N; ++i)
+        if (!a.taken[hN + i]) {
+            a.idx[(size_t)h * a.K + m++] = i;
+            a.taken[hN + i] = 1;
+        }
+    a.st[4 * h] = m;
+}
+
 }  // namespace asmk
 
 // ============================================================ init / norms ==
@@ -1666,6 +1957,107 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
         return d == 128 ? seed_all<T, 128>((const T *)x, s, H, st) : seed_all<T, 64>((const T *)x, s, H, st);
     }
     return d == 128 ? seed_all<float, 128>((const float *)x, s, H, st) : seed_all<float, 64>((const float *)x, s, H, st);
+}
+
+// ---- batched seeding: workspace and the host loop of rounds
+namespace {
+struct BSeedWs {
+    size_t off_d2, off_bs1, off_bs2, off_taken, off_st, off_key, off_cb, off_aws, total;
+    int nr1, nr2;
+};
+BSeedWs bseed_ws(int H, int N, int d, int K, int B) {
+    (void)K;
+    const size_t h = (size_t)H, n = (size_t)N;
+    BSeedWs w;
+    w.nr1 = (N + kSeedS - 1) / kSeedS;
+    w.nr2 = (w.nr1 + kSeedS - 1) / kSeedS;
+    // the assignment's workspace first: its error word (word 0) is this one's
+    w.off_aws = 0;
+    w.off_d2 = al256(w.off_aws + asm_kmeans_ws_bytes(H, N, d, B));
+    w.off_bs1 = al256(w.off_d2 + sizeof(double) * h * n);
+    w.off_bs2 = al256(w.off_bs1 + sizeof(double) * h * w.nr1);
+    w.off_taken = al256(w.off_bs2 + sizeof(double) * h * w.nr2);
+    w.off_st = al256(w.off_taken + h * n);
+    w.off_key = al256(w.off_st + sizeof(int) * 4 * h);
+    w.off_cb = al256(w.off_key + sizeof(int32_t) * h * n);
+    w.total = al256(w.off_cb + sizeof(float) * h * (size_t)B * d);
+    return w;
+}
+
+template <typename T, int D>
+cudaError_t bseed_all(const T *x, BSeedArgs &a, int H, asm_dtype dt, void *aws, cudaStream_t st) {
+    const int N = a.N;
+    bseed_first<T, D><<<dim3((N + kSeedThreads - 1) / kSeedThreads, H), kSeedThreads, 0, st>>>(x, a);
+    bseed_sums<<<dim3((a.NR1 + kSeedThreads - 1) / kSeedThreads, H), kSeedThreads, 0, st>>>(a);
+    auto round = [&]() -> cudaError_t {
+        bseed_pick<T, D><<<H, kSeedThreads, 0, st>>>(x, a);
+        cudaError_t e = asm_kmeans_assign_launch(x, a.cb, H, N, D, a.B, 0, dt, a.key, aws, 0, st);
+        if (e != cudaSuccess) return e;
+        bseed_update<T, D><<<dim3(a.NR2, H), kSeedThreads, 0, st>>>(x, a);
+        return cudaGetLastError();
+    };
+    const int main_rounds = (a.K - 1 + a.B - 1) / a.B;
+    cudaError_t e = cudaGetLastError();
+    for (int r = 0; r < main_rounds && e == cudaSuccess; ++r) e = round();
+    if (e != cudaSuccess) return e;
+    // repeated draws leave a head short: up to 16 more rounds while any is
+    {
+        std::vector<int> hst(4 * (size_t)H);
+        for (int extra = 0; extra <= 16; ++extra) {
+            if ((e = cudaMemcpyAsync(hst.data(), a.st, sizeof(int) * 4 * (size_t)H, cudaMemcpyDeviceToHost, st)) !=
+                    cudaSuccess ||
+                (e = cudaStreamSynchronize(st)) != cudaSuccess)
+                return e;
+            bool short_ = false;
+            for (int h = 0; h < H; ++h) short_ |= hst[4 * (size_t)h] < a.K;
+            if (!short_) break;
+            if (extra == 16) {
+                bseed_fill<<<H, 32, 0, st>>>(a);
+                break;
+            }
+            if ((e = round()) != cudaSuccess) return e;
+        }
+    }
+    return cudaGetLastError();
+}
+}  // namespace
+
+size_t asm_kmeanspp_batched_ws_bytes(int H, int N, int d, int K, int batch) {
+    return bseed_ws(H, N, d, K, batch).total;
+}
+
+cudaError_t asm_kmeanspp_batched_launch(const void *x, int H, int N, int d, int K, int batch, const double *u,
+                                        int U, asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st) {
+    const BSeedWs w = bseed_ws(H, N, d, K, batch);
+    if (w.nr2 > kBSeedMaxNR2 || batch > kBSeedMaxB) return cudaErrorInvalidValue;
+    char *b = static_cast<char *>(ws);
+    BSeedArgs a{};
+    a.u = u;
+    a.idx = init_idx;
+    a.d2 = reinterpret_cast<double *>(b + w.off_d2);
+    a.bs1 = reinterpret_cast<double *>(b + w.off_bs1);
+    a.bs2 = reinterpret_cast<double *>(b + w.off_bs2);
+    a.taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
+    a.st = reinterpret_cast<int *>(b + w.off_st);
+    a.key = reinterpret_cast<int32_t *>(b + w.off_key);
+    a.cb = b + w.off_cb;
+    a.err = reinterpret_cast<int *>(b);
+    a.N = N;
+    a.K = K;
+    a.B = batch;
+    a.U = U;
+    a.NR1 = w.nr1;
+    a.NR2 = w.nr2;
+    cudaError_t e = cudaMemsetAsync(a.taken, 0, (size_t)H * N, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(b, 0, sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    if (dt == ASM_BF16) {
+        using T = __nv_bfloat16;
+        return d == 128 ? bseed_all<T, 128>((const T *)x, a, H, dt, b + w.off_aws, st)
+                        : bseed_all<T, 64>((const T *)x, a, H, dt, b + w.off_aws, st);
+    }
+    return d == 128 ? bseed_all<float, 128>((const float *)x, a, H, dt, b + w.off_aws, st)
+                    : bseed_all<float, 64>((const float *)x, a, H, dt, b + w.off_aws, st);
 }
 
 size_t asm_kmeans_ws_bytes(int H, int N, int d, int K) {

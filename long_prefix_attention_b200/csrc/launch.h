@@ -74,6 +74,9 @@ size_t asm_kmeans_ws_bytes(int H, int N, int d, int K);
 cudaError_t asm_kmeans_init_launch(const void *x, int H, int N, int d, int K, asm_dtype dt,
                                    const int32_t *init_idx, float *centroids, void *centroids_dt,
                                    cudaStream_t st);
+size_t asm_kmeanspp_batched_ws_bytes(int H, int N, int d, int K, int batch);
+cudaError_t asm_kmeanspp_batched_launch(const void *x, int H, int N, int d, int K, int batch, const double *u,
+                                        int U, asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st);
 cudaError_t asm_kmeans_assign_launch(const void *x, const void *centroids_dt, int H, int N, int d,
                                      int K, int metric, asm_dtype dt, int32_t *assign, void *ws,
                                      int num_sms, cudaStream_t st);

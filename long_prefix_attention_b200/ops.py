@@ -108,6 +108,22 @@ def asm_kmeanspp_seed(x, u, init_idx, ws, stream=None):
         _stream(stream)))
 
 
+def asm_kmeanspp_batched_workspace_size(H: int, N: int, d: int, K: int, batch: int) -> int:
+    return int(_lib.load().asm_kmeanspp_batched_workspace_size(H, N, d, K, batch))
+
+
+def asm_kmeanspp_seed_batched(x, u, init_idx, batch: int, ws, stream=None):
+    """Batched k-means++ indices init_idx[H,K] of x[H,N,d]: up to `batch`
+    draws per round from the same D2 distribution, draws u[H,U] (fp64) used
+    in order."""
+    _contig(x, u, init_idx)
+    H, N, d = x.shape
+    K = init_idx.shape[1]
+    _check("asm_kmeanspp_seed_batched", _lib.load().asm_kmeanspp_seed_batched(
+        _p(x), H, N, d, K, int(batch), _p(u), u.shape[1], _dt(x), _p(init_idx), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
 def asm_kmeans_workspace_size(H: int, N: int, d: int, K: int) -> int:
     return int(_lib.load().asm_kmeans_workspace_size(H, N, d, K))
 
