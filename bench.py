@@ -9,7 +9,7 @@ streams its bytes from HBM); the 32 layer steps (two kernels each) are
 replayed from a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl asm|reference]
-    python bench.py --only states|assign|seed|lloyd|aggregate [--steps K] [--warmup W]
+    python bench.py --only states|assign|seed|seed_batched|lloyd|aggregate [--steps K] [--warmup W]
     python bench.py --sweep [--steps K] [--warmup W]
     python bench.py --index [--steps K] [--warmup W]
     python bench.py --whiten [--steps K] [--warmup W]
@@ -332,6 +332,15 @@ def build_head_shard(Hq, Hkv, world, rank):
     return sharding.head_shard(Hq, Hkv, world, rank)
 
 
+SEED_BATCH = 128  # draws per round of the opt-in batched seeding
+
+
+def batched_seed_draws(H, K):
+    """Draws of the batched seeding: twice K per head, so that rounds that
+    drop repeated draws still use fresh ones."""
+    return inputs.kmeanspp_uniforms(inputs.BASE_SEED + 4, H, 2 * K)
+
+
 def run_build(cfg, with_cpu=True, world=1, rank=0):
     """Full offline build at the 32/8-head, N=65536, L=16384, K=8192 shape.
     With several ranks each builds its shard of the heads (heads are
@@ -345,8 +354,8 @@ def run_build(cfg, with_cpu=True, world=1, rank=0):
     if h1 == h0:  # nothing to build on this rank: it joins the same collectives
         for _ in range(2):
             barrier(world)  # the two stage_times() calls
-        for _ in range(4):
-            max_over_ranks(0.0, world)  # the four stage maxima
+        for _ in range(5):
+            max_over_ranks(0.0, world)  # the five stage maxima
         return None
     x, u = bi["q"][h0:h1].cuda(), bi["u"][h0:h1].cuda()
     k, v = bi["k"][h0 // G:h1 // G].cuda(), bi["v"][h0 // G:h1 // G].cuda()
@@ -364,6 +373,11 @@ def run_build(cfg, with_cpu=True, world=1, rank=0):
     perm = torch.empty(H, N, dtype=torch.int32, device="cuda")
     seg = torch.empty(H, K + 1, dtype=torch.int32, device="cuda")
     ws = ops.alloc_workspace(ops.asm_kmeans_workspace_size(H, N, d, K), "cuda", zero=False)
+    # the opt-in batched seeding (BATCH draws per round), timed beside the exact one
+    ub = batched_seed_draws(Htot, K)[h0:h1].cuda()
+    init_b = torch.empty(H, K, dtype=torch.int32, device="cuda")
+    ws_b = ops.alloc_workspace(ops.asm_kmeanspp_batched_workspace_size(H, N, d, K, SEED_BATCH), "cuda",
+                               zero=False)
     a_bar = torch.empty(H, K, d, dtype=x.dtype, device="cuda")
     lz_bar = torch.empty(H, K, dtype=torch.float32, device="cuda")
     cl = L // chunks
@@ -372,7 +386,7 @@ def run_build(cfg, with_cpu=True, world=1, rank=0):
 
     def stage_times():
         barrier(world)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
         ev[0].record()
         for i in range(chunks):
             ops.asm_build_states(x, kc[i], vc[i], bi["scale"], a, logz, accumulate=i > 0)
@@ -383,13 +397,16 @@ def run_build(cfg, with_cpu=True, world=1, rank=0):
         ev[3].record()
         ops.asm_aggregate(a, logz, perm, seg, a_bar, lz_bar)
         ev[4].record()
+        ops.asm_kmeanspp_seed_batched(x, ub, init_b, SEED_BATCH, ws_b)
+        ev[5].record()
         torch.cuda.synchronize()
-        return [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
+        return [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
 
     stage_times()  # warm-up
     t = stage_times()
     t = [max_over_ranks(x, world) for x in t]  # the slowest rank, stage by stage
-    total = sum(t)
+    total = sum(t[:4])
+    total_b = total - t[1] + t[4]
     hbm, tf, tfs, src = peaks()
     states_flops = 4.0 * N * L * d * Htot
     assign_flops = 2.0 * N * K * d * Htot * iters
@@ -399,7 +416,10 @@ def run_build(cfg, with_cpu=True, world=1, rank=0):
         "ranks": world, "heads_per_rank": H,
         "value": Htot * N / (total / 1e3), "unit": "queries/s",
         "ms": {"states_4chunks": t[0], "kmeanspp_seed": t[1], "lloyd_10": t[2], "aggregate": t[3],
-               "total": total},
+               "total": total, f"kmeanspp_seed_batched{SEED_BATCH}": t[4]},
+        f"value_with_batched{SEED_BATCH}_seeding": Htot * N / (total_b / 1e3),
+        "seeding": f"exact sequential k-means++ (value); batched, {SEED_BATCH} draws per round from one "
+                   f"D2 distribution (value_with_batched{SEED_BATCH}_seeding, opt-in)",
         "states_tflops": states_flops / (t[0] / 1e3) / 1e12,
         "states_frac_of_bf16_peak": states_flops / (t[0] / 1e3) / 1e12 / tf,
         "lloyd_assign_tflops_incl_update": assign_flops / (t[2] / 1e3) / 1e12,
@@ -457,6 +477,13 @@ def run_stage(name, steps, warmup):
             lz_bar = torch.empty(H, K, dtype=torch.float32, device="cuda")
             fn = lambda: ops.asm_aggregate(a, logz, perm, seg, a_bar, lz_bar)
             flops = None
+    elif name == "seed_batched":
+        u = batched_seed_draws(H, K).cuda()
+        init = torch.empty(H, K, dtype=torch.int32, device="cuda")
+        ws = ops.alloc_workspace(ops.asm_kmeanspp_batched_workspace_size(H, N, d, K, SEED_BATCH), "cuda",
+                                 zero=False)
+        fn = lambda: ops.asm_kmeanspp_seed_batched(x, u, init, SEED_BATCH, ws)
+        flops = None
     else:
         u = bi["u"].cuda()
         init = torch.empty(H, K, dtype=torch.int32, device="cuda")
@@ -890,7 +917,23 @@ def build_rooflines(build, tf, hbm, src):
                       "peak_source": f"{src} HBM copy", "bytes": agg_bytes},
         "kmeanspp_seed": {"bound": "sequential rounds", "rounds": K,
                           "us_per_round": ms["kmeanspp_seed"] * 1e3 / K},
+        f"kmeanspp_seed_batched{SEED_BATCH}": batched_seed_roofline(
+            ms[f"kmeanspp_seed_batched{SEED_BATCH}"], H, N, d, K, hbm, src),
     }
+
+
+def batched_seed_roofline(ms, H, N, d, K, hbm, src):
+    """Per round of the batched seeding: the assignment reads the points and
+    writes their nearest centre, the update reads the points, that index and
+    D2 and writes D2 back: H * N * (4 d + 24) bytes (the round's centres,
+    draws and range sums are negligible)."""
+    rounds = (K - 1 + SEED_BATCH - 1) // SEED_BATCH
+    per_round = H * N * (4 * d + 24)
+    us = ms * 1e3 / rounds
+    achieved = per_round / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "rounds": rounds, "us_per_round": us, "bytes_per_round": per_round,
+            "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "peak_source": f"{src} HBM copy"}
 
 
 def main():
@@ -906,7 +949,7 @@ def main():
     ap.add_argument("--no-prefetch", action="store_true",
                     help="do not let a layer's kernel stream its (static) centroids before the "
                          "preceding kernel finishes")
-    ap.add_argument("--only", choices=["states", "assign", "seed", "lloyd", "aggregate"],
+    ap.add_argument("--only", choices=["states", "assign", "seed", "seed_batched", "lloyd", "aggregate"],
                     help="time one build stage alone (single-kernel profiling) and exit")
     ap.add_argument("--index", action="store_true",
                     help="two-level (hierarchical) search against the flat search (time and recall) and exit")

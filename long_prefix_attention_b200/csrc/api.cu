@@ -118,7 +118,7 @@ asm_status asm_kmeanspp_seed_batched(const void *x, int H, int N, int d, int K, 
     if (!d_ok(d) || batch > 256 || N > (1 << 21)) return ASM_ERR_UNSUPPORTED;
     if (!aligned(x, 16) || !aligned(u, 8) || !aligned(init_idx, 4)) return ASM_ERR_INVALID_ARG;
     if (!aligned(ws, 16) || ws_bytes < asm_kmeanspp_batched_ws_bytes(H, N, d, K, batch)) return ASM_ERR_WORKSPACE;
-    return cuda_status(asm_kmeanspp_batched_launch(x, H, N, d, K, batch, u, U, dt, init_idx, ws, stream));
+    return cuda_status(asm_kmeanspp_batched_launch(x, H, N, d, K, batch, u, U, dt, init_idx, ws, num_sms(), stream));
 }
 
 size_t asm_kmeans_workspace_size(int H, int N, int d, int K) {

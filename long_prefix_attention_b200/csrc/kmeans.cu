@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <vector>
 #include <stdint.h>
 
@@ -1232,7 +1233,8 @@ struct BSeedArgs {
     const double *u;        // [H][U] draws
     int32_t *idx;           // [H][K] picks
     double *d2;             // [H][N]
-    double *bs1, *bs2;      // [H][NR1], [H][NR2] sums of D2 (index order)
+    double *bs1;            // [H][NR1] sums of D2 over 32-point ranges (index order)
+    float *xn;              // [H][N] |x|^2 (fp32), or null where no round uses it
     unsigned char *taken;   // [H][N]
     int *st;                // [H][4]: centres chosen, draws used, kept this round
     int32_t *key;           // [H][N] nearest centre of the round
@@ -1270,31 +1272,26 @@ bseed_first(const T *__restrict__ x, const BSeedArgs a) {
     load32<T, D, true>(xh, i, m, lane, buf);
     const double dist = dist32<T, D>(buf, cv, lane);
     if ((m >> q) & 1u) a.d2[hN + base + q] = dist;
+    if (a.xn != nullptr) {
+        double zero[Gm::E16];
+#pragma unroll
+        for (int e = 0; e < Gm::E16; ++e) zero[e] = 0.0;
+        const double nrm = dist32<T, D>(buf, zero, lane);
+        if ((m >> q) & 1u) a.xn[hN + base + q] = (float)nrm;
+    }
 }
 
-// S1 sums (32 points) and S2 sums (32 S1 sums) of every head, index order.
+// S1 sums (32 points) of every head, index order.
 __global__ void __launch_bounds__(kSeedThreads)
 bseed_sums(const BSeedArgs a) {
     const int h = blockIdx.y, N = a.N;
     const double *d2h = a.d2 + (size_t)h * N;
-    __shared__ double s1[kSeedThreads];
     const int k = blockIdx.x * kSeedThreads + threadIdx.x;  // S1 range
-    double v = 0.0;
     if (k < a.NR1) {
+        double v = 0.0;
         const int q0 = k * kSeedS, q1 = min(N, q0 + kSeedS);
         for (int i = q0; i < q1; ++i) v += __ldcg(d2h + i);
         a.bs1[(size_t)h * a.NR1 + k] = v;
-    }
-    s1[threadIdx.x] = v;
-    __syncthreads();
-    if (threadIdx.x < kSeedThreads / kSeedS) {
-        const int k2 = blockIdx.x * (kSeedThreads / kSeedS) + threadIdx.x;
-        if (k2 < a.NR2) {
-            double w = 0.0;
-            const int k0 = k2 * kSeedS, k1 = min(a.NR1, k0 + kSeedS);
-            for (int kk = k0; kk < k1; ++kk) w += s1[kk - blockIdx.x * kSeedThreads];
-            a.bs2[(size_t)h * a.NR2 + k2] = w;
-        }
     }
 }
 
@@ -1305,10 +1302,9 @@ constexpr int kBSeedMaxNR2 = 2048;              // S2 prefix in shared memory (N
 // prefix first exceeds thr, then the S1 range, then the point, each a running
 // sum in index order from the range's base; where rounding keeps a range's
 // running sum at or below thr, its last element with positive mass is taken.
-__device__ int bseed_search(const BSeedArgs &a, int h, const double *P2, double thr) {
+__device__ int bseed_search(const BSeedArgs &a, int h, const double *S2, const double *P2, double thr) {
     const int NR1 = a.NR1, NR2 = a.NR2, N = a.N;
     const double *b1 = a.bs1 + (size_t)h * NR1;
-    const double *b2 = a.bs2 + (size_t)h * NR2;
     const double *d2h = a.d2 + (size_t)h * N;
     int lo = 0, hi = NR2;  // first k2 with P2[k2] > thr (NR2 if none)
     while (lo < hi) {
@@ -1319,7 +1315,7 @@ __device__ int bseed_search(const BSeedArgs &a, int h, const double *P2, double 
     bool exact = k2 < NR2;
     if (!exact) {  // the last S2 range with positive mass
         k2 = NR2 - 1;
-        while (k2 > 0 && !(__ldcg(b2 + k2) > 0.0)) --k2;
+        while (k2 > 0 && !(S2[k2] > 0.0)) --k2;
     }
     double run = k2 > 0 ? P2[k2 - 1] : 0.0;
     const int s0 = k2 * kSeedS, s1 = min(NR1, s0 + kSeedS);
@@ -1362,7 +1358,7 @@ __global__ void __launch_bounds__(kSeedThreads)
 bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
     const int h = blockIdx.x, N = a.N, K = a.K, B = a.B, tid = threadIdx.x;
     const size_t hN = (size_t)h * N;
-    __shared__ double P2[kBSeedMaxNR2];
+    __shared__ double S2[kBSeedMaxNR2], P2[kBSeedMaxNR2];
     __shared__ int picks[kBSeedMaxB], keep[kBSeedMaxB], pos[kBSeedMaxB], slotpick[kBSeedMaxB], nkept;
     __shared__ double total_s;
     int *st = a.st + 4 * h;
@@ -1372,7 +1368,15 @@ bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
         return;
     }
     const int nb = min(B, K - m);
-    for (int k = tid; k < a.NR2; k += kSeedThreads) P2[k] = __ldcg(a.bs2 + (size_t)h * a.NR2 + k);
+    // S2 sums (32 S1 sums each, index order) and their prefix
+    const double *b1 = a.bs1 + (size_t)h * a.NR1;
+    for (int k = tid; k < a.NR2; k += kSeedThreads) {
+        const int k0 = k * kSeedS, k1 = min(a.NR1, k0 + kSeedS);
+        double w = 0.0;
+        for (int kk = k0; kk < k1; ++kk) w += __ldcg(b1 + kk);
+        S2[k] = w;
+        P2[k] = w;
+    }
     __syncthreads();
     if (tid == 0) {
         double r = 0.0;
@@ -1388,7 +1392,7 @@ bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
         const double uj = a.u[(size_t)h * a.U + (p + j) % a.U];
         int pick;
         if (total > 0.0) {
-            pick = bseed_search(a, h, P2, uj * total);
+            pick = bseed_search(a, h, S2, P2, uj * total);
         } else {
             // every remaining point coincides with a centre: the j-th
             // smallest index not yet chosen
@@ -1444,7 +1448,7 @@ bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
 }
 
 // D2 = min(D2, |x - the assigned centre of the round|^2) (exact fp64), then
-// the S1 and S2 sums of this 1024-position range from the registers.
+// the S1 sums of this 1024-position range from the registers.
 template <typename T, int D>
 __global__ void __launch_bounds__(kSeedThreads)
 bseed_update(const T *__restrict__ x, const BSeedArgs a) {
@@ -1455,7 +1459,6 @@ bseed_update(const T *__restrict__ x, const BSeedArgs a) {
     const T *xh = x + hN * D;
     const T *cbh = static_cast<const T *>(a.cb) + (size_t)h * a.B * D;
     double *d2h = a.d2 + hN;
-    __shared__ double s1own[kSeedS];
     const int p0 = blockIdx.x * kSeedS * kSeedS, p1 = min(N, p0 + kSeedS * kSeedS);
     const int q = seed_row<T, D>(lane);
     for (int base = p0 + warp * 32; base < p1; base += kSeedWarps * 32) {
@@ -1476,17 +1479,7 @@ bseed_update(const T *__restrict__ x, const BSeedArgs a) {
 #pragma unroll
         for (int j = 0; j < kSeedS; ++j)
             v += __shfl_sync(0xffffffffu, fin, (j % Gm::PPL) * Gm::LPP + j / Gm::PPL);
-        if (lane == 0) {
-            a.bs1[(size_t)h * a.NR1 + base / kSeedS] = v;
-            s1own[(base - p0) / kSeedS] = v;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const int k0 = p0 / kSeedS, k1 = (p1 + kSeedS - 1) / kSeedS;
-        double v = 0.0;
-        for (int k = k0; k < k1; ++k) v += s1own[k - k0];
-        a.bs2[(size_t)h * a.NR2 + blockIdx.x] = v;
+        if (lane == 0) a.bs1[(size_t)h * a.NR1 + base / kSeedS] = v;
     }
 }
 
@@ -1962,7 +1955,7 @@ cudaError_t asm_kmeanspp_launch(const void *x, int H, int N, int d, int K, const
 // ---- batched seeding: workspace and the host loop of rounds
 namespace {
 struct BSeedWs {
-    size_t off_d2, off_bs1, off_bs2, off_taken, off_st, off_key, off_cb, off_aws, total;
+    size_t off_d2, off_bs1, off_xn, off_taken, off_st, off_key, off_cb, off_aws, total;
     int nr1, nr2;
 };
 BSeedWs bseed_ws(int H, int N, int d, int K, int B) {
@@ -1975,8 +1968,8 @@ BSeedWs bseed_ws(int H, int N, int d, int K, int B) {
     w.off_aws = 0;
     w.off_d2 = al256(w.off_aws + asm_kmeans_ws_bytes(H, N, d, B));
     w.off_bs1 = al256(w.off_d2 + sizeof(double) * h * n);
-    w.off_bs2 = al256(w.off_bs1 + sizeof(double) * h * w.nr1);
-    w.off_taken = al256(w.off_bs2 + sizeof(double) * h * w.nr2);
+    w.off_xn = al256(w.off_bs1 + sizeof(double) * h * w.nr1);
+    w.off_taken = al256(w.off_xn + sizeof(float) * h * n);
     w.off_st = al256(w.off_taken + h * n);
     w.off_key = al256(w.off_st + sizeof(int) * 4 * h);
     w.off_cb = al256(w.off_key + sizeof(int32_t) * h * n);
@@ -1985,16 +1978,32 @@ BSeedWs bseed_ws(int H, int N, int d, int K, int B) {
 }
 
 template <typename T, int D>
-cudaError_t bseed_all(const T *x, BSeedArgs &a, int H, asm_dtype dt, void *aws, cudaStream_t st) {
+cudaError_t bseed_all(const T *x, BSeedArgs &a, int H, asm_dtype dt, void *aws, int num_sms, cudaStream_t st) {
     const int N = a.N;
     bseed_first<T, D><<<dim3((N + kSeedThreads - 1) / kSeedThreads, H), kSeedThreads, 0, st>>>(x, a);
     bseed_sums<<<dim3((a.NR1 + kSeedThreads - 1) / kSeedThreads, H), kSeedThreads, 0, st>>>(a);
+    const KmWs kw = km_ws(H, N, a.B);
+    float *norms = reinterpret_cast<float *>(static_cast<char *>(aws) + kw.off_norm);
+    __nv_bfloat16 *bias = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(aws) + kw.off_bias);
+    const int sms = num_sms;
     auto round = [&]() -> cudaError_t {
         bseed_pick<T, D><<<H, kSeedThreads, 0, st>>>(x, a);
-        cudaError_t e = asm_kmeans_assign_launch(x, a.cb, H, N, D, a.B, 0, dt, a.key, aws, 0, st);
-        if (e != cudaSuccess) return e;
-        bseed_update<T, D><<<dim3(a.NR2, H), kSeedThreads, 0, st>>>(x, a);
-        return cudaGetLastError();
+        if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
+            // fused: tensor-core nearest centre, screened exact D2 update, S1 sums
+            const int HB = H * a.B;
+            centroid_norms<T, 128><<<(HB * 32 + 255) / 256, 256, 0, st>>>(static_cast<const T *>(a.cb), HB, norms,
+                                                                          bias);
+            return asm_bseed_round_tc_launch(x, a.cb, norms, bias, a.xn, a.d2, a.bs1, a.st, H, N, a.B, a.NR1, sms,
+                                             a.err, st);
+        } else {
+            (void)norms;
+            (void)bias;
+            (void)sms;
+            cudaError_t e = asm_kmeans_assign_launch(x, a.cb, H, N, D, a.B, 0, dt, a.key, aws, 0, st);
+            if (e != cudaSuccess) return e;
+            bseed_update<T, D><<<dim3(a.NR2, H), kSeedThreads, 0, st>>>(x, a);
+            return cudaGetLastError();
+        }
     };
     const int main_rounds = (a.K - 1 + a.B - 1) / a.B;
     cudaError_t e = cudaGetLastError();
@@ -2027,7 +2036,8 @@ size_t asm_kmeanspp_batched_ws_bytes(int H, int N, int d, int K, int batch) {
 }
 
 cudaError_t asm_kmeanspp_batched_launch(const void *x, int H, int N, int d, int K, int batch, const double *u,
-                                        int U, asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st) {
+                                        int U, asm_dtype dt, int32_t *init_idx, void *ws, int num_sms,
+                                        cudaStream_t st) {
     const BSeedWs w = bseed_ws(H, N, d, K, batch);
     if (w.nr2 > kBSeedMaxNR2 || batch > kBSeedMaxB) return cudaErrorInvalidValue;
     char *b = static_cast<char *>(ws);
@@ -2036,7 +2046,7 @@ cudaError_t asm_kmeanspp_batched_launch(const void *x, int H, int N, int d, int 
     a.idx = init_idx;
     a.d2 = reinterpret_cast<double *>(b + w.off_d2);
     a.bs1 = reinterpret_cast<double *>(b + w.off_bs1);
-    a.bs2 = reinterpret_cast<double *>(b + w.off_bs2);
+    a.xn = (dt == ASM_BF16 && d == 128) ? reinterpret_cast<float *>(b + w.off_xn) : nullptr;
     a.taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
     a.st = reinterpret_cast<int *>(b + w.off_st);
     a.key = reinterpret_cast<int32_t *>(b + w.off_key);
@@ -2053,11 +2063,11 @@ cudaError_t asm_kmeanspp_batched_launch(const void *x, int H, int N, int d, int 
     if (e != cudaSuccess) return e;
     if (dt == ASM_BF16) {
         using T = __nv_bfloat16;
-        return d == 128 ? bseed_all<T, 128>((const T *)x, a, H, dt, b + w.off_aws, st)
-                        : bseed_all<T, 64>((const T *)x, a, H, dt, b + w.off_aws, st);
+        return d == 128 ? bseed_all<T, 128>((const T *)x, a, H, dt, b + w.off_aws, num_sms, st)
+                        : bseed_all<T, 64>((const T *)x, a, H, dt, b + w.off_aws, num_sms, st);
     }
-    return d == 128 ? bseed_all<float, 128>((const float *)x, a, H, dt, b + w.off_aws, st)
-                    : bseed_all<float, 64>((const float *)x, a, H, dt, b + w.off_aws, st);
+    return d == 128 ? bseed_all<float, 128>((const float *)x, a, H, dt, b + w.off_aws, num_sms, st)
+                    : bseed_all<float, 64>((const float *)x, a, H, dt, b + w.off_aws, num_sms, st);
 }
 
 size_t asm_kmeans_ws_bytes(int H, int N, int d, int K) {

@@ -76,7 +76,8 @@ cudaError_t asm_kmeans_init_launch(const void *x, int H, int N, int d, int K, as
                                    cudaStream_t st);
 size_t asm_kmeanspp_batched_ws_bytes(int H, int N, int d, int K, int batch);
 cudaError_t asm_kmeanspp_batched_launch(const void *x, int H, int N, int d, int K, int batch, const double *u,
-                                        int U, asm_dtype dt, int32_t *init_idx, void *ws, cudaStream_t st);
+                                        int U, asm_dtype dt, int32_t *init_idx, void *ws, int num_sms,
+                                        cudaStream_t st);
 cudaError_t asm_kmeans_assign_launch(const void *x, const void *centroids_dt, int H, int N, int d,
                                      int K, int metric, asm_dtype dt, int32_t *assign, void *ws,
                                      int num_sms, cudaStream_t st);
@@ -88,6 +89,11 @@ cudaError_t asm_kmeans_update_launch(const void *x, const int32_t *assign, int H
 // assign_tc.cu: bf16, d = 128 assignment on tcgen05; `err` is the workspace error word
 cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norms, const void *bias, int H, int N,
                                  int K, int metric, int32_t *assign, int *err, cudaStream_t st);
+
+// assign_tc.cu: one fused round of batched k-means++ seeding (bf16, d = 128, B <= 256)
+cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const float *norms, const void *bias,
+                                      const float *xn, double *d2, double *bs1, const int *st, int H, int N,
+                                      int B, int NR1, int num_sms, int *err, cudaStream_t stream);
 
 // merge.cu: online-softmax merge of two state arrays, row by row
 cudaError_t asm_selftest_wait_launch(int polls, int *err, unsigned long long *elapsed_ns, cudaStream_t st);

@@ -34,12 +34,14 @@ def test_batch_of_one_is_kmeanspp(dt, d, N, K):
 
 
 @pytest.mark.parametrize("dt,d,N,K,batch", [("bf16", 128, 8192, 1024, 128), ("bf16", 128, 5000, 700, 32),
+                                             ("bf16", 128, 3001, 900, 200), ("bf16", 128, 2600, 800, 256),
                                              ("f32", 64, 4097, 500, 64), ("bf16", 64, 2048, 256, 256),
                                              ("f32", 128, 1500, 300, 7)])
 def test_batched_seeding_matches_the_oracle(dt, d, N, K, batch):
     """Clustered points, ragged N and K, batches from 7 to 256 draws, both
     storage types and head dims: every pick equals the oracle's, and every
-    head gets K distinct points."""
+    head gets K distinct points.  bf16 with d = 128 runs the fused rounds
+    (one or two centre tiles, the second ragged at 200 draws)."""
     x = inputs.mixture(inputs.BASE_SEED + 62 + N, "bseed_q", 2, N, d, 64, 0.3, dt)
     u = inputs.kmeanspp_uniforms(inputs.BASE_SEED + 63 + K, 2, 2 * K)
     got = gpu_seed_batched(x, u, K, batch)
@@ -47,10 +49,11 @@ def test_batched_seeding_matches_the_oracle(dt, d, N, K, batch):
     assert all(len(set(r.tolist())) == K for r in got)
 
 
-def test_batched_repeats_and_exhausted_points():
+@pytest.mark.parametrize("dt,d", [("f32", 64), ("bf16", 128)])
+def test_batched_repeats_and_exhausted_points(dt, d):
     """Fewer distinct points than centres (sum(D2) reaches 0, then the
     smallest unchosen indices), and draws that repeat within a round."""
-    base = inputs.mixture(inputs.BASE_SEED + 64, "bseed_q", 1, 100, 64, 4, 0.3, "f32")
+    base = inputs.mixture(inputs.BASE_SEED + 64, "bseed_q", 1, 100, d, 4, 0.3, dt)
     x = base.repeat(1, 5, 1).contiguous()  # 500 points, 100 distinct
     u = inputs.kmeanspp_uniforms(inputs.BASE_SEED + 65, 1, 600)
     u[:, 1:9] = 0.37                        # round 1: eight equal draws, one kept
