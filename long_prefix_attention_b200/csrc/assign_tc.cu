@@ -326,59 +326,57 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
 // One round of batched k-means++ seeding (bf16, d = 128, up to 256 centres
 // per round), fused: the nearest of the round's centres for every point (the
 // L2 arg-max above, on tcgen05) and D2 = min(D2, |x - that centre|^2), then
-// the sums of D2 over each 32-point range in index order.
+// the sum of D2 over each 32-point range.
 //
 // D2 must stay exact (fp64 from the stored values), but most points do not
 // move in a round.  The accumulator gives <x, c> - |c|^2 / 2 in fp32, so
 // |x|^2 - 2 * acc approximates |x - c|^2 to within a few 1e-5 of
 // |x|^2 + |c|^2 (131 roundings of 2^-23 each, relative to sum |x_i c_i| and
-// |c|^2 / 2, plus the fp32 norms).  A point whose estimate exceeds its D2 by
-// more than 2^-10 (|x|^2 + |c|^2) keeps D2 unchanged, which the exact
-// distance would also do; the others get the exact fp64 distance from the
-// shared-memory copies of their row and centre, one warp per point (each
-// lane four elements, a butterfly sum).  Points with D2 = 0 cannot move.
+// |c|^2 / 2, plus the fp32 norms).  As |c|^2 <= 2 |x|^2 + 2 |x - c|^2, the
+// margin 2^-9 (3 |x|^2 + 2 |estimate|) is, to first order, at least
+// 2^-9 (|x|^2 + |c|^2), some 40 times the error, and needs no |c|^2.  A
+// point whose estimate exceeds its D2 by more than that keeps D2 unchanged,
+// which the exact distance would also do; the others get the exact fp64
+// distance from the shared-memory copies of their row and centre, one warp
+// per point (each lane four elements, a butterfly sum).  Points with D2 = 0
+// cannot move.
 //
-// Persistent: CTA i owns a contiguous run of the (head, 256-point tile)
-// items, so the round's centres of a head are loaded once per CTA (at most
-// twice).  Warp 0 streams the point tiles (two stages) and the centre tiles,
-// warp 1 issues the MMAs into one TMEM accumulator set ([half][tile] x 128
-// columns), warps 2-9 reduce, screen, update and sum.  Heads with no centre
-// this round are skipped by every role alike.  Every wait is bounded; after a
-// timeout a role stops and the workspace error word is set.
+// Grid (CTAs per head, heads): a CTA owns a contiguous run of one head's
+// 128-point tiles and loads that head's centres once.  Warp 0 streams the
+// point tiles (four stages), warp 1 issues the MMAs into 512 TMEM columns
+// (four accumulators of up to 128 centres, two of up to 256), warps 2-17 are
+// four groups of four (one per TMEM lane quarter), one per accumulator (the
+// last two idle when B > 128), that take the tiles in turn: arg-max, screen,
+// exact update, sums.  A head with no centre this
+// round exits at once.  Every wait is bounded; after a timeout a role stops
+// and the workspace error word is set.
 namespace bsr {
 
+constexpr int kTile = 128;                    // points per item (one M = 128 MMA)
 constexpr int kMaxTiles = 2;                  // centre tiles of 128: B <= 256
-constexpr int kXStages = 2;
-constexpr int kThreads = (2 + atc::kEpiWarps) * 32;
-constexpr uint32_t kTmemCols = 512;           // [half][tile] x 128 fp32 columns
+constexpr int kXStages = 4;
+constexpr int kGroups = 4;                    // epilogue groups of four warps
+constexpr int kThreads = (2 + 4 * kGroups) * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kXBytes = 2 * atc::kSub;        // [k-half] 128-row boxes
 
 struct Smem {
-    unsigned char x[kXStages][atc::kABytes];    // [half][k-half] 128-row boxes
+    unsigned char x[kXStages][kXBytes];
     unsigned char c[kMaxTiles][atc::kBBytes];   // [k-half] 128-row boxes
     unsigned char ce[kMaxTiles][atc::kEBytes];  // bias parts of the centres
     unsigned char ae[atc::kEBytes];             // the ones they multiply
-    uint64_t x_full[kXStages], x_empty[kXStages], c_full, c_empty, acc_full, acc_empty;
+    uint64_t x_full[kXStages], x_empty[kXStages], acc_full[4], acc_empty[4], c_full;
     uint32_t tmem_base;
 };
 
 struct Args {
     const float *xn;     // [H][N] |x|^2 (fp32)
-    const float *cn;     // [H][B] |c|^2 (fp32) of the round's centres
     double *d2;          // [H][N]
     double *bs1;         // [H][NR1] D2 sums of 32-point ranges
     const int *st;       // [H][4]; st[4h + 2] = centres kept this round (0: none)
     int *err;
-    int N, B, NR1, tiles, items;  // tiles: 256-point tiles per head; items = H * tiles
+    int N, B, NR1, tiles;  // tiles: 128-point tiles per head
 };
-
-__device__ __forceinline__ bool live(const Args &a, int it) { return a.st[4 * (it / a.tiles) + 2] != 0; }
-
-// The first live item after `it` in [it + 1, i1), or i1.
-__device__ __forceinline__ int next_live(const Args &a, int it, int i1) {
-    for (++it; it < i1; ++it)
-        if (live(a, it)) break;
-    return it;
-}
 
 __device__ __forceinline__ double bf16_lo(uint32_t w) { return (double)__uint_as_float(w << 16); }
 __device__ __forceinline__ double bf16_hi(uint32_t w) { return (double)__uint_as_float(w & 0xFFFF0000u); }
@@ -388,20 +386,29 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
     using namespace atc;
     extern __shared__ unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int h = blockIdx.y;
+    if (a.st[4 * h + 2] == 0) return;  // no centre this round: D2 and the sums stand
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int i0 = (int)((long long)blockIdx.x * a.items / gridDim.x);
-    const int i1 = (int)((long long)(blockIdx.x + 1) * a.items / gridDim.x);
+    const int t0 = (int)((long long)blockIdx.x * a.tiles / gridDim.x);
+    const int t1 = (int)((long long)(blockIdx.x + 1) * a.tiles / gridDim.x);
+    const int nitems = t1 - t0;
     const int B = a.B, N = a.N, ntiles = (B + kN - 1) / kN;
+    // accumulators of ntiles x 128 columns, one per epilogue group: a group
+    // consumes every phase of its accumulator's barriers (sharing one between
+    // two groups would let a group's parity wait pass on the other's phase)
+    const int nacc = ntiles == 1 ? 4 : 2;
+    const size_t hN = (size_t)h * N;
 
     if (tid == 0) {
         for (int s = 0; s < kXStages; ++s) {
             mbar_init(&sm.x_full[s], 1);
-            mbar_init(&sm.x_empty[s], kEpiWarps);
+            mbar_init(&sm.x_empty[s], 4);
+        }
+        for (int b = 0; b < 4; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 4);
         }
         mbar_init(&sm.c_full, 1);
-        mbar_init(&sm.c_empty, 1 + kEpiWarps);
-        mbar_init(&sm.acc_full, 1);
-        mbar_init(&sm.acc_empty, kEpiWarps);
         fence_mbar_init();
     }
     for (int i = tid; i < kEBytes / 16; i += kThreads) {  // the ones of the bias step
@@ -423,28 +430,19 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            int j = 0, cur_h = -1, loads = 0;
-            for (int it = i0; it < i1 && ok; ++it) {
-                if (!live(a, it)) continue;
-                const int h = it / a.tiles, p0 = (it - h * a.tiles) * kM, s = j & 1;
-                if (j >= kXStages && !(ok = mbar_wait(&sm.x_empty[s], ((j >> 1) - 1) & 1))) break;
-                mbar_arrive_expect_tx(&sm.x_full[s], kABytes);
-                for (int m = 0; m < 2; ++m)
-                    for (int kh = 0; kh < 2; ++kh)
-                        tma_load_3d(sm.x[s] + (m * 2 + kh) * kSub, &maps.x, kh * 64, p0 + m * kMH, h, &sm.x_full[s]);
-                if (h != cur_h) {
-                    // the previous head's MMAs and exact distances are done with the centres
-                    if (loads > 0 && !(ok = mbar_wait(&sm.c_empty, (loads - 1) & 1))) break;
-                    mbar_arrive_expect_tx(&sm.c_full, (uint32_t)ntiles * (kBBytes + kEBytes));
-                    for (int t = 0; t < ntiles; ++t) {
-                        tma_load_3d(sm.c[t], &maps.c, 0, t * kN, h, &sm.c_full);
-                        tma_load_3d(sm.c[t] + kSub, &maps.c, 64, t * kN, h, &sm.c_full);
-                        tma_load_3d(sm.ce[t], &maps.e, 0, t * kN, h, &sm.c_full);
-                    }
-                    cur_h = h;
-                    ++loads;
-                }
-                ++j;
+            mbar_arrive_expect_tx(&sm.c_full, (uint32_t)ntiles * (kBBytes + kEBytes));
+            for (int t = 0; t < ntiles; ++t) {
+                tma_load_3d(sm.c[t], &maps.c, 0, t * kN, h, &sm.c_full);
+                tma_load_3d(sm.c[t] + kSub, &maps.c, 64, t * kN, h, &sm.c_full);
+                tma_load_3d(sm.ce[t], &maps.e, 0, t * kN, h, &sm.c_full);
+            }
+            for (int j = 0; j < nitems; ++j) {
+                const int s = j % kXStages;
+                if (j >= kXStages && !(ok = mbar_wait(&sm.x_empty[s], ((j / kXStages) - 1) & 1))) break;
+                mbar_arrive_expect_tx(&sm.x_full[s], kXBytes);
+                const int p0 = (t0 + j) * kTile;
+                tma_load_3d(sm.x[s], &maps.x, 0, p0, h, &sm.x_full[s]);
+                tma_load_3d(sm.x[s] + kSub, &maps.x, 64, p0, h, &sm.x_full[s]);
             }
         }
         __syncwarp();
@@ -452,90 +450,65 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
         // ------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kN >> 3) << 17) |
-                                   ((uint32_t)(kMH >> 4) << 24);
-            int j = 0, cur_h = -1, loads = 0;
-            for (int it = i0; it < i1 && ok; ++it) {
-                if (!live(a, it)) continue;
-                const int h = it / a.tiles, s = j & 1;
-                if (h != cur_h) {
-                    if (!(ok = mbar_wait(&sm.c_full, loads & 1))) break;
-                    cur_h = h;
-                    ++loads;
-                }
-                if (!(ok = mbar_wait(&sm.x_full[s], (j >> 1) & 1))) break;
-                if (j >= 1 && !(ok = mbar_wait(&sm.acc_empty, (j - 1) & 1))) break;
+                                   ((uint32_t)(kTile >> 4) << 24);
+            ok = mbar_wait(&sm.c_full, 0);
+            for (int j = 0; j < nitems && ok; ++j) {
+                const int s = j % kXStages, b = j % nacc, u = j / nacc;
+                if (!(ok = mbar_wait(&sm.x_full[s], (j / kXStages) & 1))) break;
+                if (u >= 1 && !(ok = mbar_wait(&sm.acc_empty[b], (u - 1) & 1))) break;
                 tc_fence_after();
                 const uint32_t x_base = smem_addr(sm.x[s]);
-                for (int m = 0; m < 2; ++m)
-                    for (int t = 0; t < ntiles; ++t) {
-                        const uint32_t d = tmem + (uint32_t)((m * kMaxTiles + t) * kN);
-                        const uint32_t c_base = smem_addr(sm.c[t]);
+                for (int t = 0; t < ntiles; ++t) {
+                    const uint32_t d = tmem + (uint32_t)((b * ntiles + t) * kN);
+                    const uint32_t c_base = smem_addr(sm.c[t]);
 #pragma unroll
-                        for (int k = 0; k < kD / 16; ++k) {
-                            const uint32_t koff = (uint32_t)((k >> 2) * kSub + (k & 3) * 32);
-                            umma_bf16(d, sdesc_sw128(x_base + (uint32_t)(m * 2 * kSub) + koff),
-                                      sdesc_sw128(c_base + koff), idesc, k > 0 ? 1u : 0u);
-                        }
-                        umma_bf16(d, sdesc_sw32(smem_addr(sm.ae)), sdesc_sw32(smem_addr(sm.ce[t])), idesc, 1u);
+                    for (int k = 0; k < kD / 16; ++k) {
+                        const uint32_t koff = (uint32_t)((k >> 2) * kSub + (k & 3) * 32);
+                        umma_bf16(d, sdesc_sw128(x_base + koff), sdesc_sw128(c_base + koff), idesc, k > 0 ? 1u : 0u);
                     }
-                umma_commit(&sm.acc_full);
-                const int nx = next_live(a, it, i1);
-                if (nx < i1 && nx / a.tiles != h) umma_commit(&sm.c_empty);
-                ++j;
+                    umma_bf16(d, sdesc_sw32(smem_addr(sm.ae)), sdesc_sw32(smem_addr(sm.ce[t])), idesc, 1u);
+                }
+                umma_commit(&sm.acc_full[b]);
             }
         }
         __syncwarp();
     } else {
         // ------------------------------- arg-max, screen, exact D2, sums
-        const int e = warp - 2, m = e >> 2, q = warp & 3;
-        const int r = q * 32 + lane;                // row within the half
+        const int e = warp - 2, g = e >> 2, q = warp & 3;  // group, TMEM lane quarter
         const int kh = lane >> 4, ch = (lane & 15) >> 1, hb = (lane & 1) << 3;  // this lane's 4 elements
-        int j = 0, cur_h = -1, loads = 0;
-        for (int it = i0; it < i1 && ok; ++it) {
-            if (!live(a, it)) continue;
-            const int h = it / a.tiles, s = j & 1;
-            if (h != cur_h) {  // the head's centres are read below for exact distances
-                if (!(ok = mbar_wait(&sm.c_full, loads & 1))) break;
-                cur_h = h;
-                ++loads;
-            }
-            const int base = (it - h * a.tiles) * kM + m * kMH + q * 32;  // this warp's 32 points
+        if (g >= nacc) goto done;                          // two groups when B > 128
+        if (!(ok = mbar_wait(&sm.c_full, 0))) goto done;  // centres read below for exact distances
+        for (int j = g; j < nitems; j += nacc) {
+            const int s = j % kXStages, b = j % nacc;
+            const int base = (t0 + j) * kTile + q * 32;  // this warp's 32 points
             const int p = base + lane;
-            const size_t hN = (size_t)h * N;
             const bool inb = p < N;
             const double dold = inb ? __ldcg(a.d2 + hN + p) : 0.0;
             const float xnv = inb ? __ldg(a.xn + hN + p) : 0.f;
-            if (!(ok = mbar_wait(&sm.x_full[s], (j >> 1) & 1))) break;
-            if (!(ok = mbar_wait(&sm.acc_full, j & 1))) break;
+            if (!(ok = mbar_wait(&sm.x_full[s], (j / kXStages) & 1))) break;
+            if (!(ok = mbar_wait(&sm.acc_full[b], (j / nacc) & 1))) break;
             tc_fence_after();
             float best = kNegInf;
             int bidx = 0;
             for (int t = 0; t < ntiles; ++t) {
                 const int nv = min(kN, B - t * kN);
-                const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((m * kMaxTiles + t) * kN);
+                const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((b * ntiles + t) * kN);
 #pragma unroll 1
-                for (int c0 = 0; c0 < kN; c0 += 64) {
+                for (int c0 = 0; c0 < kN; c0 += 32) {
                     if (c0 >= nv) break;
-                    uint32_t r0[32], r1[32];
+                    uint32_t r0[32];
                     tmem_ld32(tb + (uint32_t)c0, r0);
-                    tmem_ld32(tb + (uint32_t)c0 + 32, r1);
                     tmem_wait_ld();
-                    if (nv == kN) {
-                        fold32<0, true>(r0, nullptr, t * kN + c0, 32, best, bidx);
-                        fold32<0, true>(r1, nullptr, t * kN + c0 + 32, 32, best, bidx);
-                    } else {
-                        fold32<0, false>(r0, nullptr, t * kN + c0, nv - c0, best, bidx);
-                        fold32<0, false>(r1, nullptr, t * kN + c0 + 32, nv - c0 - 32, best, bidx);
-                    }
+                    if (nv - c0 >= 32) fold32<0, true>(r0, nullptr, t * kN + c0, 32, best, bidx);
+                    else fold32<0, false>(r0, nullptr, t * kN + c0, nv - c0, best, bidx);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.acc_empty);
+            if (lane == 0) mbar_arrive(&sm.acc_empty[b]);
             // screen: keep D2 where the estimate is clearly above it
-            const float cnv = __ldg(a.cn + (size_t)h * B + bidx);
             const float est = xnv - 2.f * best;
-            const float margin = (xnv + cnv) * 0x1p-10f;
+            const float margin = (3.f * xnv + 2.f * fabsf(est)) * 0x1p-9f;
             const bool flag = inb && dold > 0.0 && !((double)(est - margin) > dold);
             unsigned fm = __ballot_sync(0xffffffffu, flag);
             double fin = dold;
@@ -545,32 +518,27 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
                 const int c = __shfl_sync(0xffffffffu, bidx, src);
                 const int xr = q * 32 + src, cr = c & (kN - 1);
                 const uint2 xv = *reinterpret_cast<const uint2 *>(
-                    sm.x[s] + (m * 2 + kh) * kSub + xr * 128 + (((ch ^ (xr & 7)) << 4) | hb));
+                    sm.x[s] + kh * kSub + xr * 128 + (((ch ^ (xr & 7)) << 4) | hb));
                 const uint2 cv = *reinterpret_cast<const uint2 *>(
                     sm.c[c >> 7] + kh * kSub + cr * 128 + (((ch ^ (cr & 7)) << 4) | hb));
-                double t0 = bf16_lo(xv.x) - bf16_lo(cv.x), t1 = bf16_hi(xv.x) - bf16_hi(cv.x);
-                double t2 = bf16_lo(xv.y) - bf16_lo(cv.y), t3 = bf16_hi(xv.y) - bf16_hi(cv.y);
-                double acc = fma(t3, t3, fma(t2, t2, fma(t1, t1, t0 * t0)));
+                const double u0 = bf16_lo(xv.x) - bf16_lo(cv.x), u1 = bf16_hi(xv.x) - bf16_hi(cv.x);
+                const double u2 = bf16_lo(xv.y) - bf16_lo(cv.y), u3 = bf16_hi(xv.y) - bf16_hi(cv.y);
+                double acc = fma(u3, u3, fma(u2, u2, fma(u1, u1, u0 * u0)));
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
                 if (lane == src && acc < fin) fin = acc;
             }
             if (inb && fin < dold) a.d2[hN + p] = fin;
-            // the 32-point range sum, in index order
-            const double mine = inb ? fin : 0.0;
-            double v = 0.0;
+            // the 32-point range sum (a butterfly: every lane ends with the same value)
+            double v = inb ? fin : 0.0;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) v += __shfl_sync(0xffffffffu, mine, k);
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
             if (lane == 0 && base < N) a.bs1[(size_t)h * a.NR1 + base / 32] = v;
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sm.x_empty[s]);
-                const int nx = next_live(a, it, i1);
-                if (nx < i1 && nx / a.tiles != h) mbar_arrive(&sm.c_empty);
-            }
-            ++j;
+            if (lane == 0) mbar_arrive(&sm.x_empty[s]);
         }
     }
+done:
     if (!ok) atomicExch(a.err, (int)ASM_ERR_TIMEOUT);
     tc_fence_before();
     __syncthreads();
@@ -608,16 +576,16 @@ cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norm
 }
 
 // One fused round of batched seeding (bf16, d = 128, B <= 256 centres per
-// head in `c` [H][B][128]); `norms` [H][B] and `bias` [H][B][16] as for the
-// assignment, `xn` [H][N] |x|^2; D2 and the 32-point sums are updated in place.
-cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const float *norms, const void *bias,
+// head in `c` [H][B][128]); `bias` [H][B][16] as for the assignment, `xn`
+// [H][N] |x|^2; D2 and the 32-point sums are updated in place.
+cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const void *bias,
                                       const float *xn, double *d2, double *bs1, const int *st, int H, int N,
                                       int B, int NR1, int num_sms, int *err, cudaStream_t stream) {
     using namespace asmk;
     if (B < 1 || B > bsr::kMaxTiles * atc::kN) return cudaErrorInvalidValue;
     atc::Maps maps;
     memset(&maps, 0, sizeof(maps));
-    if (!make_map_3d(&maps.x, x, atc::kD, N, H, atc::kMH) || !make_map_3d(&maps.c, c, atc::kD, B, H, atc::kN) ||
+    if (!make_map_3d(&maps.x, x, atc::kD, N, H, bsr::kTile) || !make_map_3d(&maps.c, c, atc::kD, B, H, atc::kN) ||
         !make_map_rows16(&maps.e, bias, B, H, atc::kN))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(bsr::Smem) + 1024;
@@ -625,7 +593,6 @@ cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const float 
     if (e != cudaSuccess) return e;
     bsr::Args a{};
     a.xn = xn;
-    a.cn = norms;
     a.d2 = d2;
     a.bs1 = bs1;
     a.st = st;
@@ -633,9 +600,9 @@ cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const float 
     a.N = N;
     a.B = B;
     a.NR1 = NR1;
-    a.tiles = (N + atc::kM - 1) / atc::kM;
-    a.items = H * a.tiles;
-    const int grid = std::min(std::max(num_sms, 1), a.items);
-    bsr::bseed_round_tc<<<grid, bsr::kThreads, smem, stream>>>(maps, a);
+    a.tiles = (N + bsr::kTile - 1) / bsr::kTile;
+    // CTAs per head: one wave over the heads (at least one), at most one per tile
+    const int per = std::min(std::max(num_sms / H, 1), a.tiles);
+    bsr::bseed_round_tc<<<dim3(per, H), bsr::kThreads, smem, stream>>>(maps, a);
     return cudaGetLastError();
 }

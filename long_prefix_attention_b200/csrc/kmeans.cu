@@ -1993,7 +1993,7 @@ cudaError_t bseed_all(const T *x, BSeedArgs &a, int H, asm_dtype dt, void *aws, 
             const int HB = H * a.B;
             centroid_norms<T, 128><<<(HB * 32 + 255) / 256, 256, 0, st>>>(static_cast<const T *>(a.cb), HB, norms,
                                                                           bias);
-            return asm_bseed_round_tc_launch(x, a.cb, norms, bias, a.xn, a.d2, a.bs1, a.st, H, N, a.B, a.NR1, sms,
+            return asm_bseed_round_tc_launch(x, a.cb, bias, a.xn, a.d2, a.bs1, a.st, H, N, a.B, a.NR1, sms,
                                              a.err, st);
         } else {
             (void)norms;

@@ -91,7 +91,7 @@ cudaError_t asm_assign_tc_launch(const void *x, const void *c, const float *norm
                                  int K, int metric, int32_t *assign, int *err, cudaStream_t st);
 
 // assign_tc.cu: one fused round of batched k-means++ seeding (bf16, d = 128, B <= 256)
-cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const float *norms, const void *bias,
+cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const void *bias,
                                       const float *xn, double *d2, double *bs1, const int *st, int H, int N,
                                       int B, int NR1, int num_sms, int *err, cudaStream_t stream);
 

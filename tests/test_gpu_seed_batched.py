@@ -49,6 +49,16 @@ def test_batched_seeding_matches_the_oracle(dt, d, N, K, batch):
     assert all(len(set(r.tolist())) == K for r in got)
 
 
+@pytest.mark.parametrize("batch", [128, 200])
+def test_batched_many_tiles_per_cta(batch):
+    """32 heads of 4096 points: each CTA of a fused round takes several
+    128-point tiles in turn (four accumulators at 128 draws, two at 200)."""
+    x = inputs.mixture(inputs.BASE_SEED + 69, "bseed_q", 32, 4096, 128, 64, 0.3, "bf16")
+    u = inputs.kmeanspp_uniforms(inputs.BASE_SEED + 70, 32, 1200)
+    got = gpu_seed_batched(x, u, 600, batch)
+    np.testing.assert_array_equal(got, O.kmeanspp_seed_batched(x, u, 600, batch))
+
+
 @pytest.mark.parametrize("dt,d", [("f32", 64), ("bf16", 128)])
 def test_batched_repeats_and_exhausted_points(dt, d):
     """Fewer distinct points than centres (sum(D2) reaches 0, then the
