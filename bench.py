@@ -923,17 +923,18 @@ def build_rooflines(build, tf, hbm, src):
 
 
 def batched_seed_roofline(ms, H, N, d, K, hbm, src):
-    """Per round of the batched seeding: the assignment reads the points and
-    writes their nearest centre, the update reads the points, that index and
-    D2 and writes D2 back: H * N * (4 d + 24) bytes (the round's centres,
-    draws and range sums are negligible)."""
+    """Per round of the batched seeding (bf16, d = 128: one fused kernel): the
+    points are read once, D2 and |x|^2 are read and D2 is written back:
+    H * N * (2 d + 20) bytes (the round's centres, draws and range sums are
+    negligible; D2 is written only where it changed, so this is an upper
+    bound on the writes).  The time per round includes the pick kernel."""
     rounds = (K - 1 + SEED_BATCH - 1) // SEED_BATCH
-    per_round = H * N * (4 * d + 24)
+    per_round = H * N * (2 * d + 20)
     us = ms * 1e3 / rounds
     achieved = per_round / (us * 1e-6) / 1e9
     return {"bound": "hbm", "rounds": rounds, "us_per_round": us, "bytes_per_round": per_round,
             "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-            "peak_source": f"{src} HBM copy"}
+            "peak_source": f"{src} HBM copy", "note": "round time includes the pick kernel"}
 
 
 def main():

@@ -337,39 +337,43 @@ assign_tc_kernel(const __grid_constant__ Maps maps, const float *__restrict__ no
 // 2^-9 (|x|^2 + |c|^2), some 40 times the error, and needs no |c|^2.  A
 // point whose estimate exceeds its D2 by more than that keeps D2 unchanged,
 // which the exact distance would also do; the others get the exact fp64
-// distance from the shared-memory copies of their row and centre, one warp
-// per point (each lane four elements, a butterfly sum).  Points with D2 = 0
-// cannot move.
+// distance, one warp per point (each lane four elements, a butterfly sum),
+// from their row re-read in L2 (streamed in moments before) and their centre
+// in shared memory.  Points with D2 = 0 cannot move.
 //
 // Grid (CTAs per head, heads): a CTA owns a contiguous run of one head's
 // 128-point tiles and loads that head's centres once.  Warp 0 streams the
-// point tiles (four stages), warp 1 issues the MMAs into 512 TMEM columns
-// (four accumulators of up to 128 centres, two of up to 256), warps 2-17 are
-// four groups of four (one per TMEM lane quarter), one per accumulator (the
-// last two idle when B > 128), that take the tiles in turn: arg-max, screen,
-// exact update, sums.  A head with no centre this
-// round exits at once.  Every wait is bounded; after a timeout a role stops
+// point tiles (four stages, each free again once its MMAs finish), warp 1
+// issues the MMAs into 512 TMEM columns (four accumulators of
+// up to 128 centres, two of up to 256), warps 2-17 are four groups of four
+// (one per TMEM lane quarter), one per accumulator (the last two idle when
+// B > 128), that take the tiles in turn: arg-max, screen, exact update, sums.
+// Launched as a dependent of the kernel that picks the round's centres: the
+// set-up and the first point tiles overlap its end.  A head with no centre
+// this round does no more.  Every wait is bounded; after a timeout a role stops
 // and the workspace error word is set.
 namespace bsr {
 
 constexpr int kTile = 128;                    // points per item (one M = 128 MMA)
 constexpr int kMaxTiles = 2;                  // centre tiles of 128: B <= 256
-constexpr int kXStages = 4;
+constexpr int kXStages = 4;                   // point stages (five were measured slower)
 constexpr int kGroups = 4;                    // epilogue groups of four warps
 constexpr int kThreads = (2 + 4 * kGroups) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kXBytes = 2 * atc::kSub;        // [k-half] 128-row boxes
+constexpr int kExact = 4;                     // flagged points per batch of exact distances
 
 struct Smem {
-    unsigned char x[kXStages][kXBytes];
-    unsigned char c[kMaxTiles][atc::kBBytes];   // [k-half] 128-row boxes
+    unsigned char ae[atc::kEBytes];             // the ones the bias parts multiply
     unsigned char ce[kMaxTiles][atc::kEBytes];  // bias parts of the centres
-    unsigned char ae[atc::kEBytes];             // the ones they multiply
+    unsigned char c[kMaxTiles][atc::kBBytes];   // centre tiles ([k-half] 128-row boxes)
+    unsigned char x[kXStages][kXBytes];         // point stages
     uint64_t x_full[kXStages], x_empty[kXStages], acc_full[4], acc_empty[4], c_full;
     uint32_t tmem_base;
 };
 
 struct Args {
+    const __nv_bfloat16 *x;  // [H][N][128] the points (exact distances re-read them from L2)
     const float *xn;     // [H][N] |x|^2 (fp32)
     double *d2;          // [H][N]
     double *bs1;         // [H][NR1] D2 sums of 32-point ranges
@@ -387,7 +391,6 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
     extern __shared__ unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int h = blockIdx.y;
-    if (a.st[4 * h + 2] == 0) return;  // no centre this round: D2 and the sums stand
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t0 = (int)((long long)blockIdx.x * a.tiles / gridDim.x);
     const int t1 = (int)((long long)(blockIdx.x + 1) * a.tiles / gridDim.x);
@@ -397,12 +400,15 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
     // consumes every phase of its accumulator's barriers (sharing one between
     // two groups would let a group's parity wait pass on the other's phase)
     const int nacc = ntiles == 1 ? 4 : 2;
+    constexpr int nst = kXStages;
+    unsigned char *const xs0 = sm.x[0];
+    auto ctile = [&](int t) -> unsigned char * { return t ? sm.c[1] : sm.c[0]; };  // no local array
     const size_t hN = (size_t)h * N;
 
     if (tid == 0) {
         for (int s = 0; s < kXStages; ++s) {
             mbar_init(&sm.x_full[s], 1);
-            mbar_init(&sm.x_empty[s], 4);
+            mbar_init(&sm.x_empty[s], 1);
         }
         for (int b = 0; b < 4; ++b) {
             mbar_init(&sm.acc_full[b], 1);
@@ -427,22 +433,40 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
     const uint32_t tmem = sm.tmem_base;
     bool ok = true;
 
+    // The points do not depend on the preceding kernel (the round's picks):
+    // the first stages stream in before waiting for it.
+    const int pre = min(nst, nitems);
+    auto load_x = [&](int j) {
+        const int s = j % nst;
+        unsigned char *dst = xs0 + (size_t)s * kXBytes;
+        mbar_arrive_expect_tx(&sm.x_full[s], kXBytes);
+        const int p0 = (t0 + j) * kTile;
+        tma_load_3d(dst, &maps.x, 0, p0, h, &sm.x_full[s]);
+        tma_load_3d(dst + kSub, &maps.x, 64, p0, h, &sm.x_full[s]);
+    };
+    if (warp == 0 && lane == 0)
+        for (int j = 0; j < pre; ++j) load_x(j);
+    pdl_wait();
+    if (a.st[4 * h + 2] == 0) {
+        // no centre this round: D2 and the sums stand; the early copies land first
+        if (warp == 0 && lane == 0)
+            for (int j = 0; j < pre; ++j) ok &= mbar_wait(&sm.x_full[j], 0);
+        goto done;
+    }
+
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             mbar_arrive_expect_tx(&sm.c_full, (uint32_t)ntiles * (kBBytes + kEBytes));
             for (int t = 0; t < ntiles; ++t) {
-                tma_load_3d(sm.c[t], &maps.c, 0, t * kN, h, &sm.c_full);
-                tma_load_3d(sm.c[t] + kSub, &maps.c, 64, t * kN, h, &sm.c_full);
+                tma_load_3d(ctile(t), &maps.c, 0, t * kN, h, &sm.c_full);
+                tma_load_3d(ctile(t) + kSub, &maps.c, 64, t * kN, h, &sm.c_full);
                 tma_load_3d(sm.ce[t], &maps.e, 0, t * kN, h, &sm.c_full);
             }
-            for (int j = 0; j < nitems; ++j) {
-                const int s = j % kXStages;
-                if (j >= kXStages && !(ok = mbar_wait(&sm.x_empty[s], ((j / kXStages) - 1) & 1))) break;
-                mbar_arrive_expect_tx(&sm.x_full[s], kXBytes);
-                const int p0 = (t0 + j) * kTile;
-                tma_load_3d(sm.x[s], &maps.x, 0, p0, h, &sm.x_full[s]);
-                tma_load_3d(sm.x[s] + kSub, &maps.x, 64, p0, h, &sm.x_full[s]);
+            for (int j = pre; j < nitems; ++j) {
+                const int s = j % nst;
+                if (!(ok = mbar_wait(&sm.x_empty[s], ((j / nst) - 1) & 1))) break;
+                load_x(j);
             }
         }
         __syncwarp();
@@ -453,14 +477,14 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
                                    ((uint32_t)(kTile >> 4) << 24);
             ok = mbar_wait(&sm.c_full, 0);
             for (int j = 0; j < nitems && ok; ++j) {
-                const int s = j % kXStages, b = j % nacc, u = j / nacc;
-                if (!(ok = mbar_wait(&sm.x_full[s], (j / kXStages) & 1))) break;
+                const int s = j % nst, b = j % nacc, u = j / nacc;
+                if (!(ok = mbar_wait(&sm.x_full[s], (j / nst) & 1))) break;
                 if (u >= 1 && !(ok = mbar_wait(&sm.acc_empty[b], (u - 1) & 1))) break;
                 tc_fence_after();
-                const uint32_t x_base = smem_addr(sm.x[s]);
+                const uint32_t x_base = smem_addr(xs0 + (size_t)s * kXBytes);
                 for (int t = 0; t < ntiles; ++t) {
                     const uint32_t d = tmem + (uint32_t)((b * ntiles + t) * kN);
-                    const uint32_t c_base = smem_addr(sm.c[t]);
+                    const uint32_t c_base = smem_addr(ctile(t));
 #pragma unroll
                     for (int k = 0; k < kD / 16; ++k) {
                         const uint32_t koff = (uint32_t)((k >> 2) * kSub + (k & 3) * 32);
@@ -468,6 +492,7 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
                     }
                     umma_bf16(d, sdesc_sw32(smem_addr(sm.ae)), sdesc_sw32(smem_addr(sm.ce[t])), idesc, 1u);
                 }
+                umma_commit(&sm.x_empty[s]);   // the point stage is free once these MMAs finish
                 umma_commit(&sm.acc_full[b]);
             }
         }
@@ -479,13 +504,12 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
         if (g >= nacc) goto done;                          // two groups when B > 128
         if (!(ok = mbar_wait(&sm.c_full, 0))) goto done;  // centres read below for exact distances
         for (int j = g; j < nitems; j += nacc) {
-            const int s = j % kXStages, b = j % nacc;
+            const int b = j % nacc;
             const int base = (t0 + j) * kTile + q * 32;  // this warp's 32 points
             const int p = base + lane;
             const bool inb = p < N;
             const double dold = inb ? __ldcg(a.d2 + hN + p) : 0.0;
             const float xnv = inb ? __ldg(a.xn + hN + p) : 0.f;
-            if (!(ok = mbar_wait(&sm.x_full[s], (j / kXStages) & 1))) break;
             if (!(ok = mbar_wait(&sm.acc_full[b], (j / nacc) & 1))) break;
             tc_fence_after();
             float best = kNegInf;
@@ -512,21 +536,31 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
             const bool flag = inb && dold > 0.0 && !((double)(est - margin) > dold);
             unsigned fm = __ballot_sync(0xffffffffu, flag);
             double fin = dold;
+            const uint2 *xw = reinterpret_cast<const uint2 *>(a.x + (hN + base) * kD) + lane;  // 4 elements per lane
             while (fm) {
-                const int src = __ffs(fm) - 1;
-                fm &= fm - 1;
-                const int c = __shfl_sync(0xffffffffu, bidx, src);
-                const int xr = q * 32 + src, cr = c & (kN - 1);
-                const uint2 xv = *reinterpret_cast<const uint2 *>(
-                    sm.x[s] + kh * kSub + xr * 128 + (((ch ^ (xr & 7)) << 4) | hb));
-                const uint2 cv = *reinterpret_cast<const uint2 *>(
-                    sm.c[c >> 7] + kh * kSub + cr * 128 + (((ch ^ (cr & 7)) << 4) | hb));
-                const double u0 = bf16_lo(xv.x) - bf16_lo(cv.x), u1 = bf16_hi(xv.x) - bf16_hi(cv.x);
-                const double u2 = bf16_lo(xv.y) - bf16_lo(cv.y), u3 = bf16_hi(xv.y) - bf16_hi(cv.y);
-                double acc = fma(u3, u3, fma(u2, u2, fma(u1, u1, u0 * u0)));
+                // up to kExact flagged points at a time: their rows from L2 (just
+                // streamed), their centres from shared memory
+                int src[kExact];
+                uint2 xv[kExact], cv[kExact];
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (lane == src && acc < fin) fin = acc;
+                for (int k = 0; k < kExact; ++k) {
+                    src[k] = fm ? __ffs(fm) - 1 : -1;
+                    fm &= fm - 1;
+                    const int c = __shfl_sync(0xffffffffu, bidx, max(src[k], 0)), cr = c & (kN - 1);
+                    xv[k] = src[k] >= 0 ? __ldcg(xw + src[k] * (kD / 4)) : make_uint2(0u, 0u);
+                    cv[k] = *reinterpret_cast<const uint2 *>(
+                        ctile(c >> 7) + kh * kSub + cr * 128 + (((ch ^ (cr & 7)) << 4) | hb));
+                }
+#pragma unroll
+                for (int k = 0; k < kExact; ++k) {
+                    if (src[k] < 0) break;  // the same for every lane
+                    const double u0 = bf16_lo(xv[k].x) - bf16_lo(cv[k].x), u1 = bf16_hi(xv[k].x) - bf16_hi(cv[k].x);
+                    const double u2 = bf16_lo(xv[k].y) - bf16_lo(cv[k].y), u3 = bf16_hi(xv[k].y) - bf16_hi(cv[k].y);
+                    double acc = fma(u3, u3, fma(u2, u2, fma(u1, u1, u0 * u0)));
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                    if (lane == src[k] && acc < fin) fin = acc;
+                }
             }
             if (inb && fin < dold) a.d2[hN + p] = fin;
             // the 32-point range sum (a butterfly: every lane ends with the same value)
@@ -534,8 +568,6 @@ bseed_round_tc(const __grid_constant__ atc::Maps maps, const Args a) {
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
             if (lane == 0 && base < N) a.bs1[(size_t)h * a.NR1 + base / 32] = v;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.x_empty[s]);
         }
     }
 done:
@@ -592,6 +624,7 @@ cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const void *
     cudaError_t e = cudaFuncSetAttribute(bsr::bseed_round_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     bsr::Args a{};
+    a.x = static_cast<const __nv_bfloat16 *>(x);
     a.xn = xn;
     a.d2 = d2;
     a.bs1 = bs1;
@@ -603,6 +636,15 @@ cudaError_t asm_bseed_round_tc_launch(const void *x, const void *c, const void *
     a.tiles = (N + bsr::kTile - 1) / bsr::kTile;
     // CTAs per head: one wave over the heads (at least one), at most one per tile
     const int per = std::min(std::max(num_sms / H, 1), a.tiles);
-    bsr::bseed_round_tc<<<dim3(per, H), bsr::kThreads, smem, stream>>>(maps, a);
-    return cudaGetLastError();
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(per, H);
+    cfg.blockDim = dim3(bsr::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, bsr::bseed_round_tc, maps, a);
 }

@@ -1239,6 +1239,7 @@ struct BSeedArgs {
     int *st;                // [H][4]: centres chosen, draws used, kept this round
     int32_t *key;           // [H][N] nearest centre of the round
     void *cb;               // [H][B][D] the round's centres (storage type)
+    __nv_bfloat16 *cbias;   // [H][B][16] bf16 parts of -|c|^2 / 2 (fused rounds), or null
     int *err;
     int N, K, B, U, NR1, NR2;
 };
@@ -1358,6 +1359,7 @@ __global__ void __launch_bounds__(kSeedThreads)
 bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
     const int h = blockIdx.x, N = a.N, K = a.K, B = a.B, tid = threadIdx.x;
     const size_t hN = (size_t)h * N;
+    pdl_launch_dependents();  // the round kernel may set up meanwhile
     __shared__ double S2[kBSeedMaxNR2], P2[kBSeedMaxNR2];
     __shared__ int picks[kBSeedMaxB], keep[kBSeedMaxB], pos[kBSeedMaxB], slotpick[kBSeedMaxB], nkept;
     __shared__ double total_s;
@@ -1438,12 +1440,39 @@ bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
     __syncthreads();
     // the round's centres, then copies of the first one
     const int kept = nkept;
-    constexpr int C16 = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
-    uint4 *cbh = reinterpret_cast<uint4 *>(static_cast<T *>(a.cb) + (size_t)h * B * D);
-    for (int w = tid; w < B * C16; w += kSeedThreads) {
-        const int slot = w / C16, c = w - slot * C16;
-        const int src = slot < kept ? slotpick[slot] : picks[0];
-        cbh[w] = __ldg(reinterpret_cast<const uint4 *>(x + (hN + src) * D) + c);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
+        // one warp per centre, with the three bf16 parts of -|c|^2 / 2 that the
+        // fused round adds on the tensor cores (the sums of centroid_norms)
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int slot = warp; slot < B; slot += kSeedWarps) {
+            const int src = slot < kept ? slotpick[slot] : picks[0];
+            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(x + (hN + src) * D) + lane);
+            reinterpret_cast<uint2 *>(static_cast<T *>(a.cb) + ((size_t)h * B + slot) * D)[lane] = v;
+            const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xFFFF0000u);
+            const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xFFFF0000u);
+            const float sq = warp_sum(fmaf(f3, f3, fmaf(f2, f2, fmaf(f1, f1, f0 * f0))));
+            if (lane < 2) {
+                uint4 row = make_uint4(0u, 0u, 0u, 0u);
+                if (lane == 0) {
+                    const float bb = -0.5f * sq;
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(bb);
+                    const float r1 = bb - __bfloat162float(hi);
+                    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+                    row.x = (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(mid) << 16);
+                    row.y = (uint32_t)__bfloat16_as_ushort(lo);
+                }
+                reinterpret_cast<uint4 *>(a.cbias + ((size_t)h * B + slot) * 16)[lane] = row;
+            }
+        }
+    } else {
+        constexpr int C16 = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
+        uint4 *cbh = reinterpret_cast<uint4 *>(static_cast<T *>(a.cb) + (size_t)h * B * D);
+        for (int w = tid; w < B * C16; w += kSeedThreads) {
+            const int slot = w / C16, c = w - slot * C16;
+            const int src = slot < kept ? slotpick[slot] : picks[0];
+            cbh[w] = __ldg(reinterpret_cast<const uint4 *>(x + (hN + src) * D) + c);
+        }
     }
 }
 
@@ -1982,22 +2011,15 @@ cudaError_t bseed_all(const T *x, BSeedArgs &a, int H, asm_dtype dt, void *aws, 
     const int N = a.N;
     bseed_first<T, D><<<dim3((N + kSeedThreads - 1) / kSeedThreads, H), kSeedThreads, 0, st>>>(x, a);
     bseed_sums<<<dim3((a.NR1 + kSeedThreads - 1) / kSeedThreads, H), kSeedThreads, 0, st>>>(a);
-    const KmWs kw = km_ws(H, N, a.B);
-    float *norms = reinterpret_cast<float *>(static_cast<char *>(aws) + kw.off_norm);
-    __nv_bfloat16 *bias = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(aws) + kw.off_bias);
     const int sms = num_sms;
     auto round = [&]() -> cudaError_t {
         bseed_pick<T, D><<<H, kSeedThreads, 0, st>>>(x, a);
         if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
             // fused: tensor-core nearest centre, screened exact D2 update, S1 sums
-            const int HB = H * a.B;
-            centroid_norms<T, 128><<<(HB * 32 + 255) / 256, 256, 0, st>>>(static_cast<const T *>(a.cb), HB, norms,
-                                                                          bias);
-            return asm_bseed_round_tc_launch(x, a.cb, bias, a.xn, a.d2, a.bs1, a.st, H, N, a.B, a.NR1, sms,
+            // (the pick wrote the centres' bias parts)
+            return asm_bseed_round_tc_launch(x, a.cb, a.cbias, a.xn, a.d2, a.bs1, a.st, H, N, a.B, a.NR1, sms,
                                              a.err, st);
         } else {
-            (void)norms;
-            (void)bias;
             (void)sms;
             cudaError_t e = asm_kmeans_assign_launch(x, a.cb, H, N, D, a.B, 0, dt, a.key, aws, 0, st);
             if (e != cudaSuccess) return e;
@@ -2046,7 +2068,9 @@ cudaError_t asm_kmeanspp_batched_launch(const void *x, int H, int N, int d, int 
     a.idx = init_idx;
     a.d2 = reinterpret_cast<double *>(b + w.off_d2);
     a.bs1 = reinterpret_cast<double *>(b + w.off_bs1);
-    a.xn = (dt == ASM_BF16 && d == 128) ? reinterpret_cast<float *>(b + w.off_xn) : nullptr;
+    const bool fused = dt == ASM_BF16 && d == 128;
+    a.xn = fused ? reinterpret_cast<float *>(b + w.off_xn) : nullptr;
+    a.cbias = fused ? reinterpret_cast<__nv_bfloat16 *>(b + w.off_aws + km_ws(H, N, batch).off_bias) : nullptr;
     a.taken = reinterpret_cast<unsigned char *>(b + w.off_taken);
     a.st = reinterpret_cast<int *>(b + w.off_st);
     a.key = reinterpret_cast<int32_t *>(b + w.off_key);
