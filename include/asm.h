@@ -162,9 +162,11 @@ size_t asm_kmeanspp_workspace_size(int H, int N, int d, int K);
  *   ws       asm_kmeanspp_batched_workspace_size(H, N, d, K, batch) bytes;
  *            its word 0 is the error word (asm_workspace_error)
  * Requires 1 <= K <= N, 1 <= batch <= 256, U >= 1; N > 2^21 returns
- * ASM_ERR_UNSUPPORTED.  Four launches per round; synchronises `stream`
- * once, after about K / batch rounds, to see whether repeated draws left
- * any head short.
+ * ASM_ERR_UNSUPPORTED.  Two launches per round for bf16 with d = 128 (the
+ * draws, then one fused pass: tensor-core nearest centre, D2 update, sums),
+ * four otherwise.  Synchronises `stream` after about K / batch rounds to see
+ * whether repeated draws left any head short, and again after each of the
+ * (at most 16) extra rounds that then run.
  */
 size_t asm_kmeanspp_batched_workspace_size(int H, int N, int d, int K, int batch);
 asm_status asm_kmeanspp_seed_batched(const void *x, int H, int N, int d, int K, int batch,

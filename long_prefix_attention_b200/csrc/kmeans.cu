@@ -1444,25 +1444,36 @@ bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
         // one warp per centre, with the three bf16 parts of -|c|^2 / 2 that the
         // fused round adds on the tensor cores (the sums of centroid_norms)
         const int warp = tid >> 5, lane = tid & 31;
-        for (int slot = warp; slot < B; slot += kSeedWarps) {
-            const int src = slot < kept ? slotpick[slot] : picks[0];
-            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(x + (hN + src) * D) + lane);
-            reinterpret_cast<uint2 *>(static_cast<T *>(a.cb) + ((size_t)h * B + slot) * D)[lane] = v;
-            const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xFFFF0000u);
-            const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xFFFF0000u);
-            const float sq = warp_sum(fmaf(f3, f3, fmaf(f2, f2, fmaf(f1, f1, f0 * f0))));
-            if (lane < 2) {
-                uint4 row = make_uint4(0u, 0u, 0u, 0u);
-                if (lane == 0) {
-                    const float bb = -0.5f * sq;
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(bb);
-                    const float r1 = bb - __bfloat162float(hi);
-                    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-                    row.x = (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(mid) << 16);
-                    row.y = (uint32_t)__bfloat16_as_ushort(lo);
+        constexpr int kRows = 8;  // rows in flight per warp
+        for (int s0 = warp; s0 < B; s0 += kSeedWarps * kRows) {
+            uint2 v[kRows];
+#pragma unroll
+            for (int k = 0; k < kRows; ++k) {
+                const int slot = s0 + k * kSeedWarps;
+                const int src = slot < kept ? slotpick[slot] : picks[0];
+                v[k] = slot < B ? __ldg(reinterpret_cast<const uint2 *>(x + (hN + src) * D) + lane) : make_uint2(0u, 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < kRows; ++k) {
+                const int slot = s0 + k * kSeedWarps;
+                if (slot >= B) break;  // the same for every lane
+                reinterpret_cast<uint2 *>(static_cast<T *>(a.cb) + ((size_t)h * B + slot) * D)[lane] = v[k];
+                const float f0 = __uint_as_float(v[k].x << 16), f1 = __uint_as_float(v[k].x & 0xFFFF0000u);
+                const float f2 = __uint_as_float(v[k].y << 16), f3 = __uint_as_float(v[k].y & 0xFFFF0000u);
+                const float sq = warp_sum(fmaf(f3, f3, fmaf(f2, f2, fmaf(f1, f1, f0 * f0))));
+                if (lane < 2) {
+                    uint4 row = make_uint4(0u, 0u, 0u, 0u);
+                    if (lane == 0) {
+                        const float bb = -0.5f * sq;
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(bb);
+                        const float r1 = bb - __bfloat162float(hi);
+                        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+                        const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+                        row.x = (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(mid) << 16);
+                        row.y = (uint32_t)__bfloat16_as_ushort(lo);
+                    }
+                    reinterpret_cast<uint4 *>(a.cbias + ((size_t)h * B + slot) * 16)[lane] = row;
                 }
-                reinterpret_cast<uint4 *>(a.cbias + ((size_t)h * B + slot) * 16)[lane] = row;
             }
         }
     } else {
