@@ -894,6 +894,38 @@ def run_decode_large(cfg, layers, steps, warmup, world, rank, hbm, src):
     return out
 
 
+# ncu's sm__pipe_tensor_cycles_active (percent of active cycles) of the build
+# stages' tensor-core kernels, from one `--set full` capture each (the
+# profiles named), with the digest of the kernel's source text they were taken
+# on: a changed kernel reports null until it is captured again.
+NCU_TENSOR = {
+    "states": {"pct": None, "profile": "profiles/states_tc_build_n65536_l4096.md",
+               "file": "build_states_tc.cu", "begin": "states_tc_kernel(const __grid_constant__",
+               "end": "}  // namespace stc", "source": "36063807717c30d6"},
+    "lloyd": {"pct": 59.7, "profile": "profiles/assign_tc_build_n65536_k8192.md",
+              "file": "assign_tc.cu", "begin": "assign_tc_kernel(const __grid_constant__",
+              "end": "}  // namespace atc", "source": "d76c541cd98fb6cd"},
+}
+
+
+def kernel_digest(name, begin, end):
+    import hashlib
+    with open(os.path.join(ROOT, "long_prefix_attention_b200", "csrc", name)) as f:
+        text = f.read()
+    i = text.find(begin)
+    j = text.find(end, i) if i >= 0 else -1
+    if i < 0 or j < 0:
+        return None
+    return hashlib.sha256(text[i:j].encode()).hexdigest()[:16]
+
+
+def recorded_tensor_pipe(stage):
+    rec = NCU_TENSOR[stage]
+    if rec["pct"] is None or kernel_digest(rec["file"], rec["begin"], rec["end"]) != rec["source"]:
+        return None
+    return {"sm__pipe_tensor_cycles_active_pct": rec["pct"], "profile": rec["profile"]}
+
+
 def build_rooflines(build, tf, hbm, src):
     """Each build stage against the roofline that bounds it: the states and
     the assignment on the bf16 tensor peak (flops of the definition), the
@@ -909,10 +941,12 @@ def build_rooflines(build, tf, hbm, src):
     agg = agg_bytes / (ms["aggregate"] / 1e3) / 1e9
     return {
         "states": {"bound": "tensor", "achieved": states, "peak": tf, "unit": "TFLOP/s", "frac": states / tf,
-                   "peak_source": f"{src} bf16", "flops": 4.0 * N * L * d * H},
+                   "peak_source": f"{src} bf16", "flops": 4.0 * N * L * d * H,
+                   "ncu": recorded_tensor_pipe("states")},
         "lloyd": {"bound": "tensor", "achieved": lloyd, "peak": tf, "unit": "TFLOP/s", "frac": lloyd / tf,
                   "peak_source": f"{src} bf16", "flops": 2.0 * N * K * d * H * iters,
-                  "note": "assignment flops over the 10 rounds, update included in the time"},
+                  "note": "assignment flops over the 10 rounds, update included in the time",
+                  "ncu": recorded_tensor_pipe("lloyd")},
         "aggregate": {"bound": "hbm", "achieved": agg, "peak": hbm, "unit": "GB/s", "frac": agg / hbm,
                       "peak_source": f"{src} HBM copy", "bytes": agg_bytes},
         "kmeanspp_seed": {"bound": "sequential rounds", "rounds": K,
