@@ -87,6 +87,8 @@ def test_workspace_sizes_grow_with_the_problem(lib):
     assert lib.asm_flash_decode_workspace_size(1, 32, 8, 32768, 2048, 128, 1) > 0
     assert lib.asm_kmeans_workspace_size(32, 65536, 128, 8192) > 0
     assert lib.asm_kmeanspp_workspace_size(32, 65536, 128, 8192) > 0
+    assert 0 < lib.asm_kmeanspp_batched_workspace_size(2, 4096, 128, 256, 32) < \
+        lib.asm_kmeanspp_batched_workspace_size(32, 65536, 128, 8192, 128)
 
 
 def test_build_and_kmeans_validation(lib):
@@ -98,6 +100,17 @@ def test_build_and_kmeans_validation(lib):
     # k-means++: K > N, small workspace
     assert lib.asm_kmeanspp_seed(P, 2, 10, 64, 11, P, 0, P, P, 1 << 30, None) == INVALID
     assert lib.asm_kmeanspp_seed(P, 2, 10, 64, 4, P, 0, P, P, 8, None) == WORKSPACE
+    # batched k-means++: batch 0 or above 256, no draws, K > N, N above 2^21, small workspace
+    sb = lib.asm_kmeanspp_batched_workspace_size(2, 10, 64, 4, 2)
+    assert sb > 0 and lib.asm_kmeanspp_batched_workspace_size(2, 10, 64, 4, 0) == 0
+    assert lib.asm_kmeanspp_batched_workspace_size(2, 10, 64, 4, 257) == 0
+    assert lib.asm_kmeanspp_seed_batched(P, 2, 10, 64, 4, 0, P, 8, 0, P, P, 1 << 30, None) == INVALID
+    assert lib.asm_kmeanspp_seed_batched(P, 2, 10, 64, 4, 257, P, 8, 0, P, P, 1 << 30, None) == UNSUPPORTED
+    assert lib.asm_kmeanspp_seed_batched(P, 2, 10, 64, 4, 2, P, 0, 0, P, P, 1 << 30, None) == INVALID
+    assert lib.asm_kmeanspp_seed_batched(P, 2, 10, 64, 11, 2, P, 8, 0, P, P, 1 << 30, None) == INVALID
+    assert lib.asm_kmeanspp_seed_batched(P, 1, (1 << 21) + 1, 64, 4, 2, P, 8, 0, P, P, 1 << 40,
+                                         None) == UNSUPPORTED
+    assert lib.asm_kmeanspp_seed_batched(P, 2, 10, 64, 4, 2, P, 8, 0, P, P, sb - 1, None) == WORKSPACE
     # k-means: iters < 1, bad metric
     assert lib.asm_kmeans(P, 2, 10, 64, 4, 0, 0, 0, P, P, P, P, P, P, P, P, 1 << 30, None) == INVALID
     assert lib.asm_kmeans(P, 2, 10, 64, 4, 3, 5, 0, P, P, P, P, P, P, P, P, 1 << 30, None) == INVALID

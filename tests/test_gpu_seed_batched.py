@@ -97,3 +97,44 @@ def test_batched_build_shape_prefix():
     assert all(len(set(r.tolist())) == K for r in got[[0, H - 1]])
     ref = O.kmeanspp_seed_batched(bi["q"][:1], u[:1], 1025, batch)
     np.testing.assert_array_equal(got[0, :1000], ref[0, :1000])
+
+
+def test_batched_seeds_feed_lloyd_like_kmeanspp():
+    """The free-running k-means rule applied to batched seeds (bf16, d = 128,
+    the fused rounds): ten Lloyd iterations from the GPU's batched seeds end
+    within 1e-3 relative inertia of the oracle's k-means from the same seeds,
+    with the same number of non-empty clusters.  The seeds' own potential
+    (sum of D2 to the nearest seed, by the oracle's assignment) is within 10%
+    of sequential k-means++'s on the same points."""
+    H, N, d, K, batch = 2, 4096, 128, 256, 32
+    x = inputs.mixture(inputs.BASE_SEED + 71, "bseed_q", H, N, d, 64, 0.3, "bf16")
+    u = inputs.kmeanspp_uniforms(inputs.BASE_SEED + 72, H, 2 * K)
+    seeds = gpu_seed_batched(x, u, K, batch)
+    np.testing.assert_array_equal(seeds, O.kmeanspp_seed_batched(x, u, K, batch))
+
+    xd = x.cuda()
+    c = torch.empty(H, K, d, dtype=torch.float32, device="cuda")
+    cdt = torch.empty(H, K, d, dtype=x.dtype, device="cuda")
+    assign = torch.empty(H, N, dtype=torch.int32, device="cuda")
+    counts = torch.empty(H, K, dtype=torch.int32, device="cuda")
+    perm = torch.empty(H, N, dtype=torch.int32, device="cuda")
+    seg = torch.empty(H, K + 1, dtype=torch.int32, device="cuda")
+    ws = ops.alloc_workspace(ops.asm_kmeans_workspace_size(H, N, d, K), "cuda", zero=False)
+    ops.asm_kmeans(xd, torch.from_numpy(seeds).cuda(), 10, c, cdt, assign, counts, perm, seg, ws)
+    torch.cuda.synchronize()
+    oC, _, oa, ocounts, _ = O.kmeans(x, seeds, 10, O.L2, O.BF16)
+    xs = x.to(torch.float64).numpy()
+    ga, gc = assign.cpu().numpy(), c.cpu().to(torch.float64).numpy()
+    for h in range(H):
+        g_in = ((xs[h] - gc[h][ga[h]]) ** 2).sum()
+        o_in = ((xs[h] - oC[h][oa[h]]) ** 2).sum()
+        assert abs(g_in - o_in) <= 1e-3 * o_in
+        assert (counts.cpu().numpy()[h] > 0).sum() == (ocounts[h] > 0).sum()
+
+    seq = O.kmeanspp_seed(x, u[:, :K].contiguous())
+    for h in range(H):
+        pot = []
+        for idx in (seeds[h], seq[h]):
+            a, _ = O.assign(xs[h], xs[h][idx])
+            pot.append(((xs[h] - xs[h][idx][a]) ** 2).sum())
+        assert pot[0] <= 1.1 * pot[1], pot
