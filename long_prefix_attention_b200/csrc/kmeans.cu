@@ -1221,12 +1221,14 @@ __global__ void seed_group_pieces(const SeedArgs s, int G, int ch, int is_static
 // Up to b draws per round from one D2 distribution, repeats within a round
 // dropped, then one D2 update with all the round's centres (the batched
 // seeding of k-means||, Bahmani et al. 2012, without its reclustering): about
-// K / b rounds instead of K.  A round is four launches: the pick (one CTA per
-// head: the draws' inverse-CDF searches over the S2 / S1 / point sums), the
-// norms and the nearest-centre assignment of every point to the round's
-// centres (the tensor-core assignment for bf16, d = 128), and the update
-// (D2 = min(D2, exact fp64 distance to the assigned centre) and the S1 / S2
-// sums of each 1024-position range, in index order).  Heads that have all K
+// K / b rounds instead of K.  A round starts with the pick (one CTA per head:
+// the S2 sums of the S1 sums and their prefix, the draws' inverse-CDF
+// searches over S2 / S1 / point, the kept centres gathered).  For bf16 with
+// d = 128 one fused kernel then does the rest (bseed_round_tc in
+// assign_tc.cu: tensor-core nearest centre, screened exact D2 update, S1
+// sums); otherwise the assignment kernel finds each point's nearest centre
+// of the round and bseed_update sets D2 = min(D2, exact fp64 distance to it)
+// and the S1 sums (32 points each, index order).  Heads that have all K
 // centres skip their work.
 
 struct BSeedArgs {
