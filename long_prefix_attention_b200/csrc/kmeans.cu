@@ -255,6 +255,41 @@ __device__ __forceinline__ double dist32(const uint4 (&buf)[SeedGeo<T, D>::LPP],
     }
     return part[0];
 }
+// |row|^2 in fp32 of the rows load32 read (same lane layout as dist32); for
+// the screen of the fused batched rounds, which allows far more than its error.
+template <typename T, int D>
+__device__ __forceinline__ float sumsq32(const uint4 (&buf)[SeedGeo<T, D>::LPP], int lane) {
+    using G = SeedGeo<T, D>;
+    float part[G::LPP];
+#pragma unroll
+    for (int i = 0; i < G::LPP; ++i) {
+        const uint32_t w[4] = {buf[i].x, buf[i].y, buf[i].z, buf[i].w};
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if constexpr (sizeof(T) == 4) {
+                const float v = __uint_as_float(w[e]);
+                acc = fmaf(v, v, acc);
+            } else {
+                const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+                acc = fmaf(hi, hi, fmaf(lo, lo, acc));
+            }
+        }
+        part[i] = acc;
+    }
+#pragma unroll
+    for (int n = G::LPP; n > 1; n >>= 1) {
+        const int half = n >> 1;
+        const bool up = (lane & half) != 0;
+#pragma unroll
+        for (int k = 0; k < half; ++k) {
+            const float send = up ? part[k] : part[k + half];
+            const float keep = up ? part[k + half] : part[k];
+            part[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+    }
+    return part[0];
+}
 template <typename T, int D>
 __device__ __forceinline__ int seed_row(int lane) {
     using G = SeedGeo<T, D>;
@@ -1276,11 +1311,8 @@ bseed_first(const T *__restrict__ x, const BSeedArgs a) {
     const double dist = dist32<T, D>(buf, cv, lane);
     if ((m >> q) & 1u) a.d2[hN + base + q] = dist;
     if (a.xn != nullptr) {
-        double zero[Gm::E16];
-#pragma unroll
-        for (int e = 0; e < Gm::E16; ++e) zero[e] = 0.0;
-        const double nrm = dist32<T, D>(buf, zero, lane);
-        if ((m >> q) & 1u) a.xn[hN + base + q] = (float)nrm;
+        const float nrm = sumsq32<T, D>(buf, lane);
+        if ((m >> q) & 1u) a.xn[hN + base + q] = nrm;
     }
 }
 
@@ -1421,16 +1453,26 @@ bseed_pick(const T *__restrict__ x, const BSeedArgs a) {
         keep[j] = k;
     }
     __syncthreads();
-    if (tid == 0) {
-        int c = 0;
-        for (int j = 0; j < nb; ++j) {
-            pos[j] = c;
-            c += keep[j];
+    {
+        // positions of the kept draws: a ballot per warp, the warps' counts in order
+        // (nb <= kSeedThreads: one draw per thread)
+        __shared__ int wcnt[kSeedWarps];
+        const int lane = tid & 31, warp = tid >> 5;
+        const unsigned bal = __ballot_sync(0xffffffffu, tid < nb && keep[tid]);
+        if (lane == 0) wcnt[warp] = __popc(bal);
+        __syncthreads();
+        int off = 0, c = 0;
+        for (int w = 0; w < kSeedWarps; ++w) {
+            off += w < warp ? wcnt[w] : 0;
+            c += wcnt[w];
         }
-        nkept = c;
-        st[0] = m + c;
-        st[1] = p + nb;
-        st[2] = c;
+        if (tid < nb) pos[tid] = off + __popc(bal & ((1u << lane) - 1u));
+        if (tid == 0) {
+            nkept = c;
+            st[0] = m + c;
+            st[1] = p + nb;
+            st[2] = c;
+        }
     }
     __syncthreads();
     for (int j = tid; j < nb; j += kSeedThreads)
