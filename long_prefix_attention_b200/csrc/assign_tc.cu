@@ -25,6 +25,10 @@
 //              (cosine: divides by |c|) and keeps a running arg-max (ties go
 //              to the smaller index) while the next tile is multiplied.
 // Every wait is bounded; a timeout sets the workspace error word to 5.
+//
+// The same contraction, against the few centres of one round, drives the
+// fused round of batched k-means++ seeding further down (bseed_round_tc):
+// nearest centre, screened exact D2 update and range sums in one pass.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
